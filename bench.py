@@ -1,0 +1,439 @@
+"""Benchmark of the KDA hot path on B200.
+
+One step = one kda_chunk_fwd over the bf16 prefill workload (B=4, H=16,
+T=2048, d_k=d_v=128, chunk 64, per-channel gates, S0 ~ N(0, 0.02^2)): every
+chunkwise step (cumulative decay, decay-masked products, triangular solve,
+state scan and outputs) runs inside that one launch.  The decode step
+(256 x 32 heads, d=128, fp32 state in HBM, 128 one-token calls after a
+512-token prefill) is measured after it and reported under "decode".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line on rank 0.  Under torchrun each rank runs its own
+replica (weak scaling; the path has no exchange step).  The reference arm
+(--impl reference) times the float64 CPU oracle on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch
+
+METRIC = "KDA prefill tokens/s (% bf16 TC peak); decode step HBM GB/s (% of peak)"
+WORKLOAD = "prefill_b4_h16_t2048"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------ helpers
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def prefill_bytes(w, tokens_per_seq=None):
+    """Algorithmic HBM bytes of one kda_chunk_fwd launch: every input read once,
+    every output written once."""
+    ht = w.B * w.T * w.H
+    el = 2 if w.dtype == "bf16" else 4
+    g = {"channel": 4 * w.d_k, "scalar": 4, "none": 0}[w.gate_mode]
+    per_ht = el * (2 * w.d_k + w.d_v) + g + 4 + el * w.d_v
+    states = w.B * w.H * w.d_v * w.d_k * 4 * ((1 if w.s0_std is not None else 0) + 1)
+    return ht * per_ht + states
+
+
+def prefill_flops(w):
+    """Algorithmic FLOPs of the chunkwise form (multiply-add = 2), counting the
+    causal halves of the in-chunk products; per head-token at chunk C:
+    A_kk, A_qk: 2 * C*d_k (half of C^2 d_k * 2 each, per token: C*d_k);
+    W = T (beta K) and U = T (beta V): C*d_k + C*d_v; E = U - W S^T: 2 d_k d_v;
+    O = Q S^T + A_qk E: 2 d_k d_v + C d_v; S update: 2 d_k d_v; triangular solve C^2/3."""
+    C, dk, dv = w.chunk, w.d_k, w.d_v
+    per_ht = (2 * C * dk) + (C * dk + C * dv) + 2 * dk * dv + (2 * dk * dv + C * dv) + \
+        2 * dk * dv + C * C / 3.0
+    return w.B * w.T * w.H * per_ht
+
+
+def source_sha(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def dram_traffic(kernel_tag, workload, src_paths):
+    """Per-launch DRAM bytes from the committed ncu summary, if it was taken on
+    the current kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    sha = source_sha(src_paths)
+    with open(p) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) >= 4 and not line.startswith("#") and parts[0] == kernel_tag and \
+                    parts[1] == workload and parts[2] == sha:
+                return float(parts[3])
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling in the background."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        # nvidia-smi numbers GPUs physically; address this process's GPU by UUID
+        try:
+            self.idx = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+        except Exception:
+            self.idx = str(device_index)
+        self.proc = None
+        self.path = f"/tmp/kda_bench_clocks_{os.getpid()}.csv"
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}",
+                                          f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                          "-lms", "100"], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                p = [x.strip() for x in line.split(",")]
+                if len(p) >= 10:
+                    rows.append(p)
+        os.unlink(self.path)
+        busy = [r for r in rows if r[4].isdigit() and int(r[4]) > 0] or rows
+        sm = [float(r[1]) for r in busy if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in busy for i in range(4) if r[6 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows), "samples_busy": len(busy)}
+
+
+def init_dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64,
+                     device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------- CPU (oracle)
+
+def oracle_prefill(d, nthreads=0):
+    import oracle
+
+    t0 = time.perf_counter()
+    oracle.forward(d["q"], d["k"], d["v"], d["g"], d["beta"], S0=d["S0"], nthreads=nthreads)
+    return time.perf_counter() - t0
+
+
+def cpu_inputs(w, seed_offset=0):
+    from kimi_delta_attention_22_b200 import inputs
+
+    return inputs.draw(w.B, w.T, w.H, w.d_k, w.d_v, dtype=w.torch_dtype, gate=w.gate,
+                       beta=w.beta, s0_std=w.s0_std, seed=w.seed + seed_offset, device="cpu")
+
+
+def run_reference(args, world, rank):
+    """--impl reference: the float64 oracle on the host cores, each step the
+    whole prefill workload (64 (sequence, head) pairs x 2048 tokens)."""
+    from kimi_delta_attention_22_b200 import inputs
+
+    import oracle
+
+    if rank != 0:
+        return
+    w = inputs.WORKLOADS[WORKLOAD]
+    d = cpu_inputs(w)
+    cores = oracle.max_threads()
+    for _ in range(args.warmup):
+        oracle_prefill(d)
+    times = [oracle_prefill(d) for _ in range(args.steps)]
+    total = sum(times)
+    val = args.steps * w.tokens / total
+    line = {"metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": WORKLOAD, "B": w.B, "T": w.T, "H": w.H, "d_k": w.d_k,
+                       "d_v": w.d_v, "chunk": w.chunk, "gate": w.gate, "parallelism": "none"},
+            "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": f"whole workload per step ({w.B * w.H} (sequence, head) "
+                                       f"pairs x {w.T} tokens), float64 token loop"},
+            "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- GPU path
+
+def bench_prefill(args, world, rank, peaks, peak_kind):
+    import kimi_delta_attention_22_b200 as kda
+    from kimi_delta_attention_22_b200 import inputs
+
+    kda.load_library()
+    w = inputs.WORKLOADS[WORKLOAD]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream(dev)
+    n_sets = 3  # rotating input sets (3 x ~210 MB > 126 MB L2): no step re-reads from L2
+    sets = [inputs.draw(w.B, w.T, w.H, w.d_k, w.d_v, dtype=w.torch_dtype, gate=w.gate,
+                        beta=w.beta, s0_std=w.s0_std, seed=w.seed + 100 * rank + i, device=dev)
+            for i in range(n_sets)]
+    outs = [torch.empty_like(s["v"]) for s in sets]
+    STs = [torch.empty(w.B, w.H, w.d_v, w.d_k, dtype=torch.float32, device=dev) for _ in sets]
+
+    def step(i):
+        s = sets[i % n_sets]
+        kda.kda_chunk_fwd(s["q"], s["k"], s["v"], s["g"], s["beta"], S0=s["S0"], chunk=w.chunk,
+                          out=outs[i % n_sets], S_T=STs[i % n_sets])
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        step(i)
+        ev[i][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    elapsed_ms = max_over_ranks(t0.elapsed_time(t1), world)
+    launch_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    launch_ms = max_over_ranks(launch_ms, world)
+
+    alg_bytes = prefill_bytes(w)
+    flops = prefill_flops(w)
+    achieved_gbs = alg_bytes / (launch_ms * 1e-3) / 1e9
+    achieved_tf = flops / (launch_ms * 1e-3) / 1e12
+    src = ["kimi_delta_attention_22_b200/csrc/kda_chunk_tc.cu",
+           "kimi_delta_attention_22_b200/csrc/kda_chunk_f32.cu"]
+    traffic = dram_traffic("chunk_fwd", WORKLOAD, src)
+    res = {
+        "w": w, "elapsed_ms": elapsed_ms, "launch_ms": launch_ms,
+        "value": world * args.steps * w.tokens / (elapsed_ms * 1e-3),
+        "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": achieved_gbs / peaks["hbm_gbs"],
+                     "traffic": traffic, "peak_source": f"{peak_kind} hbm_gbs",
+                     "algorithmic_bytes_per_launch": alg_bytes,
+                     "kernel": "kda_chunk_fwd kernel"},
+        "tensor": {"achieved_tflops": achieved_tf, "flops_per_launch": flops,
+                   "peak_tflops": peaks["bf16_tflops"],
+                   "frac": achieved_tf / peaks["bf16_tflops"],
+                   "peak_source": f"{peak_kind} bf16_tflops (burst)"},
+    }
+    # ---- end to end through the public API with host buffers: pinned H2D of
+    #      the step's inputs, the call, D2H of out and S_T, all inside the timed region
+    host = {k: (None if v is None else v.cpu().pin_memory()) for k, v in sets[0].items()}
+    dbuf = sets[1]
+    hout = torch.empty(outs[0].shape, dtype=outs[0].dtype).pin_memory()
+    hST = torch.empty(STs[0].shape, dtype=torch.float32).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
+    d2h = hout.numel() * hout.element_size() + hST.numel() * 4
+
+    def e2e_step():
+        for k, v in host.items():
+            if v is not None:
+                dbuf[k].copy_(v, non_blocking=True)
+        kda.kda_chunk_fwd(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["g"], dbuf["beta"],
+                          S0=dbuf["S0"], chunk=w.chunk, out=outs[1], S_T=STs[1])
+        hout.copy_(outs[1], non_blocking=True)
+        hST.copy_(STs[1], non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 50))
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(a.elapsed_time(b), world) / e2e_steps
+    res["e2e"] = {"value": world * w.tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
+                  "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                  "steps": e2e_steps}
+    del sets, outs, STs, dbuf
+    torch.cuda.empty_cache()
+    return res
+
+
+def bench_decode(args, world, rank, peaks, peak_kind):
+    import kimi_delta_attention_22_b200 as kda
+    from kimi_delta_attention_22_b200 import inputs
+
+    D = inputs.DECODE
+    N, H, dk, dv, steps = D["N"], D["H"], D["d_k"], D["d_v"], D["steps"]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream(dev)
+    pre = inputs.draw(N, D["prefill_T"], H, dk, dv, seed=D["seed"] + 7 * rank, device=dev)
+    _, S = kda.kda_chunk_fwd(pre["q"], pre["k"], pre["v"], pre["g"], pre["beta"])
+    del pre
+    dec = inputs.decode_inputs(N, H, dk, dv, steps, D["seed"] + 1000 + rank, device=dev)
+    out = torch.empty(N, H, dv, dtype=torch.bfloat16, device=dev)
+    for t in range(args.warmup):
+        kda.kda_decode_step(dec["q"][t], dec["k"][t], dec["v"][t], dec["g"][t], dec["beta"][t], S,
+                            out=out)
+    torch.cuda.synchronize()
+    barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for t in range(steps):
+        kda.kda_decode_step(dec["q"][t], dec["k"][t], dec["v"][t], dec["g"][t], dec["beta"][t], S,
+                            out=out)
+    b.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    us = max_over_ranks(a.elapsed_time(b), world) * 1e3 / steps
+    state_bytes = N * H * dv * dk * 4
+    per_step = 2 * state_bytes + N * H * (2 * (2 * dk + dv) + 4 * dk + 4)
+    gbs = per_step / (us * 1e-6) / 1e9
+    del dec, S
+    torch.cuda.empty_cache()
+    return {"metric": "decode step HBM GB/s", "value": world * gbs, "unit": "GB/s",
+            "us_per_step": us, "steps": steps,
+            "config": {"workload": D["name"], "N": N, "H": H, "d_k": dk, "d_v": dv,
+                       "state_MB": state_bytes / 1e6, "state_from": f"{D['prefill_T']}-token prefill"},
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"], "peak_source": f"{peak_kind} hbm_gbs",
+                         "algorithmic_bytes_per_launch": per_step,
+                         "traffic": dram_traffic("decode", D["name"],
+                                                 ["kimi_delta_attention_22_b200/csrc/kda_decode.cu"]),
+                         "kernel": "kda_decode_kernel"},
+            "gpu_launches": steps}
+
+
+def run_ours(args, world, rank, local):
+    peaks, peak_kind = load_peaks()
+    clocks = ClockSampler(local)
+    clocks.start()
+    pre = bench_prefill(args, world, rank, peaks, peak_kind)
+    dec = bench_decode(args, world, rank, peaks, peak_kind)
+    clk = clocks.stop()
+    w = pre["w"]
+    cpu = None
+    if rank == 0 and world == 1:
+        import oracle
+
+        d = cpu_inputs(w)
+        secs = oracle_prefill(d)
+        cpu = {"value": w.tokens / secs, "unit": "tokens/s", "cores": oracle.max_threads(),
+               "kind": "oracle",
+               "sample": f"whole prefill workload once ({w.B * w.H} (sequence, head) pairs x "
+                         f"{w.T} tokens, {secs:.1f} s wall), float64 token loop, OpenMP over pairs"}
+    if rank == 0:
+        line = {"metric": METRIC, "value": pre["value"], "unit": "tokens/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": pre["elapsed_ms"] / args.steps, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic (seeded N(0,1) q/k/v, L2-normalised k, sigmoid beta, "
+                        "-softplus gates)",
+                "config": {"workload": WORKLOAD, "B": w.B, "T": w.T, "H": w.H, "d_k": w.d_k,
+                           "d_v": w.d_v, "chunk": w.chunk, "gate": w.gate,
+                           "global_batch": w.B * world, "seq_len": w.T,
+                           "parallelism": f"replicas x{world}",
+                           "l2": "3 rotating input sets (~630 MB) > 126 MB L2"},
+                "roofline": pre["roofline"], "tensor": pre["tensor"], "cpu_baseline": cpu,
+                "e2e": pre["e2e"], "decode": dec, "clocks": clk, "gpu_launches": args.steps,
+                "kernel_ms_per_launch": pre["launch_ms"]}
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = init_dist()
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            if not torch.cuda.is_available():
+                raise SystemExit("bench.py --impl ours needs a CUDA device")
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,146 @@
+/*
+ * kda.h -- C ABI of libkda, the B200 (sm_100a) hot path of Kimi Delta
+ * Attention (KDA).
+ *
+ * The operation.  For one attention head, a d_v x d_k state S maps key space
+ * to value space.  Each token t updates it in five steps ("You could have come
+ * up with Kimi Delta Attention", the KDA state update at the top of the
+ * article; the same steps in the GeekNews summary, topic 31925, section
+ * "Kimi Delta Attention: per-channel decay"):
+ *
+ *     S~_t   = S_{t-1} Diag(alpha_t)          forget, one rate per key channel
+ *     vhat_t = S~_t k_t                       predict
+ *     e_t    = beta_t (v_t - vhat_t)          correct
+ *     S_t    = S~_t + e_t k_t^T               write
+ *     o_t    = S_t (d_k^{-1/2} q_t)           read (post-write state)
+ *
+ * The gate is passed as g = log(alpha) <= 0 (GeekNews summary, end of the
+ * "diagonal-plus-low-rank transition" section).  Keys are expected to be
+ * L2-normalised by the caller (the pages assume normalised keys); the
+ * library uses k as given and applies the d_k^{-1/2} query scale itself.
+ *
+ * Common conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller, contiguous,
+ *     row-major, 16-byte aligned.  The library allocates no memory and keeps
+ *     no state between calls.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream) and never synchronise.  Host-side validation happens
+ *     before any launch and returns an error status with nothing launched.
+ *   - Errors only the device can see (inconsistent cu_seqlens) are reported
+ *     through the optional `dev_status` device word: the kernel ORs in a
+ *     KDA_DEV_* bit and skips the offending work; read it after a sync.
+ *   - Outputs must not alias inputs (except S in kda_decode_step, which is
+ *     updated in place by design).
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1,  /* null pointer, negative or inconsistent size */
+    KDA_ERR_UNSUPPORTED = 2,  /* valid but not implemented (head size, chunk, dtype) */
+    KDA_ERR_MISALIGNED = 3,   /* a pointer is not 16-byte aligned */
+    KDA_ERR_CUDA = 4,         /* a CUDA launch or attribute call failed */
+    KDA_ERR_TIMEOUT = 5       /* reserved: a bounded device wait expired */
+} kda_status_t;
+
+/* Element type of q, k, v and out.  g, beta and every state are always fp32. */
+typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype_t;
+
+/* Gate layout (GeekNews summary: "Gated DeltaNet" uses one scalar alpha per
+ * token, KDA one alpha per key channel, DeltaNet none). */
+typedef enum {
+    KDA_GATE_CHANNEL = 0,  /* g: one value per key channel, [.., H, d_k] */
+    KDA_GATE_SCALAR = 1,   /* g: one value per (token, head), [.., H]   */
+    KDA_GATE_NONE = 2      /* g must be NULL; alpha = 1                  */
+} kda_gate_t;
+
+/* Device status bits written (ORed) into *dev_status. */
+#define KDA_DEV_BAD_SEQLENS 1  /* cu_seqlens not monotone or beyond T; sequence skipped */
+#define KDA_DEV_TIMEOUT 2      /* a bounded wait on an mbarrier expired; tile skipped */
+
+typedef struct {
+    int32_t B;          /* batch of sequences (dense); 1 for varlen; decode: N */
+    int32_t T;          /* tokens per sequence (dense) or in total (varlen); decode: 1 */
+    int32_t H;          /* heads */
+    int32_t d_k;        /* key / query head size */
+    int32_t d_v;        /* value head size */
+    int32_t num_seqs;   /* sequences: B for dense, len(cu_seqlens) - 1 for varlen */
+    int32_t dtype;      /* kda_dtype_t */
+    int32_t gate;       /* kda_gate_t */
+    int32_t chunk;      /* chunk length C of kda_chunk_fwd; ignored by decode */
+    int32_t* dev_status;/* optional device int32, see KDA_DEV_*; may be NULL */
+} kda_shape_t;
+
+/*
+ * kda_chunk_fwd -- chunkwise-parallel prefill forward.
+ *
+ * Runs the recurrence above over every token of every sequence and head,
+ * returning all outputs and (optionally) each sequence's final state.  It is
+ * the chunkwise schedule of the GeekNews summary, section "Chunkwise KDA":
+ * per chunk of C tokens, the log-space cumulative decay, the decay-masked
+ * key/key and query/key products, a unit-lower-triangular solve for the
+ * in-chunk error coupling ("pseudo-values from a triangular solve", the
+ * curriculum page's objectives), and the state/output products.  The result
+ * equals the token loop up to floating-point rounding.
+ *
+ * Layouts (tok = B*T packed token rows):
+ *   q, k      [B, T, H, d_k]   dtype
+ *   v, out    [B, T, H, d_v]   dtype
+ *   g         [B, T, H, d_k] fp32 (CHANNEL) | [B, T, H] fp32 (SCALAR) | NULL (NONE)
+ *   beta      [B, T, H] fp32
+ *   S0, S_T   [num_seqs, H, d_v, d_k] fp32; row = value index, key contiguous.
+ *             S0 == NULL: zero initial state.  S_T == NULL: final state not written.
+ *   cu_seqlens NULL for a dense batch (num_seqs == B), else device int32
+ *             [num_seqs + 1] with B == 1, cu[0] = 0, cu[n] <= cu[n+1], cu[num_seqs] <= T:
+ *             sequence n is token rows [cu[n], cu[n+1]).  Chunks never cross a
+ *             sequence; the state restarts from S0[n] (or zero) per sequence.
+ *             Rows of out not covered by any sequence are left untouched.
+ * Support:
+ *   KDA_BF16: d_k = d_v = 128, chunk = 64 (tcgen05 tensor-core path), or any
+ *             shape the fp32 path takes (CUDA-core path).
+ *   KDA_F32:  d_k, d_v multiples of 16 in [16, 128], chunk in {16, 32, 64}.
+ *   Anything else returns KDA_ERR_UNSUPPORTED.
+ */
+kda_status_t kda_chunk_fwd(const kda_shape_t* shape, const void* q, const void* k,
+                           const void* v, const float* g, const float* beta,
+                           const float* S0, const int32_t* cu_seqlens, void* out,
+                           float* S_T, void* stream);
+
+/*
+ * kda_decode_step -- one fused recurrent token for N sequences.
+ *
+ * The single-token case of the recurrence (the fused recurrent schedule of the
+ * GeekNews summary, section "fused recurrent kernel for decode"): each (n, h)
+ * state is read once from HBM, decayed, used for the prediction and the
+ * query read, corrected by the rank-1 write and stored back in place.
+ *
+ * Layouts (N = shape->B, shape->T must be 1):
+ *   q, k   [N, H, d_k] dtype       v, out [N, H, d_v] dtype
+ *   g      [N, H, d_k] fp32 (CHANNEL) | [N, H] fp32 (SCALAR) | NULL (NONE)
+ *   beta   [N, H] fp32
+ *   S      [N, H, d_v, d_k] fp32, read and overwritten with the new state.
+ * Support: d_k = 128 (any dtype), d_v a positive multiple of 4.  Else
+ * KDA_ERR_UNSUPPORTED.
+ */
+kda_status_t kda_decode_step(const kda_shape_t* shape, const void* q, const void* k,
+                             const void* v, const float* g, const float* beta, float* S,
+                             void* out, void* stream);
+
+/* Human-readable text for a status code (static storage). */
+const char* kda_status_str(kda_status_t status);
+
+/* Library version string (static storage). */
+const char* kda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H_ */

@@ -1,0 +1,169 @@
+"""Python binding of libkda, the B200 (sm_100a) Kimi Delta Attention hot path.
+
+The names mirror the C ABI of include/kda.h.  This module only marshals
+arguments: it checks shapes, allocates outputs with torch when the caller
+does not pass them, and hands raw device pointers and the current CUDA stream
+to the library.  Every arithmetic step runs in the library's kernels; there is
+no CPU or PyTorch fallback, and a missing libkda.so is an error.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = ["kda_chunk_fwd", "kda_decode_step", "kda_status_str", "library_path", "load_library",
+           "KDAError", "KDA_F32", "KDA_BF16", "KDA_GATE_CHANNEL", "KDA_GATE_SCALAR",
+           "KDA_GATE_NONE", "KDA_DEV_BAD_SEQLENS", "KDA_DEV_TIMEOUT", "Shape"]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libkda.so")
+
+KDA_F32, KDA_BF16 = 0, 1
+KDA_GATE_CHANNEL, KDA_GATE_SCALAR, KDA_GATE_NONE = 0, 1, 2
+KDA_DEV_BAD_SEQLENS, KDA_DEV_TIMEOUT = 1, 2
+_STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED",
+           3: "KDA_ERR_MISALIGNED", 4: "KDA_ERR_CUDA", 5: "KDA_ERR_TIMEOUT"}
+
+
+class KDAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {_STATUS.get(status, status)} ({kda_status_str(status)})")
+        self.status = status
+
+
+class Shape(ctypes.Structure):
+    """kda_shape_t."""
+    _fields_ = [("B", ctypes.c_int32), ("T", ctypes.c_int32), ("H", ctypes.c_int32),
+                ("d_k", ctypes.c_int32), ("d_v", ctypes.c_int32), ("num_seqs", ctypes.c_int32),
+                ("dtype", ctypes.c_int32), ("gate", ctypes.c_int32), ("chunk", ctypes.c_int32),
+                ("dev_status", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library(path: str | None = None):
+    """Load libkda.so (built in-tree by __graft_entry__.build()).  Raises if it is missing."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or _LIB_PATH
+    if not os.path.exists(p):
+        raise RuntimeError(f"libkda.so not found at {p}: build it with "
+                           "`python -m kimi_delta_attention_22_b200.build`")
+    lib = ctypes.CDLL(p)
+    P = ctypes.c_void_p
+    lib.kda_chunk_fwd.argtypes = [ctypes.POINTER(Shape), P, P, P, P, P, P, P, P, P, P]
+    lib.kda_chunk_fwd.restype = ctypes.c_int
+    lib.kda_decode_step.argtypes = [ctypes.POINTER(Shape), P, P, P, P, P, P, P, P]
+    lib.kda_decode_step.restype = ctypes.c_int
+    lib.kda_status_str.argtypes = [ctypes.c_int]
+    lib.kda_status_str.restype = ctypes.c_char_p
+    lib.kda_version.restype = ctypes.c_char_p
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def kda_status_str(status: int) -> str:
+    return load_library().kda_status_str(int(status)).decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _dtype_code(dt) -> int:
+    if dt == torch.bfloat16:
+        return KDA_BF16
+    if dt == torch.float32:
+        return KDA_F32
+    raise TypeError(f"q/k/v must be bfloat16 or float32, got {dt}")
+
+
+def _gate_code(g, q) -> int:
+    if g is None:
+        return KDA_GATE_NONE
+    if g.dim() == q.dim():
+        return KDA_GATE_CHANNEL
+    if g.dim() == q.dim() - 1:
+        return KDA_GATE_SCALAR
+    raise ValueError(f"g has {g.dim()} dims; expected {q.dim()} (per channel) or {q.dim() - 1} (scalar)")
+
+
+def _check_cuda(*ts):
+    for t in ts:
+        if t is not None:
+            if not t.is_cuda:
+                raise ValueError("libkda takes device tensors (copy host data to the GPU first)")
+            if not t.is_contiguous():
+                raise ValueError("libkda takes contiguous tensors")
+
+
+def kda_chunk_fwd(q, k, v, g, beta, S0=None, cu_seqlens=None, chunk: int = 64, out=None,
+                  S_T=None, want_state: bool = True, dev_status=None, lib=None):
+    """Chunkwise KDA prefill (kda_chunk_fwd of include/kda.h).
+
+    q, k [B,T,H,d_k]; v [B,T,H,d_v] (bf16 or fp32, same dtype); g [B,T,H,d_k]
+    (per channel) | [B,T,H] (scalar) | None (no gate), fp32 log-decay;
+    beta [B,T,H] fp32; S0 [N,H,d_v,d_k] fp32 or None; cu_seqlens int32 [N+1]
+    with B == 1 for packed sequences.  Returns (out, S_T); S_T is None when
+    want_state is False and no S_T buffer is given.
+    """
+    _check_cuda(q, k, v, g, beta, S0, cu_seqlens, out, S_T, dev_status)
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    N = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    if k.shape != q.shape or v.shape[:3] != q.shape[:3] or beta.shape != q.shape[:3]:
+        raise ValueError("shape mismatch among q, k, v, beta")
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k, v must share one dtype")
+    if g is not None and g.dtype != torch.float32 or beta.dtype != torch.float32:
+        raise TypeError("g and beta are float32")
+    if cu_seqlens is not None and cu_seqlens.dtype != torch.int32:
+        raise TypeError("cu_seqlens is int32")
+    if out is None:
+        out = torch.empty_like(v)
+    if S_T is None and want_state:
+        S_T = torch.empty(N, H, Dv, Dk, dtype=torch.float32, device=q.device)
+    sh = Shape(B, T, H, Dk, Dv, N, _dtype_code(q.dtype), _gate_code(g, q), int(chunk),
+               None if dev_status is None else dev_status.data_ptr())
+    lib = lib or load_library()
+    st = lib.kda_chunk_fwd(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                           _ptr(S0), _ptr(cu_seqlens), _ptr(out), _ptr(S_T),
+                           _stream_handle(q.device))
+    if st != 0:
+        raise KDAError(st, "kda_chunk_fwd")
+    return out, S_T
+
+
+def kda_decode_step(q, k, v, g, beta, S, out=None, lib=None):
+    """One fused recurrent KDA token (kda_decode_step of include/kda.h).
+
+    q, k [N,H,d_k]; v [N,H,d_v]; g [N,H,d_k] | [N,H] | None (fp32 log-decay);
+    beta [N,H] fp32; S [N,H,d_v,d_k] fp32, updated in place.  Returns out [N,H,d_v].
+    """
+    _check_cuda(q, k, v, g, beta, S, out)
+    N, H, Dk = q.shape
+    Dv = v.shape[-1]
+    if S.shape != (N, H, Dv, Dk) or S.dtype != torch.float32:
+        raise ValueError("S must be float32 [N, H, d_v, d_k]")
+    if out is None:
+        out = torch.empty_like(v)
+    sh = Shape(N, 1, H, Dk, Dv, N, _dtype_code(q.dtype), _gate_code(g, q), 0, None)
+    lib = lib or load_library()
+    st = lib.kda_decode_step(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                             _ptr(S), _ptr(out), _stream_handle(q.device))
+    if st != 0:
+        raise KDAError(st, "kda_decode_step")
+    return out

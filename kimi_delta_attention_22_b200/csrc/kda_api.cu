@@ -1,0 +1,104 @@
+// kda_api.cu -- the C ABI of include/kda.h: host-side validation and kernel
+// selection.  Nothing here allocates memory or synchronises; every check runs
+// before any launch, so a rejected call launches nothing.
+#include <stdint.h>
+
+#include "kda_internal.cuh"
+
+namespace kda {
+size_t chunk_f32_smem_bytes(int C, int D, int V);
+bool chunk_tc_supported(int D, int V, int C);
+}  // namespace kda
+
+namespace {
+
+bool aligned16(const void* p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool f32path_supports(int D, int V, int C) {
+    return D >= 16 && D <= 128 && D % 16 == 0 && V >= 16 && V <= 128 && V % 16 == 0 &&
+           (C == 16 || C == 32 || C == 64);
+}
+
+kda_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char* kda_status_str(kda_status_t s) {
+    switch (s) {
+        case KDA_OK: return "ok";
+        case KDA_ERR_INVALID_ARG: return "invalid argument";
+        case KDA_ERR_UNSUPPORTED: return "unsupported shape, chunk or dtype";
+        case KDA_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+        case KDA_ERR_CUDA: return "CUDA launch error";
+        case KDA_ERR_TIMEOUT: return "bounded device wait expired";
+    }
+    return "unknown status";
+}
+
+const char* kda_version(void) { return "libkda 0.1 (sm_100a)"; }
+
+kda_status_t kda_chunk_fwd(const kda_shape_t* sh, const void* q, const void* k, const void* v,
+                           const float* g, const float* beta, const float* S0,
+                           const int32_t* cu_seqlens, void* out, float* S_T, void* stream) {
+    if (sh == nullptr) return KDA_ERR_INVALID_ARG;
+    const int B = sh->B, T = sh->T, H = sh->H, D = sh->d_k, V = sh->d_v, N = sh->num_seqs;
+    if (B < 0 || T < 0 || H <= 0 || D <= 0 || V <= 0 || N < 0) return KDA_ERR_INVALID_ARG;
+    if (sh->dtype != KDA_F32 && sh->dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+    if (sh->gate != KDA_GATE_CHANNEL && sh->gate != KDA_GATE_SCALAR && sh->gate != KDA_GATE_NONE)
+        return KDA_ERR_INVALID_ARG;
+    if ((sh->gate == KDA_GATE_NONE) != (g == nullptr)) return KDA_ERR_INVALID_ARG;
+    if (cu_seqlens == nullptr) {
+        if (N != B) return KDA_ERR_INVALID_ARG;
+    } else if (B != 1) {
+        return KDA_ERR_INVALID_ARG;
+    }
+    if ((long long)B * T > 0 && (!q || !k || !v || !beta || !out)) return KDA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(beta) ||
+        !aligned16(S0) || !aligned16(cu_seqlens) || !aligned16(out) || !aligned16(S_T))
+        return KDA_ERR_MISALIGNED;
+    if ((long long)N * H > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+
+    const bool bf16 = sh->dtype == KDA_BF16;
+    const int C = sh->chunk;
+    const bool tc = bf16 && kda::chunk_tc_supported(D, V, C);
+    if (!tc && !f32path_supports(D, V, C)) return KDA_ERR_UNSUPPORTED;
+    if (N == 0) return KDA_OK;
+
+    kda::ChunkArgs a;
+    a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.S0 = S0; a.cu_seqlens = cu_seqlens;
+    a.out = out; a.S_T = S_T; a.dev_status = sh->dev_status;
+    a.B = B; a.T = T; a.H = H; a.d_k = D; a.d_v = V; a.num_seqs = N; a.gate = sh->gate;
+    a.chunk = C;
+    a.scale = 1.0f / sqrtf((float)D);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return from_cuda(tc ? kda::launch_chunk_tc(a, st) : kda::launch_chunk_f32path(a, bf16, st));
+}
+
+kda_status_t kda_decode_step(const kda_shape_t* sh, const void* q, const void* k, const void* v,
+                             const float* g, const float* beta, float* S, void* out,
+                             void* stream) {
+    if (sh == nullptr) return KDA_ERR_INVALID_ARG;
+    const int N = sh->B, H = sh->H, D = sh->d_k, V = sh->d_v;
+    if (N < 0 || H <= 0 || D <= 0 || V <= 0 || sh->T != 1) return KDA_ERR_INVALID_ARG;
+    if (sh->dtype != KDA_F32 && sh->dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+    if (sh->gate != KDA_GATE_CHANNEL && sh->gate != KDA_GATE_SCALAR && sh->gate != KDA_GATE_NONE)
+        return KDA_ERR_INVALID_ARG;
+    if ((sh->gate == KDA_GATE_NONE) != (g == nullptr)) return KDA_ERR_INVALID_ARG;
+    if (N > 0 && (!q || !k || !v || !beta || !S || !out)) return KDA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(beta) ||
+        !aligned16(S) || !aligned16(out))
+        return KDA_ERR_MISALIGNED;
+    if (D != 128 || V > 65535 * 128) return KDA_ERR_UNSUPPORTED;
+    if ((long long)N * H > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+    if (N == 0) return KDA_OK;
+
+    kda::DecodeArgs a;
+    a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.S = S; a.out = out;
+    a.N = N; a.H = H; a.d_k = D; a.d_v = V; a.gate = sh->gate;
+    a.scale = 1.0f / sqrtf((float)D);
+    return from_cuda(kda::launch_decode(a, sh->dtype == KDA_BF16, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"
