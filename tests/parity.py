@@ -10,34 +10,49 @@ import oracle
 from kimi_delta_attention_22_b200 import inputs
 
 # Tolerances (see the readings of the pages): fp32 mode is compared by the
-# maximum absolute error; bf16-input/fp32-state mode by the maximum absolute
-# error divided by the RMS of the oracle's tensor, per tensor.
+# maximum absolute error.  bf16-input/fp32-state mode is compared relative to
+# the RMS of the oracle's tensor, per tensor, in two ways:
+#   * rms(gpu - oracle) / rms(oracle) <= 2e-2, and
+#   * element by element, |gpu - oracle| <= 2e-2 * rms(oracle) + q |oracle|,
+#     where q = 2^-8 (half a bf16 ulp, relative) when the library stores that
+#     tensor in bf16 and 0 when it stores fp32: the rounding of the stored
+#     result itself is not an arithmetic error of the path.
 TOL_F32_ABS = 1e-4
 TOL_BF16_REL = 2e-2
+BF16_HALF_ULP = 2.0 ** -8
 
 
 def to_dev(d, dev="cuda"):
     return {k: (None if v is None else v.to(dev)) for k, v in d.items()}
 
 
-def err(got, ref, mode):
+def err(got, ref, mode, stored_bf16=None):
+    """Returns the error figure compared against the tolerance (see above).
+    For bf16 mode: max(rms ratio, worst element-wise excess over the rounding
+    allowance, both divided by rms(oracle))."""
+    if stored_bf16 is None:
+        stored_bf16 = hasattr(got, "dtype") and got.dtype == torch.bfloat16
     got = got.detach().cpu().double().numpy() if hasattr(got, "detach") else np.asarray(got)
     ref = np.asarray(ref, dtype=np.float64)
     assert got.shape == ref.shape, (got.shape, ref.shape)
     assert np.all(np.isfinite(got)), "non-finite values in the GPU result"
     if got.size == 0:
         return 0.0
-    e = float(np.max(np.abs(got - ref)))
+    d = np.abs(got - ref)
     if mode == "f32":
-        return e
-    rms = float(np.sqrt(np.mean(ref ** 2)))
-    return e / max(rms, 1e-30)
+        return float(np.max(d))
+    rms = max(float(np.sqrt(np.mean(ref ** 2))), 1e-30)
+    # "both": two independently rounded bf16 results may differ by a full ulp
+    q = 2 * BF16_HALF_ULP if stored_bf16 == "both" else (BF16_HALF_ULP if stored_bf16 else 0.0)
+    elem = float(np.max(d - q * np.abs(ref))) / rms
+    rel_rms = float(np.sqrt(np.mean(d ** 2))) / rms
+    return max(elem, rel_rms)
 
 
-def check(got, ref, mode, what):
-    e = err(got, ref, mode)
+def check(got, ref, mode, what, stored_bf16=None):
+    e = err(got, ref, mode, stored_bf16)
     tol = TOL_F32_ABS if mode == "f32" else TOL_BF16_REL
-    assert e <= tol, f"{what}: error {e:.3e} > {tol:.1e} ({'max abs' if mode == 'f32' else 'max abs / rms'})"
+    assert e <= tol, f"{what}: error {e:.3e} > {tol:.1e} ({'max abs' if mode == 'f32' else 'rms-relative'})"
     return e
 
 
