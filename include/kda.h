@@ -21,8 +21,10 @@
  *
  * Common conventions for every entry point:
  *   - All tensor pointers are DEVICE pointers owned by the caller, contiguous,
- *     row-major, 16-byte aligned.  The library allocates no memory and keeps
- *     no state between calls.
+ *     row-major.  q, k, v, out, per-channel g and every state are 16-byte
+ *     aligned (TMA and 128-bit loads); beta, scalar g and cu_seqlens need
+ *     only their 4-byte element alignment.  The library allocates no memory
+ *     and keeps no state between calls.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
  *     default stream) and never synchronise.  Host-side validation happens
  *     before any launch and returns an error status with nothing launched.
@@ -45,7 +47,7 @@ typedef enum {
     KDA_OK = 0,
     KDA_ERR_INVALID_ARG = 1,  /* null pointer, negative or inconsistent size */
     KDA_ERR_UNSUPPORTED = 2,  /* valid but not implemented (head size, chunk, dtype) */
-    KDA_ERR_MISALIGNED = 3,   /* a pointer is not 16-byte aligned */
+    KDA_ERR_MISALIGNED = 3,   /* a pointer breaks its alignment rule (see above) */
     KDA_ERR_CUDA = 4,         /* a CUDA launch or attribute call failed */
     KDA_ERR_TIMEOUT = 5       /* reserved: a bounded device wait expired */
 } kda_status_t;
@@ -126,7 +128,7 @@ kda_status_t kda_chunk_fwd(const kda_shape_t* shape, const void* q, const void* 
  *   g      [N, H, d_k] fp32 (CHANNEL) | [N, H] fp32 (SCALAR) | NULL (NONE)
  *   beta   [N, H] fp32
  *   S      [N, H, d_v, d_k] fp32, read and overwritten with the new state.
- * Support: d_k = 128 (any dtype), d_v a positive multiple of 4.  Else
+ * Support: d_k = 128 (bf16 or fp32), any d_v from 1 to 65535*128.  Else
  * KDA_ERR_UNSUPPORTED.
  */
 kda_status_t kda_decode_step(const kda_shape_t* shape, const void* q, const void* k,

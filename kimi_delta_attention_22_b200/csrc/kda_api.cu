@@ -13,6 +13,7 @@ bool chunk_tc_supported(int D, int V, int C);
 namespace {
 
 bool aligned16(const void* p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 bool f32path_supports(int D, int V, int C) {
     return D >= 16 && D <= 128 && D % 16 == 0 && V >= 16 && V <= 128 && V % 16 == 0 &&
@@ -55,10 +56,12 @@ kda_status_t kda_chunk_fwd(const kda_shape_t* sh, const void* q, const void* k, 
         return KDA_ERR_INVALID_ARG;
     }
     if ((long long)B * T > 0 && (!q || !k || !v || !beta || !out)) return KDA_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(beta) ||
-        !aligned16(S0) || !aligned16(cu_seqlens) || !aligned16(out) || !aligned16(S_T))
+    const bool g_vec = sh->gate == KDA_GATE_CHANNEL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !(g_vec ? aligned16(g) : aligned4(g)) ||
+        !aligned4(beta) || !aligned16(S0) || !aligned4(cu_seqlens) || !aligned16(out) ||
+        !aligned16(S_T))
         return KDA_ERR_MISALIGNED;
-    if ((long long)N * H > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+    if ((long long)N * H * 2 > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
 
     const bool bf16 = sh->dtype == KDA_BF16;
     const int C = sh->chunk;
@@ -87,8 +90,9 @@ kda_status_t kda_decode_step(const kda_shape_t* sh, const void* q, const void* k
         return KDA_ERR_INVALID_ARG;
     if ((sh->gate == KDA_GATE_NONE) != (g == nullptr)) return KDA_ERR_INVALID_ARG;
     if (N > 0 && (!q || !k || !v || !beta || !S || !out)) return KDA_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(beta) ||
-        !aligned16(S) || !aligned16(out))
+    const bool g_vec = sh->gate == KDA_GATE_CHANNEL;
+    if (!aligned16(q) || !aligned16(k) || !aligned4(v) || !(g_vec ? aligned16(g) : aligned4(g)) ||
+        !aligned4(beta) || !aligned16(S) || !aligned4(out))
         return KDA_ERR_MISALIGNED;
     if (D != 128 || V > 65535 * 128) return KDA_ERR_UNSUPPORTED;
     if ((long long)N * H > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;

@@ -1,10 +1,598 @@
-// kda_chunk_tc.cu -- tensor-core (tcgen05) chunkwise prefill; not built yet.
+// kda_chunk_tc.cu -- chunkwise KDA prefill on the sm_100a tensor cores
+// (tcgen05 MMAs with fp32 accumulators in tensor memory, operands in shared
+// memory, raw tiles brought in by TMA).  bf16 q/k/v, fp32 gates / beta /
+// state, d_k = d_v = 128, chunk C = 64.
+//
+// The chunkwise form follows the GeekNews summary of "You could have come up
+// with Kimi Delta Attention", section "Chunkwise KDA" (cumulative decay,
+// provisional errors, coupling coefficients rho_ij), with the cut-off
+// dependency formula completed as the unit-lower-triangular solve the
+// curriculum page names ("pseudo-values from a triangular solve", "WY/UT
+// form").  For a chunk of C tokens with incoming state S (d_v x d_k):
+//
+//   Gamma_i = sum_{s<=i} g_s                      (log-space cumulative decay)
+//   P[i,j]  = sum_c K_ic K_jc e^{Gamma_ic - Gamma_jc}    (j <= i)
+//   Qp[i,j] = sum_c Q~_ic K_jc e^{Gamma_ic - Gamma_jc}   (j <= i)
+//   T       = (I + strict_lower(diag(beta) P))^{-1}
+//   W = T diag(beta) (K e^{Gamma}),  U = T diag(beta) V  (pseudo-values)
+//   E = U - W S^T                                     (true in-chunk errors)
+//   O = (Q~ e^{Gamma}) S^T + lower(Qp) E              (outputs, post-write)
+//   S^T <- Diag(e^{Gamma_last}) S^T + (K e^{Gamma_last - Gamma})^T E
+//
+// Log-space ratios.  A product e^{Gamma_i - Gamma_j} is split into two
+// factors with a reference row r inside each 16-token sub-block:
+// i-side x_i = e^{Gamma_i - Gamma_r(i)}, j-side e^{Gamma_r(I) - Gamma_j}; for
+// j in an earlier sub-block the j-side factor is <= 1, and inside a sub-block
+// both factors are bounded by e^{8 max|g|}, so nothing overflows in fp32/bf16
+// for |g| up to ~10 per token.  e^{-Gamma} is never formed.
+//
+// Work layout: one CTA per (sequence, head, 64-wide value tile); the CTA walks
+// its sequence's chunks in order with the fp32 state tile S^T (128 x 64) in
+// registers (thread = key channel, half the value columns per warp group) and
+// a bf16 copy in shared memory as the MMA operand.  The in-chunk phases run
+// one after another; TMA for the next chunk is issued as soon as its landing
+// buffers are free.
+#include <cudaTypedefs.h>
+
 #include "kda_internal.cuh"
+#include "sm100.cuh"
 
 namespace kda {
+namespace {
 
-bool chunk_tc_supported(int, int, int) { return false; }
+using namespace sm100;
 
-cudaError_t launch_chunk_tc(const ChunkArgs&, cudaStream_t) { return cudaErrorNotSupported; }
+constexpr int C = 64, DK = 128, DV = 128, BV = 64, NVT = DV / BV, NT = 256;
+constexpr uint64_t kWaitNs = 1000000000ull;  // 1 s bound on every wait
+
+// Shared-memory map (bytes from a 1024-aligned base).
+constexpr int OFF_RAW = 0;                       // raw K | raw Q | raw G  (64 KB)
+constexpr int OFF_RK = OFF_RAW;                  //   [64][128] bf16
+constexpr int OFF_RQ = OFF_RAW + 16384;          //   [64][128] bf16
+constexpr int OFF_RG = OFF_RAW + 32768;          //   [64][128] fp32
+constexpr int OFF_OX = OFF_RAW;                  // after prep: Gram B operand (K-major, 128 rows)
+constexpr int OFF_KG = OFF_RAW + 32768;          //   K e^Gamma        (MN-major, MN = c, K = j)
+constexpr int OFF_QG = OFF_RAW + 49152;          //   Q~ e^Gamma       (K-major, 64 rows)
+constexpr int OFF_RV = 65536;                    // raw V tile, TMA 128B swizzle = MN-major operand
+constexpr int OFF_A = 73728;                     // 64 KB, reused per phase:
+constexpr int OFF_OY = OFF_A;                    //   4 Gram A operands (K-major, 64 rows each)
+constexpr int OFF_AKK = OFF_A;                   //   fp32 [64][64] coupling matrix
+constexpr int OFF_AQK = OFF_A + 16384;           //   fp32 [64][64] Qp, then block scratch
+constexpr int OFF_TF = OFF_A + 32768;            //   fp32 [64][64] T
+constexpr int OFF_W = OFF_A;                     //   W bf16 (K-major, 64 rows)
+constexpr int OFF_E = OFF_A + 16384;             //   E bf16 (MN-major, MN = v, K = j)
+constexpr int OFF_TB = OFF_A + 65536;            // T diag(beta) bf16 (K-major 64 x 64)
+constexpr int OFF_AQB = OFF_TB + 8192;           // lower(Qp) bf16 (K-major 64 x 64)
+constexpr int OFF_KD = OFF_AQB + 8192;           // K e^{Gamma_last - Gamma} (MN-major, MN = c)
+constexpr int OFF_S = OFF_KD + 16384;            // S^T bf16 (MN-major, MN = v, K = c)
+constexpr int OFF_SMALL = OFF_S + 16384;
+constexpr int OFF_TOT = OFF_SMALL;               // fp32 [4][128] sub-block sums of g
+constexpr int OFF_SUB = OFF_TOT + 2048;          // fp32 [4][128] cumsum at each reference row
+constexpr int OFF_BETA = OFF_SUB + 2048;         // fp32 [64]
+constexpr int OFF_DECAY = OFF_BETA + 256;        // fp32 [128] e^{Gamma_last}
+constexpr int OFF_BAR = OFF_DECAY + 512;         // mbarriers + tmem base + flags
+constexpr int SMEM_USED = OFF_BAR + 64;
+constexpr int SMEM_BYTES = SMEM_USED + 1024;     // + alignment slack
+constexpr uint32_t TMEM_COLS = 256;
+
+// TMEM columns (lane base 0 or 16 for M = 64 accumulators).
+constexpr uint32_t TM_GRAM = 0;     // lanes 0-15 : [j][32 I + u]  P^T | Qp^T
+constexpr uint32_t TM_W = 0;        // lanes 16-31: W   [i][c]   (128 cols)
+constexpr uint32_t TM_UE = 128;     // lanes 0-15 : U, then E = U - W S^T  [j][v]
+constexpr uint32_t TM_O = 128;      // lanes 16-31: O   [i][v]
+constexpr uint32_t TM_DS = 192;     // all lanes  : dS^T [c][v]
+constexpr uint32_t LANE16 = 16u << 16;
+
+struct TcParams {
+    CUtensorMap map_k, map_q, map_v, map_g;
+    ChunkArgs a;
+};
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 t = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&t);
+}
+__device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
+    __nv_bfloat162 t = *reinterpret_cast<__nv_bfloat162*>(&u);
+    return __bfloat1622float2(t);
+}
+__device__ __forceinline__ void st_shared_u32(uint8_t* base, uint32_t off, uint32_t v) {
+    *reinterpret_cast<uint32_t*>(base + off) = v;
+}
+__device__ __forceinline__ void st_shared_v4(uint8_t* base, uint32_t off, uint4 v) {
+    *reinterpret_cast<uint4*>(base + off) = v;
+}
+
+// Store 8 consecutive fp32 values as one 16-byte bf16 chunk.
+__device__ __forceinline__ uint4 pack8(const float* v) {
+    return make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
+                      pack_bf16(v[6], v[7]));
+}
+
+template <int GATE>
+__global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_constant__ TcParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+    const ChunkArgs& a = p.a;
+    const int H = a.H;
+    const int vt = blockIdx.x % NVT;
+    const int h = (blockIdx.x / NVT) % H;
+    const int n = blockIdx.x / (NVT * H);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int sp = warp & 3;           // TMEM sub-partition of this warp
+    const int vhalf = warp >> 2;       // which 32 of the tile's 64 value columns
+    const uint32_t lane_base = (uint32_t)(32 * sp) << 16;
+
+    float* tot = reinterpret_cast<float*>(sm + OFF_TOT);
+    float* sub = reinterpret_cast<float*>(sm + OFF_SUB);
+    float* beta_s = reinterpret_cast<float*>(sm + OFF_BETA);
+    float* decay_s = reinterpret_cast<float*>(sm + OFF_DECAY);
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
+    uint64_t* mma_bar = full_bar + 1;
+    uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(full_bar + 2);
+    int* abort_s = reinterpret_cast<int*>(full_bar + 3);
+    const uint32_t sbase = smem_u32(sm);
+
+    long long bos, eos;
+    const bool seq_ok = seq_bounds(a.cu_seqlens, n, a.T, a.num_seqs, a.dev_status, bos, eos);
+    if (!seq_ok) return;  // uniform across the CTA
+
+    if (tid == 0) {
+        mbar_init(full_bar, 1);
+        mbar_init(mma_bar, 1);
+        *abort_s = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_base_s, TMEM_COLS);
+        tmem_relinquish();
+    }
+
+    // ---- initial state: thread owns key channel c, value columns v0..v0+31
+    const int c_own = 32 * sp + lane;
+    const int v0 = 32 * vhalf;
+    float S[32];
+    {
+        const size_t sbase_g = ((size_t)n * H + h) * DV * DK;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const int v = vt * BV + v0 + j;
+            S[j] = a.S0 ? a.S0[sbase_g + (size_t)v * DK + c_own] : 0.f;
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            st_shared_v4(sm + OFF_S, mnmaj_off(v0 + 8 * q, c_own, BV), pack8(S + 8 * q));
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = *tmem_base_s;
+
+    const uint32_t raw_bytes = 16384 * 2 + 8192 + (GATE == KDA_GATE_CHANNEL ? 32768 : 0);
+    auto issue_tma = [&](long long c0) {
+        mbar_arrive_expect_tx(full_bar, raw_bytes);
+        tma_load_3d(sm + OFF_RK, &p.map_k, full_bar, 0, h, (int)c0);
+        tma_load_3d(sm + OFF_RQ, &p.map_q, full_bar, 0, h, (int)c0);
+        tma_load_3d(sm + OFF_RV, &p.map_v, full_bar, vt * BV, h, (int)c0);
+        if (GATE == KDA_GATE_CHANNEL) tma_load_3d(sm + OFF_RG, &p.map_g, full_bar, 0, h, (int)c0);
+    };
+
+    uint32_t full_phase = 0, mma_phase = 0;
+    bool tma_pending = false, mma_pending = false;
+    // Uniform bounded wait: every thread waits; any expiry aborts the CTA.
+    // The phase flips only on success, so after an abort `phase` still names the
+    // phase the cleanup has to wait for.
+    auto wait_bar = [&](uint64_t* bar, uint32_t& phase) -> bool {
+        const bool ok = mbar_wait(bar, phase, kWaitNs);
+        if (!ok) atomicOr(abort_s, 1);
+        __syncthreads();
+        if (*abort_s != 0) return false;
+        phase ^= 1u;
+        return true;
+    };
+
+    if (tid == 0 && bos < eos) issue_tma(bos);
+    tma_pending = bos < eos;
+
+    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out);
+
+    bool aborted = false;
+    for (long long c0 = bos; c0 < eos; c0 += C) {
+        const int L = (int)min((long long)C, eos - c0);
+        // ================= phase 1: decay, reference factors, operands
+        if (!wait_bar(full_bar, full_phase)) { aborted = true; break; }
+        tma_pending = false;
+        const int blk = tid >> 6;        // 16-row sub-block
+        const int pr = tid & 63;         // channel pair
+        const int ch = 2 * pr;
+        float gl[16][2];
+        uint32_t kr[16], qr[16];
+        {
+            float run0 = 0.f, run1 = 0.f;
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const int i = 16 * blk + u;
+                const bool valid = i < L;
+                float g0 = 0.f, g1 = 0.f;
+                if (GATE == KDA_GATE_CHANNEL) {
+                    const float2 gg = *reinterpret_cast<const float2*>(sm + OFF_RG + (i * DK + ch) * 4);
+                    g0 = gg.x; g1 = gg.y;
+                } else if (GATE == KDA_GATE_SCALAR) {
+                    g0 = g1 = valid ? a.g[(size_t)(c0 + i) * H + h] : 0.f;
+                }
+                if (!valid) { g0 = 0.f; g1 = 0.f; }
+                run0 += g0; run1 += g1;
+                gl[u][0] = run0; gl[u][1] = run1;
+                const uint32_t kk = *reinterpret_cast<const uint32_t*>(sm + OFF_RK + (i * DK + ch) * 2);
+                const uint32_t qq = *reinterpret_cast<const uint32_t*>(sm + OFF_RQ + (i * DK + ch) * 2);
+                kr[u] = valid ? kk : 0u;
+                qr[u] = valid ? qq : 0u;
+            }
+            tot[blk * DK + ch] = run0; tot[blk * DK + ch + 1] = run1;
+            sub[blk * DK + ch] = gl[7][0]; sub[blk * DK + ch + 1] = gl[7][1];
+            if (tid < C) beta_s[tid] = (tid < L) ? a.beta[(size_t)(c0 + tid) * H + h] : 0.f;
+        }
+        __syncthreads();   // raw K/Q/G are consumed; their space now takes operands
+        {
+            // prefix sums of the sub-block totals for this thread's two channels
+            float pre[2] = {0.f, 0.f}, last[2] = {0.f, 0.f}, gref[4][2];
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    gref[b][e] = last[e] + sub[b * DK + ch + e];   // Gamma at reference row of sub-block b
+                    if (b < blk) pre[e] += tot[b * DK + ch + e];
+                    last[e] += tot[b * DK + ch + e];
+                }
+            }
+            float Er[2], Lr[2], z[4][2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const float gr = gref[blk][e];
+                Er[e] = __expf(gr);                 // e^{Gamma_r}
+                Lr[e] = __expf(last[e] - gr);       // e^{Gamma_last - Gamma_r}
+#pragma unroll
+                for (int I = 0; I < 4; ++I) z[I][e] = (I > blk) ? __expf(gref[I][e] - gr) : 0.f;
+            }
+            if (blk == 0) {
+                decay_s[ch] = __expf(last[0]);
+                decay_s[ch + 1] = __expf(last[1]);
+            }
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const int i = 16 * blk + u;
+                float x[2], y[2];
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const float dlt = gl[u][e] - gl[7][e];   // Gamma_i - Gamma_r
+                    x[e] = __expf(dlt);
+                    y[e] = __expf(-dlt);
+                }
+                const float2 kf = unpack_bf16(kr[u]);
+                const float2 qf = unpack_bf16(qr[u]);
+                const float k0 = kf.x, k1 = kf.y;
+                const float q0 = qf.x * a.scale, q1 = qf.y * a.scale;
+                // Gram B operand: K rows at 32 blk + u, Q rows at 32 blk + 16 + u
+                st_shared_u32(sm + OFF_OX, kmaj_off(32 * blk + u, ch, 128), pack_bf16(k0 * x[0], k1 * x[1]));
+                st_shared_u32(sm + OFF_OX, kmaj_off(32 * blk + 16 + u, ch, 128), pack_bf16(q0 * x[0], q1 * x[1]));
+                // Gram A operands (j-side) for target sub-blocks I >= blk; zero rows for I < blk
+#pragma unroll
+                for (int I = 0; I < 4; ++I) {
+                    uint32_t val = 0u;
+                    if (I == blk) val = pack_bf16(k0 * y[0], k1 * y[1]);
+                    else if (I > blk) val = pack_bf16(k0 * y[0] * z[I][0], k1 * y[1] * z[I][1]);
+                    st_shared_u32(sm + OFF_OY + I * 16384, kmaj_off(i, ch, 64), val);
+                }
+                const float eg0 = Er[0] * x[0], eg1 = Er[1] * x[1];   // e^{Gamma_i}
+                const float ed0 = Lr[0] * y[0], ed1 = Lr[1] * y[1];   // e^{Gamma_last - Gamma_i}
+                // (ch, ch + 1) are adjacent in both layouts (ch even)
+                st_shared_u32(sm + OFF_KG, mnmaj_off(ch, i, 128), pack_bf16(k0 * eg0, k1 * eg1));
+                st_shared_u32(sm + OFF_QG, kmaj_off(i, ch, 64), pack_bf16(q0 * eg0, q1 * eg1));
+                st_shared_u32(sm + OFF_KD, mnmaj_off(ch, i, 128), pack_bf16(k0 * ed0, k1 * ed1));
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        // ================= phase 2: Gram MMAs  (D[j][32 I + u] = Ky_I[j] . X[32 I + u])
+        if (tid == 0) {
+            const uint32_t ox = sbase + OFF_OX;
+#pragma unroll
+            for (int I = 0; I < 4; ++I) {
+                const uint32_t oy = sbase + OFF_OY + I * 16384;
+#pragma unroll
+                for (int s = 0; s < 8; ++s)
+                    mma_bf16(tm + TM_GRAM + 32 * I, kmaj_desc(oy, 64, s),
+                             kmaj_desc(ox + I * 32 * 128, 128, s) /* rows 32I.. of a 128-row tile */,
+                             idesc_bf16(64, 32, false, false), s > 0);
+            }
+            mma_commit(mma_bar);
+        }
+        if (!wait_bar(mma_bar, mma_phase)) { aborted = true; mma_pending = true; break; }
+        tc_fence_after();
+        // ================= phase 3: coupling matrix, Qp, and T = (I + L)^{-1}
+        float* Akk = reinterpret_cast<float*>(sm + OFF_AKK);
+        float* Aqk = reinterpret_cast<float*>(sm + OFF_AQK);
+        float* TF = reinterpret_cast<float*>(sm + OFF_TF);
+        if (warp < 4) {
+            const int j = 16 * sp + lane;   // valid for lane < 16
+#pragma unroll
+            for (int I = 0; I < 4; ++I) {
+                float v[32];
+                tmem_ld32(tm + lane_base + TM_GRAM + 32 * I, v);
+                if (lane < 16) {
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) {
+                        const int i = 16 * I + u;
+                        Akk[i * C + j] = (j < i) ? beta_s[i] * v[u] : 0.f;
+                        Aqk[i * C + j] = (j <= i) ? v[16 + u] : 0.f;
+                    }
+                }
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+        // lower(Qp) -> bf16 operand; diagonal blocks of T by forward substitution
+        for (int e = tid; e < C * C / 2; e += NT) {
+            const int i = e / (C / 2), j = 2 * (e % (C / 2));
+            st_shared_u32(sm + OFF_AQB, kmaj_off(i, j, 64), pack_bf16(Aqk[i * C + j], Aqk[i * C + j + 1]));
+        }
+        if (warp < 4) {
+            const int I = warp, cc = lane & 15;
+            float t[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                float acc = 0.f;
+#pragma unroll
+                for (int k = 0; k < r; ++k) acc = fmaf(Akk[(16 * I + r) * C + 16 * I + k], t[k], acc);
+                t[r] = (r < cc) ? 0.f : ((r == cc) ? 1.f : -acc);
+            }
+            if (lane < 16) {
+#pragma unroll
+                for (int r = 0; r < 16; ++r) TF[(16 * I + r) * C + 16 * I + cc] = t[r];
+            }
+        } else {
+            // zero the strictly-upper blocks of T
+            for (int e = tid - 128; e < 6 * 256; e += 128) {
+                const int bidx = e >> 8, r = (e >> 4) & 15, cc = e & 15;
+                const int I = (bidx < 3) ? 0 : ((bidx < 5) ? 1 : 2);
+                const int J = (bidx < 3) ? bidx + 1 : ((bidx < 5) ? bidx - 1 : 3);
+                TF[(16 * I + r) * C + 16 * J + cc] = 0.f;
+            }
+        }
+        __syncthreads();
+        // off-diagonal blocks, level by level: T_IJ = -T_II sum_{K=J}^{I-1} L_IK T_KJ
+        float* X = Aqk;   // scratch: Qp is already in its bf16 tile
+#pragma unroll 1
+        for (int d = 1; d < 4; ++d) {
+            const int nb = 4 - d;
+            for (int e = tid; e < nb * 256; e += NT) {
+                const int J = e >> 8, I = J + d, r = (e >> 4) & 15, cc = e & 15;
+                float acc = 0.f;
+                for (int K = J; K < I; ++K)
+#pragma unroll
+                    for (int k = 0; k < 16; ++k)
+                        acc = fmaf(Akk[(16 * I + r) * C + 16 * K + k], TF[(16 * K + k) * C + 16 * J + cc], acc);
+                X[(16 * J + r) * 16 + cc] = acc;
+            }
+            __syncthreads();
+            for (int e = tid; e < nb * 256; e += NT) {
+                const int J = e >> 8, I = J + d, r = (e >> 4) & 15, cc = e & 15;
+                float acc = 0.f;
+#pragma unroll
+                for (int k = 0; k < 16; ++k)
+                    acc = fmaf(TF[(16 * I + r) * C + 16 * I + k], X[(16 * J + k) * 16 + cc], acc);
+                TF[(16 * I + r) * C + 16 * J + cc] = -acc;
+            }
+            __syncthreads();
+        }
+        // T diag(beta) -> bf16 operand (K-major, rows i, K = j)
+        for (int e = tid; e < C * C / 2; e += NT) {
+            const int i = e / (C / 2), j = 2 * (e % (C / 2));
+            const float t0 = (j <= i) ? TF[i * C + j] * beta_s[j] : 0.f;
+            const float t1 = (j + 1 <= i) ? TF[i * C + j + 1] * beta_s[j + 1] : 0.f;
+            st_shared_u32(sm + OFF_TB, kmaj_off(i, j, 64), pack_bf16(t0, t1));
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        // ================= phase 4: W = T_b (K e^Gamma), U = T_b V
+        if (tid == 0) {
+            const uint32_t tb = sbase + OFF_TB;
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                mma_bf16(tm + LANE16 + TM_W, kmaj_desc(tb, 64, s), mnmaj_desc(sbase + OFF_KG, 128, s),
+                         idesc_bf16(64, 128, false, true), s > 0);
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                mma_bf16(tm + TM_UE, kmaj_desc(tb, 64, s), mnmaj_desc(sbase + OFF_RV, 64, s),
+                         idesc_bf16(64, 64, false, true), s > 0);
+            mma_commit(mma_bar);
+        }
+        if (!wait_bar(mma_bar, mma_phase)) { aborted = true; mma_pending = true; break; }
+        tc_fence_after();
+        // ================= phase 5: W -> bf16 (K-major, 64 rows, K = c)
+        {
+            const int i = 16 * sp + lane - 16;   // valid for lane >= 16
+#pragma unroll
+            for (int m = 0; m < 2; ++m) {
+                const int col = 64 * vhalf + 32 * m;
+                float v[32];
+                tmem_ld32(tm + lane_base + TM_W + col, v);
+                if (lane >= 16) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        st_shared_v4(sm + OFF_W, kmaj_off(i, col + 8 * q, 64), pack8(v + 8 * q));
+                }
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        // ================= phase 6: E = U - W S^T ; O = (Q~ e^Gamma) S^T
+        if (tid == 0) {
+            const uint32_t s_op = sbase + OFF_S;
+#pragma unroll
+            for (int s = 0; s < 8; ++s)
+                mma_bf16(tm + TM_UE, kmaj_desc(sbase + OFF_W, 64, s), mnmaj_desc(s_op, BV, s),
+                         idesc_bf16(64, BV, false, true, true), 1);
+#pragma unroll
+            for (int s = 0; s < 8; ++s)
+                mma_bf16(tm + LANE16 + TM_O, kmaj_desc(sbase + OFF_QG, 64, s), mnmaj_desc(s_op, BV, s),
+                         idesc_bf16(64, BV, false, true), s > 0);
+            mma_commit(mma_bar);
+        }
+        if (!wait_bar(mma_bar, mma_phase)) { aborted = true; mma_pending = true; break; }
+        tc_fence_after();
+        // the raw buffers are free again: fetch the next chunk
+        if (tid == 0 && c0 + C < eos) issue_tma(c0 + C);
+        tma_pending = c0 + C < eos;
+        // ================= phase 7: E -> bf16 (MN-major, MN = v, K = j)
+        {
+            const int j = 16 * sp + lane;   // valid for lane < 16
+            float v[32];
+            tmem_ld32(tm + lane_base + TM_UE + 32 * vhalf, v);
+            if (lane < 16) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    st_shared_v4(sm + OFF_E, mnmaj_off(32 * vhalf + 8 * q, j, BV), pack8(v + 8 * q));
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        // ================= phase 8: O += lower(Qp) E ; dS^T = (K e^{G_last - G})^T E
+        if (tid == 0) {
+            const uint32_t e_op = sbase + OFF_E;
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                mma_bf16(tm + LANE16 + TM_O, kmaj_desc(sbase + OFF_AQB, 64, s), mnmaj_desc(e_op, BV, s),
+                         idesc_bf16(64, BV, false, true), 1);
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                mma_bf16(tm + TM_DS, mnmaj_desc(sbase + OFF_KD, 128, s), mnmaj_desc(e_op, BV, s),
+                         idesc_bf16(128, BV, true, true), s > 0);
+            mma_commit(mma_bar);
+        }
+        if (!wait_bar(mma_bar, mma_phase)) { aborted = true; mma_pending = true; break; }
+        tc_fence_after();
+        // ================= phase 9: outputs and the state update
+        {
+            const int i = 16 * sp + lane - 16;   // valid for lane >= 16
+            float v[32];
+            tmem_ld32(tm + lane_base + TM_O + 32 * vhalf, v);
+            if (lane >= 16 && i < L) {
+                __nv_bfloat16* op = out + ((size_t)(c0 + i) * H + h) * DV + vt * BV + 32 * vhalf;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) reinterpret_cast<uint4*>(op)[q] = pack8(v + 8 * q);
+            }
+            float ds[32];
+            tmem_ld32(tm + lane_base + TM_DS + 32 * vhalf, ds);
+            const float dec = decay_s[c_own];
+#pragma unroll
+            for (int jv = 0; jv < 32; ++jv) S[jv] = fmaf(S[jv], dec, ds[jv]);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                st_shared_v4(sm + OFF_S, mnmaj_off(v0 + 8 * q, c_own, BV), pack8(S + 8 * q));
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    }
+
+    if (aborted) {
+        if (a.dev_status && tid == 0) atomicOr(a.dev_status, KDA_DEV_TIMEOUT);
+        // let copies / MMAs still in flight land before the memory goes away
+        if (tma_pending) (void)mbar_wait(full_bar, full_phase, kWaitNs);
+        if (mma_pending) (void)mbar_wait(mma_bar, mma_phase, kWaitNs);
+    } else if (a.S_T) {
+        const size_t sbase_g = ((size_t)n * H + h) * DV * DK;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const int v = vt * BV + v0 + j;
+            a.S_T[sbase_g + (size_t)v * DK + c_own] = S[j];
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tm, TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------- host side
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void* ptr = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// 3-D map over [tokens][H][width] (innermost first: width, H, tokens).
+bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, int width,
+              int H, long long tokens, int box_w, int box_t, CUtensorMapSwizzle sw) {
+    auto enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)width, (cuuint64_t)H, (cuuint64_t)tokens};
+    cuuint64_t strides[2] = {(cuuint64_t)width * esize, (cuuint64_t)width * esize * H};
+    cuuint32_t box[3] = {(cuuint32_t)box_w, 1u, (cuuint32_t)box_t};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    return enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int GATE>
+cudaError_t launch_gate(const TcParams& p, int grid, cudaStream_t st) {
+    auto kern = kda_chunk_tc_kernel<GATE>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, NT, SMEM_BYTES, st>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool chunk_tc_supported(int D, int V, int Cc) { return D == DK && V == DV && Cc == C; }
+
+cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t st) {
+    TcParams p;
+    memset(&p, 0, sizeof(p));
+    p.a = a;
+    const long long tokens = (long long)a.B * a.T;
+    if (tokens > 0) {  // with no tokens the kernel only copies S0 to S_T and never issues TMA
+        bool ok = make_map(&p.map_k, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DK, a.H, tokens, DK,
+                           C, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+                  make_map(&p.map_q, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DK, a.H, tokens, DK,
+                           C, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+                  make_map(&p.map_v, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DV, a.H, tokens, BV,
+                           C, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (ok && a.gate == KDA_GATE_CHANNEL)
+            ok = make_map(&p.map_g, a.g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, DK, a.H, tokens, DK, C,
+                          CU_TENSOR_MAP_SWIZZLE_NONE);
+        if (!ok) return cudaErrorInvalidValue;
+    }
+    const int grid = a.num_seqs * a.H * NVT;
+    switch (a.gate) {
+        case KDA_GATE_CHANNEL: return launch_gate<KDA_GATE_CHANNEL>(p, grid, st);
+        case KDA_GATE_SCALAR: return launch_gate<KDA_GATE_SCALAR>(p, grid, st);
+        default: return launch_gate<KDA_GATE_NONE>(p, grid, st);
+    }
+}
 
 }  // namespace kda

@@ -81,6 +81,9 @@ def test_chunk_validation(lib):
     # misaligned pointers
     assert _chunk(lib, _shape(B=0, N=0), q=P(0x10004)) == 3
     assert _chunk(lib, _shape(B=0, N=0), S0=P(0x10008)) == 3
+    assert _chunk(lib, _shape(B=0, N=0), g=P(0x10004)) == 3                       # per-channel g
+    assert _chunk(lib, _shape(B=0, N=0, gate=kda.KDA_GATE_SCALAR), g=P(0x10004)) == 0  # scalar g
+    assert _chunk(lib, _shape(B=1, N=0), cu=P(0x10004)) == 0                      # cu_seqlens
     # unsupported head sizes / chunks
     assert _chunk(lib, _shape(B=0, N=0, dk=24, dv=24, dtype=kda.KDA_F32)) == 2
     assert _chunk(lib, _shape(B=0, N=0, dk=256, dv=128, dtype=kda.KDA_F32)) == 2
