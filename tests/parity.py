@@ -9,16 +9,21 @@ import kimi_delta_attention_22_b200 as kda
 import oracle
 from kimi_delta_attention_22_b200 import inputs
 
-# Tolerances (see the readings of the pages): fp32 mode is compared by the
-# maximum absolute error.  bf16-input/fp32-state mode is compared relative to
-# the RMS of the oracle's tensor, per tensor, in two ways:
-#   * rms(gpu - oracle) / rms(oracle) <= 2e-2, and
-#   * element by element, |gpu - oracle| <= 2e-2 * rms(oracle) + q |oracle|,
-#     where q = 2^-8 (half a bf16 ulp, relative) when the library stores that
-#     tensor in bf16 and 0 when it stores fp32: the rounding of the stored
-#     result itself is not an arithmetic error of the path.
+# Tolerances (see the readings of the pages).  fp32 mode: the maximum
+# absolute error, max |gpu - oracle| <= 1e-4.  bf16-input/fp32-state mode:
+# the error relative to the RMS of the oracle's tensor, per tensor:
+#   * rms(gpu - oracle) / rms(oracle) <= 2e-2 (the stated tolerance), and
+#   * element by element, |gpu - oracle| <= 5 * 2e-2 * rms(oracle) + q |oracle|.
+#     Rounding errors summed over many bf16 products are close to Gaussian, and
+#     the largest of 1e5..1e6 such errors sits near 5 sigma, so this bound is
+#     the worst element consistent with the RMS tolerance.  It catches
+#     localised defects (one bad row or chunk) that an RMS could dilute.
+#     q = 2^-8 (half a bf16 ulp, relative) when the library stores that tensor
+#     in bf16, 0 for fp32 tensors: rounding the stored result is not an
+#     arithmetic error of the path.
 TOL_F32_ABS = 1e-4
 TOL_BF16_REL = 2e-2
+ELEM_FACTOR = 5.0
 BF16_HALF_ULP = 2.0 ** -8
 
 
@@ -27,9 +32,10 @@ def to_dev(d, dev="cuda"):
 
 
 def err(got, ref, mode, stored_bf16=None):
-    """Returns the error figure compared against the tolerance (see above).
-    For bf16 mode: max(rms ratio, worst element-wise excess over the rounding
-    allowance, both divided by rms(oracle))."""
+    """Returns the error figure compared against TOL_F32_ABS (fp32 mode) or
+    TOL_BF16_REL (bf16 mode: the larger of the RMS ratio and the worst
+    element-wise excess over the rounding allowance divided by ELEM_FACTOR,
+    both relative to rms(oracle))."""
     if stored_bf16 is None:
         stored_bf16 = hasattr(got, "dtype") and got.dtype == torch.bfloat16
     got = got.detach().cpu().double().numpy() if hasattr(got, "detach") else np.asarray(got)
@@ -46,7 +52,7 @@ def err(got, ref, mode, stored_bf16=None):
     q = 2 * BF16_HALF_ULP if stored_bf16 == "both" else (BF16_HALF_ULP if stored_bf16 else 0.0)
     elem = float(np.max(d - q * np.abs(ref))) / rms
     rel_rms = float(np.sqrt(np.mean(d ** 2))) / rms
-    return max(elem, rel_rms)
+    return max(rel_rms, elem / ELEM_FACTOR)
 
 
 def check(got, ref, mode, what, stored_bf16=None):
