@@ -50,15 +50,23 @@ constexpr int OFF_RAW = 0;                       // raw K | raw Q | raw G  (64 K
 constexpr int OFF_RK = OFF_RAW;                  //   [64][128] bf16
 constexpr int OFF_RQ = OFF_RAW + 16384;          //   [64][128] bf16
 constexpr int OFF_RG = OFF_RAW + 32768;          //   [64][128] fp32
-constexpr int OFF_OX = OFF_RAW;                  // after prep: Gram B operand (K-major, 128 rows)
-constexpr int OFF_KG = OFF_RAW + 32768;          //   K e^Gamma        (MN-major, MN = c, K = j)
-constexpr int OFF_QG = OFF_RAW + 49152;          //   Q~ e^Gamma       (K-major, 64 rows)
+constexpr int OFF_OX = OFF_RAW;                  // after prep (sub-block path): Gram B operand
+constexpr int OFF_KYG = OFF_RAW;                 // after prep (one-reference path): K e^{-Gamma}
+constexpr int OFF_KQG = OFF_RAW + 32768;         //   rows 0-63 K e^Gamma, rows 64-127 Q~ e^Gamma
+// K e^{-Gamma}, the K|Q e^Gamma tile and K e^{Gamma_last - Gamma} share one layout,
+// element (row n, channel c) at mnmaj_off(c, n, 128): 8-row groups 2048 bytes apart,
+// 64-channel halves 1024 apart.  Read as MN-major (MN = c) or as K-major (K = c).
+constexpr float kFastLimit2 = 112.f;             // one-reference path while max |Gamma_last| <= 2^112
 constexpr int OFF_RV = 65536;                    // raw V tile, TMA 128B swizzle = MN-major operand
 constexpr int OFF_A = 73728;                     // 64 KB, reused per phase:
-constexpr int OFF_OY = OFF_A;                    //   4 Gram A operands (K-major, 64 rows each)
-constexpr int OFF_AKK = OFF_A;                   //   fp32 [64][64] coupling matrix
-constexpr int OFF_AQK = OFF_A + 16384;           //   fp32 [64][64] Qp, then block scratch
-constexpr int OFF_TF = OFF_A + 32768;            //   fp32 [64][64] T
+constexpr int OFF_OY = OFF_A;                    //   Gram A operands: 2 K-major tiles of 128 rows
+                                                 //   (tile g: rows 0-63 version 2g, 64-127 version 2g+1)
+constexpr int LDT = 68;                          //   fp32 row stride of L and T (bank spread)
+constexpr int LDX = 24;                          //   fp32 row stride of the per-warp block scratch
+constexpr int OFF_L = OFF_A;                     //   fp32 [64][LDT] coupling matrix L
+constexpr int OFF_TF = OFF_A + 64 * LDT * 4;     //   fp32 [64][LDT] T = (I + L)^{-1}
+constexpr int OFF_XS = OFF_TF + 64 * LDT * 4;    //   fp32 [4][16][LDX] block-product scratch
+constexpr int OFF_Q32 = OFF_XS + 4 * 16 * LDX * 4; //   fp32 [64][LDT] lower(Qp) before its bf16 tile
 constexpr int OFF_W = OFF_A;                     //   W bf16 (K-major, 64 rows)
 constexpr int OFF_E = OFF_A + 16384;             //   E bf16 (MN-major, MN = v, K = j)
 constexpr int OFF_TB = OFF_A + 65536;            // T diag(beta) bf16 (K-major 64 x 64)
@@ -66,21 +74,24 @@ constexpr int OFF_AQB = OFF_TB + 8192;           // lower(Qp) bf16 (K-major 64 x
 constexpr int OFF_KD = OFF_AQB + 8192;           // K e^{Gamma_last - Gamma} (MN-major, MN = c)
 constexpr int OFF_S = OFF_KD + 16384;            // S^T bf16 (MN-major, MN = v, K = c)
 constexpr int OFF_SMALL = OFF_S + 16384;
-constexpr int OFF_TOT = OFF_SMALL;               // fp32 [4][128] sub-block sums of g
-constexpr int OFF_SUB = OFF_TOT + 2048;          // fp32 [4][128] cumsum at each reference row
-constexpr int OFF_BETA = OFF_SUB + 2048;         // fp32 [64]
+constexpr int OFF_TOT4 = OFF_SMALL;              // fp32 [16][128] row-group sums of g (log2), then prefixes
+constexpr int OFF_GREF = OFF_TOT4 + 8192;        // fp32 [4][128] Gamma (log2) at each reference row
+constexpr int OFF_GLAST = OFF_GREF + 2048;       // fp32 [128] Gamma (log2) at the chunk's last row
+constexpr int OFF_RED = OFF_GLAST + 512;         // fp32 [4] per-warp max |Gamma_last| (log2)
+constexpr int OFF_BETA = OFF_RED + 16;           // fp32 [64]
 constexpr int OFF_DECAY = OFF_BETA + 256;        // fp32 [128] e^{Gamma_last}
 constexpr int OFF_BAR = OFF_DECAY + 512;         // mbarriers + tmem base + flags
 constexpr int SMEM_USED = OFF_BAR + 64;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;     // + alignment slack
-constexpr uint32_t TMEM_COLS = 256;
+static_assert(OFF_Q32 + 64 * LDT * 4 <= OFF_A + 65536, "phase-3 scratch overflows region A");
+constexpr uint32_t TMEM_COLS = 512;
 
 // TMEM columns (lane base 0 or 16 for M = 64 accumulators).
-constexpr uint32_t TM_GRAM = 0;     // lanes 0-15 : [j][32 I + u]  P^T | Qp^T
-constexpr uint32_t TM_W = 0;        // lanes 16-31: W   [i][c]   (128 cols)
+constexpr uint32_t TM_GRAM = 0;     // all lanes  : group g at cols 64 g: [version rows j][X rows]
 constexpr uint32_t TM_UE = 128;     // lanes 0-15 : U, then E = U - W S^T  [j][v]
 constexpr uint32_t TM_O = 128;      // lanes 16-31: O   [i][v]
 constexpr uint32_t TM_DS = 192;     // all lanes  : dS^T [c][v]
+constexpr uint32_t TM_W = 256;      // lanes 0-15 : W   [i][c]   (128 cols)
 constexpr uint32_t LANE16 = 16u << 16;
 
 struct TcParams {
@@ -96,11 +107,71 @@ __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
     __nv_bfloat162 t = *reinterpret_cast<__nv_bfloat162*>(&u);
     return __bfloat1622float2(t);
 }
-__device__ __forceinline__ void st_shared_u32(uint8_t* base, uint32_t off, uint32_t v) {
-    *reinterpret_cast<uint32_t*>(base + off) = v;
-}
 __device__ __forceinline__ void st_shared_v4(uint8_t* base, uint32_t off, uint4 v) {
     *reinterpret_cast<uint4*>(base + off) = v;
+}
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// 2^x on the special-function unit (inputs here are differences of
+// cumulative log2 decays, so |x| stays far below the exponent range).
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
+// acc (16x16, two m16n8 C fragments) += A (16x16) * B (16x16), both fp32 in
+// shared memory (row-major, strides lda / ldb), on the warp-level tf32 MMA.
+__device__ __forceinline__ void blk_mma(float (&acc)[2][4], const float* A, int lda, const float* B,
+                                        int ldb, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+        const uint32_t a0 = to_tf32(A[g * lda + 8 * ks + t]);
+        const uint32_t a1 = to_tf32(A[(g + 8) * lda + 8 * ks + t]);
+        const uint32_t a2 = to_tf32(A[g * lda + 8 * ks + t + 4]);
+        const uint32_t a3 = to_tf32(A[(g + 8) * lda + 8 * ks + t + 4]);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            const uint32_t b0 = to_tf32(B[(8 * ks + t) * ldb + 8 * nt + g]);
+            const uint32_t b1 = to_tf32(B[(8 * ks + t + 4) * ldb + 8 * nt + g]);
+            asm volatile(
+                "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, "
+                "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};\n"
+                : "+f"(acc[nt][0]), "+f"(acc[nt][1]), "+f"(acc[nt][2]), "+f"(acc[nt][3])
+                : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+        }
+    }
+}
+
+// K-major view (K = channel) of rows laid out by mnmaj_off(c, row, 128): k-step s.
+__device__ __forceinline__ uint64_t rowview_desc(uint32_t base, int s) {
+    return desc_sw128(base + (uint32_t)((s >> 2) * 1024 + (s & 3) * 32), 16, 2048);
+}
+
+// Store a 16x16 C-fragment pair, scaled by s, to shared memory (row stride ld).
+__device__ __forceinline__ void blk_store(float* Cm, int ld, const float (&acc)[2][4], int lane,
+                                          float s) {
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        Cm[g * ld + 8 * nt + 2 * t] = s * acc[nt][0];
+        Cm[g * ld + 8 * nt + 2 * t + 1] = s * acc[nt][1];
+        Cm[(g + 8) * ld + 8 * nt + 2 * t] = s * acc[nt][2];
+        Cm[(g + 8) * ld + 8 * nt + 2 * t + 1] = s * acc[nt][3];
+    }
+}
+
+__device__ __forceinline__ void unpack8(uint4 u, float* f) {
+    const float2 a = unpack_bf16(u.x), b = unpack_bf16(u.y), c = unpack_bf16(u.z), d = unpack_bf16(u.w);
+    f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y; f[4] = c.x; f[5] = c.y; f[6] = d.x; f[7] = d.y;
 }
 
 // Store 8 consecutive fp32 values as one 16-byte bf16 chunk.
@@ -124,8 +195,9 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
     const int vhalf = warp >> 2;       // which 32 of the tile's 64 value columns
     const uint32_t lane_base = (uint32_t)(32 * sp) << 16;
 
-    float* tot = reinterpret_cast<float*>(sm + OFF_TOT);
-    float* sub = reinterpret_cast<float*>(sm + OFF_SUB);
+    float* tot4 = reinterpret_cast<float*>(sm + OFF_TOT4);
+    float* gref_s = reinterpret_cast<float*>(sm + OFF_GREF);
+    float* glast_s = reinterpret_cast<float*>(sm + OFF_GLAST);
     float* beta_s = reinterpret_cast<float*>(sm + OFF_BETA);
     float* decay_s = reinterpret_cast<float*>(sm + OFF_DECAY);
     uint64_t* full_bar = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
@@ -201,145 +273,282 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
     bool aborted = false;
     for (long long c0 = bos; c0 < eos; c0 += C) {
         const int L = (int)min((long long)C, eos - c0);
-        // ================= phase 1: decay, reference factors, operands
+        // ================= phase 1: log-space decay, reference factors, operands
+        bool fast;   // one reference (chunk start) for the whole chunk, else 16-row sub-blocks
+        const float beta_pf = (tid < L) ? a.beta[(size_t)(c0 + tid) * H + h] : 0.f;  // overlaps the wait
         if (!wait_bar(full_bar, full_phase)) { aborted = true; break; }
         tma_pending = false;
-        const int blk = tid >> 6;        // 16-row sub-block
-        const int pr = tid & 63;         // channel pair
-        const int ch = 2 * pr;
-        float gl[16][2];
-        uint32_t kr[16], qr[16];
         {
-            float run0 = 0.f, run1 = 0.f;
+            // thread tile: channels c8..c8+7 of rows 4 rg .. 4 rg + 3 (log2 units throughout)
+            const int cq = tid & 15, rg = tid >> 4, c8 = 8 * cq;
+            float g2[4][8], run[8];
+            uint4 kraw[4], qraw[4];
 #pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                const int i = 16 * blk + u;
+            for (int e = 0; e < 8; ++e) run[e] = 0.f;
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const int i = 4 * rg + r;
                 const bool valid = i < L;
-                float g0 = 0.f, g1 = 0.f;
+                float gv[8];
                 if (GATE == KDA_GATE_CHANNEL) {
-                    const float2 gg = *reinterpret_cast<const float2*>(sm + OFF_RG + (i * DK + ch) * 4);
-                    g0 = gg.x; g1 = gg.y;
+                    const float4 a0 = *reinterpret_cast<const float4*>(sm + OFF_RG + (i * DK + c8) * 4);
+                    const float4 a1 = *reinterpret_cast<const float4*>(sm + OFF_RG + (i * DK + c8 + 4) * 4);
+                    gv[0] = a0.x; gv[1] = a0.y; gv[2] = a0.z; gv[3] = a0.w;
+                    gv[4] = a1.x; gv[5] = a1.y; gv[6] = a1.z; gv[7] = a1.w;
                 } else if (GATE == KDA_GATE_SCALAR) {
-                    g0 = g1 = valid ? a.g[(size_t)(c0 + i) * H + h] : 0.f;
+                    const float gs = valid ? a.g[(size_t)(c0 + i) * H + h] : 0.f;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) gv[e] = gs;
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) gv[e] = 0.f;
                 }
-                if (!valid) { g0 = 0.f; g1 = 0.f; }
-                run0 += g0; run1 += g1;
-                gl[u][0] = run0; gl[u][1] = run1;
-                const uint32_t kk = *reinterpret_cast<const uint32_t*>(sm + OFF_RK + (i * DK + ch) * 2);
-                const uint32_t qq = *reinterpret_cast<const uint32_t*>(sm + OFF_RQ + (i * DK + ch) * 2);
-                kr[u] = valid ? kk : 0u;
-                qr[u] = valid ? qq : 0u;
-            }
-            tot[blk * DK + ch] = run0; tot[blk * DK + ch + 1] = run1;
-            sub[blk * DK + ch] = gl[7][0]; sub[blk * DK + ch + 1] = gl[7][1];
-            if (tid < C) beta_s[tid] = (tid < L) ? a.beta[(size_t)(c0 + tid) * H + h] : 0.f;
-        }
-        __syncthreads();   // raw K/Q/G are consumed; their space now takes operands
-        {
-            // prefix sums of the sub-block totals for this thread's two channels
-            float pre[2] = {0.f, 0.f}, last[2] = {0.f, 0.f}, gref[4][2];
 #pragma unroll
-            for (int b = 0; b < 4; ++b) {
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    gref[b][e] = last[e] + sub[b * DK + ch + e];   // Gamma at reference row of sub-block b
-                    if (b < blk) pre[e] += tot[b * DK + ch + e];
-                    last[e] += tot[b * DK + ch + e];
+                for (int e = 0; e < 8; ++e) {
+                    run[e] += valid ? gv[e] * kLog2e : 0.f;
+                    g2[r][e] = run[e];
                 }
+                const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+                kraw[r] = valid ? *reinterpret_cast<const uint4*>(sm + OFF_RK + (i * DK + c8) * 2) : z4;
+                qraw[r] = valid ? *reinterpret_cast<const uint4*>(sm + OFF_RQ + (i * DK + c8) * 2) : z4;
             }
-            float Er[2], Lr[2], z[4][2];
+            *reinterpret_cast<float4*>(tot4 + rg * DK + c8) = make_float4(run[0], run[1], run[2], run[3]);
+            *reinterpret_cast<float4*>(tot4 + rg * DK + c8 + 4) = make_float4(run[4], run[5], run[6], run[7]);
+            if (tid < C) beta_s[tid] = beta_pf;
+            __syncthreads();   // raw K/Q/G are consumed; their space now takes operands
+            // exclusive prefix over the 16 row groups, one thread per channel; the
+            // reference row of sub-block b is row 16 b + 7 (prefix before group 4 b + 2)
+            if (tid < DK) {
+                float tv[16];
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const float gr = gref[blk][e];
-                Er[e] = __expf(gr);                 // e^{Gamma_r}
-                Lr[e] = __expf(last[e] - gr);       // e^{Gamma_last - Gamma_r}
+                for (int q = 0; q < 16; ++q) tv[q] = tot4[q * DK + tid];
+                float acc = 0.f;
 #pragma unroll
-                for (int I = 0; I < 4; ++I) z[I][e] = (I > blk) ? __expf(gref[I][e] - gr) : 0.f;
-            }
-            if (blk == 0) {
-                decay_s[ch] = __expf(last[0]);
-                decay_s[ch + 1] = __expf(last[1]);
-            }
-#pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                const int i = 16 * blk + u;
-                float x[2], y[2];
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const float dlt = gl[u][e] - gl[7][e];   // Gamma_i - Gamma_r
-                    x[e] = __expf(dlt);
-                    y[e] = __expf(-dlt);
+                for (int q = 0; q < 16; ++q) {
+                    if ((q & 3) == 2) gref_s[(q >> 2) * DK + tid] = acc;
+                    const float t = tv[q];
+                    tv[q] = acc;
+                    acc += t;
                 }
-                const float2 kf = unpack_bf16(kr[u]);
-                const float2 qf = unpack_bf16(qr[u]);
-                const float k0 = kf.x, k1 = kf.y;
-                const float q0 = qf.x * a.scale, q1 = qf.y * a.scale;
-                // Gram B operand: K rows at 32 blk + u, Q rows at 32 blk + 16 + u
-                st_shared_u32(sm + OFF_OX, kmaj_off(32 * blk + u, ch, 128), pack_bf16(k0 * x[0], k1 * x[1]));
-                st_shared_u32(sm + OFF_OX, kmaj_off(32 * blk + 16 + u, ch, 128), pack_bf16(q0 * x[0], q1 * x[1]));
-                // Gram A operands (j-side) for target sub-blocks I >= blk; zero rows for I < blk
 #pragma unroll
-                for (int I = 0; I < 4; ++I) {
-                    uint32_t val = 0u;
-                    if (I == blk) val = pack_bf16(k0 * y[0], k1 * y[1]);
-                    else if (I > blk) val = pack_bf16(k0 * y[0] * z[I][0], k1 * y[1] * z[I][1]);
-                    st_shared_u32(sm + OFF_OY + I * 16384, kmaj_off(i, ch, 64), val);
+                for (int q = 0; q < 16; ++q) tot4[q * DK + tid] = tv[q];
+                glast_s[tid] = acc;
+                decay_s[tid] = ex2(acc);
+                float m = -acc;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                if (lane == 0) reinterpret_cast<float*>(sm + OFF_RED)[warp] = m;
+            }
+            __syncthreads();
+            const float* red = reinterpret_cast<const float*>(sm + OFF_RED);
+            fast = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3])) <= kFastLimit2;
+            const uint32_t basemn_f = (uint32_t)((rg >> 1) * 2048 + (cq >> 3) * 1024 + (rg & 1) * 512);
+            if (fast) {
+                // one reference: e^{Gamma_i} <= 1 on the i-side, e^{-Gamma_j} <= 2^112 on the j-side
+                float pre[8], dec[8];
+                {
+                    const float4* pp = reinterpret_cast<const float4*>(tot4 + rg * DK + c8);
+                    const float4* dp = reinterpret_cast<const float4*>(decay_s + c8);
+                    const float4 p0 = pp[0], p1 = pp[1], d0 = dp[0], d1 = dp[1];
+                    pre[0] = p0.x; pre[1] = p0.y; pre[2] = p0.z; pre[3] = p0.w;
+                    pre[4] = p1.x; pre[5] = p1.y; pre[6] = p1.z; pre[7] = p1.w;
+                    dec[0] = d0.x; dec[1] = d0.y; dec[2] = d0.z; dec[3] = d0.w;
+                    dec[4] = d1.x; dec[5] = d1.y; dec[6] = d1.z; dec[7] = d1.w;
                 }
-                const float eg0 = Er[0] * x[0], eg1 = Er[1] * x[1];   // e^{Gamma_i}
-                const float ed0 = Lr[0] * y[0], ed1 = Lr[1] * y[1];   // e^{Gamma_last - Gamma_i}
-                // (ch, ch + 1) are adjacent in both layouts (ch even)
-                st_shared_u32(sm + OFF_KG, mnmaj_off(ch, i, 128), pack_bf16(k0 * eg0, k1 * eg1));
-                st_shared_u32(sm + OFF_QG, kmaj_off(i, ch, 64), pack_bf16(q0 * eg0, q1 * eg1));
-                st_shared_u32(sm + OFF_KD, mnmaj_off(ch, i, 128), pack_bf16(k0 * ed0, k1 * ed1));
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const uint32_t omn = basemn_f + (((uint32_t)(cq & 7) ^ (uint32_t)(4 * (rg & 1) + r)) << 4) +
+                                         (uint32_t)(r * 128);
+                    float kf[8], qf[8], t1[8], t2[8], t3[8], t4[8];
+                    unpack8(kraw[r], kf);
+                    unpack8(qraw[r], qf);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float gm = pre[e] + g2[r][e];   // Gamma_i (log2), <= 0
+                        const float eg = ex2(gm), ey = ex2(-gm);
+                        t1[e] = kf[e] * eg;                    // K e^{Gamma}
+                        t2[e] = (qf[e] * a.scale) * eg;        // Q~ e^{Gamma}
+                        t3[e] = kf[e] * ey;                    // K e^{-Gamma}
+                        t4[e] = kf[e] * (dec[e] * ey);         // K e^{Gamma_last - Gamma}
+                    }
+                    st_shared_v4(sm + OFF_KQG, omn, pack8(t1));
+                    st_shared_v4(sm + OFF_KQG, omn + 16384, pack8(t2));
+                    st_shared_v4(sm + OFF_KYG, omn, pack8(t3));
+                    st_shared_v4(sm + OFF_KD, omn, pack8(t4));
+                }
+            } else {
+                const int b = rg >> 2;
+                float pre[8], gr[8], Er[8], Lr[8], z[4][8];
+                {
+                    const float4* pp = reinterpret_cast<const float4*>(tot4 + rg * DK + c8);
+                    const float4* gp = reinterpret_cast<const float4*>(gref_s + b * DK + c8);
+                    const float4* lp = reinterpret_cast<const float4*>(glast_s + c8);
+                    const float4 p0 = pp[0], p1 = pp[1], r0 = gp[0], r1 = gp[1], l0 = lp[0], l1 = lp[1];
+                    const float pv[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+                    const float rv[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+                    const float lv[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
+    #pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        pre[e] = pv[e];
+                        gr[e] = rv[e];
+                        Er[e] = ex2(rv[e]);            // e^{Gamma_r}
+                        Lr[e] = ex2(lv[e] - rv[e]);    // e^{Gamma_last - Gamma_r}
+                    }
+    #pragma unroll
+                    for (int I = 1; I < 4; ++I) {
+                        if (I > b) {
+                            const float4* ip = reinterpret_cast<const float4*>(gref_s + I * DK + c8);
+                            const float4 i0 = ip[0], i1 = ip[1];
+                            const float iv[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
+    #pragma unroll
+                            for (int e = 0; e < 8; ++e) z[I][e] = ex2(iv[e] - rv[e]);   // e^{Gamma_rI - Gamma_r} <= 1
+                        }
+                    }
+                }
+                // swizzled byte offsets of this thread's 16-byte chunks (row i = 4 rg + r)
+                const uint32_t sw0 = (uint32_t)(cq & 7);
+                    // the same rows inside a 128-row tile (Gram A operands): K-atom stride 16 KB
+                const uint32_t baseY = (uint32_t)((cq >> 3) * 16384 + (rg >> 1) * 1024 + (rg & 1) * 512);
+                const uint32_t base128 = (uint32_t)((cq >> 3) * 16384 + ((rg >> 1) + 2 * b) * 1024 + (rg & 1) * 512);
+                const uint32_t basemn = (uint32_t)((rg >> 1) * 2048 + (cq >> 3) * 1024 + (rg & 1) * 512);
+    #pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const uint32_t swz = ((sw0 ^ (uint32_t)(4 * (rg & 1) + r)) << 4) + (uint32_t)(r * 128);
+                    const uint32_t o128 = base128 + swz, omn = basemn + swz;
+                    const uint32_t oy = baseY + swz;   // + (I >> 1) * 32768 + (I & 1) * 8192 for version I
+                    float kf[8], qf[8], x[8], y[8], t[8];
+                    unpack8(kraw[r], kf);
+                    unpack8(qraw[r], qf);
+    #pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float dl = (pre[e] + g2[r][e]) - gr[e];   // Gamma_i - Gamma_r (log2)
+                        x[e] = ex2(dl);
+                        y[e] = ex2(-dl);
+                        qf[e] *= a.scale;
+                    }
+                    // Gram i-side: K rows at 32 b + (i - 16 b), Q rows 16 further
+    #pragma unroll
+                    for (int e = 0; e < 8; ++e) t[e] = kf[e] * x[e];
+                    st_shared_v4(sm + OFF_OX, o128, pack8(t));
+    #pragma unroll
+                    for (int e = 0; e < 8; ++e) t[e] = qf[e] * x[e];
+                    st_shared_v4(sm + OFF_OX, o128 + 2048, pack8(t));
+                    // Gram j-side for this sub-block and the later ones
+                    float ky[8];
+    #pragma unroll
+                    for (int e = 0; e < 8; ++e) ky[e] = kf[e] * y[e];
+                    st_shared_v4(sm + OFF_OY + (b >> 1) * 32768 + (b & 1) * 8192, oy, pack8(ky));
+    #pragma unroll
+                    for (int I = 1; I < 4; ++I) {
+                        if (I > b) {
+    #pragma unroll
+                            for (int e = 0; e < 8; ++e) t[e] = ky[e] * z[I][e];
+                            st_shared_v4(sm + OFF_OY + (I >> 1) * 32768 + (I & 1) * 8192, oy, pack8(t));
+                        }
+                    }
+                    // K e^Gamma (MN-major), Q~ e^Gamma (K-major), K e^{Gamma_last - Gamma} (MN-major)
+                    float t2[8];
+    #pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float eg = Er[e] * x[e];
+                        t[e] = kf[e] * eg;
+                        t2[e] = qf[e] * eg;
+                    }
+                    st_shared_v4(sm + OFF_KQG, omn, pack8(t));
+                    st_shared_v4(sm + OFF_KQG, omn + 16384, pack8(t2));
+    #pragma unroll
+                    for (int e = 0; e < 8; ++e) t[e] = kf[e] * (Lr[e] * y[e]);
+                    st_shared_v4(sm + OFF_KD, omn, pack8(t));
+                }
             }
         }
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
-        // ================= phase 2: Gram MMAs  (D[j][32 I + u] = Ky_I[j] . X[32 I + u])
+        // ================= phase 2: Gram MMAs.  Group g (M = 128, N = 64): A rows 0-63 are
+        // the j-side operand of sub-block 2g, rows 64-127 that of sub-block 2g+1; B rows
+        // are the i-side rows of sub-blocks 2g and 2g+1 (K then Q~ for each).
+        // One-reference path: a single group, D[n][j] = [K e^G ; Q~ e^G]_n . (K e^-G)_j.
         if (tid == 0) {
-            const uint32_t ox = sbase + OFF_OX;
+            if (fast) {
 #pragma unroll
-            for (int I = 0; I < 4; ++I) {
-                const uint32_t oy = sbase + OFF_OY + I * 16384;
+                for (int s8 = 0; s8 < 8; ++s8)
+                    mma_bf16(tm + TM_GRAM, rowview_desc(sbase + OFF_KQG, s8),
+                             rowview_desc(sbase + OFF_KYG, s8), idesc_bf16(128, 64, false, false),
+                             s8 > 0);
+            } else {
+                const uint32_t ox = sbase + OFF_OX, oy = sbase + OFF_OY;
 #pragma unroll
-                for (int s = 0; s < 8; ++s)
-                    mma_bf16(tm + TM_GRAM + 32 * I, kmaj_desc(oy, 64, s),
-                             kmaj_desc(ox + I * 32 * 128, 128, s) /* rows 32I.. of a 128-row tile */,
-                             idesc_bf16(64, 32, false, false), s > 0);
+                for (int s8 = 0; s8 < 8; ++s8)
+#pragma unroll
+                    for (int g = 0; g < 2; ++g)
+                        mma_bf16(tm + TM_GRAM + 64 * g, kmaj_desc(oy + g * 32768, 128, s8),
+                                 kmaj_desc(ox + g * 8192, 128, s8), idesc_bf16(128, 64, false, false),
+                                 s8 > 0);
             }
             mma_commit(mma_bar);
         }
         if (!wait_bar(mma_bar, mma_phase)) { aborted = true; mma_pending = true; break; }
         tc_fence_after();
-        // ================= phase 3: coupling matrix, Qp, and T = (I + L)^{-1}
-        float* Akk = reinterpret_cast<float*>(sm + OFF_AKK);
-        float* Aqk = reinterpret_cast<float*>(sm + OFF_AQK);
+        // ================= phase 3: coupling matrix L, lower(Qp), T = (I + L)^{-1}
+        float* Lm = reinterpret_cast<float*>(sm + OFF_L);
         float* TF = reinterpret_cast<float*>(sm + OFF_TF);
-        if (warp < 4) {
-            const int j = 16 * sp + lane;   // valid for lane < 16
+        if (fast) {
+            // lane n = 32 sp + lane: rows i of P (n < 64) or of Qp (n >= 64); warp group
+            // vhalf reads columns j = 32 vhalf .. 32 vhalf + 31
+            const int n = 32 * sp + lane, j0 = 32 * vhalf;
+            float v[32];
+            tmem_ld32(tm + lane_base + TM_GRAM + j0, v);
+            if (n < 64) {
+                const int i = n;
+                const float bi = beta_s[i];
 #pragma unroll
-            for (int I = 0; I < 4; ++I) {
-                float v[32];
-                tmem_ld32(tm + lane_base + TM_GRAM + 32 * I, v);
-                if (lane < 16) {
-#pragma unroll
-                    for (int u = 0; u < 16; ++u) {
-                        const int i = 16 * I + u;
-                        Akk[i * C + j] = (j < i) ? beta_s[i] * v[u] : 0.f;
-                        Aqk[i * C + j] = (j <= i) ? v[16 + u] : 0.f;
-                    }
+                for (int q = 0; q < 8; ++q) {
+                    float4 o;
+                    o.x = (j0 + 4 * q + 0 < i) ? bi * v[4 * q + 0] : 0.f;
+                    o.y = (j0 + 4 * q + 1 < i) ? bi * v[4 * q + 1] : 0.f;
+                    o.z = (j0 + 4 * q + 2 < i) ? bi * v[4 * q + 2] : 0.f;
+                    o.w = (j0 + 4 * q + 3 < i) ? bi * v[4 * q + 3] : 0.f;
+                    *reinterpret_cast<float4*>(Lm + i * LDT + j0 + 4 * q) = o;
                 }
+            } else {
+                const int i = n - 64;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    float t8[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) t8[e] = (j0 + 8 * q + e <= i) ? v[8 * q + e] : 0.f;
+                    st_shared_v4(sm + OFF_AQB, kmaj_off(i, j0 + 8 * q, 64), pack8(t8));
+                }
+            }
+        } else {
+            // warp group g reads Gram group g; lanes of sub-partitions 0-1 hold rows j of
+            // sub-block 2g's version, those of 2-3 rows j of sub-block 2g+1's version
+            const int g = vhalf, hi = sp >> 1;
+            const int I = 2 * g + hi, j = 32 * (sp & 1) + lane;
+            float* Q32 = reinterpret_cast<float*>(sm + OFF_Q32);
+            float bi[16];
+            {
+                const float4* bp = reinterpret_cast<const float4*>(beta_s + 16 * I);
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const float4 t4 = bp[q4];
+                    bi[4 * q4] = t4.x; bi[4 * q4 + 1] = t4.y; bi[4 * q4 + 2] = t4.z; bi[4 * q4 + 3] = t4.w;
+                }
+            }
+            float v[32];
+            tmem_ld32(tm + lane_base + TM_GRAM + 64 * g + 32 * hi, v);
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const int i = 16 * I + u;
+                Lm[i * LDT + j] = (j < i) ? bi[u] * v[u] : 0.f;
+                Q32[i * LDT + j] = (j <= i) ? v[16 + u] : 0.f;
             }
         }
         tc_fence_before();
         __syncthreads();
-        // lower(Qp) -> bf16 operand; diagonal blocks of T by forward substitution
-        for (int e = tid; e < C * C / 2; e += NT) {
-            const int i = e / (C / 2), j = 2 * (e % (C / 2));
-            st_shared_u32(sm + OFF_AQB, kmaj_off(i, j, 64), pack_bf16(Aqk[i * C + j], Aqk[i * C + j + 1]));
-        }
+        // diagonal 16x16 blocks of T by forward substitution (lane = column)
         if (warp < 4) {
             const int I = warp, cc = lane & 15;
             float t[16];
@@ -347,54 +556,53 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
             for (int r = 0; r < 16; ++r) {
                 float acc = 0.f;
 #pragma unroll
-                for (int k = 0; k < r; ++k) acc = fmaf(Akk[(16 * I + r) * C + 16 * I + k], t[k], acc);
+                for (int k = 0; k < r; ++k) acc = fmaf(Lm[(16 * I + r) * LDT + 16 * I + k], t[k], acc);
                 t[r] = (r < cc) ? 0.f : ((r == cc) ? 1.f : -acc);
             }
             if (lane < 16) {
 #pragma unroll
-                for (int r = 0; r < 16; ++r) TF[(16 * I + r) * C + 16 * I + cc] = t[r];
-            }
-        } else {
-            // zero the strictly-upper blocks of T
-            for (int e = tid - 128; e < 6 * 256; e += 128) {
-                const int bidx = e >> 8, r = (e >> 4) & 15, cc = e & 15;
-                const int I = (bidx < 3) ? 0 : ((bidx < 5) ? 1 : 2);
-                const int J = (bidx < 3) ? bidx + 1 : ((bidx < 5) ? bidx - 1 : 3);
-                TF[(16 * I + r) * C + 16 * J + cc] = 0.f;
+                for (int r = 0; r < 16; ++r) TF[(16 * I + r) * LDT + 16 * I + cc] = t[r];
             }
         }
         __syncthreads();
-        // off-diagonal blocks, level by level: T_IJ = -T_II sum_{K=J}^{I-1} L_IK T_KJ
-        float* X = Aqk;   // scratch: Qp is already in its bf16 tile
+        // off-diagonal blocks by level: T_IJ = -T_II sum_{K=J}^{I-1} L_IK T_KJ (warp J at level I-J)
 #pragma unroll 1
         for (int d = 1; d < 4; ++d) {
-            const int nb = 4 - d;
-            for (int e = tid; e < nb * 256; e += NT) {
-                const int J = e >> 8, I = J + d, r = (e >> 4) & 15, cc = e & 15;
-                float acc = 0.f;
+            if (warp < 4 - d) {
+                const int J = warp, I = J + d;
+                float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
                 for (int K = J; K < I; ++K)
-#pragma unroll
-                    for (int k = 0; k < 16; ++k)
-                        acc = fmaf(Akk[(16 * I + r) * C + 16 * K + k], TF[(16 * K + k) * C + 16 * J + cc], acc);
-                X[(16 * J + r) * 16 + cc] = acc;
-            }
-            __syncthreads();
-            for (int e = tid; e < nb * 256; e += NT) {
-                const int J = e >> 8, I = J + d, r = (e >> 4) & 15, cc = e & 15;
-                float acc = 0.f;
-#pragma unroll
-                for (int k = 0; k < 16; ++k)
-                    acc = fmaf(TF[(16 * I + r) * C + 16 * I + k], X[(16 * J + k) * 16 + cc], acc);
-                TF[(16 * I + r) * C + 16 * J + cc] = -acc;
+                    blk_mma(acc, Lm + 16 * I * LDT + 16 * K, LDT, TF + 16 * K * LDT + 16 * J, LDT, lane);
+                float* Xs = reinterpret_cast<float*>(sm + OFF_XS) + warp * 16 * LDX;
+                blk_store(Xs, LDX, acc, lane, 1.f);
+                __syncwarp();
+                float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                blk_mma(acc2, TF + 16 * I * LDT + 16 * I, LDT, Xs, LDX, lane);
+                blk_store(TF + 16 * I * LDT + 16 * J, LDT, acc2, lane, -1.f);
             }
             __syncthreads();
         }
-        // T diag(beta) -> bf16 operand (K-major, rows i, K = j)
-        for (int e = tid; e < C * C / 2; e += NT) {
-            const int i = e / (C / 2), j = 2 * (e % (C / 2));
-            const float t0 = (j <= i) ? TF[i * C + j] * beta_s[j] : 0.f;
-            const float t1 = (j + 1 <= i) ? TF[i * C + j + 1] * beta_s[j + 1] : 0.f;
-            st_shared_u32(sm + OFF_TB, kmaj_off(i, j, 64), pack_bf16(t0, t1));
+        // lower(Qp) and T diag(beta) -> bf16 operands (K-major, rows i, K = j), 8 columns per step
+        for (int e = tid; !fast && e < C * 8; e += NT) {
+            const int i = e >> 3, j0 = 8 * (e & 7);
+            const float* Q32 = reinterpret_cast<const float*>(sm + OFF_Q32);
+            const float4 a0 = *reinterpret_cast<const float4*>(Q32 + i * LDT + j0);
+            const float4 a1 = *reinterpret_cast<const float4*>(Q32 + i * LDT + j0 + 4);
+            const float t8[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            st_shared_v4(sm + OFF_AQB, kmaj_off(i, j0, 64), pack8(t8));
+        }
+        for (int e = tid; e < C * 8; e += NT) {
+            const int i = e >> 3, j0 = 8 * (e & 7);
+            const float4 a0 = *reinterpret_cast<const float4*>(TF + i * LDT + j0);
+            const float4 a1 = *reinterpret_cast<const float4*>(TF + i * LDT + j0 + 4);
+            const float tv[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            const float4 b0 = *reinterpret_cast<const float4*>(beta_s + j0);
+            const float4 b1 = *reinterpret_cast<const float4*>(beta_s + j0 + 4);
+            const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+            float t8[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) t8[k] = (j0 + k <= i) ? tv[k] * bv[k] : 0.f;
+            st_shared_v4(sm + OFF_TB, kmaj_off(i, j0, 64), pack8(t8));
         }
         fence_async_smem();
         tc_fence_before();
@@ -405,7 +613,7 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
             const uint32_t tb = sbase + OFF_TB;
 #pragma unroll
             for (int s = 0; s < 4; ++s)
-                mma_bf16(tm + LANE16 + TM_W, kmaj_desc(tb, 64, s), mnmaj_desc(sbase + OFF_KG, 128, s),
+                mma_bf16(tm + TM_W, kmaj_desc(tb, 64, s), mnmaj_desc(sbase + OFF_KQG, 128, s),
                          idesc_bf16(64, 128, false, true), s > 0);
 #pragma unroll
             for (int s = 0; s < 4; ++s)
@@ -417,13 +625,13 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
         tc_fence_after();
         // ================= phase 5: W -> bf16 (K-major, 64 rows, K = c)
         {
-            const int i = 16 * sp + lane - 16;   // valid for lane >= 16
+            const int i = 16 * sp + lane;   // valid for lane < 16
 #pragma unroll
             for (int m = 0; m < 2; ++m) {
                 const int col = 64 * vhalf + 32 * m;
                 float v[32];
                 tmem_ld32(tm + lane_base + TM_W + col, v);
-                if (lane >= 16) {
+                if (lane < 16) {
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
                         st_shared_v4(sm + OFF_W, kmaj_off(i, col + 8 * q, 64), pack8(v + 8 * q));
@@ -438,13 +646,12 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
         if (tid == 0) {
             const uint32_t s_op = sbase + OFF_S;
 #pragma unroll
-            for (int s = 0; s < 8; ++s)
+            for (int s = 0; s < 8; ++s) {
                 mma_bf16(tm + TM_UE, kmaj_desc(sbase + OFF_W, 64, s), mnmaj_desc(s_op, BV, s),
                          idesc_bf16(64, BV, false, true, true), 1);
-#pragma unroll
-            for (int s = 0; s < 8; ++s)
-                mma_bf16(tm + LANE16 + TM_O, kmaj_desc(sbase + OFF_QG, 64, s), mnmaj_desc(s_op, BV, s),
+                mma_bf16(tm + LANE16 + TM_O, rowview_desc(sbase + OFF_KQG + 16384, s), mnmaj_desc(s_op, BV, s),
                          idesc_bf16(64, BV, false, true), s > 0);
+            }
             mma_commit(mma_bar);
         }
         if (!wait_bar(mma_bar, mma_phase)) { aborted = true; mma_pending = true; break; }
