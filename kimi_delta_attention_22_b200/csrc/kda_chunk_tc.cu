@@ -68,21 +68,22 @@ constexpr int OFF_TF = OFF_A + 64 * LDT * 4;     //   fp32 [64][LDT] T = (I + L)
 constexpr int OFF_XS = OFF_TF + 64 * LDT * 4;    //   fp32 [4][16][LDX] block-product scratch
 constexpr int OFF_Q32 = OFF_XS + 4 * 16 * LDX * 4; //   fp32 [64][LDT] lower(Qp) before its bf16 tile
 constexpr int OFF_W = OFF_A;                     //   W bf16 (K-major, 64 rows)
-constexpr int OFF_E = OFF_A + 16384;             //   E bf16 (MN-major, MN = v, K = j)
 constexpr int OFF_TB = OFF_A + 65536;            // T diag(beta) bf16 (K-major 64 x 64)
 constexpr int OFF_AQB = OFF_TB + 8192;           // lower(Qp) bf16 (K-major 64 x 64)
-constexpr int OFF_KD = OFF_AQB + 8192;           // K e^{Gamma_last - Gamma} (MN-major, MN = c)
-constexpr int OFF_S = OFF_KD + 16384;            // S^T bf16 (MN-major, MN = v, K = c)
+constexpr int OFF_KD = OFF_AQB + 8192;           // 2 x K e^{Gamma_last - Gamma} (by chunk parity)
+constexpr int OFF_E = OFF_KD + 2 * 16384;        // E bf16 (MN-major, MN = v, K = j)
+constexpr int OFF_S = OFF_E + 8192;              // S^T bf16 (MN-major, MN = v, K = c)
 constexpr int OFF_SMALL = OFF_S + 16384;
 constexpr int OFF_TOT4 = OFF_SMALL;              // fp32 [16][128] row-group sums of g (log2), then prefixes
 constexpr int OFF_GREF = OFF_TOT4 + 8192;        // fp32 [4][128] Gamma (log2) at each reference row
 constexpr int OFF_GLAST = OFF_GREF + 2048;       // fp32 [128] Gamma (log2) at the chunk's last row
 constexpr int OFF_RED = OFF_GLAST + 512;         // fp32 [4] per-warp max |Gamma_last| (log2)
 constexpr int OFF_BETA = OFF_RED + 16;           // fp32 [64]
-constexpr int OFF_DECAY = OFF_BETA + 256;        // fp32 [128] e^{Gamma_last}
-constexpr int OFF_BAR = OFF_DECAY + 512;         // mbarriers + tmem base + flags
+constexpr int OFF_DECAY = OFF_BETA + 256;        // fp32 [2][128] e^{Gamma_last} (by chunk parity)
+constexpr int OFF_BAR = OFF_DECAY + 1024;        // mbarriers + tmem base + flags
 constexpr int SMEM_USED = OFF_BAR + 64;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;     // + alignment slack
+static_assert(SMEM_BYTES <= 232448, "shared memory over the sm_100 per-block limit");
 static_assert(OFF_Q32 + 64 * LDT * 4 <= OFF_A + 65536, "phase-3 scratch overflows region A");
 constexpr uint32_t TMEM_COLS = 512;
 
@@ -201,9 +202,10 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
     float* beta_s = reinterpret_cast<float*>(sm + OFF_BETA);
     float* decay_s = reinterpret_cast<float*>(sm + OFF_DECAY);
     uint64_t* full_bar = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
-    uint64_t* mma_bar = full_bar + 1;
-    uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(full_bar + 2);
-    int* abort_s = reinterpret_cast<int*>(full_bar + 3);
+    uint64_t* ut_bar = full_bar + 1;   // commits of the state-independent MMAs (Gram, W/U)
+    uint64_t* st_bar = full_bar + 2;   // commits of the state MMAs (E/O1, O2/dS)
+    uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(full_bar + 3);
+    int* abort_s = reinterpret_cast<int*>(full_bar + 4);
     const uint32_t sbase = smem_u32(sm);
 
     long long bos, eos;
@@ -212,7 +214,8 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
 
     if (tid == 0) {
         mbar_init(full_bar, 1);
-        mbar_init(mma_bar, 1);
+        mbar_init(ut_bar, 1);
+        mbar_init(st_bar, 1);
         *abort_s = 0;
         fence_mbar_init();
     }
@@ -251,8 +254,8 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
         if (GATE == KDA_GATE_CHANNEL) tma_load_3d(sm + OFF_RG, &p.map_g, full_bar, 0, h, (int)c0);
     };
 
-    uint32_t full_phase = 0, mma_phase = 0;
-    bool tma_pending = false, mma_pending = false;
+    uint32_t full_phase = 0, ut_phase = 0, st_phase = 0;
+    bool tma_pending = false, ut_pending = false, st_pending = false;
     // Uniform bounded wait: every thread waits; any expiry aborts the CTA.
     // The phase flips only on success, so after an abort `phase` still names the
     // phase the cleanup has to wait for.
@@ -270,9 +273,34 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
 
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out);
 
+    // Outputs and state update of a chunk whose O2 / dS MMAs have completed:
+    // O rows go to HBM, S^T <- Diag(e^{Gamma_last}) S^T + dS^T (fp32 registers) and
+    // its bf16 copy becomes the next chunk's MMA operand.
+    auto finish_chunk = [&](long long cp, int Lp, const float* dec_buf) {
+        const int i = 16 * sp + lane - 16;   // O rows live in lanes 16-31
+        float v[32];
+        tmem_ld32(tm + lane_base + TM_O + 32 * vhalf, v);
+        if (lane >= 16 && i < Lp) {
+            __nv_bfloat16* op = out + ((size_t)(cp + i) * H + h) * DV + vt * BV + 32 * vhalf;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) reinterpret_cast<uint4*>(op)[q] = pack8(v + 8 * q);
+        }
+        float ds[32];
+        tmem_ld32(tm + lane_base + TM_DS + 32 * vhalf, ds);
+        const float dec = dec_buf[c_own];
+#pragma unroll
+        for (int jv = 0; jv < 32; ++jv) S[jv] = fmaf(S[jv], dec, ds[jv]);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            st_shared_v4(sm + OFF_S, mnmaj_off(v0 + 8 * q, c_own, BV), pack8(S + 8 * q));
+    };
+
     bool aborted = false;
-    for (long long c0 = bos; c0 < eos; c0 += C) {
+    long long c0_prev = 0;
+    int L_prev = 0, par = 0;
+    for (long long c0 = bos; c0 < eos; c0 += C, par ^= 1) {
         const int L = (int)min((long long)C, eos - c0);
+        float* dec_cur = decay_s + par * DK;
         // ================= phase 1: log-space decay, reference factors, operands
         bool fast;   // one reference (chunk start) for the whole chunk, else 16-row sub-blocks
         const float beta_pf = (tid < L) ? a.beta[(size_t)(c0 + tid) * H + h] : 0.f;  // overlaps the wait
@@ -333,7 +361,7 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
 #pragma unroll
                 for (int q = 0; q < 16; ++q) tot4[q * DK + tid] = tv[q];
                 glast_s[tid] = acc;
-                decay_s[tid] = ex2(acc);
+                dec_cur[tid] = ex2(acc);
                 float m = -acc;
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -348,7 +376,7 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
                 float pre[8], dec[8];
                 {
                     const float4* pp = reinterpret_cast<const float4*>(tot4 + rg * DK + c8);
-                    const float4* dp = reinterpret_cast<const float4*>(decay_s + c8);
+                    const float4* dp = reinterpret_cast<const float4*>(dec_cur + c8);
                     const float4 p0 = pp[0], p1 = pp[1], d0 = dp[0], d1 = dp[1];
                     pre[0] = p0.x; pre[1] = p0.y; pre[2] = p0.z; pre[3] = p0.w;
                     pre[4] = p1.x; pre[5] = p1.y; pre[6] = p1.z; pre[7] = p1.w;
@@ -374,7 +402,7 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
                     st_shared_v4(sm + OFF_KQG, omn, pack8(t1));
                     st_shared_v4(sm + OFF_KQG, omn + 16384, pack8(t2));
                     st_shared_v4(sm + OFF_KYG, omn, pack8(t3));
-                    st_shared_v4(sm + OFF_KD, omn, pack8(t4));
+                    st_shared_v4(sm + OFF_KD + par * 16384, omn, pack8(t4));
                 }
             } else {
                 const int b = rg >> 2;
@@ -458,7 +486,7 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
                     st_shared_v4(sm + OFF_KQG, omn + 16384, pack8(t2));
     #pragma unroll
                     for (int e = 0; e < 8; ++e) t[e] = kf[e] * (Lr[e] * y[e]);
-                    st_shared_v4(sm + OFF_KD, omn, pack8(t));
+                    st_shared_v4(sm + OFF_KD + par * 16384, omn, pack8(t));
                 }
             }
         }
@@ -487,9 +515,20 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
                                  kmaj_desc(ox + g * 8192, 128, s8), idesc_bf16(128, 64, false, false),
                                  s8 > 0);
             }
-            mma_commit(mma_bar);
+            mma_commit(ut_bar);
         }
-        if (!wait_bar(mma_bar, mma_phase)) { aborted = true; mma_pending = true; break; }
+        ut_pending = true;
+        // while the Gram MMAs run: finish the previous chunk (its O2 / dS MMAs)
+        if (st_pending) {
+            if (!wait_bar(st_bar, st_phase)) { aborted = true; break; }
+            st_pending = false;
+            tc_fence_after();
+            finish_chunk(c0_prev, L_prev, decay_s + (par ^ 1) * DK);
+            fence_async_smem();
+            tc_fence_before();
+        }
+        if (!wait_bar(ut_bar, ut_phase)) { aborted = true; break; }
+        ut_pending = false;
         tc_fence_after();
         // ================= phase 3: coupling matrix L, lower(Qp), T = (I + L)^{-1}
         float* Lm = reinterpret_cast<float*>(sm + OFF_L);
@@ -565,44 +604,45 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
             }
         }
         __syncthreads();
-        // off-diagonal blocks by level: T_IJ = -T_II sum_{K=J}^{I-1} L_IK T_KJ (warp J at level I-J)
-#pragma unroll 1
-        for (int d = 1; d < 4; ++d) {
-            if (warp < 4 - d) {
-                const int J = warp, I = J + d;
+        if (warp < 4) {
+            // column block J walks down: T_IJ = -T_II sum_{K=J}^{I-1} L_IK T_KJ, all in this warp
+            const int J = warp;
+            float* Xs = reinterpret_cast<float*>(sm + OFF_XS) + warp * 16 * LDX;
+            for (int I = J + 1; I < 4; ++I) {
                 float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
                 for (int K = J; K < I; ++K)
                     blk_mma(acc, Lm + 16 * I * LDT + 16 * K, LDT, TF + 16 * K * LDT + 16 * J, LDT, lane);
-                float* Xs = reinterpret_cast<float*>(sm + OFF_XS) + warp * 16 * LDX;
                 blk_store(Xs, LDX, acc, lane, 1.f);
                 __syncwarp();
                 float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
                 blk_mma(acc2, TF + 16 * I * LDT + 16 * I, LDT, Xs, LDX, lane);
                 blk_store(TF + 16 * I * LDT + 16 * J, LDT, acc2, lane, -1.f);
+                __syncwarp();
             }
-            __syncthreads();
-        }
-        // lower(Qp) and T diag(beta) -> bf16 operands (K-major, rows i, K = j), 8 columns per step
-        for (int e = tid; !fast && e < C * 8; e += NT) {
-            const int i = e >> 3, j0 = 8 * (e & 7);
-            const float* Q32 = reinterpret_cast<const float*>(sm + OFF_Q32);
-            const float4 a0 = *reinterpret_cast<const float4*>(Q32 + i * LDT + j0);
-            const float4 a1 = *reinterpret_cast<const float4*>(Q32 + i * LDT + j0 + 4);
-            const float t8[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-            st_shared_v4(sm + OFF_AQB, kmaj_off(i, j0, 64), pack8(t8));
-        }
-        for (int e = tid; e < C * 8; e += NT) {
-            const int i = e >> 3, j0 = 8 * (e & 7);
-            const float4 a0 = *reinterpret_cast<const float4*>(TF + i * LDT + j0);
-            const float4 a1 = *reinterpret_cast<const float4*>(TF + i * LDT + j0 + 4);
-            const float tv[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-            const float4 b0 = *reinterpret_cast<const float4*>(beta_s + j0);
-            const float4 b1 = *reinterpret_cast<const float4*>(beta_s + j0 + 4);
-            const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-            float t8[8];
+            // T diag(beta), column block J -> bf16 operand (K-major, rows i, K = j)
+            for (int e = lane; e < 128; e += 32) {
+                const int i = e >> 1, j0 = 16 * J + 8 * (e & 1);
+                const float4 a0 = *reinterpret_cast<const float4*>(TF + i * LDT + j0);
+                const float4 a1 = *reinterpret_cast<const float4*>(TF + i * LDT + j0 + 4);
+                const float4 b0 = *reinterpret_cast<const float4*>(beta_s + j0);
+                const float4 b1 = *reinterpret_cast<const float4*>(beta_s + j0 + 4);
+                const float tv[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+                const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+                float t8[8];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) t8[k] = (j0 + k <= i) ? tv[k] * bv[k] : 0.f;
-            st_shared_v4(sm + OFF_TB, kmaj_off(i, j0, 64), pack8(t8));
+                for (int k = 0; k < 8; ++k) t8[k] = (j0 + k <= i) ? tv[k] * bv[k] : 0.f;
+                st_shared_v4(sm + OFF_TB, kmaj_off(i, j0, 64), pack8(t8));
+            }
+        } else if (!fast) {
+            // sub-block path: lower(Qp) -> bf16 operand
+            for (int e = tid - 128; e < C * 8; e += 128) {
+                const int i = e >> 3, j0 = 8 * (e & 7);
+                const float* Q32 = reinterpret_cast<const float*>(sm + OFF_Q32);
+                const float4 a0 = *reinterpret_cast<const float4*>(Q32 + i * LDT + j0);
+                const float4 a1 = *reinterpret_cast<const float4*>(Q32 + i * LDT + j0 + 4);
+                const float t8[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+                st_shared_v4(sm + OFF_AQB, kmaj_off(i, j0, 64), pack8(t8));
+            }
         }
         fence_async_smem();
         tc_fence_before();
@@ -619,9 +659,11 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
             for (int s = 0; s < 4; ++s)
                 mma_bf16(tm + TM_UE, kmaj_desc(tb, 64, s), mnmaj_desc(sbase + OFF_RV, 64, s),
                          idesc_bf16(64, 64, false, true), s > 0);
-            mma_commit(mma_bar);
+            mma_commit(ut_bar);
         }
-        if (!wait_bar(mma_bar, mma_phase)) { aborted = true; mma_pending = true; break; }
+        ut_pending = true;
+        if (!wait_bar(ut_bar, ut_phase)) { aborted = true; break; }
+        ut_pending = false;
         tc_fence_after();
         // ================= phase 5: W -> bf16 (K-major, 64 rows, K = c)
         {
@@ -652,9 +694,11 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
                 mma_bf16(tm + LANE16 + TM_O, rowview_desc(sbase + OFF_KQG + 16384, s), mnmaj_desc(s_op, BV, s),
                          idesc_bf16(64, BV, false, true), s > 0);
             }
-            mma_commit(mma_bar);
+            mma_commit(st_bar);
         }
-        if (!wait_bar(mma_bar, mma_phase)) { aborted = true; mma_pending = true; break; }
+        st_pending = true;
+        if (!wait_bar(st_bar, st_phase)) { aborted = true; break; }
+        st_pending = false;
         tc_fence_after();
         // the raw buffers are free again: fetch the next chunk
         if (tid == 0 && c0 + C < eos) issue_tma(c0 + C);
@@ -675,50 +719,38 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
         __syncthreads();
         tc_fence_after();
         // ================= phase 8: O += lower(Qp) E ; dS^T = (K e^{G_last - G})^T E
+        // (issued without waiting: the next chunk's prep runs while they execute)
         if (tid == 0) {
             const uint32_t e_op = sbase + OFF_E;
 #pragma unroll
-            for (int s = 0; s < 4; ++s)
+            for (int s = 0; s < 4; ++s) {
                 mma_bf16(tm + LANE16 + TM_O, kmaj_desc(sbase + OFF_AQB, 64, s), mnmaj_desc(e_op, BV, s),
                          idesc_bf16(64, BV, false, true), 1);
-#pragma unroll
-            for (int s = 0; s < 4; ++s)
-                mma_bf16(tm + TM_DS, mnmaj_desc(sbase + OFF_KD, 128, s), mnmaj_desc(e_op, BV, s),
-                         idesc_bf16(128, BV, true, true), s > 0);
-            mma_commit(mma_bar);
-        }
-        if (!wait_bar(mma_bar, mma_phase)) { aborted = true; mma_pending = true; break; }
-        tc_fence_after();
-        // ================= phase 9: outputs and the state update
-        {
-            const int i = 16 * sp + lane - 16;   // valid for lane >= 16
-            float v[32];
-            tmem_ld32(tm + lane_base + TM_O + 32 * vhalf, v);
-            if (lane >= 16 && i < L) {
-                __nv_bfloat16* op = out + ((size_t)(c0 + i) * H + h) * DV + vt * BV + 32 * vhalf;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) reinterpret_cast<uint4*>(op)[q] = pack8(v + 8 * q);
+                mma_bf16(tm + TM_DS, mnmaj_desc(sbase + OFF_KD + par * 16384, 128, s),
+                         mnmaj_desc(e_op, BV, s), idesc_bf16(128, BV, true, true), s > 0);
             }
-            float ds[32];
-            tmem_ld32(tm + lane_base + TM_DS + 32 * vhalf, ds);
-            const float dec = decay_s[c_own];
-#pragma unroll
-            for (int jv = 0; jv < 32; ++jv) S[jv] = fmaf(S[jv], dec, ds[jv]);
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                st_shared_v4(sm + OFF_S, mnmaj_off(v0 + 8 * q, c_own, BV), pack8(S + 8 * q));
+            mma_commit(st_bar);
         }
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
+        st_pending = true;
+        c0_prev = c0;
+        L_prev = L;
+    }
+    if (!aborted && st_pending) {
+        if (!wait_bar(st_bar, st_phase)) {
+            aborted = true;
+        } else {
+            st_pending = false;
+            tc_fence_after();
+            finish_chunk(c0_prev, L_prev, decay_s + (par ^ 1) * DK);
+        }
     }
 
     if (aborted) {
         if (a.dev_status && tid == 0) atomicOr(a.dev_status, KDA_DEV_TIMEOUT);
         // let copies / MMAs still in flight land before the memory goes away
         if (tma_pending) (void)mbar_wait(full_bar, full_phase, kWaitNs);
-        if (mma_pending) (void)mbar_wait(mma_bar, mma_phase, kWaitNs);
+        if (ut_pending) (void)mbar_wait(ut_bar, ut_phase, kWaitNs);
+        if (st_pending) (void)mbar_wait(st_bar, st_phase, kWaitNs);
     } else if (a.S_T) {
         const size_t sbase_g = ((size_t)n * H + h) * DV * DK;
 #pragma unroll
