@@ -44,6 +44,11 @@ using namespace sm100;
 
 constexpr int C = 64, DK = 128, DV = 128, BV = 64, NVT = DV / BV, NT = 256;
 constexpr uint64_t kWaitNs = 1000000000ull;  // 1 s bound on every wait
+// Issuing a tcgen05.mma holds the issuing thread while the tensor pipe takes it, so
+// each batch is issued by a lane of a warp with no SIMT work in the phase that follows.
+constexpr int kGramTid = 128;   // warp 4: only the dS / S update in finish_chunk
+constexpr int kIssA = 192;      // warp 6: [-K e^G S^T ; O1], then O2
+constexpr int kIssB = 224;      // warp 7: E, the next chunk's TMA, then dS
 
 // Shared-memory map (bytes from a 1024-aligned base).
 constexpr int OFF_RAW = 0;                       // raw K | raw Q | raw G  (64 KB)
@@ -61,39 +66,37 @@ constexpr int OFF_RV = 65536;                    // raw V tile, TMA 128B swizzle
 constexpr int OFF_A = 73728;                     // 64 KB, reused per phase:
 constexpr int OFF_OY = OFF_A;                    //   Gram A operands: 2 K-major tiles of 128 rows
                                                  //   (tile g: rows 0-63 version 2g, 64-127 version 2g+1)
+constexpr int OFF_TOT4 = OFF_A;                  //   decay scan (prep, before any operand write here):
+constexpr int OFF_GREF = OFF_TOT4 + 8192;        //     fp32 [16][128] row-group sums then prefixes,
+constexpr int OFF_GLAST = OFF_GREF + 2048;       //     [4][128] Gamma at reference rows, [128] at the
+constexpr int OFF_RED = OFF_GLAST + 512;         //     last row, [4] per-warp max |Gamma_last| (log2)
 constexpr int LDT = 68;                          //   fp32 row stride of L and T (bank spread)
-constexpr int LDX = 24;                          //   fp32 row stride of the per-warp block scratch
+constexpr int LDX = 20;                          //   fp32 row stride of 16x16 block scratch
 constexpr int OFF_L = OFF_A;                     //   fp32 [64][LDT] coupling matrix L
-constexpr int OFF_TF = OFF_A + 64 * LDT * 4;     //   fp32 [64][LDT] T = (I + L)^{-1}
-constexpr int OFF_XS = OFF_TF + 64 * LDT * 4;    //   fp32 [4][16][LDX] block-product scratch
-constexpr int OFF_Q32 = OFF_XS + 4 * 16 * LDX * 4; //   fp32 [64][LDT] lower(Qp) before its bf16 tile
-constexpr int OFF_W = OFF_A;                     //   W bf16 (K-major, 64 rows)
-constexpr int OFF_TB = OFF_A + 65536;            // T diag(beta) bf16 (K-major 64 x 64)
-constexpr int OFF_AQB = OFF_TB + 8192;           // lower(Qp) bf16 (K-major 64 x 64)
-constexpr int OFF_KD = OFF_AQB + 8192;           // 2 x K e^{Gamma_last - Gamma} (by chunk parity)
+constexpr int OFF_TF = OFF_L + 64 * LDT * 4;     //   fp32 [64][LDT] T = (I + L)^{-1}
+constexpr int OFF_Q32 = OFF_TF + 64 * LDT * 4;   //   fp32 [64][LDT] lower(Qp), sub-block path
+constexpr int OFF_NS = OFF_Q32 + 64 * LDT * 4;   //   fp32 [10][16][LDX] Neumann-series blocks
+constexpr int OFF_TB = OFF_A + 65536;            // K-major, K = 64, 192 rows: T diag(beta) (rows 0-63),
+constexpr int OFF_AQB = OFF_TB + 16384;          //   zeros (64-127), lower(Qp) (128-191)
+constexpr int OFF_KD = OFF_TB + 24576;           // 2 x K e^{Gamma_last - Gamma} (by chunk parity)
 constexpr int OFF_E = OFF_KD + 2 * 16384;        // E bf16 (MN-major, MN = v, K = j)
 constexpr int OFF_S = OFF_E + 8192;              // S^T bf16 (MN-major, MN = v, K = c)
 constexpr int OFF_SMALL = OFF_S + 16384;
-constexpr int OFF_TOT4 = OFF_SMALL;              // fp32 [16][128] row-group sums of g (log2), then prefixes
-constexpr int OFF_GREF = OFF_TOT4 + 8192;        // fp32 [4][128] Gamma (log2) at each reference row
-constexpr int OFF_GLAST = OFF_GREF + 2048;       // fp32 [128] Gamma (log2) at the chunk's last row
-constexpr int OFF_RED = OFF_GLAST + 512;         // fp32 [4] per-warp max |Gamma_last| (log2)
-constexpr int OFF_BETA = OFF_RED + 16;           // fp32 [64]
+constexpr int OFF_BETA = OFF_SMALL;              // fp32 [64]
 constexpr int OFF_DECAY = OFF_BETA + 256;        // fp32 [2][128] e^{Gamma_last} (by chunk parity)
 constexpr int OFF_BAR = OFF_DECAY + 1024;        // mbarriers + tmem base + flags
 constexpr int SMEM_USED = OFF_BAR + 64;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;     // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory over the sm_100 per-block limit");
-static_assert(OFF_Q32 + 64 * LDT * 4 <= OFF_A + 65536, "phase-3 scratch overflows region A");
+static_assert(OFF_NS + 10 * 16 * LDX * 4 <= OFF_A + 65536, "phase-3 scratch overflows region A");
+static_assert(OFF_RED + 16 <= OFF_A + 65536, "scan scratch overflows region A");
 constexpr uint32_t TMEM_COLS = 512;
 
-// TMEM columns (lane base 0 or 16 for M = 64 accumulators).
-constexpr uint32_t TM_GRAM = 0;     // all lanes  : group g at cols 64 g: [version rows j][X rows]
-constexpr uint32_t TM_UE = 128;     // lanes 0-15 : U, then E = U - W S^T  [j][v]
-constexpr uint32_t TM_O = 128;      // lanes 16-31: O   [i][v]
+// TMEM columns.
+constexpr uint32_t TM_GRAM = 0;     // all lanes  : Gram groups (cols 0-63 or 0-127)
+constexpr uint32_t TM_UE = 128;     // all lanes  : rows 0-63 -K e^G S^T, rows 64-127 O
 constexpr uint32_t TM_DS = 192;     // all lanes  : dS^T [c][v]
-constexpr uint32_t TM_W = 256;      // lanes 0-15 : W   [i][c]   (128 cols)
-constexpr uint32_t LANE16 = 16u << 16;
+constexpr uint32_t TM_E = 256;      // all lanes  : rows 0-63 E = T diag(beta) (V - K e^G S^T)
 
 struct TcParams {
     CUtensorMap map_k, map_q, map_v, map_g;
@@ -157,6 +160,35 @@ __device__ __forceinline__ uint64_t rowview_desc(uint32_t base, int s) {
     return desc_sw128(base + (uint32_t)((s >> 2) * 1024 + (s & 3) * 32), 16, 2048);
 }
 
+// As blk_mma with A = s0 A0 + s1 A1 (+ s2 A2 when A2 is not null), all stride lda.
+__device__ __forceinline__ void blk_mma2(float (&acc)[2][4], const float* A0, float s0,
+                                         const float* A1, float s1, const float* A2, float s2,
+                                         int lda, const float* B, int ldb, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    auto av = [&](int off) {
+        float x = s0 * A0[off] + s1 * A1[off];
+        if (A2) x += s2 * A2[off];
+        return to_tf32(x);
+    };
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+        const uint32_t a0 = av(g * lda + 8 * ks + t);
+        const uint32_t a1 = av((g + 8) * lda + 8 * ks + t);
+        const uint32_t a2 = av(g * lda + 8 * ks + t + 4);
+        const uint32_t a3 = av((g + 8) * lda + 8 * ks + t + 4);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            const uint32_t b0 = to_tf32(B[(8 * ks + t) * ldb + 8 * nt + g]);
+            const uint32_t b1 = to_tf32(B[(8 * ks + t + 4) * ldb + 8 * nt + g]);
+            asm volatile(
+                "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, "
+                "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};\n"
+                : "+f"(acc[nt][0]), "+f"(acc[nt][1]), "+f"(acc[nt][2]), "+f"(acc[nt][3])
+                : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+        }
+    }
+}
+
 // Store a 16x16 C-fragment pair, scaled by s, to shared memory (row stride ld).
 __device__ __forceinline__ void blk_store(float* Cm, int ld, const float (&acc)[2][4], int lane,
                                           float s) {
@@ -204,8 +236,9 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
     uint64_t* full_bar = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
     uint64_t* ut_bar = full_bar + 1;   // commits of the state-independent MMAs (Gram, W/U)
     uint64_t* st_bar = full_bar + 2;   // commits of the state MMAs (E/O1, O2/dS)
-    uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(full_bar + 3);
-    int* abort_s = reinterpret_cast<int*>(full_bar + 4);
+    uint64_t* v_bar = full_bar + 3;    // the V tile (waited only by the warps that read it)
+    uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(full_bar + 4);
+    int* abort_s = reinterpret_cast<int*>(full_bar + 5);
     const uint32_t sbase = smem_u32(sm);
 
     long long bos, eos;
@@ -215,7 +248,8 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
     if (tid == 0) {
         mbar_init(full_bar, 1);
         mbar_init(ut_bar, 1);
-        mbar_init(st_bar, 1);
+        mbar_init(st_bar, 2);   // each state-MMA phase: two arrivals (kIssA, kIssB)
+        mbar_init(v_bar, 1);
         *abort_s = 0;
         fence_mbar_init();
     }
@@ -239,23 +273,35 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
         for (int q = 0; q < 4; ++q)
             st_shared_v4(sm + OFF_S, mnmaj_off(v0 + 8 * q, c_own, BV), pack8(S + 8 * q));
     }
+    // the zero rows 64-127 of the T diag(beta) | 0 | lower(Qp) tile never change
+    for (int e = tid; e < 512; e += NT)
+        st_shared_v4(sm + OFF_TB + 8192, (uint32_t)(16 * e), make_uint4(0u, 0u, 0u, 0u));
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tm = *tmem_base_s;
 
-    const uint32_t raw_bytes = 16384 * 2 + 8192 + (GATE == KDA_GATE_CHANNEL ? 32768 : 0);
-    auto issue_tma = [&](long long c0) {
-        mbar_arrive_expect_tx(full_bar, raw_bytes);
-        tma_load_3d(sm + OFF_RK, &p.map_k, full_bar, 0, h, (int)c0);
-        tma_load_3d(sm + OFF_RQ, &p.map_q, full_bar, 0, h, (int)c0);
-        tma_load_3d(sm + OFF_RV, &p.map_v, full_bar, vt * BV, h, (int)c0);
-        if (GATE == KDA_GATE_CHANNEL) tma_load_3d(sm + OFF_RG, &p.map_g, full_bar, 0, h, (int)c0);
+    // K, Q, g of a chunk complete on full_bar, V on v_bar.  Inside the chunk loop the
+    // next chunk's tiles go out as soon as their buffers free: K and Q after the Gram
+    // MMAs, g after the K|Q S^T MMAs, V after the E MMAs.
+    auto issue_kq = [&](long long c1) {
+        if (GATE == KDA_GATE_CHANNEL) mbar_expect_tx(full_bar, 32768u);   // g arrives later
+        else mbar_arrive_expect_tx(full_bar, 32768u);
+        tma_load_3d(sm + OFF_RK, &p.map_k, full_bar, 0, h, (int)c1);
+        tma_load_3d(sm + OFF_RQ, &p.map_q, full_bar, 0, h, (int)c1);
     };
-
-    uint32_t full_phase = 0, ut_phase = 0, st_phase = 0;
-    bool tma_pending = false, ut_pending = false, st_pending = false;
+    auto issue_g = [&](long long c1) {
+        mbar_arrive_expect_tx(full_bar, 32768u);
+        tma_load_3d(sm + OFF_RG, &p.map_g, full_bar, 0, h, (int)c1);
+    };
+    auto issue_v = [&](long long c1) {
+        mbar_arrive_expect_tx(v_bar, 8192u);
+        tma_load_3d(sm + OFF_RV, &p.map_v, v_bar, vt * BV, h, (int)c1);
+    };
+    uint32_t full_phase = 0, ut_phase = 0, st_phase = 0, v_phase = 0;
+    bool tma_pending = false, ut_pending = false, st_pending = false, v_pending = false;
+    bool g_issued = true;   // the pending full_bar phase already has its arrival
     // Uniform bounded wait: every thread waits; any expiry aborts the CTA.
     // The phase flips only on success, so after an abort `phase` still names the
     // phase the cleanup has to wait for.
@@ -268,8 +314,12 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
         return true;
     };
 
-    if (tid == 0 && bos < eos) issue_tma(bos);
-    tma_pending = bos < eos;
+    if (tid == 0 && bos < eos) {
+        issue_kq(bos);
+        if (GATE == KDA_GATE_CHANNEL) issue_g(bos);
+        issue_v(bos);
+    }
+    tma_pending = v_pending = bos < eos;
 
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out);
 
@@ -277,10 +327,10 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
     // O rows go to HBM, S^T <- Diag(e^{Gamma_last}) S^T + dS^T (fp32 registers) and
     // its bf16 copy becomes the next chunk's MMA operand.
     auto finish_chunk = [&](long long cp, int Lp, const float* dec_buf) {
-        const int i = 16 * sp + lane - 16;   // O rows live in lanes 16-31
+        const int i = 32 * (sp - 2) + lane;   // O rows live in lanes 64-127
         float v[32];
-        tmem_ld32(tm + lane_base + TM_O + 32 * vhalf, v);
-        if (lane >= 16 && i < Lp) {
+        if (sp >= 2) tmem_ld32(tm + lane_base + TM_UE + 32 * vhalf, v);
+        if (sp >= 2 && i < Lp) {
             __nv_bfloat16* op = out + ((size_t)(cp + i) * H + h) * DV + vt * BV + 32 * vhalf;
 #pragma unroll
             for (int q = 0; q < 4; ++q) reinterpret_cast<uint4*>(op)[q] = pack8(v + 8 * q);
@@ -395,7 +445,7 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
                         const float gm = pre[e] + g2[r][e];   // Gamma_i (log2), <= 0
                         const float eg = ex2(gm), ey = ex2(-gm);
                         t1[e] = kf[e] * eg;                    // K e^{Gamma}
-                        t2[e] = (qf[e] * a.scale) * eg;        // Q~ e^{Gamma}
+                        t2[e] = -(qf[e] * a.scale) * eg;       // -Q~ e^{Gamma} (see phase 6)
                         t3[e] = kf[e] * ey;                    // K e^{-Gamma}
                         t4[e] = kf[e] * (dec[e] * ey);         // K e^{Gamma_last - Gamma}
                     }
@@ -433,6 +483,7 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
                         }
                     }
                 }
+                __syncthreads();   // the scan scratch shares region A with the j-side operands
                 // swizzled byte offsets of this thread's 16-byte chunks (row i = 4 rg + r)
                 const uint32_t sw0 = (uint32_t)(cq & 7);
                     // the same rows inside a 128-row tile (Gram A operands): K-atom stride 16 KB
@@ -480,7 +531,7 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
                     for (int e = 0; e < 8; ++e) {
                         const float eg = Er[e] * x[e];
                         t[e] = kf[e] * eg;
-                        t2[e] = qf[e] * eg;
+                        t2[e] = -qf[e] * eg;
                     }
                     st_shared_v4(sm + OFF_KQG, omn, pack8(t));
                     st_shared_v4(sm + OFF_KQG, omn + 16384, pack8(t2));
@@ -498,7 +549,7 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
         // the j-side operand of sub-block 2g, rows 64-127 that of sub-block 2g+1; B rows
         // are the i-side rows of sub-blocks 2g and 2g+1 (K then Q~ for each).
         // One-reference path: a single group, D[n][j] = [K e^G ; Q~ e^G]_n . (K e^-G)_j.
-        if (tid == 0) {
+        if (tid == kGramTid) {
             if (fast) {
 #pragma unroll
                 for (int s8 = 0; s8 < 8; ++s8)
@@ -530,35 +581,58 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
         if (!wait_bar(ut_bar, ut_phase)) { aborted = true; break; }
         ut_pending = false;
         tc_fence_after();
+        // S is current: [-K e^G S^T ; Q~ e^G S^T] with A = [K e^G ; -Q~ e^G] negated (M = 128).
+        // It needs no T, so it runs while the coupling matrix is read out and inverted.
+        if (tid == kIssA) {
+            const uint32_t s_op = sbase + OFF_S;
+#pragma unroll
+            for (int s = 0; s < 8; ++s)
+                mma_bf16(tm + TM_UE, rowview_desc(sbase + OFF_KQG, s), mnmaj_desc(s_op, BV, s),
+                         idesc_bf16(128, BV, false, true, true), s > 0);
+            mma_commit(st_bar);
+        } else if (tid == kIssB) {
+            mbar_arrive(st_bar);
+        }
+        st_pending = true;
+        const bool more = c0 + C < eos;
+        if (tid == 32 && more) issue_kq(c0 + C);   // K|e^-G operand rows are consumed
+        tma_pending = more;
+        g_issued = !(more && GATE == KDA_GATE_CHANNEL);
         // ================= phase 3: coupling matrix L, lower(Qp), T = (I + L)^{-1}
         float* Lm = reinterpret_cast<float*>(sm + OFF_L);
         float* TF = reinterpret_cast<float*>(sm + OFF_TF);
         if (fast) {
-            // lane n = 32 sp + lane: rows i of P (n < 64) or of Qp (n >= 64); warp group
-            // vhalf reads columns j = 32 vhalf .. 32 vhalf + 31
-            const int n = 32 * sp + lane, j0 = 32 * vhalf;
-            float v[32];
-            tmem_ld32(tm + lane_base + TM_GRAM + j0, v);
-            if (n < 64) {
-                const int i = n;
-                const float bi = beta_s[i];
+            // lane n = 32 sp + lane: rows i of P (n < 64) or of Qp (n >= 64); warps 4-7
+            // read all 64 columns j (warp 0 may still be issuing MMAs)
+            if (vhalf == 1) {
+                const int n = 32 * sp + lane;
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    float4 o;
-                    o.x = (j0 + 4 * q + 0 < i) ? bi * v[4 * q + 0] : 0.f;
-                    o.y = (j0 + 4 * q + 1 < i) ? bi * v[4 * q + 1] : 0.f;
-                    o.z = (j0 + 4 * q + 2 < i) ? bi * v[4 * q + 2] : 0.f;
-                    o.w = (j0 + 4 * q + 3 < i) ? bi * v[4 * q + 3] : 0.f;
-                    *reinterpret_cast<float4*>(Lm + i * LDT + j0 + 4 * q) = o;
-                }
-            } else {
-                const int i = n - 64;
+                for (int hj = 0; hj < 2; ++hj) {
+                    const int j0 = 32 * hj;
+                    float v[32];
+                    tmem_ld32(tm + lane_base + TM_GRAM + j0, v);
+                    if (n < 64) {
+                        const int i = n;
+                        const float bi = beta_s[i];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    float t8[8];
+                        for (int q = 0; q < 8; ++q) {
+                            float4 o;
+                            o.x = (j0 + 4 * q + 0 < i) ? bi * v[4 * q + 0] : 0.f;
+                            o.y = (j0 + 4 * q + 1 < i) ? bi * v[4 * q + 1] : 0.f;
+                            o.z = (j0 + 4 * q + 2 < i) ? bi * v[4 * q + 2] : 0.f;
+                            o.w = (j0 + 4 * q + 3 < i) ? bi * v[4 * q + 3] : 0.f;
+                            *reinterpret_cast<float4*>(Lm + i * LDT + j0 + 4 * q) = o;
+                        }
+                    } else {
+                        const int i = n - 64;
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) t8[e] = (j0 + 8 * q + e <= i) ? v[8 * q + e] : 0.f;
-                    st_shared_v4(sm + OFF_AQB, kmaj_off(i, j0 + 8 * q, 64), pack8(t8));
+                        for (int q = 0; q < 4; ++q) {
+                            float t8[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) t8[e] = (j0 + 8 * q + e <= i) ? -v[8 * q + e] : 0.f;
+                            st_shared_v4(sm + OFF_AQB, kmaj_off(i, j0 + 8 * q, 64), pack8(t8));
+                        }
+                    }
                 }
             }
         } else {
@@ -593,47 +667,44 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
             float t[16];
 #pragma unroll
             for (int r = 0; r < 16; ++r) {
-                float acc = 0.f;
+                float a4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int k = 0; k < r; ++k) acc = fmaf(Lm[(16 * I + r) * LDT + 16 * I + k], t[k], acc);
+                for (int k = 0; k < r; ++k)
+                    a4[k & 3] = fmaf(Lm[(16 * I + r) * LDT + 16 * I + k], t[k], a4[k & 3]);
+                const float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
                 t[r] = (r < cc) ? 0.f : ((r == cc) ? 1.f : -acc);
             }
             if (lane < 16) {
 #pragma unroll
                 for (int r = 0; r < 16; ++r) TF[(16 * I + r) * LDT + 16 * I + cc] = t[r];
             }
-        }
-        __syncthreads();
-        if (warp < 4) {
-            // column block J walks down: T_IJ = -T_II sum_{K=J}^{I-1} L_IK T_KJ, all in this warp
-            const int J = warp;
-            float* Xs = reinterpret_cast<float*>(sm + OFF_XS) + warp * 16 * LDX;
-            for (int I = J + 1; I < 4; ++I) {
-                float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-                for (int K = J; K < I; ++K)
-                    blk_mma(acc, Lm + 16 * I * LDT + 16 * K, LDT, TF + 16 * K * LDT + 16 * J, LDT, lane);
-                blk_store(Xs, LDX, acc, lane, 1.f);
-                __syncwarp();
-                float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-                blk_mma(acc2, TF + 16 * I * LDT + 16 * I, LDT, Xs, LDX, lane);
-                blk_store(TF + 16 * I * LDT + 16 * J, LDT, acc2, lane, -1.f);
-                __syncwarp();
-            }
-            // T diag(beta), column block J -> bf16 operand (K-major, rows i, K = j)
-            for (int e = lane; e < 128; e += 32) {
-                const int i = e >> 1, j0 = 16 * J + 8 * (e & 1);
-                const float4 a0 = *reinterpret_cast<const float4*>(TF + i * LDT + j0);
-                const float4 a1 = *reinterpret_cast<const float4*>(TF + i * LDT + j0 + 4);
-                const float4 b0 = *reinterpret_cast<const float4*>(beta_s + j0);
-                const float4 b1 = *reinterpret_cast<const float4*>(beta_s + j0 + 4);
-                const float tv[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-                const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-                float t8[8];
+        } else {
+            if (sp < 2) {
+                // E' = V - K e^G S^T, rows j = lanes 0-63, written over the V tile (MN-major)
+                if (!mbar_wait(st_bar, st_phase, kWaitNs)) atomicOr(abort_s, 1);
+                if (!mbar_wait(v_bar, v_phase, kWaitNs)) atomicOr(abort_s, 1);
+                tc_fence_after();
+                // the K e^G | -Q~ e^G tile is consumed: g of the next chunk can land there
+                if (GATE == KDA_GATE_CHANNEL && tid == 128 && more) issue_g(c0 + C);
+                const int j = 32 * sp + lane;
 #pragma unroll
-                for (int k = 0; k < 8; ++k) t8[k] = (j0 + k <= i) ? tv[k] * bv[k] : 0.f;
-                st_shared_v4(sm + OFF_TB, kmaj_off(i, j0, 64), pack8(t8));
+                for (int hv = 0; hv < 2; ++hv) {
+                    float v[32];
+                    tmem_ld32(tm + lane_base + TM_UE + 32 * hv, v);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint32_t off = mnmaj_off(32 * hv + 8 * q, j, BV);
+                        float vv[8];
+                        unpack8(*reinterpret_cast<const uint4*>(sm + OFF_RV + off), vv);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) vv[e] += v[8 * q + e];
+                        st_shared_v4(sm + OFF_RV, off, pack8(vv));
+                    }
+                }
+                fence_async_smem();
             }
-        } else if (!fast) {
+        }
+        if (warp >= 4 && !fast) {
             // sub-block path: lower(Qp) -> bf16 operand
             for (int e = tid - 128; e < C * 8; e += 128) {
                 const int i = e >> 3, j0 = 8 * (e & 7);
@@ -644,75 +715,114 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
                 st_shared_v4(sm + OFF_AQB, kmaj_off(i, j0, 64), pack8(t8));
             }
         }
+        __syncthreads();
+        if (*abort_s != 0) { aborted = true; break; }
+        st_phase ^= 1u;    // the [-K e^G S^T ; O1] MMAs and the V tile were waited for above
+        st_pending = false;
+        v_phase ^= 1u;
+        v_pending = false;
+        tc_fence_before();
+        // Off-diagonal blocks by a block Neumann series.  With D = blockdiag(T_II) and
+        // N = D L_off (strictly block-lower, N^4 = 0):
+        //   T = (I + N)^{-1} D = (I - N + N^2 - N^3) D,  so  T_IJ = M_IJ T_JJ (I > J)
+        // with M = -N + N^2 - N^3.  Four levels of independent 16x16 products.
+        {
+            float* NS = reinterpret_cast<float*>(sm + OFF_NS);
+            auto nb = [&](int idx) { return NS + idx * 16 * LDX; };
+            auto tf = [&](int I, int J) { return TF + 16 * I * LDT + 16 * J; };
+            auto lb = [&](int I, int J) { return Lm + 16 * I * LDT + 16 * J; };
+            // N blocks: 0:(1,0) 1:(2,0) 2:(3,0) 3:(2,1) 4:(3,1) 5:(3,2); 6: N^2_20, 7: N^2_31,
+            // 8: N^2_30, 9: N^3_30
+            if (warp < 6) {
+                const int I = (warp < 3) ? warp + 1 : ((warp < 5) ? warp - 1 : 3);
+                const int K = (warp < 3) ? 0 : ((warp < 5) ? 1 : 2);
+                float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                blk_mma(acc, tf(I, I), LDT, lb(I, K), LDT, lane);
+                blk_store(nb(warp), LDX, acc, lane, 1.f);
+            }
+            __syncthreads();
+            if (warp < 6) {
+                float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                if (warp < 3) {   // T_{J+1,J} = -N_{J+1,J} T_JJ
+                    const int J = warp, nidx = (J == 0) ? 0 : ((J == 1) ? 3 : 5);
+                    blk_mma(acc, nb(nidx), LDX, tf(J, J), LDT, lane);
+                    blk_store(tf(J + 1, J), LDT, acc, lane, -1.f);
+                } else if (warp == 3) {   // N^2_20 = N_21 N_10
+                    blk_mma(acc, nb(3), LDX, nb(0), LDX, lane);
+                    blk_store(nb(6), LDX, acc, lane, 1.f);
+                } else if (warp == 4) {   // N^2_31 = N_32 N_21
+                    blk_mma(acc, nb(5), LDX, nb(3), LDX, lane);
+                    blk_store(nb(7), LDX, acc, lane, 1.f);
+                } else {                  // N^2_30 = N_31 N_10 + N_32 N_20
+                    blk_mma(acc, nb(4), LDX, nb(0), LDX, lane);
+                    blk_mma(acc, nb(5), LDX, nb(1), LDX, lane);
+                    blk_store(nb(8), LDX, acc, lane, 1.f);
+                }
+            }
+            __syncthreads();
+            if (warp < 3) {
+                float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                if (warp == 0) {          // T_20 = (N^2_20 - N_20) T_00
+                    blk_mma2(acc, nb(6), 1.f, nb(1), -1.f, nullptr, 0.f, LDX, tf(0, 0), LDT, lane);
+                    blk_store(tf(2, 0), LDT, acc, lane, 1.f);
+                } else if (warp == 1) {   // T_31 = (N^2_31 - N_31) T_11
+                    blk_mma2(acc, nb(7), 1.f, nb(4), -1.f, nullptr, 0.f, LDX, tf(1, 1), LDT, lane);
+                    blk_store(tf(3, 1), LDT, acc, lane, 1.f);
+                } else {                  // N^3_30 = N_32 N^2_20
+                    blk_mma(acc, nb(5), LDX, nb(6), LDX, lane);
+                    blk_store(nb(9), LDX, acc, lane, 1.f);
+                }
+            }
+            __syncthreads();
+            if (warp == 0) {              // T_30 = (N^2_30 - N_30 - N^3_30) T_00
+                float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                blk_mma2(acc, nb(8), 1.f, nb(2), -1.f, nb(9), -1.f, LDX, tf(0, 0), LDT, lane);
+                blk_store(tf(3, 0), LDT, acc, lane, 1.f);
+            }
+            __syncthreads();
+        }
+        // T diag(beta) -> bf16 operand rows 0-63 (K-major, K = j), 8 columns per step
+        for (int e = tid; e < C * 8; e += NT) {
+            const int i = e >> 3, j0 = 8 * (e & 7);
+            const float4 a0 = *reinterpret_cast<const float4*>(TF + i * LDT + j0);
+            const float4 a1 = *reinterpret_cast<const float4*>(TF + i * LDT + j0 + 4);
+            const float4 b0 = *reinterpret_cast<const float4*>(beta_s + j0);
+            const float4 b1 = *reinterpret_cast<const float4*>(beta_s + j0 + 4);
+            const float tv[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+            float t8[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) t8[k] = (j0 + k <= i) ? tv[k] * bv[k] : 0.f;
+            st_shared_v4(sm + OFF_TB, kmaj_off(i, j0, 64), pack8(t8));
+        }
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
-        // ================= phase 4: W = T_b (K e^Gamma), U = T_b V
-        if (tid == 0) {
-            const uint32_t tb = sbase + OFF_TB;
+        // ================= phase 4: [E ; 0] = [T diag(beta) ; 0] E'  (M = 128, K = 64)
+        if (tid == kIssB) {
 #pragma unroll
             for (int s = 0; s < 4; ++s)
-                mma_bf16(tm + TM_W, kmaj_desc(tb, 64, s), mnmaj_desc(sbase + OFF_KQG, 128, s),
-                         idesc_bf16(64, 128, false, true), s > 0);
-#pragma unroll
-            for (int s = 0; s < 4; ++s)
-                mma_bf16(tm + TM_UE, kmaj_desc(tb, 64, s), mnmaj_desc(sbase + OFF_RV, 64, s),
-                         idesc_bf16(64, 64, false, true), s > 0);
+                mma_bf16(tm + TM_E, kmaj_desc(sbase + OFF_TB, 128, s), mnmaj_desc(sbase + OFF_RV, 64, s),
+                         idesc_bf16(128, 64, false, true), s > 0);
             mma_commit(ut_bar);
         }
         ut_pending = true;
         if (!wait_bar(ut_bar, ut_phase)) { aborted = true; break; }
         ut_pending = false;
         tc_fence_after();
-        // ================= phase 5: W -> bf16 (K-major, 64 rows, K = c)
-        {
-            const int i = 16 * sp + lane;   // valid for lane < 16
-#pragma unroll
-            for (int m = 0; m < 2; ++m) {
-                const int col = 64 * vhalf + 32 * m;
-                float v[32];
-                tmem_ld32(tm + lane_base + TM_W + col, v);
-                if (lane < 16) {
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        st_shared_v4(sm + OFF_W, kmaj_off(i, col + 8 * q, 64), pack8(v + 8 * q));
-                }
-            }
-        }
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        // ================= phase 6: E = U - W S^T ; O = (Q~ e^Gamma) S^T
-        if (tid == 0) {
-            const uint32_t s_op = sbase + OFF_S;
-#pragma unroll
-            for (int s = 0; s < 8; ++s) {
-                mma_bf16(tm + TM_UE, kmaj_desc(sbase + OFF_W, 64, s), mnmaj_desc(s_op, BV, s),
-                         idesc_bf16(64, BV, false, true, true), 1);
-                mma_bf16(tm + LANE16 + TM_O, rowview_desc(sbase + OFF_KQG + 16384, s), mnmaj_desc(s_op, BV, s),
-                         idesc_bf16(64, BV, false, true), s > 0);
-            }
-            mma_commit(st_bar);
-        }
-        st_pending = true;
-        if (!wait_bar(st_bar, st_phase)) { aborted = true; break; }
-        st_pending = false;
-        tc_fence_after();
-        // the raw buffers are free again: fetch the next chunk
-        if (tid == 0 && c0 + C < eos) issue_tma(c0 + C);
-        tma_pending = c0 + C < eos;
-        // ================= phase 7: E -> bf16 (MN-major, MN = v, K = j)
-        {
-            const int j = 16 * sp + lane;   // valid for lane < 16
+        // E' (written over V) is consumed: the next chunk's V completes the TMA phase
+        if (tid == kIssB && more) issue_v(c0 + C);
+        v_pending = more;
+        g_issued = true;
+        // ================= phase 7: E -> bf16 (MN-major, MN = v, K = j); E rows are lanes 0-63
+        if (sp < 2) {
+            const int j = 32 * sp + lane;
             float v[32];
-            tmem_ld32(tm + lane_base + TM_UE + 32 * vhalf, v);
-            if (lane < 16) {
+            tmem_ld32(tm + lane_base + TM_E + 32 * vhalf, v);
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    st_shared_v4(sm + OFF_E, mnmaj_off(32 * vhalf + 8 * q, j, BV), pack8(v + 8 * q));
-            }
+            for (int q = 0; q < 4; ++q)
+                st_shared_v4(sm + OFF_E, mnmaj_off(32 * vhalf + 8 * q, j, BV), pack8(v + 8 * q));
         }
         fence_async_smem();
         tc_fence_before();
@@ -720,15 +830,19 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
         tc_fence_after();
         // ================= phase 8: O += lower(Qp) E ; dS^T = (K e^{G_last - G})^T E
         // (issued without waiting: the next chunk's prep runs while they execute)
-        if (tid == 0) {
+        if (tid == kIssA) {
             const uint32_t e_op = sbase + OFF_E;
 #pragma unroll
-            for (int s = 0; s < 4; ++s) {
-                mma_bf16(tm + LANE16 + TM_O, kmaj_desc(sbase + OFF_AQB, 64, s), mnmaj_desc(e_op, BV, s),
-                         idesc_bf16(64, BV, false, true), 1);
+            for (int s = 0; s < 4; ++s)   // rows 64-127: O += lower(Qp) E; rows 0-63 add zero
+                mma_bf16(tm + TM_UE, kmaj_desc(sbase + OFF_TB + 8192, 128, s), mnmaj_desc(e_op, BV, s),
+                         idesc_bf16(128, BV, false, true), 1);
+            mma_commit(st_bar);
+        } else if (tid == kIssB) {
+            const uint32_t e_op = sbase + OFF_E;
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
                 mma_bf16(tm + TM_DS, mnmaj_desc(sbase + OFF_KD + par * 16384, 128, s),
                          mnmaj_desc(e_op, BV, s), idesc_bf16(128, BV, true, true), s > 0);
-            }
             mma_commit(st_bar);
         }
         st_pending = true;
@@ -748,7 +862,11 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
     if (aborted) {
         if (a.dev_status && tid == 0) atomicOr(a.dev_status, KDA_DEV_TIMEOUT);
         // let copies / MMAs still in flight land before the memory goes away
-        if (tma_pending) (void)mbar_wait(full_bar, full_phase, kWaitNs);
+        if (tma_pending) {
+            if (tid == 0 && !g_issued) mbar_arrive(full_bar);   // let the landed bytes close it
+            (void)mbar_wait(full_bar, full_phase, kWaitNs);
+        }
+        if (v_pending) (void)mbar_wait(v_bar, v_phase, kWaitNs);
         if (ut_pending) (void)mbar_wait(ut_bar, ut_phase, kWaitNs);
         if (st_pending) (void)mbar_wait(st_bar, st_phase, kWaitNs);
     } else if (a.S_T) {
