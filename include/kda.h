@@ -24,7 +24,8 @@
  *     row-major.  q, k, v, out, per-channel g and every state are 16-byte
  *     aligned (TMA and 128-bit loads); beta, scalar g and cu_seqlens need
  *     only their 4-byte element alignment.  The library allocates no memory
- *     and keeps no state between calls.
+ *     (scratch comes from the caller's workspace) and keeps no state between
+ *     calls.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
  *     default stream) and never synchronise.  Host-side validation happens
  *     before any launch and returns an error status with nothing launched.
@@ -37,6 +38,7 @@
 #ifndef KDA_H_
 #define KDA_H_
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -109,11 +111,31 @@ typedef struct {
  *             shape the fp32 path takes (CUDA-core path).
  *   KDA_F32:  d_k, d_v multiples of 16 in [16, 128], chunk in {16, 32, 64}.
  *   Anything else returns KDA_ERR_UNSUPPORTED.
+ * Workspace (caller-owned device memory, 256-byte aligned, contents need no
+ *   initialisation and are garbage afterwards):
+ *   workspace_bytes >= kda_chunk_fwd_workspace_size(shape) selects, on the
+ *   tensor-core path, the two-kernel schedule: every (chunk, head) computes its
+ *   state-independent operands in parallel into the workspace, then one short
+ *   sequential scan per (sequence, head) applies the state.  With workspace ==
+ *   NULL (workspace_bytes ignored) one fused kernel walks each sequence and
+ *   nothing else is needed.  A non-NULL workspace that is too small or
+ *   misaligned returns KDA_ERR_INVALID_ARG / KDA_ERR_MISALIGNED.  Both
+ *   schedules compute the same result up to rounding order.  The CUDA-core
+ *   path ignores the workspace.
  */
 kda_status_t kda_chunk_fwd(const kda_shape_t* shape, const void* q, const void* k,
                            const void* v, const float* g, const float* beta,
                            const float* S0, const int32_t* cu_seqlens, void* out,
-                           float* S_T, void* stream);
+                           float* S_T, void* workspace, size_t workspace_bytes,
+                           void* stream);
+
+/*
+ * Bytes of workspace the two-kernel schedule of kda_chunk_fwd needs for this
+ * shape; varlen != 0 for a packed batch (a cu_seqlens array will be passed).
+ * Returns 0 for a NULL shape or for shapes whose path uses no workspace (the
+ * fp32 CUDA-core path).  About 73 KB per (chunk, head) plus bookkeeping.
+ */
+size_t kda_chunk_fwd_workspace_size(const kda_shape_t* shape, int varlen);
 
 /*
  * kda_decode_step -- one fused recurrent token for N sequences.

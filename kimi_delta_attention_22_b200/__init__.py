@@ -13,7 +13,7 @@ import os
 
 import torch
 
-__all__ = ["kda_chunk_fwd", "kda_decode_step", "kda_status_str", "library_path", "load_library",
+__all__ = ["kda_chunk_fwd", "kda_chunk_fwd_workspace_size", "kda_decode_step", "kda_status_str", "library_path", "load_library",
            "KDAError", "KDA_F32", "KDA_BF16", "KDA_GATE_CHANNEL", "KDA_GATE_SCALAR",
            "KDA_GATE_NONE", "KDA_DEV_BAD_SEQLENS", "KDA_DEV_TIMEOUT", "Shape"]
 
@@ -59,7 +59,10 @@ def load_library(path: str | None = None):
                            "`python -m kimi_delta_attention_22_b200.build`")
     lib = ctypes.CDLL(p)
     P = ctypes.c_void_p
-    lib.kda_chunk_fwd.argtypes = [ctypes.POINTER(Shape), P, P, P, P, P, P, P, P, P, P]
+    lib.kda_chunk_fwd.argtypes = [ctypes.POINTER(Shape), P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t,
+                                  P]
+    lib.kda_chunk_fwd_workspace_size.argtypes = [ctypes.POINTER(Shape), ctypes.c_int]
+    lib.kda_chunk_fwd_workspace_size.restype = ctypes.c_size_t
     lib.kda_chunk_fwd.restype = ctypes.c_int
     lib.kda_decode_step.argtypes = [ctypes.POINTER(Shape), P, P, P, P, P, P, P, P]
     lib.kda_decode_step.restype = ctypes.c_int
@@ -111,7 +114,7 @@ def _check_cuda(*ts):
 
 
 def kda_chunk_fwd(q, k, v, g, beta, S0=None, cu_seqlens=None, chunk: int = 64, out=None,
-                  S_T=None, want_state: bool = True, dev_status=None, lib=None):
+                  S_T=None, want_state: bool = True, dev_status=None, workspace=True, lib=None):
     """Chunkwise KDA prefill (kda_chunk_fwd of include/kda.h).
 
     q, k [B,T,H,d_k]; v [B,T,H,d_v] (bf16 or fp32, same dtype); g [B,T,H,d_k]
@@ -119,6 +122,10 @@ def kda_chunk_fwd(q, k, v, g, beta, S0=None, cu_seqlens=None, chunk: int = 64, o
     beta [B,T,H] fp32; S0 [N,H,d_v,d_k] fp32 or None; cu_seqlens int32 [N+1]
     with B == 1 for packed sequences.  Returns (out, S_T); S_T is None when
     want_state is False and no S_T buffer is given.
+
+    workspace: True allocates the scratch of the two-kernel schedule with torch
+    (when the shape takes a path that uses one), a uint8 CUDA tensor supplies
+    it, None / False runs the single fused kernel with no scratch.
     """
     _check_cuda(q, k, v, g, beta, S0, cu_seqlens, out, S_T, dev_status)
     B, T, H, Dk = q.shape
@@ -139,12 +146,29 @@ def kda_chunk_fwd(q, k, v, g, beta, S0=None, cu_seqlens=None, chunk: int = 64, o
     sh = Shape(B, T, H, Dk, Dv, N, _dtype_code(q.dtype), _gate_code(g, q), int(chunk),
                None if dev_status is None else dev_status.data_ptr())
     lib = lib or load_library()
+    if isinstance(workspace, torch.Tensor):
+        _check_cuda(workspace)
+    if workspace is True:
+        nbytes = lib.kda_chunk_fwd_workspace_size(ctypes.byref(sh), int(cu_seqlens is not None))
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device) if nbytes else None
+    elif workspace is False:
+        workspace = None
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = lib.kda_chunk_fwd(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
-                           _ptr(S0), _ptr(cu_seqlens), _ptr(out), _ptr(S_T),
-                           _stream_handle(q.device))
+                           _ptr(S0), _ptr(cu_seqlens), _ptr(out), _ptr(S_T), _ptr(workspace),
+                           ws_bytes, _stream_handle(q.device))
     if st != 0:
         raise KDAError(st, "kda_chunk_fwd")
     return out, S_T
+
+
+def kda_chunk_fwd_workspace_size(q, v, g=None, cu_seqlens=None, chunk: int = 64, lib=None) -> int:
+    """Bytes of scratch the two-kernel schedule needs for these inputs (0: none)."""
+    B, T, H, Dk = q.shape
+    N = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    sh = Shape(B, T, H, Dk, v.shape[-1], N, _dtype_code(q.dtype), _gate_code(g, q), int(chunk), None)
+    lib = lib or load_library()
+    return int(lib.kda_chunk_fwd_workspace_size(ctypes.byref(sh), int(cu_seqlens is not None)))
 
 
 def kda_decode_step(q, k, v, g, beta, S, out=None, lib=None):

@@ -40,9 +40,16 @@ const char* kda_status_str(kda_status_t s) {
 
 const char* kda_version(void) { return "libkda 0.1 (sm_100a)"; }
 
+size_t kda_chunk_fwd_workspace_size(const kda_shape_t* sh, int varlen) {
+    if (sh == nullptr || sh->B < 0 || sh->T < 0 || sh->H <= 0 || sh->num_seqs < 0) return 0;
+    if (sh->dtype != KDA_BF16 || !kda::chunk_tc_supported(sh->d_k, sh->d_v, sh->chunk)) return 0;
+    return kda::rec::layout(sh->B, sh->T, sh->H, sh->num_seqs, varlen != 0).bytes;
+}
+
 kda_status_t kda_chunk_fwd(const kda_shape_t* sh, const void* q, const void* k, const void* v,
                            const float* g, const float* beta, const float* S0,
-                           const int32_t* cu_seqlens, void* out, float* S_T, void* stream) {
+                           const int32_t* cu_seqlens, void* out, float* S_T, void* workspace,
+                           size_t workspace_bytes, void* stream) {
     if (sh == nullptr) return KDA_ERR_INVALID_ARG;
     const int B = sh->B, T = sh->T, H = sh->H, D = sh->d_k, V = sh->d_v, N = sh->num_seqs;
     if (B < 0 || T < 0 || H <= 0 || D <= 0 || V <= 0 || N < 0) return KDA_ERR_INVALID_ARG;
@@ -67,6 +74,14 @@ kda_status_t kda_chunk_fwd(const kda_shape_t* sh, const void* q, const void* k, 
     const int C = sh->chunk;
     const bool tc = bf16 && kda::chunk_tc_supported(D, V, C);
     if (!tc && !f32path_supports(D, V, C)) return KDA_ERR_UNSUPPORTED;
+    kda::rec::Layout lay{};
+    const bool split = tc && workspace != nullptr;
+    if (split) {
+        if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KDA_ERR_MISALIGNED;
+        lay = kda::rec::layout(B, T, H, N, cu_seqlens != nullptr);
+        if (workspace_bytes < lay.bytes) return KDA_ERR_INVALID_ARG;
+        if (lay.slots * H > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+    }
     if (N == 0) return KDA_OK;
 
     kda::ChunkArgs a;
@@ -76,6 +91,12 @@ kda_status_t kda_chunk_fwd(const kda_shape_t* sh, const void* q, const void* k, 
     a.chunk = C;
     a.scale = 1.0f / sqrtf((float)D);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (split) {
+        uint8_t* ws = static_cast<uint8_t*>(workspace);
+        cudaError_t e = kda::launch_chunk_wy(a, ws, lay, st);
+        if (e == cudaSuccess) e = kda::launch_chunk_scan(a, ws, lay, st);
+        return from_cuda(e);
+    }
     return from_cuda(tc ? kda::launch_chunk_tc(a, st) : kda::launch_chunk_f32path(a, bf16, st));
 }
 

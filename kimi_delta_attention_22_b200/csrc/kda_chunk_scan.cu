@@ -1,0 +1,294 @@
+// kda_chunk_scan.cu -- the sequential half of the two-kernel tensor-core
+// prefill: the inter-chunk state scan plus outputs, from the records the WY
+// kernel wrote (layout and formulas in kda_chunk_record.cuh).
+//
+// One CTA per (sequence, head, 64-wide value tile) walks its sequence's
+// chunks in order with the fp32 state tile S^T (128 x 64) in registers
+// (thread = key channel, 32 value columns per warp group) and a bf16 copy in
+// shared memory as the MMA operand.  Per chunk, three groups of tcgen05 MMAs:
+//
+//   [W ; Qg] S^T          (M = 128, N = 64, K = 128)  -> E = U - W S^T  (lanes 0-63)
+//   Kd^T E                (M = 128, N = 64, K = 64)   -> S^T <- Diag(dec) S^T + Kd^T E
+//   [* ; Aqk] E  (accum.) (M = 128, N = 64, K = 64)   -> O = Qg S^T + Aqk E (lanes 64-127)
+//
+// The records of the next two chunks stream in by bulk copy while a chunk
+// runs; the outputs of a chunk are read out while the next chunk's first MMA
+// runs, so the dependent chain per chunk is MMA -> E -> MMA -> state update.
+#include "kda_chunk_record.cuh"
+#include "kda_internal.cuh"
+#include "kda_tc_common.cuh"
+#include "sm100.cuh"
+
+namespace kda {
+namespace {
+
+using namespace sm100;
+using namespace tc;
+
+constexpr int C = rec::C, DK = rec::DK, DV = rec::DV, BV = rec::BV, NVT = rec::NVT, NT = 256;
+constexpr uint64_t kWaitNs = 1000000000ull;   // 1 s bound on every wait
+constexpr int NSTAGE = 3;
+// One stage = one chunk's record slice: W|Qg, Kd, Aqk (one copy), U of this value
+// tile, dec.
+constexpr int ST_WQ = 0, ST_KD = 32768, ST_AQ = 49152, ST_U = 57344, ST_DEC = 65536;
+constexpr int STAGE = 66560;
+constexpr uint32_t STAGE_TX = 57344u + 8192u + 512u;
+constexpr int OFF_S = NSTAGE * STAGE;          // S^T bf16 (MN-major, MN = v, K = c)
+constexpr int OFF_BAR = OFF_S + 16384;         // full[NSTAGE], mma1, ds, o2, tmem base, flag
+constexpr int SMEM_BYTES = OFF_BAR + 128 + 1024;
+static_assert(SMEM_BYTES <= 232448, "shared memory over the sm_100 per-block limit");
+static_assert(ST_AQ - ST_KD == 16384 && ST_U - ST_AQ == 8192, "the [* ; Aqk] window needs Kd|Aqk adjacent");
+constexpr uint32_t TMEM_COLS = 256;
+constexpr uint32_t TM_D1 = 0;                  // 2 x 64 columns by chunk parity: [W ; Qg] S^T, then O
+constexpr uint32_t TM_DS = 128;                // Kd^T E
+constexpr int kIss = 64;                       // warp 2 (an output warp, off the E path)
+
+struct ScanParams {
+    const uint8_t* rec;
+    const int32_t* coff;
+    const int32_t* cu_seqlens;
+    const float* S0;
+    float* S_T;
+    __nv_bfloat16* out;
+    int32_t* dev_status;
+    int T, H, num_seqs, nc;
+};
+
+__global__ void __launch_bounds__(NT, 1) kda_chunk_scan_kernel(const __grid_constant__ ScanParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+    const int H = p.H;
+    const int vt = blockIdx.x % NVT;
+    const int h = (blockIdx.x / NVT) % H;
+    const int n = blockIdx.x / (NVT * H);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int sp = warp & 3, vh = warp >> 2;
+    const uint32_t lane_base = (uint32_t)(32 * sp) << 16;
+    const uint32_t sbase = smem_u32(sm);
+    uint64_t* full = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
+    uint64_t* bar1 = full + NSTAGE;
+    uint64_t* bar2 = bar1 + 1;
+    uint64_t* bar3 = bar1 + 2;
+    uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(bar1 + 3);
+    volatile int* flag_s = reinterpret_cast<volatile int*>(bar1 + 4);
+    uint64_t* drain = bar1 + 5;        // error path: completion of every MMA issued so far
+
+    long long bos, eos;
+    if (!seq_bounds(p.cu_seqlens, n, p.T, p.num_seqs, p.dev_status, bos, eos)) return;
+    const int nch = (int)((eos - bos + C - 1) / C);
+    const long long first = p.cu_seqlens ? (long long)p.coff[n] : (long long)n * p.nc;
+
+    if (tid == 0) {
+        for (int s = 0; s < NSTAGE; ++s) mbar_init(full + s, 1);
+        mbar_init(bar1, 1);
+        mbar_init(bar2, 1);
+        mbar_init(bar3, 1);
+        mbar_init(drain, 1);
+        *flag_s = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_base_s, TMEM_COLS);
+        tmem_relinquish();
+    }
+    __syncthreads();
+
+    int loaded = -1;                 // last chunk whose record copy was issued (issuing thread)
+    auto load_chunk = [&](int m) {   // issuing thread only
+        loaded = m;
+        uint8_t* dst = sm + (m % NSTAGE) * STAGE;
+        const uint8_t* src = p.rec + ((size_t)(first + m) * H + h) * rec::BYTES;
+        uint64_t* bar = full + (m % NSTAGE);
+        mbar_arrive_expect_tx(bar, STAGE_TX);
+        bulk_load(dst + ST_WQ, src + rec::WQ, 57344u, bar);
+        bulk_load(dst + ST_U, src + rec::U + 8192 * vt, 8192u, bar);
+        bulk_load(dst + ST_DEC, src + rec::DEC, 512u, bar);
+    };
+    if (tid == kIss) {
+        if (nch > 0) load_chunk(0);
+        if (nch > 1) load_chunk(1);
+    }
+
+    // ---- initial state: thread owns key channel c, value columns v0..v0+31
+    const int c_own = 32 * sp + lane;
+    const int v0 = 32 * vh;
+    const size_t sg = ((size_t)n * H + h) * DV * DK;
+    float S[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        const int v = vt * BV + v0 + j;
+        S[j] = p.S0 ? p.S0[sg + (size_t)v * DK + c_own] : 0.f;
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) st_shared_v4(sm + OFF_S, mnmaj_off(v0 + 8 * q, c_own, BV), pack8(S + 8 * q));
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = *tmem_base_s;
+
+    // Outputs of chunk m (its O2 MMAs complete on bar3): rows live in lanes 64-127.
+    auto read_out = [&](long long cp, int Lp, uint32_t col) {
+        const int i = 32 * (sp - 2) + lane;
+        float v[32];
+        tmem_ld32(tm + lane_base + col + 32 * vh, v);
+        if (i < Lp) {
+            __nv_bfloat16* op = p.out + ((size_t)(cp + i) * H + h) * DV + vt * BV + v0;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) reinterpret_cast<uint4*>(op)[q] = pack8(v + 8 * q);
+        }
+    };
+
+    uint32_t ph1 = 0, ph2 = 0, ph3 = 0;
+    bool aborted = false;
+    int m_stop = 0;
+    long long c_prev = 0;
+    int L_prev = 0;
+    for (int m = 0; m < nch; ++m) {
+        const int st = m % NSTAGE, par = m & 1;
+        const uint32_t full_ph = (uint32_t)((m / NSTAGE) & 1);
+        uint8_t* stg = sm + st * STAGE;
+        const uint32_t sstg = sbase + st * STAGE;
+        const long long c0 = bos + (long long)m * C;
+        const int L = (int)min((long long)C, eos - c0);
+        const uint32_t d1 = TM_D1 + 64 * par;
+        if (tid == kIss) {
+            if (!mbar_wait(full + st, full_ph, kWaitNs)) *flag_s = 1;
+            tc_fence_after();
+#pragma unroll
+            for (int s = 0; s < 8; ++s)
+                mma_bf16(tm + d1, rowview_desc(sstg + ST_WQ, s), mnmaj_desc(sbase + OFF_S, BV, s),
+                         idesc_bf16(128, BV, false, true), s > 0);
+            mma_commit(bar1);
+            // the stage of chunk m - 1 is free once its output MMAs are done
+            if (m + 2 < nch) {
+                if (m > 0 && !mbar_wait(bar3, ph3, kWaitNs)) *flag_s = 1;
+                load_chunk(m + 2);
+            }
+        }
+        if (sp >= 2) {
+            if (m > 0) {
+                if (!mbar_wait(bar3, ph3, kWaitNs)) *flag_s = 1;
+                tc_fence_after();
+                read_out(c_prev, L_prev, TM_D1 + 64 * (par ^ 1));
+            }
+        } else {
+            // E = U - W S^T over the U tile (same MN-major layout), rows j = lanes 0-63
+            if (!mbar_wait(bar1, ph1, kWaitNs)) *flag_s = 1;
+            tc_fence_after();
+            const int j = 32 * sp + lane;
+            float d[32];
+            tmem_ld32(tm + lane_base + d1 + 32 * vh, d);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const uint32_t off = ST_U + mnmaj_off(v0 + 8 * q, j, BV);
+                float u[8];
+                unpack8(*reinterpret_cast<const uint4*>(stg + off), u);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) u[e] -= d[8 * q + e];
+                st_shared_v4(stg, off, pack8(u));
+            }
+            fence_async_smem();
+        }
+        if (m > 0) ph3 ^= 1u;
+        ph1 ^= 1u;
+        tc_fence_before();
+        __syncthreads();
+        if (*flag_s != 0) { aborted = true; m_stop = m; break; }
+        if (tid == kIss) {
+            tc_fence_after();
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                mma_bf16(tm + TM_DS, mnmaj_desc(sstg + ST_KD, 128, s), mnmaj_desc(sstg + ST_U, BV, s),
+                         idesc_bf16(128, BV, true, true), s > 0);
+            mma_commit(bar2);
+            // rows 0-63 of the window are the second half of Kd: their products land in
+            // lanes 0-63, which hold nothing that is read again
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                mma_bf16(tm + d1, kmaj_desc(sstg + ST_KD + 8192, 128, s), mnmaj_desc(sstg + ST_U, BV, s),
+                         idesc_bf16(128, BV, false, true), 1);
+            mma_commit(bar3);
+        }
+        // ---- S^T <- Diag(dec) S^T + Kd^T E (fp32 registers) and its bf16 operand copy
+        if (!mbar_wait(bar2, ph2, kWaitNs)) *flag_s = 1;
+        ph2 ^= 1u;
+        tc_fence_after();
+        {
+            float ds[32];
+            tmem_ld32(tm + lane_base + TM_DS + 32 * vh, ds);
+            const float dec = reinterpret_cast<const float*>(stg + ST_DEC)[c_own];
+#pragma unroll
+            for (int jv = 0; jv < 32; ++jv) S[jv] = fmaf(S[jv], dec, ds[jv]);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                st_shared_v4(sm + OFF_S, mnmaj_off(v0 + 8 * q, c_own, BV), pack8(S + 8 * q));
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (*flag_s != 0) { aborted = true; m_stop = m; break; }
+        c_prev = c0;
+        L_prev = L;
+    }
+    if (!aborted && nch > 0) {
+        if (sp >= 2) {
+            if (!mbar_wait(bar3, ph3, kWaitNs)) {
+                *flag_s = 1;
+            } else {
+                tc_fence_after();
+                read_out(c_prev, L_prev, TM_D1 + 64 * ((nch - 1) & 1));
+            }
+        }
+        __syncthreads();
+        aborted = *flag_s != 0;
+        m_stop = nch;
+    }
+    if (aborted) {
+        if (p.dev_status && tid == 0) atomicOr(p.dev_status, KDA_DEV_TIMEOUT);
+        // let copies / MMAs still in flight land before the memory goes away
+        if (tid == kIss) {
+            mma_commit(drain);
+            (void)mbar_wait(drain, 0, kWaitNs);
+            for (int c = m_stop; c <= loaded; ++c)
+                (void)mbar_wait(full + c % NSTAGE, (uint32_t)((c / NSTAGE) & 1), kWaitNs);
+        }
+    } else if (p.S_T) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const int v = vt * BV + v0 + j;
+            p.S_T[sg + (size_t)v * DK + c_own] = S[j];
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tm, TMEM_COLS);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_chunk_scan(const ChunkArgs& a, const uint8_t* ws, const rec::Layout& lay, cudaStream_t st) {
+    ScanParams p;
+    p.rec = ws + lay.rec_off;
+    p.coff = a.cu_seqlens ? reinterpret_cast<const int32_t*>(ws + lay.coff_off) : nullptr;
+    p.cu_seqlens = a.cu_seqlens;
+    p.S0 = a.S0;
+    p.S_T = a.S_T;
+    p.out = static_cast<__nv_bfloat16*>(a.out);
+    p.dev_status = a.dev_status;
+    p.T = a.T;
+    p.H = a.H;
+    p.num_seqs = a.num_seqs;
+    p.nc = (a.T + C - 1) / C;
+    cudaError_t e = cudaFuncSetAttribute(kda_chunk_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    kda_chunk_scan_kernel<<<a.num_seqs * a.H * NVT, NT, SMEM_BYTES, st>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace kda

@@ -1,0 +1,756 @@
+// kda_chunk_wy.cu -- the state-independent half of the two-kernel
+// tensor-core prefill: one CTA per (chunk, head) computes the log-space
+// cumulative decay, the decay-masked key/key and query/key products (tcgen05
+// MMAs), the unit-lower-triangular inverse T = (I + L)^{-1} and the WY/UT
+// pseudo-value products W and U, and writes them as a record (layout in
+// kda_chunk_record.cuh).  Chunks are independent, so the whole grid runs in
+// parallel; only the state scan that follows is sequential.
+//
+// Chunkwise form: GeekNews summary of "You could have come up with Kimi
+// Delta Attention", section "Chunkwise KDA" (cumulative decay, coupling of
+// the in-chunk errors); the triangular solve into pseudo-values is the one
+// the curriculum page names ("WY/UT form").  For a chunk of C tokens:
+//
+//   Gamma_i = sum_{s<=i} g_s                                   (log2 units)
+//   P[i,j]  = sum_c K_ic K_jc 2^{Gamma_ic - Gamma_jc}    L = strict_lower(diag(beta) P)
+//   Qp[i,j] = sum_c Q~_ic K_jc 2^{Gamma_ic - Gamma_jc}   T = (I + L)^{-1}
+//
+// Two ways to split 2^{Gamma_i - Gamma_j} into an i-side and a j-side factor:
+//  * one reference (chunk start): i-side 2^{Gamma_i} <= 1, j-side 2^{-Gamma_j},
+//    used while max_c |Gamma_last,c| <= 112 so that the j-side stays finite;
+//  * sub-block references (16-token sub-blocks, reference row r(I)): i-side
+//    2^{Gamma_i - Gamma_r(I)}, j-side 2^{Gamma_r(I) - Gamma_j} (one version of
+//    the j-side per sub-block I), bounded for any decay a token can carry.
+// The fast kernel takes every chunk; a chunk that needs sub-block references
+// is put on a list that the slow kernel (more shared memory, one CTA per SM)
+// works through afterwards.
+#include <cudaTypedefs.h>
+
+#include "kda_chunk_record.cuh"
+#include "kda_internal.cuh"
+#include "kda_tc_common.cuh"
+#include "sm100.cuh"
+
+namespace kda {
+namespace {
+
+using namespace sm100;
+using namespace tc;
+
+constexpr int C = rec::C, DK = rec::DK, NT = 256;
+constexpr uint64_t kWaitNs = 1000000000ull;   // 1 s bound on every wait
+constexpr float kFastLimit2 = 112.f;          // one reference while max |Gamma_last| <= 2^112
+constexpr int LDT = 68;                       // fp32 row stride of L and T (bank spread)
+constexpr int LDX = 20;                       // fp32 row stride of 16x16 block scratch
+constexpr uint32_t TMEM_COLS = 256;
+constexpr uint32_t TM_GRAM = 0;               // Gram: 64 (one reference) or 128 columns
+constexpr uint32_t TM_WU = 128;               // W (lanes 0-15 of each sub-partition), U (16-31)
+
+// Shared-memory maps (bytes from a 1024-aligned base).
+template <bool SLOW>
+struct WyMap;
+template <>
+struct WyMap<false> {                          // one-reference chunks, two CTAs per SM
+    static constexpr int RK = 0, RQ = 16384, RG = 32768, RV = 65536;   // raw K, Q, g, V (2 tiles)
+    static constexpr int KQG = 0;              // after prep: rows 0-63 K e^G, rows 64-127 Q~ e^G
+    static constexpr int KYG = 32768;          //   K e^{-G}
+    static constexpr int KG = KQG;             //   K e^G as the B operand of W
+    static constexpr int L = 16384;            // after the Gram: fp32 L, T, Neumann blocks
+    static constexpr int TF = L + 64 * LDT * 4;
+    static constexpr int NS = TF + 64 * LDT * 4;
+    static constexpr int TOT4 = 81920;         // decay scan scratch (prep only)
+    static constexpr int GREF = TOT4 + 8192, GLAST = GREF + 2048, RED = GLAST + 512;
+    static constexpr int TB = 81920;           // after prep: T diag(beta) bf16 (K-major, 64 rows)
+    static constexpr int OX = 0, OY = 0, AQS = 0;   // sub-block path only
+    static constexpr int DECS = RED + 64, BETA = DECS + 512, BAR = BETA + 256, END = BAR + 64;
+    static_assert(NS + 10 * 16 * LDX * 4 <= RV, "phase-3 scratch overflows into V");
+    static_assert(TB + 8192 <= DECS, "T diag(beta) overlaps live scratch");
+};
+template <>
+struct WyMap<true> {                           // sub-block references, one CTA per SM
+    static constexpr int RK = 0, RQ = 16384, RG = 32768, RV = 65536;
+    static constexpr int OX = 0;               // after prep: Gram i-side rows (K-major, 128 rows)
+    static constexpr int KG = 32768;           //   K e^G (MN-major, MN = channel)
+    static constexpr int A = 81920;            // 64 KB, reused: scan scratch, Gram j-side
+    static constexpr int TOT4 = A, GREF = TOT4 + 8192, GLAST = GREF + 2048, RED = GLAST + 512;
+    static constexpr int OY = A;               //   2 K-major tiles of 128 rows (versions 2g, 2g+1)
+    static constexpr int L = A;                //   after the Gram: fp32 L, T, Neumann blocks,
+    static constexpr int TF = L + 64 * LDT * 4;
+    static constexpr int NS = TF + 64 * LDT * 4;
+    static constexpr int AQS = NS + 10 * 16 * LDX * 4;   // bf16 lower(Qp) staging
+    static constexpr int TB = A + 65536;
+    static constexpr int KQG = 0, KYG = 0;     // one-reference path only
+    static constexpr int DECS = TB + 8192, BETA = DECS + 512, BAR = BETA + 256, END = BAR + 64;
+    static_assert(AQS + 8192 <= A + 65536, "phase-3 scratch overflows region A");
+};
+template <bool SLOW>
+constexpr int wy_smem_bytes() { return WyMap<SLOW>::END + 1024; }
+static_assert(2 * (wy_smem_bytes<false>() + 1024) <= 233472, "fast kernel must fit twice per SM");
+static_assert(wy_smem_bytes<true>() <= 232448, "shared memory over the sm_100 per-block limit");
+
+struct WyParams {
+    CUtensorMap map_k, map_q, map_v, map_g;
+    const float* g;
+    const float* beta;
+    const int32_t* cu_seqlens;
+    const int32_t* coff;      // packed batches: first slot of each sequence, [num_seqs + 1]
+    int32_t* slow;            // [0] count, [1 + x] = slot * H + head
+    int32_t* dev_status;
+    uint8_t* rec;
+    int T, H, num_seqs, nc;   // nc: slots per sequence of a dense batch
+    float scale;
+};
+
+// Slot -> (sequence, first row, length).  False for slots past the last chunk.
+__device__ __forceinline__ bool decode_slot(const WyParams& p, int slot, long long& c0, int& L) {
+    long long bos, eos, first;
+    if (p.cu_seqlens == nullptr) {
+        const int n = slot / p.nc;
+        bos = (long long)n * p.T;
+        eos = bos + p.T;
+        first = (long long)n * p.nc;
+    } else {
+        if (slot >= p.coff[p.num_seqs]) return false;
+        int lo = 0, hi = p.num_seqs - 1;   // largest n with coff[n] <= slot
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (p.coff[mid] <= slot) lo = mid; else hi = mid - 1;
+        }
+        bos = p.cu_seqlens[lo];
+        eos = p.cu_seqlens[lo + 1];
+        first = p.coff[lo];
+    }
+    c0 = bos + (slot - first) * C;
+    L = (int)min((long long)C, eos - c0);
+    return L > 0;
+}
+
+// Off-diagonal 16x16 blocks of T = (I + L)^{-1} from its diagonal blocks by a block
+// Neumann series: with D = blockdiag(T_II) and N = D L_off (strictly block-lower,
+// N^4 = 0), T = (I - N + N^2 - N^3) D, i.e. T_IJ = M_IJ T_JJ (I > J) with
+// M = -N + N^2 - N^3.  Four levels of independent 16x16 tf32 products.
+__device__ __forceinline__ void neumann_offdiag(float* TF, const float* Lm, float* NS, int warp,
+                                                int lane) {
+    auto nb = [&](int idx) { return NS + idx * 16 * LDX; };
+    auto tf = [&](int I, int J) { return TF + 16 * I * LDT + 16 * J; };
+    auto lb = [&](int I, int J) { return Lm + 16 * I * LDT + 16 * J; };
+    // N blocks: 0:(1,0) 1:(2,0) 2:(3,0) 3:(2,1) 4:(3,1) 5:(3,2); 6: N^2_20, 7: N^2_31,
+    // 8: N^2_30, 9: N^3_30
+    if (warp < 6) {
+        const int I = (warp < 3) ? warp + 1 : ((warp < 5) ? warp - 1 : 3);
+        const int K = (warp < 3) ? 0 : ((warp < 5) ? 1 : 2);
+        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        blk_mma(acc, tf(I, I), LDT, lb(I, K), LDT, lane);
+        blk_store(nb(warp), LDX, acc, lane, 1.f);
+    }
+    __syncthreads();
+    if (warp < 6) {
+        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        if (warp < 3) {   // T_{J+1,J} = -N_{J+1,J} T_JJ
+            const int J = warp, nidx = (J == 0) ? 0 : ((J == 1) ? 3 : 5);
+            blk_mma(acc, nb(nidx), LDX, tf(J, J), LDT, lane);
+            blk_store(tf(J + 1, J), LDT, acc, lane, -1.f);
+        } else if (warp == 3) {   // N^2_20 = N_21 N_10
+            blk_mma(acc, nb(3), LDX, nb(0), LDX, lane);
+            blk_store(nb(6), LDX, acc, lane, 1.f);
+        } else if (warp == 4) {   // N^2_31 = N_32 N_21
+            blk_mma(acc, nb(5), LDX, nb(3), LDX, lane);
+            blk_store(nb(7), LDX, acc, lane, 1.f);
+        } else {                  // N^2_30 = N_31 N_10 + N_32 N_20
+            blk_mma(acc, nb(4), LDX, nb(0), LDX, lane);
+            blk_mma(acc, nb(5), LDX, nb(1), LDX, lane);
+            blk_store(nb(8), LDX, acc, lane, 1.f);
+        }
+    }
+    __syncthreads();
+    if (warp < 3) {
+        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        if (warp == 0) {          // T_20 = (N^2_20 - N_20) T_00
+            blk_mma2(acc, nb(6), 1.f, nb(1), -1.f, nullptr, 0.f, LDX, tf(0, 0), LDT, lane);
+            blk_store(tf(2, 0), LDT, acc, lane, 1.f);
+        } else if (warp == 1) {   // T_31 = (N^2_31 - N_31) T_11
+            blk_mma2(acc, nb(7), 1.f, nb(4), -1.f, nullptr, 0.f, LDX, tf(1, 1), LDT, lane);
+            blk_store(tf(3, 1), LDT, acc, lane, 1.f);
+        } else {                  // N^3_30 = N_32 N^2_20
+            blk_mma(acc, nb(5), LDX, nb(6), LDX, lane);
+            blk_store(nb(9), LDX, acc, lane, 1.f);
+        }
+    }
+    __syncthreads();
+    if (warp == 0) {              // T_30 = (N^2_30 - N_30 - N^3_30) T_00
+        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        blk_mma2(acc, nb(8), 1.f, nb(2), -1.f, nb(9), -1.f, LDX, tf(0, 0), LDT, lane);
+        blk_store(tf(3, 0), LDT, acc, lane, 1.f);
+    }
+    __syncthreads();
+}
+
+// One (chunk, head).  Returns 0 when the record is written, 1 when the chunk
+// needs sub-block references (fast kernel only; nothing written), 2 when a
+// bounded wait expired (everything in flight has been waited for again).
+template <int GATE, bool SLOW>
+__device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t tm, int slot, int h,
+                                      uint32_t& full_phase, uint32_t& mma_phase) {
+    using M = WyMap<SLOW>;
+    const int H = p.H;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int sp = warp & 3, half = warp >> 2;
+    const uint32_t lane_base = (uint32_t)(32 * sp) << 16;
+    const uint32_t sbase = smem_u32(sm);
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(sm + M::BAR);
+    uint64_t* mma_bar = full_bar + 1;
+    volatile int* flag_s = reinterpret_cast<volatile int*>(full_bar + 3);
+    float* tot4 = reinterpret_cast<float*>(sm + M::TOT4);
+    float* gref_s = reinterpret_cast<float*>(sm + M::GREF);
+    float* glast_s = reinterpret_cast<float*>(sm + M::GLAST);
+    float* dec_s = reinterpret_cast<float*>(sm + M::DECS);
+    float* beta_s = reinterpret_cast<float*>(sm + M::BETA);
+
+    long long c0;
+    int L;
+    if (!decode_slot(p, slot, c0, L)) return 0;
+    uint8_t* rec_p = p.rec + ((size_t)slot * H + h) * rec::BYTES;
+
+    // Uniform bounded wait: on expiry every thread leaves with `false` after
+    // waiting once more for the same phase (copies / MMAs still in flight).
+    auto wait_all = [&](uint64_t* bar, uint32_t& phase) -> bool {
+        if (!mbar_wait(bar, phase, kWaitNs)) *flag_s = 1;
+        __syncthreads();
+        if (*flag_s != 0) {
+            (void)mbar_wait(bar, phase, kWaitNs);
+            if (p.dev_status && tid == 0) atomicOr(p.dev_status, KDA_DEV_TIMEOUT);
+            return false;
+        }
+        phase ^= 1u;
+        return true;
+    };
+
+    if (tid == 0) {
+        // K, Q (16 KB each), V (two 8 KB tiles), per-channel g (32 KB)
+        const uint32_t bytes = 16384u * 3u + (GATE == KDA_GATE_CHANNEL ? 32768u : 0u);
+        mbar_arrive_expect_tx(full_bar, bytes);
+        tma_load_3d(sm + M::RK, &p.map_k, full_bar, 0, h, (int)c0);
+        tma_load_3d(sm + M::RQ, &p.map_q, full_bar, 0, h, (int)c0);
+        tma_load_3d(sm + M::RV, &p.map_v, full_bar, 0, h, (int)c0);
+        tma_load_3d(sm + M::RV + 8192, &p.map_v, full_bar, 64, h, (int)c0);
+        if (GATE == KDA_GATE_CHANNEL) tma_load_3d(sm + M::RG, &p.map_g, full_bar, 0, h, (int)c0);
+    }
+    const float beta_pf = (tid < L) ? p.beta[(size_t)(c0 + tid) * H + h] : 0.f;
+    if (!wait_all(full_bar, full_phase)) return 2;
+
+    // ================= log-space decay: thread tile = channels c8..c8+7 of rows 4 rg .. 4 rg + 3
+    bool fast;
+    const int cq = tid & 15, rg = tid >> 4, c8 = 8 * cq;
+    float g2[4][8], run[8];
+    uint4 kraw[4], qraw[4];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) run[e] = 0.f;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const int i = 4 * rg + r;
+        const bool valid = i < L;
+        float gv[8];
+        if (GATE == KDA_GATE_CHANNEL) {
+            const float4 a0 = *reinterpret_cast<const float4*>(sm + M::RG + (i * DK + c8) * 4);
+            const float4 a1 = *reinterpret_cast<const float4*>(sm + M::RG + (i * DK + c8 + 4) * 4);
+            gv[0] = a0.x; gv[1] = a0.y; gv[2] = a0.z; gv[3] = a0.w;
+            gv[4] = a1.x; gv[5] = a1.y; gv[6] = a1.z; gv[7] = a1.w;
+        } else if (GATE == KDA_GATE_SCALAR) {
+            const float gs = valid ? p.g[(size_t)(c0 + i) * H + h] : 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) gv[e] = gs;
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) gv[e] = 0.f;
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            run[e] += valid ? gv[e] * kLog2e : 0.f;
+            g2[r][e] = run[e];
+        }
+        const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+        kraw[r] = valid ? *reinterpret_cast<const uint4*>(sm + M::RK + (i * DK + c8) * 2) : z4;
+        qraw[r] = valid ? *reinterpret_cast<const uint4*>(sm + M::RQ + (i * DK + c8) * 2) : z4;
+    }
+    *reinterpret_cast<float4*>(tot4 + rg * DK + c8) = make_float4(run[0], run[1], run[2], run[3]);
+    *reinterpret_cast<float4*>(tot4 + rg * DK + c8 + 4) = make_float4(run[4], run[5], run[6], run[7]);
+    if (tid < C) beta_s[tid] = beta_pf;
+    __syncthreads();   // raw K / Q / g are consumed; their space now takes operands
+    // exclusive prefix over the 16 row groups, one thread per channel; the reference
+    // row of sub-block b is row 16 b + 7 (prefix before group 4 b + 2)
+    if (tid < DK) {
+        float tv[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q) tv[q] = tot4[q * DK + tid];
+        float acc = 0.f;
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+            if ((q & 3) == 2) gref_s[(q >> 2) * DK + tid] = acc;
+            const float t = tv[q];
+            tv[q] = acc;
+            acc += t;
+        }
+#pragma unroll
+        for (int q = 0; q < 16; ++q) tot4[q * DK + tid] = tv[q];
+        glast_s[tid] = acc;
+        const float d = ex2(acc);
+        dec_s[tid] = d;
+        reinterpret_cast<float*>(rec_p + rec::DEC)[tid] = d;
+        float m = -acc;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (lane == 0) reinterpret_cast<float*>(sm + M::RED)[warp] = m;
+    }
+    __syncthreads();
+    {
+        const float* red = reinterpret_cast<const float*>(sm + M::RED);
+        fast = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3])) <= kFastLimit2;
+    }
+    if (!SLOW && !fast) {
+        if (tid == 0) {
+            const int pos = atomicAdd(p.slow, 1);
+            p.slow[1 + pos] = slot * H + h;
+        }
+        __syncthreads();   // the scratch of this job is read no more
+        return 1;
+    }
+    uint8_t* g_wq = rec_p + rec::WQ;
+    uint8_t* g_kd = rec_p + rec::KD;
+    // the 16-byte chunks of this thread: (row 4 rg + r, channels c8..c8+7) in the
+    // mnmaj_off(c, row, 128) layout shared by K e^G, Q~ e^G, K e^{-G} and Kd
+    const uint32_t basemn = (uint32_t)((rg >> 1) * 2048 + (cq >> 3) * 1024 + (rg & 1) * 512);
+    if (!SLOW) {
+        // ================= one reference: 2^{Gamma_i} <= 1 on the i-side, 2^{-Gamma_j} <= 2^112 on the j-side
+        float pre[8], dec[8];
+        {
+            const float4* pp = reinterpret_cast<const float4*>(tot4 + rg * DK + c8);
+            const float4* dp = reinterpret_cast<const float4*>(dec_s + c8);
+            const float4 p0 = pp[0], p1 = pp[1], d0 = dp[0], d1 = dp[1];
+            pre[0] = p0.x; pre[1] = p0.y; pre[2] = p0.z; pre[3] = p0.w;
+            pre[4] = p1.x; pre[5] = p1.y; pre[6] = p1.z; pre[7] = p1.w;
+            dec[0] = d0.x; dec[1] = d0.y; dec[2] = d0.z; dec[3] = d0.w;
+            dec[4] = d1.x; dec[5] = d1.y; dec[6] = d1.z; dec[7] = d1.w;
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const uint32_t omn =
+                basemn + (((uint32_t)(cq & 7) ^ (uint32_t)(4 * (rg & 1) + r)) << 4) + (uint32_t)(r * 128);
+            float kf[8], qf[8], t1[8], t2[8], t3[8], t4[8];
+            unpack8(kraw[r], kf);
+            unpack8(qraw[r], qf);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float gm = pre[e] + g2[r][e];   // Gamma_i (log2), <= 0
+                const float eg = ex2(gm), ey = ex2(-gm);
+                t1[e] = kf[e] * eg;                    // K e^{Gamma}
+                t2[e] = (qf[e] * p.scale) * eg;        // Q~ e^{Gamma}
+                t3[e] = kf[e] * ey;                    // K e^{-Gamma}
+                t4[e] = kf[e] * (dec[e] * ey);         // K e^{Gamma_last - Gamma}
+            }
+            const uint4 q4 = pack8(t2);
+            st_shared_v4(sm + M::KQG, omn, pack8(t1));
+            st_shared_v4(sm + M::KQG, omn + 16384, q4);
+            st_shared_v4(sm + M::KYG, omn, pack8(t3));
+            *reinterpret_cast<uint4*>(g_wq + omn + 16384) = q4;
+            *reinterpret_cast<uint4*>(g_kd + omn) = pack8(t4);
+        }
+    } else {
+        // ================= sub-block references
+        const int b = rg >> 2;
+        float pre[8], gr[8], Er[8], Lr[8], z[4][8];
+        {
+            const float4* pp = reinterpret_cast<const float4*>(tot4 + rg * DK + c8);
+            const float4* gp = reinterpret_cast<const float4*>(gref_s + b * DK + c8);
+            const float4* lp = reinterpret_cast<const float4*>(glast_s + c8);
+            const float4 p0 = pp[0], p1 = pp[1], r0 = gp[0], r1 = gp[1], l0 = lp[0], l1 = lp[1];
+            const float pv[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+            const float rv[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+            const float lv[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                pre[e] = pv[e];
+                gr[e] = rv[e];
+                Er[e] = ex2(rv[e]);            // e^{Gamma_r}
+                Lr[e] = ex2(lv[e] - rv[e]);    // e^{Gamma_last - Gamma_r}
+            }
+#pragma unroll
+            for (int I = 1; I < 4; ++I) {
+                if (I > b) {
+                    const float4* ip = reinterpret_cast<const float4*>(gref_s + I * DK + c8);
+                    const float4 i0 = ip[0], i1 = ip[1];
+                    const float iv[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) z[I][e] = ex2(iv[e] - rv[e]);   // e^{Gamma_rI - Gamma_r} <= 1
+                }
+            }
+        }
+        __syncthreads();   // the scan scratch shares region A with the j-side operands
+        const uint32_t sw0 = (uint32_t)(cq & 7);
+        // the same rows inside a 128-row K-major tile: K-atom stride 16 KB
+        const uint32_t baseY = (uint32_t)((cq >> 3) * 16384 + (rg >> 1) * 1024 + (rg & 1) * 512);
+        const uint32_t base128 = (uint32_t)((cq >> 3) * 16384 + ((rg >> 1) + 2 * b) * 1024 + (rg & 1) * 512);
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const uint32_t swz = ((sw0 ^ (uint32_t)(4 * (rg & 1) + r)) << 4) + (uint32_t)(r * 128);
+            const uint32_t o128 = base128 + swz, omn = basemn + swz;
+            const uint32_t oy = baseY + swz;   // + (I >> 1) * 32768 + (I & 1) * 8192 for version I
+            float kf[8], qf[8], x[8], y[8], t[8];
+            unpack8(kraw[r], kf);
+            unpack8(qraw[r], qf);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float dl = (pre[e] + g2[r][e]) - gr[e];   // Gamma_i - Gamma_r (log2)
+                x[e] = ex2(dl);
+                y[e] = ex2(-dl);
+                qf[e] *= p.scale;
+            }
+            // Gram i-side: K rows at 32 b + (i - 16 b), Q rows 16 further
+#pragma unroll
+            for (int e = 0; e < 8; ++e) t[e] = kf[e] * x[e];
+            st_shared_v4(sm + M::OX, o128, pack8(t));
+#pragma unroll
+            for (int e = 0; e < 8; ++e) t[e] = qf[e] * x[e];
+            st_shared_v4(sm + M::OX, o128 + 2048, pack8(t));
+            // Gram j-side for this sub-block and the later ones
+            float ky[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) ky[e] = kf[e] * y[e];
+            st_shared_v4(sm + M::OY + (b >> 1) * 32768 + (b & 1) * 8192, oy, pack8(ky));
+#pragma unroll
+            for (int I = 1; I < 4; ++I) {
+                if (I > b) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) t[e] = ky[e] * z[I][e];
+                    st_shared_v4(sm + M::OY + (I >> 1) * 32768 + (I & 1) * 8192, oy, pack8(t));
+                }
+            }
+            // K e^Gamma (shared, MN-major), Q~ e^Gamma and K e^{Gamma_last - Gamma} (record)
+            float t2[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float eg = Er[e] * x[e];
+                t[e] = kf[e] * eg;
+                t2[e] = qf[e] * eg;
+            }
+            st_shared_v4(sm + M::KG, omn, pack8(t));
+            *reinterpret_cast<uint4*>(g_wq + omn + 16384) = pack8(t2);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) t[e] = kf[e] * (Lr[e] * y[e]);
+            *reinterpret_cast<uint4*>(g_kd + omn) = pack8(t);
+        }
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    // ================= Gram MMAs
+    // one reference: D[n][j] = [K e^G ; Q~ e^G]_n . (K e^-G)_j   (M = 128, N = 64)
+    // sub-blocks: group g (M = 128, N = 64): A rows 0-63 are the j-side of version 2g,
+    // rows 64-127 that of version 2g+1; B rows the i-side rows of sub-blocks 2g, 2g+1
+    if (tid == 0) {
+        if (!SLOW) {
+#pragma unroll
+            for (int s8 = 0; s8 < 8; ++s8)
+                mma_bf16(tm + TM_GRAM, rowview_desc(sbase + M::KQG, s8), rowview_desc(sbase + M::KYG, s8),
+                         idesc_bf16(128, 64, false, false), s8 > 0);
+        } else {
+            const uint32_t ox = sbase + M::OX, oy = sbase + M::OY;
+#pragma unroll
+            for (int s8 = 0; s8 < 8; ++s8)
+#pragma unroll
+                for (int g = 0; g < 2; ++g)
+                    mma_bf16(tm + TM_GRAM + 64 * g, kmaj_desc(oy + g * 32768, 128, s8),
+                             kmaj_desc(ox + g * 8192, 128, s8), idesc_bf16(128, 64, false, false), s8 > 0);
+        }
+        mma_commit(mma_bar);
+    }
+    if (!wait_all(mma_bar, mma_phase)) return 2;
+    tc_fence_after();
+    // ================= coupling matrix L (fp32, shared) and lower(Qp) (bf16, record)
+    float* Lm = reinterpret_cast<float*>(sm + M::L);
+    float* TF = reinterpret_cast<float*>(sm + M::TF);
+    if (!SLOW) {
+        // lane n = 32 sp + lane: row i of P (n < 64) or of Qp (n >= 64); columns 32 half ..
+        const int n = 32 * sp + lane, j0 = 32 * half;
+        float v[32];
+        tmem_ld32(tm + lane_base + TM_GRAM + j0, v);
+        if (n < 64) {
+            const int i = n;
+            const float bi = beta_s[i];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                float4 o;
+                o.x = (j0 + 4 * q + 0 < i) ? bi * v[4 * q + 0] : 0.f;
+                o.y = (j0 + 4 * q + 1 < i) ? bi * v[4 * q + 1] : 0.f;
+                o.z = (j0 + 4 * q + 2 < i) ? bi * v[4 * q + 2] : 0.f;
+                o.w = (j0 + 4 * q + 3 < i) ? bi * v[4 * q + 3] : 0.f;
+                *reinterpret_cast<float4*>(Lm + i * LDT + j0 + 4 * q) = o;
+            }
+        } else {
+            const int i = n - 64;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                float t8[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) t8[e] = (j0 + 8 * q + e <= i) ? v[8 * q + e] : 0.f;
+                *reinterpret_cast<uint4*>(rec_p + rec::AQ + kmaj_off(i, j0 + 8 * q, 64)) = pack8(t8);
+            }
+        }
+    } else {
+        // warp group g reads Gram group g; lanes of sub-partitions 0-1 hold rows j of
+        // sub-block 2g's version, those of 2-3 rows j of sub-block 2g+1's version
+        const int g = half, hi = sp >> 1;
+        const int I = 2 * g + hi, j = 32 * (sp & 1) + lane;
+        __nv_bfloat16* aqs = reinterpret_cast<__nv_bfloat16*>(sm + M::AQS);
+        float v[32];
+        tmem_ld32(tm + lane_base + TM_GRAM + 64 * g + 32 * hi, v);
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            const int i = 16 * I + u;
+            Lm[i * LDT + j] = (j < i) ? beta_s[i] * v[u] : 0.f;
+            aqs[kmaj_off(i, j, 64) >> 1] = __float2bfloat16_rn((j <= i) ? v[16 + u] : 0.f);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (SLOW) {   // the staged lower(Qp) tile to the record
+        for (int e = tid; e < 512; e += NT)
+            reinterpret_cast<uint4*>(rec_p + rec::AQ)[e] = reinterpret_cast<const uint4*>(sm + M::AQS)[e];
+    }
+    // ================= T = (I + L)^{-1}: diagonal 16x16 blocks by forward substitution
+    // (lane = column), then the off-diagonal blocks
+    if (warp < 4) {
+        const int I = warp, cc = lane & 15;
+        float t[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            float a4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int k = 0; k < r; ++k)
+                a4[k & 3] = fmaf(Lm[(16 * I + r) * LDT + 16 * I + k], t[k], a4[k & 3]);
+            const float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+            t[r] = (r < cc) ? 0.f : ((r == cc) ? 1.f : -acc);
+        }
+        if (lane < 16) {
+#pragma unroll
+            for (int r = 0; r < 16; ++r) TF[(16 * I + r) * LDT + 16 * I + cc] = t[r];
+        }
+    }
+    __syncthreads();
+    neumann_offdiag(TF, Lm, reinterpret_cast<float*>(sm + M::NS), warp, lane);
+    // T diag(beta) -> bf16 (K-major, K = j), 8 columns per step
+    for (int e = tid; e < C * 8; e += NT) {
+        const int i = e >> 3, j0 = 8 * (e & 7);
+        const float4 a0 = *reinterpret_cast<const float4*>(TF + i * LDT + j0);
+        const float4 a1 = *reinterpret_cast<const float4*>(TF + i * LDT + j0 + 4);
+        const float4 b0 = *reinterpret_cast<const float4*>(beta_s + j0);
+        const float4 b1 = *reinterpret_cast<const float4*>(beta_s + j0 + 4);
+        const float tv[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+        const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+        float t8[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) t8[k] = (j0 + k <= i) ? tv[k] * bv[k] : 0.f;
+        st_shared_v4(sm + M::TB, kmaj_off(i, j0, 64), pack8(t8));
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    // ================= W = T diag(beta) K e^G (M = 64, N = 128, lanes 0-15 of each
+    // sub-partition) and U = T diag(beta) V (two M = 64, N = 64 tiles, lanes 16-31)
+    if (tid == 0) {
+        const uint32_t tb = sbase + M::TB;
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+            mma_bf16(tm + TM_WU, kmaj_desc(tb, 64, s), mnmaj_desc(sbase + M::KG, 128, s),
+                     idesc_bf16(64, 128, false, true), s > 0);
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                mma_bf16(tm + TM_WU + (16u << 16) + 64 * t, kmaj_desc(tb, 64, s),
+                         mnmaj_desc(sbase + M::RV + 8192 * t, 64, s), idesc_bf16(64, 64, false, true),
+                         s > 0);
+        mma_commit(mma_bar);
+    }
+    if (!wait_all(mma_bar, mma_phase)) return 2;
+    tc_fence_after();
+    {
+        // lane l < 16: W row 16 sp + l; l >= 16: U row 16 sp + l - 16; columns 64 half ..
+        const bool isw = lane < 16;
+        const int i = 16 * sp + (lane & 15);
+#pragma unroll
+        for (int hc = 0; hc < 2; ++hc) {
+            float v[32];
+            tmem_ld32(tm + lane_base + TM_WU + 64 * half + 32 * hc, v);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int c = 64 * half + 32 * hc + 8 * q;
+                const uint32_t off = isw ? (uint32_t)rec::WQ + mnmaj_off(c, i, 128)
+                                         : (uint32_t)(rec::U + 8192 * half) + mnmaj_off(c - 64 * half, i, 64);
+                *reinterpret_cast<uint4*>(rec_p + off) = pack8(v + 8 * q);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    return 0;
+}
+
+template <int GATE, bool SLOW>
+__global__ void __launch_bounds__(NT, SLOW ? 1 : 2) kda_chunk_wy_kernel(const __grid_constant__ WyParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+    using M = WyMap<SLOW>;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(sm + M::BAR);
+    uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(full_bar + 2);
+    int* flag_s = reinterpret_cast<int*>(full_bar + 3);
+    const int count = SLOW ? *p.slow : 0;
+    if (SLOW && (int)blockIdx.x >= count) return;
+    if (tid == 0) {
+        mbar_init(full_bar, 1);
+        mbar_init(full_bar + 1, 1);
+        *flag_s = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_base_s, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = *tmem_base_s;
+    uint32_t full_phase = 0, mma_phase = 0;
+    if (!SLOW) {
+        (void)wy_job<GATE, false>(p, sm, tm, blockIdx.x, blockIdx.y, full_phase, mma_phase);
+    } else {
+        for (int x = blockIdx.x; x < count; x += gridDim.x) {
+            const int job = p.slow[1 + x];
+            if (wy_job<GATE, true>(p, sm, tm, job / p.H, job % p.H, full_phase, mma_phase) == 2) break;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tm, TMEM_COLS);
+    }
+}
+
+// Chunk offsets of a packed batch: coff[n] = sum_{m < n} ceil(len_m / C), with
+// inconsistent sequences counted as empty (and flagged, as everywhere else).
+__global__ void __launch_bounds__(1024) kda_chunk_offsets_kernel(const int32_t* cu, int num_seqs, int T,
+                                                                 int32_t* coff, int32_t* dev_status) {
+    __shared__ int32_t warp_sums[32];
+    __shared__ int32_t carry_s;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid == 0) carry_s = 0;
+    __syncthreads();
+    for (int base = 0; base < num_seqs; base += 1024) {
+        const int n = base + tid;
+        int cnt = 0;
+        if (n < num_seqs) {
+            const int a = cu[n], b = cu[n + 1];
+            if (a < 0 || b < a || b > T || (n == 0 && a != 0)) {
+                if (dev_status) atomicOr(dev_status, KDA_DEV_BAD_SEQLENS);
+            } else {
+                cnt = (b - a + C - 1) / C;
+            }
+        }
+        int x = cnt;   // inclusive warp scan
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane == 31) warp_sums[warp] = x;
+        __syncthreads();
+        if (warp == 0) {
+            int w = warp_sums[lane];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, w, o);
+                if (lane >= o) w += y;
+            }
+            warp_sums[lane] = w;   // inclusive over warps
+        }
+        __syncthreads();
+        const int carry = carry_s;
+        const int excl = carry + (warp > 0 ? warp_sums[warp - 1] : 0) + x - cnt;
+        if (n < num_seqs) coff[n] = excl;
+        __syncthreads();
+        if (tid == 0) carry_s = carry + warp_sums[31];
+        __syncthreads();
+    }
+    if (tid == 0) coff[num_seqs] = carry_s;
+}
+
+template <int GATE>
+cudaError_t launch_wy_gate(const WyParams& p, long long slots, int sm_count, cudaStream_t st) {
+    auto kf = kda_chunk_wy_kernel<GATE, false>;
+    auto ks = kda_chunk_wy_kernel<GATE, true>;
+    cudaError_t e = cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, wy_smem_bytes<false>());
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, wy_smem_bytes<true>());
+    if (e != cudaSuccess) return e;
+    kf<<<dim3((unsigned)slots, (unsigned)p.H), NT, wy_smem_bytes<false>(), st>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const long long jobs = slots * p.H;
+    const int grid = (int)(jobs < (long long)sm_count ? jobs : (long long)sm_count);
+    ks<<<grid, NT, wy_smem_bytes<true>(), st>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+// The state-independent pass of the two-kernel prefill (see kda_chunk_record.cuh).
+cudaError_t launch_chunk_wy(const ChunkArgs& a, uint8_t* ws, const rec::Layout& lay, cudaStream_t st) {
+    WyParams p;
+    memset(&p, 0, sizeof(p));
+    p.g = a.g;
+    p.beta = a.beta;
+    p.cu_seqlens = a.cu_seqlens;
+    p.dev_status = a.dev_status;
+    p.slow = reinterpret_cast<int32_t*>(ws + lay.list_off);
+    p.coff = a.cu_seqlens ? reinterpret_cast<const int32_t*>(ws + lay.coff_off) : nullptr;
+    p.rec = ws + lay.rec_off;
+    p.T = a.T;
+    p.H = a.H;
+    p.num_seqs = a.num_seqs;
+    p.nc = (a.T + C - 1) / C;
+    p.scale = a.scale;
+    const long long tokens = (long long)a.B * a.T;
+    if (tokens == 0 || lay.slots == 0) return cudaSuccess;
+    bool ok = make_map(&p.map_k, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DK, a.H, tokens, DK, C,
+                       CU_TENSOR_MAP_SWIZZLE_NONE) &&
+              make_map(&p.map_q, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DK, a.H, tokens, DK, C,
+                       CU_TENSOR_MAP_SWIZZLE_NONE) &&
+              make_map(&p.map_v, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rec::DV, a.H, tokens, 64, C,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+    if (ok && a.gate == KDA_GATE_CHANNEL)
+        ok = make_map(&p.map_g, a.g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, DK, a.H, tokens, DK, C,
+                      CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (!ok) return cudaErrorInvalidValue;
+    cudaError_t e = cudaMemsetAsync(p.slow, 0, sizeof(int32_t), st);
+    if (e != cudaSuccess) return e;
+    if (a.cu_seqlens) {
+        kda_chunk_offsets_kernel<<<1, 1024, 0, st>>>(a.cu_seqlens, a.num_seqs, a.T,
+                                                     const_cast<int32_t*>(p.coff), a.dev_status);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        (void)cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    switch (a.gate) {
+        case KDA_GATE_CHANNEL: return launch_wy_gate<KDA_GATE_CHANNEL>(p, lay.slots, sms, st);
+        case KDA_GATE_SCALAR: return launch_wy_gate<KDA_GATE_SCALAR>(p, lay.slots, sms, st);
+        default: return launch_wy_gate<KDA_GATE_NONE>(p, lay.slots, sms, st);
+    }
+}
+
+}  // namespace kda

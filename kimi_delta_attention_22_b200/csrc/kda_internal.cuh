@@ -7,6 +7,7 @@
 #include <stdint.h>
 
 #include "../../include/kda.h"
+#include "kda_chunk_record.cuh"
 
 namespace kda {
 
@@ -40,6 +41,10 @@ struct DecodeArgs {
 
 cudaError_t launch_chunk_f32path(const ChunkArgs& a, bool bf16, cudaStream_t s);
 cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t s);
+// Two-kernel tensor-core prefill over a caller workspace laid out by rec::layout().
+cudaError_t launch_chunk_wy(const ChunkArgs& a, uint8_t* ws, const rec::Layout& lay, cudaStream_t s);
+cudaError_t launch_chunk_scan(const ChunkArgs& a, const uint8_t* ws, const rec::Layout& lay,
+                              cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs& a, bool bf16, cudaStream_t s);
 
 // Rows [bos, eos) of the packed token axis that sequence n covers.  Returns

@@ -62,11 +62,13 @@ def check(got, ref, mode, what, stored_bf16=None):
     return e
 
 
-def run_chunk(d, chunk, want_state=True, cu=None):
+def run_chunk(d, chunk, want_state=True, cu=None, workspace=True):
+    """kda_chunk_fwd on the GPU copies of d.  workspace=True takes the two-kernel
+    schedule on the tensor-core path, False the single fused kernel."""
     on = to_dev(d)
     out, ST = kda.kda_chunk_fwd(on["q"], on["k"], on["v"], on["g"], on["beta"], S0=on["S0"],
                                 cu_seqlens=on.get("cu_seqlens") if cu is None else cu.cuda(),
-                                chunk=chunk, want_state=want_state)
+                                chunk=chunk, want_state=want_state, workspace=workspace)
     torch.cuda.synchronize()
     return out, ST
 

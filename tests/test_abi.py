@@ -31,7 +31,8 @@ def declared_functions():
 
 def test_header_declares_entry_points():
     names = declared_functions()
-    for n in ("kda_chunk_fwd", "kda_decode_step", "kda_status_str", "kda_version"):
+    for n in ("kda_chunk_fwd", "kda_chunk_fwd_workspace_size", "kda_decode_step", "kda_status_str",
+              "kda_version"):
         assert n in names
 
 
@@ -55,9 +56,9 @@ P = ctypes.c_void_p
 A = P(0x10000)  # a 16-byte aligned fake address: only ever seen by host-side checks
 
 
-def _chunk(lib, sh, q=A, g=A, cu=None, S0=None):
+def _chunk(lib, sh, q=A, g=A, cu=None, S0=None, ws=None, ws_bytes=0):
     return lib.kda_chunk_fwd(None if sh is None else ctypes.byref(sh), q, A, A, g, A, S0, cu, A,
-                             None, None)
+                             None, ws, ws_bytes, None)
 
 
 def test_chunk_validation(lib):
@@ -90,6 +91,26 @@ def test_chunk_validation(lib):
     assert _chunk(lib, _shape(B=0, N=0, chunk=48, dtype=kda.KDA_F32)) == 2
     # null tensors with tokens present
     assert _chunk(lib, _shape(B=1, T=4, N=1), q=None) == 1
+
+
+def test_workspace_size_and_checks(lib):
+    sh = _shape(B=4, T=2048, H=16, N=4)
+    # one record of 74240 bytes per (chunk, head) plus the job list
+    n = lib.kda_chunk_fwd_workspace_size(ctypes.byref(sh), 0)
+    assert n >= 4 * 32 * 16 * 74240 and n < 4 * 32 * 16 * 74240 + 65536
+    # packed batches reserve one extra partial chunk per sequence and the chunk offsets
+    shv = _shape(B=1, T=2048, H=16, N=4)
+    assert lib.kda_chunk_fwd_workspace_size(ctypes.byref(shv), 1) >= (32 + 4) * 16 * 74240
+    # the CUDA-core path needs none
+    sf = _shape(B=4, T=64, H=1, dk=16, dv=16, N=4, dtype=kda.KDA_F32, chunk=16)
+    assert lib.kda_chunk_fwd_workspace_size(ctypes.byref(sf), 0) == 0
+    assert lib.kda_chunk_fwd_workspace_size(None, 0) == 0
+    # zero sequences with a workspace: too small, misaligned, enough
+    z = _shape(B=0, N=0)
+    need = lib.kda_chunk_fwd_workspace_size(ctypes.byref(z), 0)
+    assert _chunk(lib, z, ws=A, ws_bytes=need) == 0
+    assert _chunk(lib, _shape(B=1, T=64, N=1), ws=A, ws_bytes=16) == 1
+    assert _chunk(lib, z, ws=P(0x10010), ws_bytes=need + 1024) == 3
 
 
 def _decode(lib, sh, g=A, S=A):

@@ -59,17 +59,19 @@ BF16_CASES = [
 ]
 
 
+@pytest.mark.parametrize("schedule", ["split", "fused"])
 @pytest.mark.parametrize("B,T,H,gate,beta,s0,chunk", BF16_CASES)
-def test_bf16(B, T, H, gate, beta, s0, chunk):
+def test_bf16(B, T, H, gate, beta, s0, chunk, schedule):
     d = inputs.draw(B, T, H, 128, 128, dtype=torch.bfloat16, gate=gate, beta=beta,
                     s0_std=0.02 if s0 else None, seed=B * 1000 + T + H)
-    out, ST = run_chunk(d, chunk)
+    out, ST = run_chunk(d, chunk, workspace=schedule == "split")
     ro, rs = oracle_chunk(d, gate_of(d))
     check(out, ro, "bf16", "out")
     check(ST, rs, "bf16", "S_T")
 
 
-def test_varlen_small_ragged_and_empty():
+@pytest.mark.parametrize("schedule", ["split", "fused"])
+def test_varlen_small_ragged_and_empty(schedule):
     """Packed sequences of lengths 0, 1, 64, 65, 127, 200 (state restarts per
     sequence; the empty one returns S0)."""
     lens = [0, 1, 64, 65, 127, 200]
@@ -77,7 +79,7 @@ def test_varlen_small_ragged_and_empty():
     d = inputs.draw(1, int(cu[-1]), 2, 128, 128, dtype=torch.bfloat16, s0_std=0.02,
                     num_states=len(lens), seed=77)
     d["cu_seqlens"] = cu
-    out, ST = run_chunk(d, 64)
+    out, ST = run_chunk(d, 64, workspace=schedule == "split")
     ro, rs = oracle_chunk(d, "channel")
     check(out, ro, "bf16", "out")
     check(ST, rs, "bf16", "S_T")
