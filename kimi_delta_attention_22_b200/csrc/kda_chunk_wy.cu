@@ -55,6 +55,7 @@ struct WyMap<false> {                          // one-reference chunks, two CTAs
     static constexpr int KQG = 0;              // after prep: rows 0-63 K e^G, rows 64-127 Q~ e^G
     static constexpr int KYG = 32768;          //   K e^{-G}
     static constexpr int KG = KQG;             //   K e^G as the B operand of W
+    static constexpr int KDST = 49152;         //   K e^{G_last - G} record image (over raw g)
     static constexpr int L = 16384;            // after the Gram: fp32 L, T, Neumann blocks
     static constexpr int TF = L + 64 * LDT * 4;
     static constexpr int NS = TF + 64 * LDT * 4;
@@ -62,6 +63,8 @@ struct WyMap<false> {                          // one-reference chunks, two CTAs
     static constexpr int GREF = TOT4 + 8192, GLAST = GREF + 2048, RED = GLAST + 512;
     static constexpr int TB = 81920;           // after prep: T diag(beta) bf16 (K-major, 64 rows)
     static constexpr int OX = 0, OY = 0, AQS = 0;   // sub-block path only
+    static constexpr int AQST = TB;            // bf16 lower(Qp) staging (before T diag(beta) exists)
+    static constexpr int WST = L, UST = L + 16384;   // after the W/U MMAs: record images of W, U
     static constexpr int DECS = RED + 64, BETA = DECS + 512, BAR = BETA + 256, END = BAR + 64;
     static_assert(NS + 10 * 16 * LDX * 4 <= RV, "phase-3 scratch overflows into V");
     static_assert(TB + 8192 <= DECS, "T diag(beta) overlaps live scratch");
@@ -79,7 +82,10 @@ struct WyMap<true> {                           // sub-block references, one CTA 
     static constexpr int NS = TF + 64 * LDT * 4;
     static constexpr int AQS = NS + 10 * 16 * LDX * 4;   // bf16 lower(Qp) staging
     static constexpr int TB = A + 65536;
-    static constexpr int KQG = 0, KYG = 0;     // one-reference path only
+    static constexpr int KQG = 0, KYG = 0, KDST = 0;   // one-reference path only
+    static constexpr int AQST = AQS;
+    static constexpr int WST = A, UST = A + 16384;   // after the W/U MMAs: record images of W, U
+    static_assert(UST + 16384 <= AQS, "W/U staging overlaps the lower(Qp) staging");
     static constexpr int DECS = TB + 8192, BETA = DECS + 512, BAR = BETA + 256, END = BAR + 64;
     static_assert(AQS + 8192 <= A + 65536, "phase-3 scratch overflows region A");
 };
@@ -98,6 +104,7 @@ struct WyParams {
     int32_t* dev_status;
     uint8_t* rec;
     int T, H, num_seqs, nc;   // nc: slots per sequence of a dense batch
+    int ahead;                // fast kernel: CTAs resident at once (L2 prefetch distance)
     float scale;
 };
 
@@ -234,6 +241,22 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
         tma_load_3d(sm + M::RV, &p.map_v, full_bar, 0, h, (int)c0);
         tma_load_3d(sm + M::RV + 8192, &p.map_v, full_bar, 64, h, (int)c0);
         if (GATE == KDA_GATE_CHANNEL) tma_load_3d(sm + M::RG, &p.map_g, full_bar, 0, h, (int)c0);
+        if (!SLOW) {
+            // the job that starts one resident wave later (blocks start in linear order):
+            // its tiles go to L2 now, so that its own loads hit there
+            const long long lin = blockIdx.x + (long long)blockIdx.y * gridDim.x + p.ahead;
+            long long c2;
+            int L2;
+            if (lin < (long long)gridDim.x * gridDim.y &&
+                decode_slot(p, (int)(lin % gridDim.x), c2, L2)) {
+                const int h2 = (int)(lin / gridDim.x);
+                tma_prefetch_l2_3d(&p.map_k, 0, h2, (int)c2);
+                tma_prefetch_l2_3d(&p.map_q, 0, h2, (int)c2);
+                tma_prefetch_l2_3d(&p.map_v, 0, h2, (int)c2);
+                tma_prefetch_l2_3d(&p.map_v, 64, h2, (int)c2);
+                if (GATE == KDA_GATE_CHANNEL) tma_prefetch_l2_3d(&p.map_g, 0, h2, (int)c2);
+            }
+        }
     }
     const float beta_pf = (tid < L) ? p.beta[(size_t)(c0 + tid) * H + h] : 0.f;
     if (!wait_all(full_bar, full_phase)) return 2;
@@ -347,12 +370,11 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
                 t3[e] = kf[e] * ey;                    // K e^{-Gamma}
                 t4[e] = kf[e] * (dec[e] * ey);         // K e^{Gamma_last - Gamma}
             }
-            const uint4 q4 = pack8(t2);
+            // rows 64-127 of K|Q e^G are also the Qg half of the record image
             st_shared_v4(sm + M::KQG, omn, pack8(t1));
-            st_shared_v4(sm + M::KQG, omn + 16384, q4);
+            st_shared_v4(sm + M::KQG, omn + 16384, pack8(t2));
             st_shared_v4(sm + M::KYG, omn, pack8(t3));
-            *reinterpret_cast<uint4*>(g_wq + omn + 16384) = q4;
-            *reinterpret_cast<uint4*>(g_kd + omn) = pack8(t4);
+            st_shared_v4(sm + M::KDST, omn, pack8(t4));
         }
     } else {
         // ================= sub-block references
@@ -463,6 +485,12 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
                              kmaj_desc(ox + g * 8192, 128, s8), idesc_bf16(128, 64, false, false), s8 > 0);
         }
         mma_commit(mma_bar);
+        if (!SLOW) {   // Qg and Kd images to the record while the Gram runs
+            bulk_store(g_wq + 16384, sm + M::KQG + 16384, 16384u);
+            bulk_store(g_kd, sm + M::KDST, 16384u);
+            bulk_commit();
+            bulk_wait_read();   // both are overwritten once the Gram is read out
+        }
     }
     if (!wait_all(mma_bar, mma_phase)) return 2;
     tc_fence_after();
@@ -493,7 +521,7 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
                 float t8[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) t8[e] = (j0 + 8 * q + e <= i) ? v[8 * q + e] : 0.f;
-                *reinterpret_cast<uint4*>(rec_p + rec::AQ + kmaj_off(i, j0 + 8 * q, 64)) = pack8(t8);
+                st_shared_v4(sm + M::AQST, kmaj_off(i, j0 + 8 * q, 64), pack8(t8));
             }
         }
     } else {
@@ -511,11 +539,12 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
             aqs[kmaj_off(i, j, 64) >> 1] = __float2bfloat16_rn((j <= i) ? v[16 + u] : 0.f);
         }
     }
+    fence_async_smem();
     tc_fence_before();
     __syncthreads();
-    if (SLOW) {   // the staged lower(Qp) tile to the record
-        for (int e = tid; e < 512; e += NT)
-            reinterpret_cast<uint4*>(rec_p + rec::AQ)[e] = reinterpret_cast<const uint4*>(sm + M::AQS)[e];
+    if (tid == 0) {   // the staged lower(Qp) tile to the record
+        bulk_store(rec_p + rec::AQ, sm + M::AQST, 8192u);
+        bulk_commit();
     }
     // ================= T = (I + L)^{-1}: diagonal 16x16 blocks by forward substitution
     // (lane = column), then the off-diagonal blocks
@@ -536,6 +565,7 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
             for (int r = 0; r < 16; ++r) TF[(16 * I + r) * LDT + 16 * I + cc] = t[r];
         }
     }
+    if (tid == 0) bulk_wait_read();   // the staging is overwritten from here on
     __syncthreads();
     neumann_offdiag(TF, Lm, reinterpret_cast<float*>(sm + M::NS), warp, lane);
     // T diag(beta) -> bf16 (K-major, K = j), 8 columns per step
@@ -586,13 +616,21 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const int c = 64 * half + 32 * hc + 8 * q;
-                const uint32_t off = isw ? (uint32_t)rec::WQ + mnmaj_off(c, i, 128)
-                                         : (uint32_t)(rec::U + 8192 * half) + mnmaj_off(c - 64 * half, i, 64);
-                *reinterpret_cast<uint4*>(rec_p + off) = pack8(v + 8 * q);
+                const uint32_t off = isw ? (uint32_t)M::WST + mnmaj_off(c, i, 128)
+                                         : (uint32_t)(M::UST + 8192 * half) + mnmaj_off(c - 64 * half, i, 64);
+                st_shared_v4(sm, off, pack8(v + 8 * q));
             }
         }
     }
+    fence_async_smem();
     tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {   // W (rows 0-63 of the W|Qg image) and both U tiles
+        bulk_store(rec_p + rec::WQ, sm + M::WST, 16384u);
+        bulk_store(rec_p + rec::U, sm + M::UST, 16384u);
+        bulk_commit();
+        bulk_wait_read();
+    }
     __syncthreads();
     return 0;
 }
@@ -632,6 +670,7 @@ __global__ void __launch_bounds__(NT, SLOW ? 1 : 2) kda_chunk_wy_kernel(const __
             if (wy_job<GATE, true>(p, sm, tm, job / p.H, job % p.H, full_phase, mma_phase) == 2) break;
         }
     }
+    if (tid == 0) bulk_wait_read();   // shared memory outlives no store that reads it
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -696,7 +735,13 @@ cudaError_t launch_wy_gate(const WyParams& p, long long slots, int sm_count, cud
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, wy_smem_bytes<true>());
     if (e != cudaSuccess) return e;
-    kf<<<dim3((unsigned)slots, (unsigned)p.H), NT, wy_smem_bytes<false>(), st>>>(p);
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kf, NT, wy_smem_bytes<false>()) != cudaSuccess ||
+        per_sm < 1)
+        per_sm = 1;
+    WyParams pf = p;
+    pf.ahead = per_sm * sm_count;
+    kf<<<dim3((unsigned)slots, (unsigned)p.H), NT, wy_smem_bytes<false>(), st>>>(pf);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const long long jobs = slots * p.H;
