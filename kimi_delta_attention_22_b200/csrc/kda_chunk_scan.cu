@@ -77,7 +77,6 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_scan_kernel(const __grid_cons
     long long bos, eos;
     if (!seq_bounds(p.cu_seqlens, n, p.T, p.num_seqs, p.dev_status, bos, eos)) return;
     const int nch = (int)((eos - bos + C - 1) / C);
-    const long long first = p.cu_seqlens ? (long long)p.coff[n] : (long long)n * p.nc;
 
     if (tid == 0) {
         for (int s = 0; s < NSTAGE; ++s) mbar_init(full + s, 1);
@@ -94,6 +93,7 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_scan_kernel(const __grid_cons
     }
     __syncthreads();
 
+    long long first = 0;             // slot of the sequence's first chunk (set after pdl_wait)
     int loaded = -1;                 // last chunk whose record copy was issued (issuing thread)
     auto load_chunk = [&](int m) {   // issuing thread only
         loaded = m;
@@ -105,11 +105,6 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_scan_kernel(const __grid_cons
         bulk_load(dst + ST_U, src + rec::U + 8192 * vt, 8192u, bar);
         bulk_load(dst + ST_DEC, src + rec::DEC, 512u, bar);
     };
-    if (tid == kIss) {
-        if (nch > 0) load_chunk(0);
-        if (nch > 1) load_chunk(1);
-    }
-
     // ---- initial state: thread owns key channel c, value columns v0..v0+31
     const int c_own = 32 * sp + lane;
     const int v0 = 32 * vh;
@@ -127,6 +122,13 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_scan_kernel(const __grid_cons
     __syncthreads();
     tc_fence_after();
     const uint32_t tm = *tmem_base_s;
+    // everything above overlaps the tail of the WY kernels; records are read below
+    pdl_wait();
+    first = p.cu_seqlens ? (long long)p.coff[n] : (long long)n * p.nc;
+    if (tid == kIss) {
+        if (nch > 0) load_chunk(0);
+        if (nch > 1) load_chunk(1);
+    }
 
     // Outputs of chunk m (its O2 MMAs complete on bar3): rows live in lanes 64-127.
     auto read_out = [&](long long cp, int Lp, uint32_t col) {
@@ -287,8 +289,7 @@ cudaError_t launch_chunk_scan(const ChunkArgs& a, const uint8_t* ws, const rec::
     cudaError_t e = cudaFuncSetAttribute(kda_chunk_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    kda_chunk_scan_kernel<<<a.num_seqs * a.H * NVT, NT, SMEM_BYTES, st>>>(p);
-    return cudaGetLastError();
+    return launch_after(kda_chunk_scan_kernel, dim3(a.num_seqs * a.H * NVT), NT, SMEM_BYTES, st, p);
 }
 
 }  // namespace kda

@@ -645,6 +645,8 @@ __global__ void __launch_bounds__(NT, SLOW ? 1 : 2) kda_chunk_wy_kernel(const __
     uint64_t* full_bar = reinterpret_cast<uint64_t*>(sm + M::BAR);
     uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(full_bar + 2);
     int* flag_s = reinterpret_cast<int*>(full_bar + 3);
+    pdl_launch_dependents();
+    if (SLOW) pdl_wait();   // the list is complete once the one-reference kernel is
     const int count = SLOW ? *p.slow : 0;
     if (SLOW && (int)blockIdx.x >= count) return;
     if (tid == 0) {
@@ -746,8 +748,7 @@ cudaError_t launch_wy_gate(const WyParams& p, long long slots, int sm_count, cud
     if (e != cudaSuccess) return e;
     const long long jobs = slots * p.H;
     const int grid = (int)(jobs < (long long)sm_count ? jobs : (long long)sm_count);
-    ks<<<grid, NT, wy_smem_bytes<true>(), st>>>(p);
-    return cudaGetLastError();
+    return launch_after(ks, dim3(grid), NT, wy_smem_bytes<true>(), st, p);
 }
 
 }  // namespace

@@ -126,6 +126,25 @@ __device__ __forceinline__ uint4 pack8(const float* v) {
 
 // ------------------------------------------------------------------ host side
 
+// Launch `kern` after the previous work of `st` with programmatic serialization:
+// it may start (prologue) while that work drains and must call pdl_wait() before
+// reading anything the previous kernel writes.
+template <typename Params>
+inline cudaError_t launch_after(void (*kern)(Params), dim3 grid, int block, int smem, cudaStream_t st,
+                                const Params& prm) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, prm);
+}
+
 inline PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     if (!fn) {

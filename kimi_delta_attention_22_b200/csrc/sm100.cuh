@@ -131,6 +131,16 @@ __device__ __forceinline__ void bulk_wait_read() {
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
+// ------------------------------------------------- programmatic dependent launch
+
+// Let the next kernel of the stream (launched with programmatic serialization)
+// begin launching; it still waits in pdl_wait() for this grid's results.
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Wait until the preceding grid has completed and its memory writes are visible.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ------------------------------------------------------------------- tcgen05
 
 // Allocate ncols tensor-memory columns (power of 2, >= 32); one full warp
