@@ -246,9 +246,10 @@ def bench_prefill(args, world, rank, peaks, peak_kind):
     outs = [torch.empty_like(s["v"]) for s in sets]
     STs = [torch.empty(w.B, w.H, w.d_v, w.d_k, dtype=torch.float32, device=dev) for _ in sets]
     # scratch of the two-kernel schedule, allocated once outside the timed region
-    ws = torch.empty(kda.kda_chunk_fwd_workspace_size(sets[0]["q"], sets[0]["v"], sets[0]["g"],
-                                                      chunk=w.chunk),
-                     dtype=torch.uint8, device=dev)
+    # (--schedule fused: no workspace, the single fused kernel)
+    ws = None if args.schedule == "fused" else torch.empty(
+        kda.kda_chunk_fwd_workspace_size(sets[0]["q"], sets[0]["v"], sets[0]["g"], chunk=w.chunk),
+        dtype=torch.uint8, device=dev)
 
     def step(i):
         s = sets[i % n_sets]
@@ -279,9 +280,10 @@ def bench_prefill(args, world, rank, peaks, peak_kind):
     flops = prefill_flops(w)
     achieved_gbs = alg_bytes / (launch_ms * 1e-3) / 1e9
     achieved_tf = flops / (launch_ms * 1e-3) / 1e12
-    src = ["kimi_delta_attention_22_b200/csrc/kda_chunk_wy.cu",
-           "kimi_delta_attention_22_b200/csrc/kda_chunk_scan.cu"]
-    traffic = dram_traffic("chunk_fwd", WORKLOAD, src)
+    src = (["kimi_delta_attention_22_b200/csrc/kda_chunk_tc.cu"] if args.schedule == "fused" else
+           ["kimi_delta_attention_22_b200/csrc/kda_chunk_wy.cu",
+            "kimi_delta_attention_22_b200/csrc/kda_chunk_scan.cu"])
+    traffic = dram_traffic("chunk_fwd_" + args.schedule, WORKLOAD, src)
     res = {
         "w": w, "elapsed_ms": elapsed_ms, "launch_ms": launch_ms,
         "value": world * args.steps * w.tokens / (elapsed_ms * 1e-3),
@@ -289,7 +291,8 @@ def bench_prefill(args, world, rank, peaks, peak_kind):
                      "unit": "GB/s", "frac": achieved_gbs / peaks["hbm_gbs"],
                      "traffic": traffic, "peak_source": f"{peak_kind} hbm_gbs",
                      "algorithmic_bytes_per_launch": alg_bytes,
-                     "kernel": "kda_chunk_fwd kernel"},
+                     "kernel": ("kda_chunk_fwd call (fused kernel)" if args.schedule == "fused"
+                                else "kda_chunk_fwd call (WY, sub-block WY and state-scan kernels)")},
         "tensor": {"achieved_tflops": achieved_tf, "flops_per_launch": flops,
                    "peak_tflops": peaks["bf16_tflops"],
                    "frac": achieved_tf / peaks["bf16_tflops"],
@@ -411,10 +414,12 @@ def run_ours(args, world, rank, local):
                            "l2": "3 rotating input sets (~630 MB) > 126 MB L2"},
                 "roofline": pre["roofline"], "tensor": pre["tensor"], "cpu_baseline": cpu,
                 "e2e": pre["e2e"], "decode": dec, "clocks": clk,
-                # per step: the WY kernel, the (empty when every chunk takes one
-                # reference) sub-block WY kernel and the state scan; plus the job-counter memset
-                "gpu_launches": 3 * args.steps,
-                "schedule": "two-kernel (parallel WY records + sequential state scan)",
+                # per step, two-kernel schedule: the WY kernel, the (empty when every chunk
+                # takes one reference) sub-block WY kernel and the state scan; fused: one kernel
+                "gpu_launches": (1 if args.schedule == "fused" else 3) * args.steps,
+                "schedule": ("fused (one kernel per sequence, head, value tile)"
+                             if args.schedule == "fused" else
+                             "two-kernel (parallel WY records + sequential state scan)"),
                 "kernel_ms_per_launch": pre["launch_ms"]}
         print(json.dumps(line), flush=True)
 
@@ -425,6 +430,8 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--schedule", choices=["split", "fused"], default="split",
+                    help="prefill schedule: two kernels over a workspace (default) or the fused kernel")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
