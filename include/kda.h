@@ -138,6 +138,22 @@ kda_status_t kda_chunk_fwd(const kda_shape_t* shape, const void* q, const void* 
 size_t kda_chunk_fwd_workspace_size(const kda_shape_t* shape, int varlen);
 
 /*
+ * kda_chunk_fwd_noalloc -- kda_chunk_fwd with library-owned scratch.
+ *
+ * Same operation, layouts, support and errors as kda_chunk_fwd, with no
+ * workspace argument: when the shape's workspace fits a 160 MiB scratch
+ * array that the library reserves in device memory at load time (module
+ * static storage; nothing is allocated per call), the two-kernel schedule
+ * runs on it; otherwise the fused kernel runs.  The scratch is shared by
+ * every call in the process: calls on different streams that may overlap
+ * must be ordered by the caller.
+ */
+kda_status_t kda_chunk_fwd_noalloc(const kda_shape_t* shape, const void* q, const void* k,
+                                   const void* v, const float* g, const float* beta,
+                                   const float* S0, const int32_t* cu_seqlens, void* out,
+                                   float* S_T, void* stream);
+
+/*
  * kda_decode_step -- one fused recurrent token for N sequences.
  *
  * The single-token case of the recurrence (the fused recurrent schedule of the

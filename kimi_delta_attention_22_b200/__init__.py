@@ -13,7 +13,7 @@ import os
 
 import torch
 
-__all__ = ["kda_chunk_fwd", "kda_chunk_fwd_workspace_size", "kda_decode_step", "kda_status_str", "library_path", "load_library",
+__all__ = ["kda_chunk_fwd", "kda_chunk_fwd_noalloc", "kda_chunk_fwd_workspace_size", "kda_decode_step", "kda_status_str", "library_path", "load_library",
            "KDAError", "KDA_F32", "KDA_BF16", "KDA_GATE_CHANNEL", "KDA_GATE_SCALAR",
            "KDA_GATE_NONE", "KDA_DEV_BAD_SEQLENS", "KDA_DEV_TIMEOUT", "Shape"]
 
@@ -61,6 +61,8 @@ def load_library(path: str | None = None):
     P = ctypes.c_void_p
     lib.kda_chunk_fwd.argtypes = [ctypes.POINTER(Shape), P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t,
                                   P]
+    lib.kda_chunk_fwd_noalloc.argtypes = [ctypes.POINTER(Shape), P, P, P, P, P, P, P, P, P, P]
+    lib.kda_chunk_fwd_noalloc.restype = ctypes.c_int
     lib.kda_chunk_fwd_workspace_size.argtypes = [ctypes.POINTER(Shape), ctypes.c_int]
     lib.kda_chunk_fwd_workspace_size.restype = ctypes.c_size_t
     lib.kda_chunk_fwd.restype = ctypes.c_int
@@ -159,6 +161,29 @@ def kda_chunk_fwd(q, k, v, g, beta, S0=None, cu_seqlens=None, chunk: int = 64, o
                            ws_bytes, _stream_handle(q.device))
     if st != 0:
         raise KDAError(st, "kda_chunk_fwd")
+    return out, S_T
+
+
+def kda_chunk_fwd_noalloc(q, k, v, g, beta, S0=None, cu_seqlens=None, chunk: int = 64, out=None,
+                          S_T=None, want_state: bool = True, dev_status=None, lib=None):
+    """kda_chunk_fwd_noalloc of include/kda.h: the library's own static scratch
+    instead of a workspace (arguments and results as kda_chunk_fwd)."""
+    _check_cuda(q, k, v, g, beta, S0, cu_seqlens, out, S_T, dev_status)
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    N = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    if out is None:
+        out = torch.empty_like(v)
+    if S_T is None and want_state:
+        S_T = torch.empty(N, H, Dv, Dk, dtype=torch.float32, device=q.device)
+    sh = Shape(B, T, H, Dk, Dv, N, _dtype_code(q.dtype), _gate_code(g, q), int(chunk),
+               None if dev_status is None else dev_status.data_ptr())
+    lib = lib or load_library()
+    st = lib.kda_chunk_fwd_noalloc(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                   _ptr(S0), _ptr(cu_seqlens), _ptr(out), _ptr(S_T),
+                                   _stream_handle(q.device))
+    if st != 0:
+        raise KDAError(st, "kda_chunk_fwd_noalloc")
     return out, S_T
 
 

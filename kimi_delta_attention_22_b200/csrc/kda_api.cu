@@ -12,6 +12,12 @@ bool chunk_tc_supported(int D, int V, int C);
 
 namespace {
 
+// Scratch of kda_chunk_fwd_noalloc: module-static device memory, reserved when
+// the library is loaded; 160 MiB holds the records of 2,200+ (chunk, head)
+// pairs (e.g. 4 sequences x 16 heads x 2048 tokens).
+constexpr size_t kStaticScratchBytes = (size_t)160 << 20;
+static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
+
 bool aligned16(const void* p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void* p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
@@ -98,6 +104,20 @@ kda_status_t kda_chunk_fwd(const kda_shape_t* sh, const void* q, const void* k, 
         return from_cuda(e);
     }
     return from_cuda(tc ? kda::launch_chunk_tc(a, st) : kda::launch_chunk_f32path(a, bf16, st));
+}
+
+kda_status_t kda_chunk_fwd_noalloc(const kda_shape_t* sh, const void* q, const void* k,
+                                   const void* v, const float* g, const float* beta, const float* S0,
+                                   const int32_t* cu_seqlens, void* out, float* S_T, void* stream) {
+    if (sh == nullptr) return KDA_ERR_INVALID_ARG;
+    const size_t need = kda_chunk_fwd_workspace_size(sh, cu_seqlens != nullptr);
+    const bool any = sh->num_seqs > 0 && (long long)sh->B * sh->T > 0;
+    void* ws = nullptr;
+    if (any && need > 0 && need <= kStaticScratchBytes &&
+        cudaGetSymbolAddress(&ws, g_static_scratch) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    return kda_chunk_fwd(sh, q, k, v, g, beta, S0, cu_seqlens, out, S_T, ws,
+                         ws ? kStaticScratchBytes : 0, stream);
 }
 
 kda_status_t kda_decode_step(const kda_shape_t* sh, const void* q, const void* k, const void* v,
