@@ -125,10 +125,26 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_scan_kernel(const __grid_cons
     // everything above overlaps the tail of the WY kernels; records are read below
     pdl_wait();
     first = p.cu_seqlens ? (long long)p.coff[n] : (long long)n * p.nc;
+    constexpr int kAhead = 3;   // records fetched into L2 this many chunks before their copy
+    auto prefetch_chunk = [&](int m) {
+        const uint8_t* src = p.rec + ((size_t)(first + m) * H + h) * rec::BYTES;
+        bulk_prefetch_l2(src + rec::WQ, 57344u);
+        bulk_prefetch_l2(src + rec::U + 8192 * vt, 8192u);
+        bulk_prefetch_l2(src + rec::DEC, 512u);
+    };
     if (tid == kIss) {
         if (nch > 0) load_chunk(0);
         if (nch > 1) load_chunk(1);
+        for (int m = 2; m < nch && m < 2 + kAhead; ++m) prefetch_chunk(m);
     }
+    // Operand descriptors of stage 0; k-step and stage offsets are added in 16-byte
+    // units (every address stays below 256 KB, inside the 14-bit address field).
+    constexpr uint32_t kStage16 = STAGE >> 4;
+    const uint64_t dWQ = rowview_desc(sbase + ST_WQ, 0);          // + (s/4)*64 + (s%4)*2
+    const uint64_t dS = mnmaj_desc(sbase + OFF_S, BV, 0);          // + s*128
+    const uint64_t dKD = mnmaj_desc(sbase + ST_KD, 128, 0);        // + s*256
+    const uint64_t dU = mnmaj_desc(sbase + ST_U, BV, 0);           // + s*128
+    const uint64_t dAQ = kmaj_desc(sbase + ST_KD + 8192, 128, 0);  // + s*2
 
     // Outputs of chunk m (its O2 MMAs complete on bar3): rows live in lanes 64-127.
     auto read_out = [&](long long cp, int Lp, uint32_t col) {
@@ -151,16 +167,16 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_scan_kernel(const __grid_cons
         const int st = m % NSTAGE, par = m & 1;
         const uint32_t full_ph = (uint32_t)((m / NSTAGE) & 1);
         uint8_t* stg = sm + st * STAGE;
-        const uint32_t sstg = sbase + st * STAGE;
         const long long c0 = bos + (long long)m * C;
         const int L = (int)min((long long)C, eos - c0);
         const uint32_t d1 = TM_D1 + 64 * par;
         if (tid == kIss) {
             if (!mbar_wait(full + st, full_ph, kWaitNs)) *flag_s = 1;
             tc_fence_after();
+            const uint64_t so = (uint64_t)(st * kStage16);
 #pragma unroll
             for (int s = 0; s < 8; ++s)
-                mma_bf16(tm + d1, rowview_desc(sstg + ST_WQ, s), mnmaj_desc(sbase + OFF_S, BV, s),
+                mma_bf16(tm + d1, dWQ + so + (uint64_t)((s >> 2) * 64 + (s & 3) * 2), dS + (uint64_t)(s * 128),
                          idesc_bf16(128, BV, false, true), s > 0);
             mma_commit(bar1);
             // the stage of chunk m - 1 is free once its output MMAs are done
@@ -168,6 +184,7 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_scan_kernel(const __grid_cons
                 if (m > 0 && !mbar_wait(bar3, ph3, kWaitNs)) *flag_s = 1;
                 load_chunk(m + 2);
             }
+            if (m + 2 + kAhead < nch) prefetch_chunk(m + 2 + kAhead);
         }
         if (sp >= 2) {
             if (m > 0) {
@@ -200,16 +217,17 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_scan_kernel(const __grid_cons
         if (*flag_s != 0) { aborted = true; m_stop = m; break; }
         if (tid == kIss) {
             tc_fence_after();
+            const uint64_t so = (uint64_t)(st * kStage16);
 #pragma unroll
             for (int s = 0; s < 4; ++s)
-                mma_bf16(tm + TM_DS, mnmaj_desc(sstg + ST_KD, 128, s), mnmaj_desc(sstg + ST_U, BV, s),
+                mma_bf16(tm + TM_DS, dKD + so + (uint64_t)(s * 256), dU + so + (uint64_t)(s * 128),
                          idesc_bf16(128, BV, true, true), s > 0);
             mma_commit(bar2);
             // rows 0-63 of the window are the second half of Kd: their products land in
             // lanes 0-63, which hold nothing that is read again
 #pragma unroll
             for (int s = 0; s < 4; ++s)
-                mma_bf16(tm + d1, kmaj_desc(sstg + ST_KD + 8192, 128, s), mnmaj_desc(sstg + ST_U, BV, s),
+                mma_bf16(tm + d1, dAQ + so + (uint64_t)(s * 2), dU + so + (uint64_t)(s * 128),
                          idesc_bf16(128, BV, false, true), 1);
             mma_commit(bar3);
         }

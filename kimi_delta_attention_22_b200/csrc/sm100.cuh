@@ -117,6 +117,13 @@ __device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int c
                  : "memory");
 }
 
+// Bring `bytes` (multiple of 16, 16-byte aligned) of global memory into L2.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)),
+                 "r"(bytes)
+                 : "memory");
+}
+
 // Untiled bulk copy shared -> global (bulk-group completion; both addresses
 // 16-byte aligned, size a multiple of 16).
 __device__ __forceinline__ void bulk_store(void* dst, const void* src, uint32_t bytes) {
