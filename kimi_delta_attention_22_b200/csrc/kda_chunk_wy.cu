@@ -132,62 +132,27 @@ __device__ __forceinline__ bool decode_slot(const WyParams& p, int slot, long lo
     return L > 0;
 }
 
-// Off-diagonal 16x16 blocks of T = (I + L)^{-1} from its diagonal blocks by a block
-// Neumann series: with D = blockdiag(T_II) and N = D L_off (strictly block-lower,
-// N^4 = 0), T = (I - N + N^2 - N^3) D, i.e. T_IJ = M_IJ T_JJ (I > J) with
-// M = -N + N^2 - N^3.  Four levels of independent 16x16 tf32 products.
-__device__ __forceinline__ void neumann_offdiag(float* TF, const float* Lm, float* NS, int warp,
+// Off-diagonal 16x16 blocks of T = (I + L)^{-1} from its diagonal blocks T_II, one
+// block column per warp (forward substitution by blocks, no CTA barrier inside):
+//   T_IJ = -T_II sum_{K=J}^{I-1} L_IK T_KJ        (I > J),
+// each product a 16x16 warp-level tf32 MMA; P is warp-private scratch.
+__device__ __forceinline__ void offdiag_columns(float* TF, const float* Lm, float* NS, int warp,
                                                 int lane) {
-    auto nb = [&](int idx) { return NS + idx * 16 * LDX; };
     auto tf = [&](int I, int J) { return TF + 16 * I * LDT + 16 * J; };
     auto lb = [&](int I, int J) { return Lm + 16 * I * LDT + 16 * J; };
-    // N blocks: 0:(1,0) 1:(2,0) 2:(3,0) 3:(2,1) 4:(3,1) 5:(3,2); 6: N^2_20, 7: N^2_31,
-    // 8: N^2_30, 9: N^3_30
-    if (warp < 6) {
-        const int I = (warp < 3) ? warp + 1 : ((warp < 5) ? warp - 1 : 3);
-        const int K = (warp < 3) ? 0 : ((warp < 5) ? 1 : 2);
-        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-        blk_mma(acc, tf(I, I), LDT, lb(I, K), LDT, lane);
-        blk_store(nb(warp), LDX, acc, lane, 1.f);
-    }
-    __syncthreads();
-    if (warp < 6) {
-        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-        if (warp < 3) {   // T_{J+1,J} = -N_{J+1,J} T_JJ
-            const int J = warp, nidx = (J == 0) ? 0 : ((J == 1) ? 3 : 5);
-            blk_mma(acc, nb(nidx), LDX, tf(J, J), LDT, lane);
-            blk_store(tf(J + 1, J), LDT, acc, lane, -1.f);
-        } else if (warp == 3) {   // N^2_20 = N_21 N_10
-            blk_mma(acc, nb(3), LDX, nb(0), LDX, lane);
-            blk_store(nb(6), LDX, acc, lane, 1.f);
-        } else if (warp == 4) {   // N^2_31 = N_32 N_21
-            blk_mma(acc, nb(5), LDX, nb(3), LDX, lane);
-            blk_store(nb(7), LDX, acc, lane, 1.f);
-        } else {                  // N^2_30 = N_31 N_10 + N_32 N_20
-            blk_mma(acc, nb(4), LDX, nb(0), LDX, lane);
-            blk_mma(acc, nb(5), LDX, nb(1), LDX, lane);
-            blk_store(nb(8), LDX, acc, lane, 1.f);
-        }
-    }
-    __syncthreads();
     if (warp < 3) {
-        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-        if (warp == 0) {          // T_20 = (N^2_20 - N_20) T_00
-            blk_mma2(acc, nb(6), 1.f, nb(1), -1.f, nullptr, 0.f, LDX, tf(0, 0), LDT, lane);
-            blk_store(tf(2, 0), LDT, acc, lane, 1.f);
-        } else if (warp == 1) {   // T_31 = (N^2_31 - N_31) T_11
-            blk_mma2(acc, nb(7), 1.f, nb(4), -1.f, nullptr, 0.f, LDX, tf(1, 1), LDT, lane);
-            blk_store(tf(3, 1), LDT, acc, lane, 1.f);
-        } else {                  // N^3_30 = N_32 N^2_20
-            blk_mma(acc, nb(5), LDX, nb(6), LDX, lane);
-            blk_store(nb(9), LDX, acc, lane, 1.f);
+        const int J = warp;
+        float* P = NS + warp * 16 * LDX;
+        for (int I = J + 1; I < 4; ++I) {
+            float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            for (int K = J; K < I; ++K) blk_mma(acc, lb(I, K), LDT, tf(K, J), LDT, lane);
+            blk_store(P, LDX, acc, lane, 1.f);
+            __syncwarp();
+            float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            blk_mma(acc2, tf(I, I), LDT, P, LDX, lane);
+            blk_store(tf(I, J), LDT, acc2, lane, -1.f);
+            __syncwarp();
         }
-    }
-    __syncthreads();
-    if (warp == 0) {              // T_30 = (N^2_30 - N_30 - N^3_30) T_00
-        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-        blk_mma2(acc, nb(8), 1.f, nb(2), -1.f, nb(9), -1.f, LDX, tf(0, 0), LDT, lane);
-        blk_store(tf(3, 0), LDT, acc, lane, 1.f);
     }
     __syncthreads();
 }
@@ -197,7 +162,7 @@ __device__ __forceinline__ void neumann_offdiag(float* TF, const float* Lm, floa
 // bounded wait expired (everything in flight has been waited for again).
 template <int GATE, bool SLOW>
 __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t tm, int slot, int h,
-                                      uint32_t& full_phase, uint32_t& mma_phase) {
+                                      uint32_t& full_phase, uint32_t& mma_phase, uint32_t& v_phase) {
     using M = WyMap<SLOW>;
     const int H = p.H;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -206,6 +171,7 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
     const uint32_t sbase = smem_u32(sm);
     uint64_t* full_bar = reinterpret_cast<uint64_t*>(sm + M::BAR);
     uint64_t* mma_bar = full_bar + 1;
+    uint64_t* v_bar = full_bar + 4;   // the V tiles, needed only by the U MMAs
     volatile int* flag_s = reinterpret_cast<volatile int*>(full_bar + 3);
     float* tot4 = reinterpret_cast<float*>(sm + M::TOT4);
     float* gref_s = reinterpret_cast<float*>(sm + M::GREF);
@@ -220,11 +186,20 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
 
     // Uniform bounded wait: on expiry every thread leaves with `false` after
     // waiting once more for the same phase (copies / MMAs still in flight).
+    bool v_pending = false;   // the V copy is in flight (every exit waits for it)
+    auto wait_v = [&]() {
+        if (v_pending) {
+            if (!mbar_wait(v_bar, v_phase, kWaitNs)) *flag_s = 1;
+            v_phase ^= 1u;
+            v_pending = false;
+        }
+    };
     auto wait_all = [&](uint64_t* bar, uint32_t& phase) -> bool {
         if (!mbar_wait(bar, phase, kWaitNs)) *flag_s = 1;
         __syncthreads();
         if (*flag_s != 0) {
             (void)mbar_wait(bar, phase, kWaitNs);
+            wait_v();
             if (p.dev_status && tid == 0) atomicOr(p.dev_status, KDA_DEV_TIMEOUT);
             return false;
         }
@@ -233,14 +208,15 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
     };
 
     if (tid == 0) {
-        // K, Q (16 KB each), V (two 8 KB tiles), per-channel g (32 KB)
-        const uint32_t bytes = 16384u * 3u + (GATE == KDA_GATE_CHANNEL ? 32768u : 0u);
+        // K, Q (16 KB each), per-channel g (32 KB); V (two 8 KB tiles) on its own barrier
+        const uint32_t bytes = 16384u * 2u + (GATE == KDA_GATE_CHANNEL ? 32768u : 0u);
         mbar_arrive_expect_tx(full_bar, bytes);
         tma_load_3d(sm + M::RK, &p.map_k, full_bar, 0, h, (int)c0);
         tma_load_3d(sm + M::RQ, &p.map_q, full_bar, 0, h, (int)c0);
-        tma_load_3d(sm + M::RV, &p.map_v, full_bar, 0, h, (int)c0);
-        tma_load_3d(sm + M::RV + 8192, &p.map_v, full_bar, 64, h, (int)c0);
         if (GATE == KDA_GATE_CHANNEL) tma_load_3d(sm + M::RG, &p.map_g, full_bar, 0, h, (int)c0);
+        mbar_arrive_expect_tx(v_bar, 16384u);
+        tma_load_3d(sm + M::RV, &p.map_v, v_bar, 0, h, (int)c0);
+        tma_load_3d(sm + M::RV + 8192, &p.map_v, v_bar, 64, h, (int)c0);
         if (!SLOW) {
             // the job that starts one resident wave later (blocks start in linear order):
             // its tiles go to L2 now, so that its own loads hit there
@@ -258,6 +234,7 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
             }
         }
     }
+    v_pending = true;
     const float beta_pf = (tid < L) ? p.beta[(size_t)(c0 + tid) * H + h] : 0.f;
     if (!wait_all(full_bar, full_phase)) return 2;
 
@@ -334,6 +311,7 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
             const int pos = atomicAdd(p.slow, 1);
             p.slow[1 + pos] = slot * H + h;
         }
+        wait_v();          // no copy may land after the CTA is gone
         __syncthreads();   // the scratch of this job is read no more
         return 1;
     }
@@ -471,6 +449,10 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
     // rows 64-127 that of version 2g+1; B rows the i-side rows of sub-blocks 2g, 2g+1
     if (tid == 0) {
         if (!SLOW) {
+            // Qg and Kd images to the record; their shared-memory reads overlap the MMA issue
+            bulk_store(g_wq + 16384, sm + M::KQG + 16384, 16384u);
+            bulk_store(g_kd, sm + M::KDST, 16384u);
+            bulk_commit();
 #pragma unroll
             for (int s8 = 0; s8 < 8; ++s8)
                 mma_bf16(tm + TM_GRAM, rowview_desc(sbase + M::KQG, s8), rowview_desc(sbase + M::KYG, s8),
@@ -485,12 +467,7 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
                              kmaj_desc(ox + g * 8192, 128, s8), idesc_bf16(128, 64, false, false), s8 > 0);
         }
         mma_commit(mma_bar);
-        if (!SLOW) {   // Qg and Kd images to the record while the Gram runs
-            bulk_store(g_wq + 16384, sm + M::KQG + 16384, 16384u);
-            bulk_store(g_kd, sm + M::KDST, 16384u);
-            bulk_commit();
-            bulk_wait_read();   // both are overwritten once the Gram is read out
-        }
+        if (!SLOW) bulk_wait_read();   // both images are overwritten once the Gram is read out
     }
     if (!wait_all(mma_bar, mma_phase)) return 2;
     tc_fence_after();
@@ -567,7 +544,7 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
     }
     if (tid == 0) bulk_wait_read();   // the staging is overwritten from here on
     __syncthreads();
-    neumann_offdiag(TF, Lm, reinterpret_cast<float*>(sm + M::NS), warp, lane);
+    offdiag_columns(TF, Lm, reinterpret_cast<float*>(sm + M::NS), warp, lane);
     // T diag(beta) -> bf16 (K-major, K = j), 8 columns per step
     for (int e = tid; e < C * 8; e += NT) {
         const int i = e >> 3, j0 = 8 * (e & 7);
@@ -588,6 +565,7 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
     tc_fence_after();
     // ================= W = T diag(beta) K e^G (M = 64, N = 128, lanes 0-15 of each
     // sub-partition) and U = T diag(beta) V (two M = 64, N = 64 tiles, lanes 16-31)
+    wait_v();   // V landed long ago; every thread observes it before its tiles are MMA operands
     if (tid == 0) {
         const uint32_t tb = sbase + M::TB;
 #pragma unroll
@@ -652,6 +630,7 @@ __global__ void __launch_bounds__(NT, SLOW ? 1 : 2) kda_chunk_wy_kernel(const __
     if (tid == 0) {
         mbar_init(full_bar, 1);
         mbar_init(full_bar + 1, 1);
+        mbar_init(full_bar + 4, 1);
         *flag_s = 0;
         fence_mbar_init();
     }
@@ -663,13 +642,13 @@ __global__ void __launch_bounds__(NT, SLOW ? 1 : 2) kda_chunk_wy_kernel(const __
     __syncthreads();
     tc_fence_after();
     const uint32_t tm = *tmem_base_s;
-    uint32_t full_phase = 0, mma_phase = 0;
+    uint32_t full_phase = 0, mma_phase = 0, v_phase = 0;
     if (!SLOW) {
-        (void)wy_job<GATE, false>(p, sm, tm, blockIdx.x, blockIdx.y, full_phase, mma_phase);
+        (void)wy_job<GATE, false>(p, sm, tm, blockIdx.x, blockIdx.y, full_phase, mma_phase, v_phase);
     } else {
         for (int x = blockIdx.x; x < count; x += gridDim.x) {
             const int job = p.slow[1 + x];
-            if (wy_job<GATE, true>(p, sm, tm, job / p.H, job % p.H, full_phase, mma_phase) == 2) break;
+            if (wy_job<GATE, true>(p, sm, tm, job / p.H, job % p.H, full_phase, mma_phase, v_phase) == 2) break;
         }
     }
     if (tid == 0) bulk_wait_read();   // shared memory outlives no store that reads it
