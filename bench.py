@@ -30,6 +30,8 @@ if ROOT not in sys.path:
 
 import torch
 
+from kimi_delta_attention_22_b200.roofline import prefill_bytes, prefill_flops
+
 METRIC = "KDA prefill tokens/s (% bf16 TC peak); decode step HBM GB/s (% of peak)"
 WORKLOAD = "prefill_b4_h16_t2048"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -44,29 +46,6 @@ def load_peaks():
             d = json.load(f)
         return d, "measured"
     return dict(FALLBACK_PEAKS), "fallback"
-
-
-def prefill_bytes(w, tokens_per_seq=None):
-    """Algorithmic HBM bytes of one kda_chunk_fwd launch: every input read once,
-    every output written once."""
-    ht = w.B * w.T * w.H
-    el = 2 if w.dtype == "bf16" else 4
-    g = {"channel": 4 * w.d_k, "scalar": 4, "none": 0}[w.gate_mode]
-    per_ht = el * (2 * w.d_k + w.d_v) + g + 4 + el * w.d_v
-    states = w.B * w.H * w.d_v * w.d_k * 4 * ((1 if w.s0_std is not None else 0) + 1)
-    return ht * per_ht + states
-
-
-def prefill_flops(w):
-    """Algorithmic FLOPs of the chunkwise form (multiply-add = 2), counting the
-    causal halves of the in-chunk products; per head-token at chunk C:
-    A_kk, A_qk: 2 * C*d_k (half of C^2 d_k * 2 each, per token: C*d_k);
-    W = T (beta K) and U = T (beta V): C*d_k + C*d_v; E = U - W S^T: 2 d_k d_v;
-    O = Q S^T + A_qk E: 2 d_k d_v + C d_v; S update: 2 d_k d_v; triangular solve C^2/3."""
-    C, dk, dv = w.chunk, w.d_k, w.d_v
-    per_ht = (2 * C * dk) + (C * dk + C * dv) + 2 * dk * dv + (2 * dk * dv + C * dv) + \
-        2 * dk * dv + C * C / 3.0
-    return w.B * w.T * w.H * per_ht
 
 
 def source_sha(paths):

@@ -236,6 +236,11 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
     }
     v_pending = true;
     const float beta_pf = (tid < L) ? p.beta[(size_t)(c0 + tid) * H + h] : 0.f;
+    // One gate value per token (or none) in the one-reference kernel: the decay is a
+    // per-row factor, so the cumulative sum runs over 64 values instead of 64 x 128.
+    constexpr bool ROWGATE = !SLOW && GATE != KDA_GATE_CHANNEL;
+    const float gsc_pf = (ROWGATE && GATE == KDA_GATE_SCALAR && tid < L)
+                             ? p.g[(size_t)(c0 + tid) * H + h] * kLog2e : 0.f;
     if (!wait_all(full_bar, full_phase)) return 2;
 
     // ================= log-space decay: thread tile = channels c8..c8+7 of rows 4 rg .. 4 rg + 3
@@ -250,7 +255,10 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
         const int i = 4 * rg + r;
         const bool valid = i < L;
         float gv[8];
-        if (GATE == KDA_GATE_CHANNEL) {
+        if (ROWGATE) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) gv[e] = 0.f;   // handled per row below
+        } else if (GATE == KDA_GATE_CHANNEL) {
             const float4 a0 = *reinterpret_cast<const float4*>(sm + M::RG + (i * DK + c8) * 4);
             const float4 a1 = *reinterpret_cast<const float4*>(sm + M::RG + (i * DK + c8 + 4) * 4);
             gv[0] = a0.x; gv[1] = a0.y; gv[2] = a0.z; gv[3] = a0.w;
@@ -272,13 +280,46 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
         kraw[r] = valid ? *reinterpret_cast<const uint4*>(sm + M::RK + (i * DK + c8) * 2) : z4;
         qraw[r] = valid ? *reinterpret_cast<const uint4*>(sm + M::RQ + (i * DK + c8) * 2) : z4;
     }
-    *reinterpret_cast<float4*>(tot4 + rg * DK + c8) = make_float4(run[0], run[1], run[2], run[3]);
-    *reinterpret_cast<float4*>(tot4 + rg * DK + c8 + 4) = make_float4(run[4], run[5], run[6], run[7]);
+    if (!ROWGATE) {
+        *reinterpret_cast<float4*>(tot4 + rg * DK + c8) = make_float4(run[0], run[1], run[2], run[3]);
+        *reinterpret_cast<float4*>(tot4 + rg * DK + c8 + 4) = make_float4(run[4], run[5], run[6], run[7]);
+    }
     if (tid < C) beta_s[tid] = beta_pf;
+    float* rowf = tot4;        // per-row gate factors 2^{Gamma_i}, 2^{-Gamma_i} (ROWGATE)
+    float* rowi = tot4 + C;
+    float* red = reinterpret_cast<float*>(sm + M::RED);
+    if (ROWGATE && GATE == KDA_GATE_SCALAR) {
+        // inclusive scan of the per-token log2 decay over the 64 rows (two warps)
+        float x = gsc_pf;
+        if (tid < C) {
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += y;
+            }
+            if (lane == 31) red[warp] = x;
+        }
+        __syncthreads();
+        if (tid < C) {
+            if (warp == 1) x += red[0];
+            rowf[tid] = ex2(x);
+            rowi[tid] = ex2(-x);   // only used when the chunk takes one reference
+            if (tid == C - 1) red[2] = x;
+        }
+    }
     __syncthreads();   // raw K / Q / g are consumed; their space now takes operands
+    if (ROWGATE) {
+        const float glast = (GATE == KDA_GATE_SCALAR) ? red[2] : 0.f;
+        fast = -glast <= kFastLimit2;
+        if (tid < DK) {
+            const float d = (GATE == KDA_GATE_SCALAR) ? ex2(glast) : 1.f;
+            dec_s[tid] = d;
+            reinterpret_cast<float*>(rec_p + rec::DEC)[tid] = d;
+        }
+    }
     // exclusive prefix over the 16 row groups, one thread per channel; the reference
     // row of sub-block b is row 16 b + 7 (prefix before group 4 b + 2)
-    if (tid < DK) {
+    if (!ROWGATE && tid < DK) {
         float tv[16];
 #pragma unroll
         for (int q = 0; q < 16; ++q) tv[q] = tot4[q * DK + tid];
@@ -302,10 +343,7 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
         if (lane == 0) reinterpret_cast<float*>(sm + M::RED)[warp] = m;
     }
     __syncthreads();
-    {
-        const float* red = reinterpret_cast<const float*>(sm + M::RED);
-        fast = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3])) <= kFastLimit2;
-    }
+    if (!ROWGATE) fast = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3])) <= kFastLimit2;
     if (!SLOW && !fast) {
         if (tid == 0) {
             const int pos = atomicAdd(p.slow, 1);
@@ -320,7 +358,33 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
     // the 16-byte chunks of this thread: (row 4 rg + r, channels c8..c8+7) in the
     // mnmaj_off(c, row, 128) layout shared by K e^G, Q~ e^G, K e^{-G} and Kd
     const uint32_t basemn = (uint32_t)((rg >> 1) * 2048 + (cq >> 3) * 1024 + (rg & 1) * 512);
-    if (!SLOW) {
+    if (ROWGATE) {
+        // ================= one reference, one decay per row: factors from the row scan
+        const float dd = dec_s[0];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const int i = 4 * rg + r;
+            const uint32_t omn =
+                basemn + (((uint32_t)(cq & 7) ^ (uint32_t)(4 * (rg & 1) + r)) << 4) + (uint32_t)(r * 128);
+            const float eg = (GATE == KDA_GATE_SCALAR) ? rowf[i] : 1.f;
+            const float ey = (GATE == KDA_GATE_SCALAR) ? rowi[i] : 1.f;
+            const float qs = p.scale * eg, kd = dd * ey;
+            float kf[8], qf[8], t1[8], t2[8], t3[8], t4[8];
+            unpack8(kraw[r], kf);
+            unpack8(qraw[r], qf);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                t1[e] = kf[e] * eg;
+                t2[e] = qf[e] * qs;
+                t3[e] = kf[e] * ey;
+                t4[e] = kf[e] * kd;
+            }
+            st_shared_v4(sm + M::KQG, omn, pack8(t1));
+            st_shared_v4(sm + M::KQG, omn + 16384, pack8(t2));
+            st_shared_v4(sm + M::KYG, omn, pack8(t3));
+            st_shared_v4(sm + M::KDST, omn, pack8(t4));
+        }
+    } else if (!SLOW) {
         // ================= one reference: 2^{Gamma_i} <= 1 on the i-side, 2^{-Gamma_j} <= 2^112 on the j-side
         float pre[8], dec[8];
         {

@@ -1,0 +1,97 @@
+"""Time kda_chunk_fwd on the named synthetic workloads (one GPU).
+
+    python -m kimi_delta_attention_22_b200.measure [--workloads a,b,...] [--schedule split|fused]
+                                                   [--iters 10] [--warmup 3]
+
+For each workload: inputs drawn once on the device (kimi_delta_attention_22_b200.inputs),
+the two-kernel schedule's workspace allocated once, `warmup` untimed calls, then `iters`
+calls timed one by one with CUDA events on the current stream; the median is reported
+with tokens/s, the algorithmic HBM bytes and FLOPs of kimi_delta_attention_22_b200.roofline
+and their fractions of MEASURED_PEAKS.json (repository root) when that file exists.
+Inputs of the prefill and sweep workloads exceed the 126 MB L2, so consecutive calls do
+not re-read them from L2; the small fp32 case is listed for completeness only.
+One JSON line per workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+
+import torch
+
+import kimi_delta_attention_22_b200 as kda
+from kimi_delta_attention_22_b200 import inputs
+from kimi_delta_attention_22_b200.roofline import prefill_bytes, prefill_flops
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        return json.load(f)
+
+
+def measure(name: str, schedule: str, iters: int, warmup: int) -> dict:
+    w = inputs.WORKLOADS[name]
+    d = inputs.workload_inputs(w, device="cuda")
+    cu = d.get("cu_seqlens")
+    ws = None
+    if schedule == "split":
+        n = kda.kda_chunk_fwd_workspace_size(d["q"], d["v"], d["g"], cu_seqlens=cu, chunk=w.chunk)
+        ws = torch.empty(n, dtype=torch.uint8, device="cuda") if n else None
+    out = torch.empty_like(d["v"])
+    N = w.num_seqs if w.varlen else w.B
+    S_T = torch.empty(N, w.H, w.d_v, w.d_k, dtype=torch.float32, device="cuda")
+
+    def call():
+        kda.kda_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], S0=d["S0"], cu_seqlens=cu,
+                          chunk=w.chunk, out=out, S_T=S_T, workspace=ws if ws is not None else False)
+
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    times = []
+    for _ in range(iters):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        call()
+        b.record(stream)
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    ms = statistics.median(times)
+    nbytes, flops = prefill_bytes(w), prefill_flops(w)
+    res = {"workload": name, "schedule": schedule, "ms_per_call": ms,
+           "tokens_per_s": w.tokens / (ms * 1e-3), "hbm_gbs": nbytes / (ms * 1e-3) / 1e9,
+           "tflops": flops / (ms * 1e-3) / 1e12, "algorithmic_bytes": nbytes, "flops": flops,
+           "iters": iters}
+    pk = peaks()
+    if pk:
+        res["hbm_frac"] = res["hbm_gbs"] / pk["hbm_gbs"]
+        res["tc_frac"] = res["tflops"] / pk["bf16_tflops"]
+    del d, ws, out, S_T
+    torch.cuda.empty_cache()
+    return res
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--workloads", default=",".join(n for n in inputs.WORKLOADS))
+    ap.add_argument("--schedule", choices=["split", "fused"], default="split")
+    ap.add_argument("--iters", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    args = ap.parse_args()
+    if not torch.cuda.is_available():
+        raise SystemExit("measure needs a CUDA device")
+    kda.load_library()
+    for name in args.workloads.split(","):
+        print(json.dumps(measure(name, args.schedule, args.iters, args.warmup)), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,29 @@
+"""Algorithmic work of one kda_chunk_fwd call on a named workload, the
+numerators of the roofline fractions that bench.py and measure.py report.
+
+Bytes: every input read once and every output written once (per head-token
+q, k, v, out at the input element size, g at 4 bytes per channel / per token /
+none, beta 4 bytes; S0 and S_T at 4 bytes per state element per sequence).
+FLOPs (multiply-add = 2): the chunkwise form at chunk C, counting only the
+causal halves of the in-chunk products."""
+from __future__ import annotations
+
+
+def prefill_bytes(w) -> int:
+    ht = w.B * w.T * w.H
+    el = 2 if w.dtype == "bf16" else 4
+    g = {"channel": 4 * w.d_k, "scalar": 4, "none": 0}[w.gate_mode]
+    per_ht = el * (2 * w.d_k + w.d_v) + g + 4 + el * w.d_v
+    seqs = w.num_seqs if w.varlen else w.B
+    states = seqs * w.H * w.d_v * w.d_k * 4 * ((1 if w.s0_std is not None else 0) + 1)
+    return ht * per_ht + states
+
+
+def prefill_flops(w) -> float:
+    """Per head-token at chunk C: A_kk and A_qk 2*C*d_k (causal halves); W and U
+    C*(d_k + d_v); E = U - W S^T 2*d_k*d_v; O = Q S^T + A_qk E 2*d_k*d_v + C*d_v;
+    state update 2*d_k*d_v; triangular solve C^2/3."""
+    C, dk, dv = w.chunk, w.d_k, w.d_v
+    per_ht = (2 * C * dk) + (C * dk + C * dv) + 2 * dk * dv + (2 * dk * dv + C * dv) + \
+        2 * dk * dv + C * C / 3.0
+    return w.B * w.T * w.H * per_ht
