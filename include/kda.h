@@ -173,6 +173,31 @@ kda_status_t kda_decode_step(const kda_shape_t* shape, const void* q, const void
                              const void* v, const float* g, const float* beta, float* S,
                              void* out, void* stream);
 
+/*
+ * kda_recurrent_fwd -- fused recurrent pass over a short run of tokens.
+ *
+ * The token loop of the recurrence for N sequences of T tokens each, with the
+ * state kept in registers across the tokens: S is read from HBM once and
+ * written once per call (the multi-token form of the fused recurrent decode
+ * schedule, GeekNews summary, section "fused recurrent kernel for decode";
+ * suited to short runs -- speculative tokens, short prefills -- where the
+ * chunkwise schedule has too few tokens per chunk).  The result equals
+ * kda_chunk_fwd with S0 = S_T = S up to floating-point rounding, and equals T
+ * calls of kda_decode_step exactly.
+ *
+ * Layouts (dense batch, N = shape->B, shape->num_seqs must equal N):
+ *   q, k   [N, T, H, d_k] dtype      v, out [N, T, H, d_v] dtype
+ *   g      [N, T, H, d_k] fp32 (CHANNEL) | [N, T, H] fp32 (SCALAR) | NULL (NONE)
+ *   beta   [N, T, H] fp32
+ *   S      [N, H, d_v, d_k] fp32, read and overwritten with the state after the T tokens.
+ * Alignment: q, k, per-channel g and S 16 bytes; v, out, beta, scalar g 4 bytes.
+ * Support: d_k = 128 (bf16 or fp32), any d_v from 1 to 65535*32; T = 0 leaves S as is.
+ * Else KDA_ERR_UNSUPPORTED.
+ */
+kda_status_t kda_recurrent_fwd(const kda_shape_t* shape, const void* q, const void* k,
+                               const void* v, const float* g, const float* beta, float* S,
+                               void* out, void* stream);
+
 /* Human-readable text for a status code (static storage). */
 const char* kda_status_str(kda_status_t status);
 

@@ -13,7 +13,7 @@ import os
 
 import torch
 
-__all__ = ["kda_chunk_fwd", "kda_chunk_fwd_noalloc", "kda_chunk_fwd_workspace_size", "kda_decode_step", "kda_status_str", "library_path", "load_library",
+__all__ = ["kda_chunk_fwd", "kda_recurrent_fwd", "kda_chunk_fwd_noalloc", "kda_chunk_fwd_workspace_size", "kda_decode_step", "kda_status_str", "library_path", "load_library",
            "KDAError", "KDA_F32", "KDA_BF16", "KDA_GATE_CHANNEL", "KDA_GATE_SCALAR",
            "KDA_GATE_NONE", "KDA_DEV_BAD_SEQLENS", "KDA_DEV_TIMEOUT", "Shape"]
 
@@ -67,6 +67,8 @@ def load_library(path: str | None = None):
     lib.kda_chunk_fwd_workspace_size.restype = ctypes.c_size_t
     lib.kda_chunk_fwd.restype = ctypes.c_int
     lib.kda_decode_step.argtypes = [ctypes.POINTER(Shape), P, P, P, P, P, P, P, P]
+    lib.kda_recurrent_fwd.argtypes = [ctypes.POINTER(Shape), P, P, P, P, P, P, P, P]
+    lib.kda_recurrent_fwd.restype = ctypes.c_int
     lib.kda_decode_step.restype = ctypes.c_int
     lib.kda_status_str.argtypes = [ctypes.c_int]
     lib.kda_status_str.restype = ctypes.c_char_p
@@ -215,4 +217,27 @@ def kda_decode_step(q, k, v, g, beta, S, out=None, lib=None):
                              _ptr(S), _ptr(out), _stream_handle(q.device))
     if st != 0:
         raise KDAError(st, "kda_decode_step")
+    return out
+
+
+def kda_recurrent_fwd(q, k, v, g, beta, S, out=None, lib=None):
+    """Fused recurrent KDA over T tokens per sequence (kda_recurrent_fwd of include/kda.h).
+
+    q, k [N,T,H,d_k]; v [N,T,H,d_v]; g [N,T,H,d_k] | [N,T,H] | None (fp32 log-decay);
+    beta [N,T,H] fp32; S [N,H,d_v,d_k] fp32, read once and overwritten with the state
+    after the T tokens.  Returns out [N,T,H,d_v].
+    """
+    _check_cuda(q, k, v, g, beta, S, out)
+    N, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    if S.shape != (N, H, Dv, Dk) or S.dtype != torch.float32:
+        raise ValueError("S must be float32 [N, H, d_v, d_k]")
+    if out is None:
+        out = torch.empty_like(v)
+    sh = Shape(N, T, H, Dk, Dv, N, _dtype_code(q.dtype), _gate_code(g, q), 0, None)
+    lib = lib or load_library()
+    st = lib.kda_recurrent_fwd(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                               _ptr(S), _ptr(out), _stream_handle(q.device))
+    if st != 0:
+        raise KDAError(st, "kda_recurrent_fwd")
     return out

@@ -120,6 +120,31 @@ kda_status_t kda_chunk_fwd_noalloc(const kda_shape_t* sh, const void* q, const v
                          ws ? kStaticScratchBytes : 0, stream);
 }
 
+kda_status_t kda_recurrent_fwd(const kda_shape_t* sh, const void* q, const void* k, const void* v,
+                               const float* g, const float* beta, float* S, void* out, void* stream) {
+    if (sh == nullptr) return KDA_ERR_INVALID_ARG;
+    const int N = sh->B, T = sh->T, H = sh->H, D = sh->d_k, V = sh->d_v;
+    if (N < 0 || T < 0 || H <= 0 || D <= 0 || V <= 0 || sh->num_seqs != N) return KDA_ERR_INVALID_ARG;
+    if (sh->dtype != KDA_F32 && sh->dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+    if (sh->gate != KDA_GATE_CHANNEL && sh->gate != KDA_GATE_SCALAR && sh->gate != KDA_GATE_NONE)
+        return KDA_ERR_INVALID_ARG;
+    if ((sh->gate == KDA_GATE_NONE) != (g == nullptr)) return KDA_ERR_INVALID_ARG;
+    if (N > 0 && (!S || (T > 0 && (!q || !k || !v || !beta || !out)))) return KDA_ERR_INVALID_ARG;
+    const bool g_vec = sh->gate == KDA_GATE_CHANNEL;
+    if (!aligned16(q) || !aligned16(k) || !aligned4(v) || !(g_vec ? aligned16(g) : aligned4(g)) ||
+        !aligned4(beta) || !aligned16(S) || !aligned4(out))
+        return KDA_ERR_MISALIGNED;
+    if (D != 128 || V > 65535 * 32) return KDA_ERR_UNSUPPORTED;
+    if ((long long)N * H > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+    if (N == 0 || T == 0) return KDA_OK;
+
+    kda::RecurrentArgs a;
+    a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.S = S; a.out = out;
+    a.N = N; a.T = T; a.H = H; a.d_k = D; a.d_v = V; a.gate = sh->gate;
+    a.scale = 1.0f / sqrtf((float)D);
+    return from_cuda(kda::launch_recurrent(a, sh->dtype == KDA_BF16, static_cast<cudaStream_t>(stream)));
+}
+
 kda_status_t kda_decode_step(const kda_shape_t* sh, const void* q, const void* k, const void* v,
                              const float* g, const float* beta, float* S, void* out,
                              void* stream) {

@@ -39,6 +39,20 @@ struct DecodeArgs {
     float scale;
 };
 
+// Multi-token recurrent pass (dense batch: N sequences of T tokens each).
+struct RecurrentArgs {
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* g;
+    const float* beta;
+    float* S;
+    void* out;
+    int N, T, H, d_k, d_v, gate;
+    float scale;
+};
+
+cudaError_t launch_recurrent(const RecurrentArgs& a, bool bf16, cudaStream_t s);
 cudaError_t launch_chunk_f32path(const ChunkArgs& a, bool bf16, cudaStream_t s);
 cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t s);
 // Two-kernel tensor-core prefill over a caller workspace laid out by rec::layout().

@@ -2,6 +2,7 @@
 
     python -m kimi_delta_attention_22_b200.measure [--workloads a,b,...] [--schedule split|fused]
                                                    [--iters 10] [--warmup 3]
+    python -m kimi_delta_attention_22_b200.measure --recurrent [--tokens 1,4,16,64]
 
 For each workload: inputs drawn once on the device (kimi_delta_attention_22_b200.inputs),
 the two-kernel schedule's workspace allocated once, `warmup` untimed calls, then `iters`
@@ -11,6 +12,11 @@ and their fractions of MEASURED_PEAKS.json (repository root) when that file exis
 Inputs of the prefill and sweep workloads exceed the 126 MB L2, so consecutive calls do
 not re-read them from L2; the small fp32 case is listed for completeness only.
 One JSON line per workload.
+
+--recurrent times kda_recurrent_fwd at the decode workload's shape (256 sequences,
+32 heads, d = 128, bf16, per-channel gates) for each token count T, next to T calls
+of kda_decode_step on the same inputs, with the algorithmic bytes of
+roofline.recurrent_bytes (state read once and written once per call).
 """
 from __future__ import annotations
 
@@ -23,7 +29,7 @@ import torch
 
 import kimi_delta_attention_22_b200 as kda
 from kimi_delta_attention_22_b200 import inputs
-from kimi_delta_attention_22_b200.roofline import prefill_bytes, prefill_flops
+from kimi_delta_attention_22_b200.roofline import prefill_bytes, prefill_flops, recurrent_bytes
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -79,16 +85,68 @@ def measure(name: str, schedule: str, iters: int, warmup: int) -> dict:
     return res
 
 
+def _time(fn, iters: int, warmup: int) -> float:
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    times = []
+    for _ in range(iters):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    return statistics.median(times)
+
+
+def measure_recurrent(T: int, iters: int, warmup: int, N: int = 256, H: int = 32) -> dict:
+    d = inputs.draw(N, T, H, 128, 128, dtype=torch.bfloat16, gate="channel", s0_std=0.05, seed=7,
+                    device="cuda")
+    S = d["S0"].clone()
+    out = torch.empty_like(d["v"])
+    steps = [{k: d[k][:, t].contiguous() for k in ("q", "k", "v", "g", "beta")} for t in range(T)]
+    step_out = torch.empty(N, H, 128, dtype=torch.bfloat16, device="cuda")
+
+    def fused():
+        kda.kda_recurrent_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], S, out=out)
+
+    def per_token():
+        for st in steps:
+            kda.kda_decode_step(st["q"], st["k"], st["v"], st["g"], st["beta"], S, out=step_out)
+
+    ms = _time(fused, iters, warmup)
+    ms_steps = _time(per_token, iters, warmup)
+    nbytes = recurrent_bytes(N, T, H, 128, 128)
+    res = {"kernel": "kda_recurrent_fwd", "N": N, "H": H, "T": T, "ms_per_call": ms,
+           "tokens_per_s": N * T / (ms * 1e-3), "hbm_gbs": nbytes / (ms * 1e-3) / 1e9,
+           "algorithmic_bytes": nbytes, "decode_steps_ms": ms_steps,
+           "speedup_vs_decode_steps": ms_steps / ms, "iters": iters}
+    pk = peaks()
+    if pk:
+        res["hbm_frac"] = res["hbm_gbs"] / pk["hbm_gbs"]
+    del d, S, out, steps
+    torch.cuda.empty_cache()
+    return res
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--workloads", default=",".join(n for n in inputs.WORKLOADS))
     ap.add_argument("--schedule", choices=["split", "fused"], default="split")
     ap.add_argument("--iters", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--recurrent", action="store_true")
+    ap.add_argument("--tokens", default="1,4,16,64")
     args = ap.parse_args()
     if not torch.cuda.is_available():
         raise SystemExit("measure needs a CUDA device")
     kda.load_library()
+    if args.recurrent:
+        for T in (int(x) for x in args.tokens.split(",")):
+            print(json.dumps(measure_recurrent(T, args.iters, args.warmup)), flush=True)
+        return
     for name in args.workloads.split(","):
         print(json.dumps(measure(name, args.schedule, args.iters, args.warmup)), flush=True)
 

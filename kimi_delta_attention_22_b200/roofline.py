@@ -27,3 +27,11 @@ def prefill_flops(w) -> float:
     per_ht = (2 * C * dk) + (C * dk + C * dv) + 2 * dk * dv + (2 * dk * dv + C * dv) + \
         2 * dk * dv + C * C / 3.0
     return w.B * w.T * w.H * per_ht
+
+
+def recurrent_bytes(N: int, T: int, H: int, d_k: int, d_v: int, el: int = 2, gate: str = "channel") -> int:
+    """Algorithmic HBM bytes of one kda_recurrent_fwd call: the fp32 state read
+    once and written once, plus every token's q, k, v, out (el bytes), g and beta."""
+    g = {"channel": 4 * d_k, "scalar": 4, "none": 0}[gate]
+    per_ht = el * (2 * d_k + 2 * d_v) + g + 4
+    return 2 * N * H * d_v * d_k * 4 + N * T * H * per_ht
