@@ -134,7 +134,7 @@ kda_status_t kda_recurrent_fwd(const kda_shape_t* sh, const void* q, const void*
     if (!aligned16(q) || !aligned16(k) || !aligned4(v) || !(g_vec ? aligned16(g) : aligned4(g)) ||
         !aligned4(beta) || !aligned16(S) || !aligned4(out))
         return KDA_ERR_MISALIGNED;
-    if (D != 128 || V > 65535 * 32) return KDA_ERR_UNSUPPORTED;
+    if (D != 128 || V > 65535 * 128) return KDA_ERR_UNSUPPORTED;
     if ((long long)N * H > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
     if (N == 0 || T == 0) return KDA_OK;
 

@@ -7,13 +7,16 @@
 // summary, section "fused recurrent kernel for decode").
 //
 // Every state row r (value index) evolves independently given the token
-// vectors, so the work layout follows the decode kernel's: a CTA owns 32 rows
-// of one (n, h) state, each warp 4 rows, one row per 8-lane group (few
-// registers, so two CTAs share an SM and hide each other's latency); lane
-// (l & 7) holds key columns 4(l & 7) + 32m, m = 0..3.  Per token:
+// vectors, so the work layout follows the decode kernel's: a CTA owns 128
+// rows of one (n, h) state, each warp 16, four at a time, one row per 8-lane
+// group; lane (l & 7) holds key columns 4(l & 7) + 32m, m = 0..3.  Per token:
 //     sd = S_r Diag(alpha_t); a = sd.k_t; b = sd.q~_t; e = beta_t (v_tr - a)
 //     S_r <- sd + e k_t;      o_tr = b + e (k_t . q~_t)
-// The next token's vectors are loaded while the current one is processed.
+// The token vectors alpha_t = exp(g_t), k_t, q~_t, beta_t and this CTA's
+// entries of v_t are formed once per CTA in shared memory (double-buffered:
+// the next token's are staged while the current one is processed); each lane
+// reads its 16 channels of them.  The per-row arithmetic, including the
+// k_t.q~_t partial sums, is the decode kernel's, operation for operation.
 #include "kda_internal.cuh"
 
 namespace kda {
@@ -21,67 +24,51 @@ namespace {
 
 constexpr int kDK = 128;           // key head size handled by this kernel
 constexpr int kThreads = 256;      // 8 warps
-constexpr int kIt = 1;             // rows per 8-lane group
+constexpr int kIt = 4;             // rows per 8-lane group
 constexpr int kRowsPerCta = 8 * 4 * kIt;
+static_assert(kRowsPerCta == 128 && kThreads == 2 * kDK, "staging assigns one channel / row per thread");
 
-__device__ __forceinline__ void load4(const float* p, float* x) {
-    const float4 t = __ldg(reinterpret_cast<const float4*>(p));
-    x[0] = t.x; x[1] = t.y; x[2] = t.z; x[3] = t.w;
-}
-__device__ __forceinline__ void load4(const __nv_bfloat16* p, float* x) {
-    const uint2 t = __ldg(reinterpret_cast<const uint2*>(p));
-    const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&t.x);
-    const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&t.y);
-    const float2 a = __bfloat1622float2(lo), b = __bfloat1622float2(hi);
-    x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
-}
-
-// One token's operands as this lane sees them.
-template <typename TI>
-struct TokenRegs {
-    float k[16], q[16], g[16], v[kIt];
-    float beta;
+struct Stage {
+    float al[kDK], k[kDK], qs[kDK], v[kRowsPerCta];
+    float beta, pad[3];
 };
 
 template <typename TI, int GATE>
-__device__ __forceinline__ void load_token(const RecurrentArgs& a, size_t tok_h, const int* rows, int sub,
-                                           TokenRegs<TI>& t) {
-    const TI* kp = static_cast<const TI*>(a.k) + tok_h * kDK;
-    const TI* qp = static_cast<const TI*>(a.q) + tok_h * kDK;
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-        const int c = 32 * m + 4 * sub;
-        load4(kp + c, t.k + 4 * m);
-        load4(qp + c, t.q + 4 * m);
-        if (GATE == KDA_GATE_CHANNEL) load4(a.g + tok_h * kDK + c, t.g + 4 * m);
-    }
-    if (GATE == KDA_GATE_SCALAR) {
-        const float s = __ldg(a.g + tok_h);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) t.g[j] = s;
-    }
-    t.beta = __ldg(a.beta + tok_h);
-    const TI* vp = static_cast<const TI*>(a.v) + tok_h * a.d_v;
-#pragma unroll
-    for (int it = 0; it < kIt; ++it) t.v[it] = rows[it] < a.d_v ? to_f32(vp[rows[it]]) : 0.f;
-}
-
-template <typename TI, int GATE>
 __global__ void __launch_bounds__(kThreads, 2) kda_recurrent_kernel(RecurrentArgs a) {
+    __shared__ __align__(16) Stage stg[2];
     const int nh = blockIdx.x;
     const int n = nh / a.H, h = nh - n * a.H;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int sub = lane & 7, rsel = lane >> 3;
-    int rows[kIt];
-#pragma unroll
-    for (int it = 0; it < kIt; ++it) rows[it] = blockIdx.y * kRowsPerCta + warp * (4 * kIt) + rsel + 4 * it;
+    const int rbase = blockIdx.y * kRowsPerCta;
+    const int row0 = rbase + warp * (4 * kIt) + rsel;
+
+    // Stage token t into buffer b: threads 0-127 own channel tid, 128-255 row tid - 128.
+    const size_t tok0 = (size_t)n * a.T;
+    auto stage = [&](int t, int b) {
+        const size_t th = (tok0 + t) * a.H + h;
+        Stage& st = stg[b];
+        if (tid < kDK) {
+            float gc = 0.f;
+            if (GATE == KDA_GATE_CHANNEL) gc = __ldg(a.g + th * kDK + tid);
+            else if (GATE == KDA_GATE_SCALAR) gc = __ldg(a.g + th);
+            st.al[tid] = (GATE == KDA_GATE_NONE) ? 1.f : expf(gc);
+            st.k[tid] = to_f32(static_cast<const TI*>(a.k)[th * kDK + tid]);
+            st.qs[tid] = to_f32(static_cast<const TI*>(a.q)[th * kDK + tid]) * a.scale;
+            if (tid == 0) st.beta = __ldg(a.beta + th);
+        } else {
+            const int r = rbase + tid - kDK;
+            st.v[tid - kDK] = r < a.d_v ? to_f32(static_cast<const TI*>(a.v)[th * a.d_v + r]) : 0.f;
+        }
+    };
 
     float* Sbase = a.S + (size_t)nh * a.d_v * kDK;
     float s[kIt][16];
 #pragma unroll
     for (int it = 0; it < kIt; ++it) {
-        if (rows[it] < a.d_v) {
-            const float* rowp = Sbase + (size_t)rows[it] * kDK + 4 * sub;
+        const int r = row0 + 4 * it;
+        if (r < a.d_v) {
+            const float* rowp = Sbase + (size_t)r * kDK + 4 * sub;
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
                 const float4 t = __ldcs(reinterpret_cast<const float4*>(rowp + 32 * m));
@@ -93,33 +80,42 @@ __global__ void __launch_bounds__(kThreads, 2) kda_recurrent_kernel(RecurrentArg
             for (int j = 0; j < 16; ++j) s[it][j] = 0.f;
         }
     }
+    if (a.T > 0) stage(0, 0);
+    __syncthreads();
 
-    TokenRegs<TI> cur, nxt;
-    const size_t tok0 = (size_t)n * a.T;
-    if (a.T > 0) load_token<TI, GATE>(a, tok0 * a.H + h, rows, sub, cur);
     TI* out = static_cast<TI*>(a.out);
     for (int t = 0; t < a.T; ++t) {
-        if (t + 1 < a.T) load_token<TI, GATE>(a, (tok0 + t + 1) * a.H + h, rows, sub, nxt);
-        float al[16], qs[16];
+        const int b = t & 1;
+        if (t + 1 < a.T) stage(t + 1, b ^ 1);   // its loads overlap the work below
+        const Stage& st = stg[b];
+        float al[16], kr[16], qr[16];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const int c = 32 * m + 4 * sub;
+            const float4 x = *reinterpret_cast<const float4*>(st.al + c);
+            const float4 y = *reinterpret_cast<const float4*>(st.k + c);
+            const float4 z = *reinterpret_cast<const float4*>(st.qs + c);
+            al[4 * m] = x.x; al[4 * m + 1] = x.y; al[4 * m + 2] = x.z; al[4 * m + 3] = x.w;
+            kr[4 * m] = y.x; kr[4 * m + 1] = y.y; kr[4 * m + 2] = y.z; kr[4 * m + 3] = y.w;
+            qr[4 * m] = z.x; qr[4 * m + 1] = z.y; qr[4 * m + 2] = z.z; qr[4 * m + 3] = z.w;
+        }
         float kq = 0.f;
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            al[j] = (GATE == KDA_GATE_NONE) ? 1.f : expf(cur.g[j]);
-            qs[j] = cur.q[j] * a.scale;
-            kq = fmaf(cur.k[j], qs[j], kq);
-        }
+        for (int j = 0; j < 16; ++j) kq = fmaf(kr[j], qr[j], kq);
         kq += __shfl_xor_sync(0xffffffffu, kq, 1);
         kq += __shfl_xor_sync(0xffffffffu, kq, 2);
         kq += __shfl_xor_sync(0xffffffffu, kq, 4);
+        const float beta = st.beta;
         const size_t orow = ((tok0 + t) * a.H + h) * a.d_v;
 #pragma unroll
         for (int it = 0; it < kIt; ++it) {
+            const int r = row0 + 4 * it;
             float pa = 0.f, pb = 0.f;
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 s[it][j] *= al[j];
-                pa = fmaf(s[it][j], cur.k[j], pa);
-                pb = fmaf(s[it][j], qs[j], pb);
+                pa = fmaf(s[it][j], kr[j], pa);
+                pb = fmaf(s[it][j], qr[j], pb);
             }
             pa += __shfl_xor_sync(0xffffffffu, pa, 1);
             pb += __shfl_xor_sync(0xffffffffu, pb, 1);
@@ -127,18 +123,19 @@ __global__ void __launch_bounds__(kThreads, 2) kda_recurrent_kernel(RecurrentArg
             pb += __shfl_xor_sync(0xffffffffu, pb, 2);
             pa += __shfl_xor_sync(0xffffffffu, pa, 4);
             pb += __shfl_xor_sync(0xffffffffu, pb, 4);
-            const float e = cur.beta * (cur.v[it] - pa);
+            const float e = beta * (st.v[r - rbase] - pa);
 #pragma unroll
-            for (int j = 0; j < 16; ++j) s[it][j] = fmaf(e, cur.k[j], s[it][j]);
-            if (sub == 0 && rows[it] < a.d_v) out[orow + rows[it]] = from_f32<TI>(fmaf(e, kq, pb));
+            for (int j = 0; j < 16; ++j) s[it][j] = fmaf(e, kr[j], s[it][j]);
+            if (sub == 0 && r < a.d_v) out[orow + r] = from_f32<TI>(fmaf(e, kq, pb));
         }
-        cur = nxt;
+        __syncthreads();   // buffer b is re-staged next iteration; b ^ 1 is complete
     }
 
 #pragma unroll
     for (int it = 0; it < kIt; ++it) {
-        if (rows[it] < a.d_v) {
-            float* rowp = Sbase + (size_t)rows[it] * kDK + 4 * sub;
+        const int r = row0 + 4 * it;
+        if (r < a.d_v) {
+            float* rowp = Sbase + (size_t)r * kDK + 4 * sub;
 #pragma unroll
             for (int m = 0; m < 4; ++m)
                 __stcs(reinterpret_cast<float4*>(rowp + 32 * m),
