@@ -87,7 +87,8 @@ constexpr int OFF_SMALL = OFF_S + 16384;
 constexpr int OFF_BETA = OFF_SMALL;              // fp32 [64]
 constexpr int OFF_DECAY = OFF_BETA + 256;        // fp32 [2][128] e^{Gamma_last} (by chunk parity)
 constexpr int OFF_BAR = OFF_DECAY + 1024;        // mbarriers + tmem base + flags
-constexpr int SMEM_USED = OFF_BAR + 64;
+constexpr int OFF_DQ = OFF_BAR + 64;             // fp32 [64] d_k^{-1/2} q_i . k_i (exact)
+constexpr int SMEM_USED = OFF_DQ + 256;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;     // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory over the sm_100 per-block limit");
 static_assert(OFF_NS + 10 * 16 * LDX * 4 <= OFF_A + 65536, "phase-3 scratch overflows region A");
@@ -121,6 +122,7 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
     const uint32_t lane_base = (uint32_t)(32 * sp) << 16;
 
     float* tot4 = reinterpret_cast<float*>(sm + OFF_TOT4);
+    float* dq_s = reinterpret_cast<float*>(sm + OFF_DQ);
     float* gref_s = reinterpret_cast<float*>(sm + OFF_GREF);
     float* glast_s = reinterpret_cast<float*>(sm + OFF_GLAST);
     float* beta_s = reinterpret_cast<float*>(sm + OFF_BETA);
@@ -285,6 +287,20 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
             *reinterpret_cast<float4*>(tot4 + rg * DK + c8) = make_float4(run[0], run[1], run[2], run[3]);
             *reinterpret_cast<float4*>(tot4 + rg * DK + c8 + 4) = make_float4(run[4], run[5], run[6], run[7]);
             if (tid < C) beta_s[tid] = beta_pf;
+            // The diagonal of lower(Qp) is the undecayed q~_i . k_i; formed from the raw
+            // inputs in fp32 (through the decayed bf16 operands the cancellation in the
+            // channel sum would amplify their rounding).
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                float kf[8], qf[8], acc = 0.f;
+                unpack8(kraw[r], kf);
+                unpack8(qraw[r], qf);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc = fmaf(kf[e], qf[e], acc);
+#pragma unroll
+                for (int o = 1; o < 16; o <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+                if (cq == 0) dq_s[4 * rg + r] = acc * a.scale;
+            }
             __syncthreads();   // raw K/Q/G are consumed; their space now takes operands
             // exclusive prefix over the 16 row groups, one thread per channel; the
             // reference row of sub-block b is row 16 b + 7 (prefix before group 4 b + 2)
@@ -517,11 +533,15 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
                         }
                     } else {
                         const int i = n - 64;
+                        const float dii = dq_s[i];
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
                             float t8[8];
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) t8[e] = (j0 + 8 * q + e <= i) ? -v[8 * q + e] : 0.f;
+                            for (int e = 0; e < 8; ++e) {
+                                const int j = j0 + 8 * q + e;
+                                t8[e] = (j < i) ? -v[8 * q + e] : ((j == i) ? dii : 0.f);
+                            }
                             st_shared_v4(sm + OFF_AQB, kmaj_off(i, j0 + 8 * q, 64), pack8(t8));
                         }
                     }
@@ -548,7 +568,7 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
             for (int u = 0; u < 16; ++u) {
                 const int i = 16 * I + u;
                 Lm[i * LDT + j] = (j < i) ? bi[u] * v[u] : 0.f;
-                Q32[i * LDT + j] = (j <= i) ? v[16 + u] : 0.f;
+                Q32[i * LDT + j] = (j < i) ? v[16 + u] : ((j == i) ? dq_s[i] : 0.f);
             }
         }
         tc_fence_before();

@@ -65,7 +65,8 @@ struct WyMap<false> {                          // one-reference chunks, two CTAs
     static constexpr int OX = 0, OY = 0, AQS = 0;   // sub-block path only
     static constexpr int AQST = TB;            // bf16 lower(Qp) staging (before T diag(beta) exists)
     static constexpr int WST = L, UST = L + 16384;   // after the W/U MMAs: record images of W, U
-    static constexpr int DECS = RED + 64, BETA = DECS + 512, BAR = BETA + 256, END = BAR + 64;
+    static constexpr int DECS = RED + 64, BETA = DECS + 512, BAR = BETA + 256, DQS = BAR + 64;
+    static constexpr int END = DQS + 256;
     static_assert(NS + 10 * 16 * LDX * 4 <= RV, "phase-3 scratch overflows into V");
     static_assert(TB + 8192 <= DECS, "T diag(beta) overlaps live scratch");
 };
@@ -86,7 +87,8 @@ struct WyMap<true> {                           // sub-block references, one CTA 
     static constexpr int AQST = AQS;
     static constexpr int WST = A, UST = A + 16384;   // after the W/U MMAs: record images of W, U
     static_assert(UST + 16384 <= AQS, "W/U staging overlaps the lower(Qp) staging");
-    static constexpr int DECS = TB + 8192, BETA = DECS + 512, BAR = BETA + 256, END = BAR + 64;
+    static constexpr int DECS = TB + 8192, BETA = DECS + 512, BAR = BETA + 256, DQS = BAR + 64;
+    static constexpr int END = DQS + 256;
     static_assert(AQS + 8192 <= A + 65536, "phase-3 scratch overflows region A");
 };
 template <bool SLOW>
@@ -178,6 +180,7 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
     float* glast_s = reinterpret_cast<float*>(sm + M::GLAST);
     float* dec_s = reinterpret_cast<float*>(sm + M::DECS);
     float* beta_s = reinterpret_cast<float*>(sm + M::BETA);
+    float* dq_s = reinterpret_cast<float*>(sm + M::DQS);   // d_k^{-1/2} q_i . k_i, exact in fp32
 
     long long c0;
     int L;
@@ -284,6 +287,19 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
         *reinterpret_cast<float4*>(tot4 + rg * DK + c8) = make_float4(run[0], run[1], run[2], run[3]);
         *reinterpret_cast<float4*>(tot4 + rg * DK + c8 + 4) = make_float4(run[4], run[5], run[6], run[7]);
     }
+    // The diagonal of lower(Qp) is the undecayed q~_i . k_i.  Through the decayed bf16
+    // operands it would carry their rounding amplified by the cancellation in the
+    // channel sum, so the operand loops below also form it from the raw inputs in fp32.
+    float dqp[4];
+    auto store_dq = [&]() {   // all threads; 16 threads share a row
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            float acc = dqp[r];
+#pragma unroll
+            for (int o = 1; o < 16; o <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+            if (cq == 0) dq_s[4 * rg + r] = acc * p.scale;
+        }
+    };
     if (tid < C) beta_s[tid] = beta_pf;
     float* rowf = tot4;        // per-row gate factors 2^{Gamma_i}, 2^{-Gamma_i} (ROWGATE)
     float* rowi = tot4 + C;
@@ -372,8 +388,10 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
             float kf[8], qf[8], t1[8], t2[8], t3[8], t4[8];
             unpack8(kraw[r], kf);
             unpack8(qraw[r], qf);
+            dqp[r] = 0.f;
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
+                dqp[r] = fmaf(kf[e], qf[e], dqp[r]);
                 t1[e] = kf[e] * eg;
                 t2[e] = qf[e] * qs;
                 t3[e] = kf[e] * ey;
@@ -403,8 +421,10 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
             float kf[8], qf[8], t1[8], t2[8], t3[8], t4[8];
             unpack8(kraw[r], kf);
             unpack8(qraw[r], qf);
+            dqp[r] = 0.f;
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
+                dqp[r] = fmaf(kf[e], qf[e], dqp[r]);
                 const float gm = pre[e] + g2[r][e];   // Gamma_i (log2), <= 0
                 const float eg = ex2(gm), ey = ex2(-gm);
                 t1[e] = kf[e] * eg;                    // K e^{Gamma}
@@ -461,8 +481,10 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
             float kf[8], qf[8], x[8], y[8], t[8];
             unpack8(kraw[r], kf);
             unpack8(qraw[r], qf);
+            dqp[r] = 0.f;
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
+                dqp[r] = fmaf(kf[e], qf[e], dqp[r]);
                 const float dl = (pre[e] + g2[r][e]) - gr[e];   // Gamma_i - Gamma_r (log2)
                 x[e] = ex2(dl);
                 y[e] = ex2(-dl);
@@ -503,6 +525,7 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
             *reinterpret_cast<uint4*>(g_kd + omn) = pack8(t);
         }
     }
+    store_dq();
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -557,11 +580,15 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
             }
         } else {
             const int i = n - 64;
+            const float dii = dq_s[i];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 float t8[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) t8[e] = (j0 + 8 * q + e <= i) ? v[8 * q + e] : 0.f;
+                for (int e = 0; e < 8; ++e) {
+                    const int j = j0 + 8 * q + e;
+                    t8[e] = (j < i) ? v[8 * q + e] : ((j == i) ? dii : 0.f);
+                }
                 st_shared_v4(sm + M::AQST, kmaj_off(i, j0 + 8 * q, 64), pack8(t8));
             }
         }
@@ -577,7 +604,7 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
         for (int u = 0; u < 16; ++u) {
             const int i = 16 * I + u;
             Lm[i * LDT + j] = (j < i) ? beta_s[i] * v[u] : 0.f;
-            aqs[kmaj_off(i, j, 64) >> 1] = __float2bfloat16_rn((j <= i) ? v[16 + u] : 0.f);
+            aqs[kmaj_off(i, j, 64) >> 1] = __float2bfloat16_rn((j < i) ? v[16 + u] : ((j == i) ? dq_s[i] : 0.f));
         }
     }
     fence_async_smem();
