@@ -25,3 +25,29 @@ def pytest_collection_modifyitems(config, items):
     for it in items:
         if "gpu" in it.keywords:
             it.add_marker(skip)
+
+
+# KDA_PARITY_REPORT=<file>: write every parity check's error figure and its
+# tolerance, per test, as JSON (the largest margin used is the number to watch).
+_REPORT = {}
+
+
+@pytest.fixture(autouse=True)
+def _parity_record(request):
+    yield
+    if not os.environ.get("KDA_PARITY_REPORT") or "parity" not in sys.modules:
+        return
+    rec = sys.modules["parity"].RECORD
+    if rec:
+        _REPORT[request.node.nodeid] = [
+            {"what": w, "mode": m, "error": e, "tol": t} for (w, m, e, t) in rec]
+        rec.clear()
+
+
+def pytest_sessionfinish(session, exitstatus):
+    path = os.environ.get("KDA_PARITY_REPORT")
+    if path and _REPORT:
+        import json
+
+        with open(path, "w") as f:
+            json.dump(_REPORT, f, indent=1)

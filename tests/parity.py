@@ -55,9 +55,14 @@ def err(got, ref, mode, stored_bf16=None):
     return max(rel_rms, elem / ELEM_FACTOR)
 
 
+# Every check's figure, for the optional per-test error report (conftest.py).
+RECORD: list[tuple[str, str, float, float]] = []
+
+
 def check(got, ref, mode, what, stored_bf16=None):
     e = err(got, ref, mode, stored_bf16)
     tol = TOL_F32_ABS if mode == "f32" else TOL_BF16_REL
+    RECORD.append((what, mode, e, tol))
     assert e <= tol, f"{what}: error {e:.3e} > {tol:.1e} ({'max abs' if mode == 'f32' else 'rms-relative'})"
     return e
 
