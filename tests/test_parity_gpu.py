@@ -70,6 +70,20 @@ def test_bf16(B, T, H, gate, beta, s0, chunk, schedule):
     check(ST, rs, "bf16", "S_T")
 
 
+@pytest.mark.parametrize("gate", ["channel", "channel_strong"])
+def test_whole_width_scan_matches_oracle(gate):
+    """More (sequence, head) pairs than SMs take the whole-width (N = 128) state
+    scan: 2 x 90 heads, ragged 130-token sequences, one- and sub-block-reference
+    chunks; every pair against the oracle."""
+    props = torch.cuda.get_device_properties(0)
+    B, T, H = 2, 130, max(90, props.multi_processor_count // 2 + 1)
+    d = inputs.draw(B, T, H, 128, 128, dtype=torch.bfloat16, gate=gate, s0_std=0.02, seed=4242)
+    out, ST = run_chunk(d, 64)
+    ro, rs = oracle_chunk(d, "channel")
+    check(out, ro, "bf16", "out")
+    check(ST, rs, "bf16", "S_T")
+
+
 @pytest.mark.parametrize("schedule", ["split", "fused"])
 def test_varlen_small_ragged_and_empty(schedule):
     """Packed sequences of lengths 0, 1, 64, 65, 127, 200 (state restarts per
