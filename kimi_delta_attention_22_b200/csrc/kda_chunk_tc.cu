@@ -287,20 +287,10 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
             *reinterpret_cast<float4*>(tot4 + rg * DK + c8) = make_float4(run[0], run[1], run[2], run[3]);
             *reinterpret_cast<float4*>(tot4 + rg * DK + c8 + 4) = make_float4(run[4], run[5], run[6], run[7]);
             if (tid < C) beta_s[tid] = beta_pf;
-            // The diagonal of lower(Qp) is the undecayed q~_i . k_i; formed from the raw
-            // inputs in fp32 (through the decayed bf16 operands the cancellation in the
-            // channel sum would amplify their rounding).
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                float kf[8], qf[8], acc = 0.f;
-                unpack8(kraw[r], kf);
-                unpack8(qraw[r], qf);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) acc = fmaf(kf[e], qf[e], acc);
-#pragma unroll
-                for (int o = 1; o < 16; o <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-                if (cq == 0) dq_s[4 * rg + r] = acc * a.scale;
-            }
+            // The diagonal of lower(Qp) is the undecayed q~_i . k_i.  Through the decayed
+            // bf16 operands the cancellation in the channel sum would amplify their
+            // rounding, so the operand loops below also form it from the raw inputs in fp32.
+            float dqp[4];
             __syncthreads();   // raw K/Q/G are consumed; their space now takes operands
             // exclusive prefix over the 16 row groups, one thread per channel; the
             // reference row of sub-block b is row 16 b + 7 (prefix before group 4 b + 2)
@@ -348,8 +338,10 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
                     float kf[8], qf[8], t1[8], t2[8], t3[8], t4[8];
                     unpack8(kraw[r], kf);
                     unpack8(qraw[r], qf);
+                    dqp[r] = 0.f;
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
+                        dqp[r] = fmaf(kf[e], qf[e], dqp[r]);
                         const float gm = pre[e] + g2[r][e];   // Gamma_i (log2), <= 0
                         const float eg = ex2(gm), ey = ex2(-gm);
                         t1[e] = kf[e] * eg;                    // K e^{Gamma}
@@ -406,8 +398,10 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
                     float kf[8], qf[8], x[8], y[8], t[8];
                     unpack8(kraw[r], kf);
                     unpack8(qraw[r], qf);
+                    dqp[r] = 0.f;
     #pragma unroll
                     for (int e = 0; e < 8; ++e) {
+                        dqp[r] = fmaf(kf[e], qf[e], dqp[r]);
                         const float dl = (pre[e] + g2[r][e]) - gr[e];   // Gamma_i - Gamma_r (log2)
                         x[e] = ex2(dl);
                         y[e] = ex2(-dl);
@@ -447,6 +441,13 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
                     for (int e = 0; e < 8; ++e) t[e] = kf[e] * (Lr[e] * y[e]);
                     st_shared_v4(sm + OFF_KD + par * 16384, omn, pack8(t));
                 }
+            }
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {   // 16 threads share a row
+                float acc = dqp[r];
+#pragma unroll
+                for (int o = 1; o < 16; o <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+                if (cq == 0) dq_s[4 * rg + r] = acc * a.scale;
             }
         }
         fence_async_smem();
