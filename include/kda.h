@@ -191,7 +191,8 @@ kda_status_t kda_decode_step(const kda_shape_t* shape, const void* q, const void
  *   beta   [N, T, H] fp32
  *   S      [N, H, d_v, d_k] fp32, read and overwritten with the state after the T tokens.
  * Alignment: q, k, per-channel g and S 16 bytes; v, out, beta, scalar g 4 bytes.
- * Support: d_k = 128 (bf16 or fp32), any d_v from 1 to 65535*128; T = 0 leaves S as is.
+ * Support: d_k = 128 (bf16 or fp32), any d_v from 1 to 65535*128; T = 0 leaves S as is;
+ * T = 1 runs the decode step's kernel (the same arithmetic, at the state-copy rate).
  * Else KDA_ERR_UNSUPPORTED.
  */
 kda_status_t kda_recurrent_fwd(const kda_shape_t* shape, const void* q, const void* k,

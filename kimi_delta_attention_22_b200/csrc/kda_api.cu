@@ -137,6 +137,15 @@ kda_status_t kda_recurrent_fwd(const kda_shape_t* sh, const void* q, const void*
     if (D != 128 || V > 65535 * 128) return KDA_ERR_UNSUPPORTED;
     if ((long long)N * H > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
     if (N == 0 || T == 0) return KDA_OK;
+    if (T == 1) {
+        // one token per sequence: [N, 1, H, .] is the decode step's [N, H, .] layout, and its
+        // kernel streams the state at the copy rate (the two are the same arithmetic)
+        kda::DecodeArgs d;
+        d.q = q; d.k = k; d.v = v; d.g = g; d.beta = beta; d.S = S; d.out = out;
+        d.N = N; d.H = H; d.d_k = D; d.d_v = V; d.gate = sh->gate;
+        d.scale = 1.0f / sqrtf((float)D);
+        return from_cuda(kda::launch_decode(d, sh->dtype == KDA_BF16, static_cast<cudaStream_t>(stream)));
+    }
 
     kda::RecurrentArgs a;
     a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.S = S; a.out = out;
