@@ -44,7 +44,7 @@ def bind(path: str):
     """Load a compiled oracle library and declare its C signatures."""
     lib = ctypes.CDLL(path)
     P = ctypes.c_void_p
-    lib.kda_oracle_forward.argtypes = [ctypes.c_int, P, P, ctypes.c_int, ctypes.c_int,
+    lib.kda_oracle_forward.argtypes = [ctypes.c_int, P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                        ctypes.c_int, ctypes.c_int, P, P, P, P, P, P, P, P,
                                        ctypes.c_int]
     lib.kda_oracle_forward.restype = ctypes.c_int
@@ -80,10 +80,12 @@ def forward(q, k, v, g, beta, S0=None, cu_seqlens=None, gate="channel", want_sta
             nthreads: int = 0, lib=None):
     """Run the float64 KDA recurrence.
 
-    Dense layout (cu_seqlens None): q,k [B,T,H,dk]; v [B,T,H,dv]; g [B,T,H,dk]
+    Dense layout (cu_seqlens None): q,k [B,T,Hk,dk]; v [B,T,H,dv]; g [B,T,H,dk]
     (channel) / [B,T,H] (scalar) / None (none); beta [B,T,H]; S0 [B,H,dv,dk] or
     None.  Varlen layout: leading batch of 1 (or none), cu_seqlens [N+1] offsets
-    into the packed token axis; S0 [N,H,dv,dk].
+    into the packed token axis; S0 [N,H,dv,dk].  H is the number of value heads
+    and a multiple of Hk: value head h reads query/key head h // (H // Hk)
+    (Hk == H is the plain one-to-one case).
 
     Returns (out [same lead shape as v], S_T [num_seqs,H,dv,dk] or None), float64.
     Inputs are converted to float64 exactly (bf16 and fp32 both embed in fp64).
@@ -91,7 +93,9 @@ def forward(q, k, v, g, beta, S0=None, cu_seqlens=None, gate="channel", want_sta
     gate_mode = _GATE_NAMES[gate] if isinstance(gate, str) else int(gate)
     q, k, v, g, beta, S0 = (_f64(a) for a in (q, k, v, g, beta, S0))
     lead = v.shape[:-2]
-    H, dk, dv = q.shape[-2], q.shape[-1], v.shape[-1]
+    H, Hk, dk, dv = v.shape[-2], q.shape[-2], q.shape[-1], v.shape[-1]
+    if k.shape != q.shape or H % Hk != 0:
+        raise ValueError(f"q/k heads {q.shape[-2]} must divide the value heads {H}")
     if cu_seqlens is None:
         B, T = (1, lead[0]) if len(lead) == 1 else lead
         starts = np.arange(B, dtype=np.int64) * T
@@ -111,7 +115,7 @@ def forward(q, k, v, g, beta, S0=None, cu_seqlens=None, gate="channel", want_sta
         raise ValueError(f"S0 shape {S0.shape} != {(N, H, dv, dk)}")
     if lens.size and int((starts + lens).max()) > rows:
         raise ValueError("sequence extends past the token axis")
-    rc = (lib or _load()).kda_oracle_forward(N, _ptr(starts), _ptr(lens), H, dk, dv, gate_mode,
+    rc = (lib or _load()).kda_oracle_forward(N, _ptr(starts), _ptr(lens), H, Hk, dk, dv, gate_mode,
                                     _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0),
                                     _ptr(out), _ptr(ST), int(nthreads))
     if rc != 0:

@@ -40,10 +40,11 @@
 
 enum { ORACLE_GATE_CHANNEL = 0, ORACLE_GATE_SCALAR = 1, ORACLE_GATE_NONE = 2 };
 
-/* One (sequence, head) pair: walk its tokens in order.
+/* One (sequence, value head) pair: walk its tokens in order.
  * Token t of the pair lives at packed row (start + t); every per-token array
- * is [rows, H, width] row-major. */
-static void oracle_one_pair(int64_t start, int64_t len, int h, int H, int dk, int dv,
+ * is [rows, heads, width] row-major: q and k have Hk heads (value head h reads
+ * q/k head hk), v, g, beta and the state have H. */
+static void oracle_one_pair(int64_t start, int64_t len, int h, int H, int hk, int Hk, int dk, int dv,
                             int gate_mode, const double* q, const double* k,
                             const double* v, const double* g, const double* beta,
                             const double* S0 /* dv*dk or NULL */, double* out,
@@ -56,8 +57,8 @@ static void oracle_one_pair(int64_t start, int64_t len, int h, int H, int dk, in
 
     for (int64_t t = 0; t < len; ++t) {
         const int64_t row = start + t;
-        const double* kt = k + (row * H + h) * dk;
-        const double* qt = q + (row * H + h) * dk;
+        const double* kt = k + (row * Hk + hk) * dk;
+        const double* qt = q + (row * Hk + hk) * dk;
         const double* vt = v + (row * H + h) * dv;
         const double bt = beta[row * H + h];
 
@@ -96,7 +97,9 @@ static void oracle_one_pair(int64_t start, int64_t len, int h, int H, int dk, in
  * kda_oracle_forward: run the recurrence over num_seqs packed sequences.
  *   seq_start[n], seq_len[n] : token rows [seq_start[n], seq_start[n]+seq_len[n])
  *                              of the packed token axis belong to sequence n.
- *   q, k : [rows, H, dk]     v, out : [rows, H, dv]
+ *   q, k : [rows, Hk, dk]    v, out : [rows, H, dv]
+ *   H a multiple of Hk: value head h reads q/k head h / (H / Hk) -- groups of
+ *   consecutive value heads share one query/key head.
  *   g    : [rows, H, dk] (channel) | [rows, H] (scalar) | NULL (none)
  *   beta : [rows, H]
  *   S0   : [num_seqs, H, dv, dk] or NULL (zero initial state)
@@ -105,12 +108,12 @@ static void oracle_one_pair(int64_t start, int64_t len, int h, int H, int dk, in
  * Returns 0 on success, -1 on a bad argument, -2 if memory runs out.
  */
 int kda_oracle_forward(int num_seqs, const int64_t* seq_start, const int64_t* seq_len,
-                       int H, int dk, int dv, int gate_mode, const double* q,
+                       int H, int Hk, int dk, int dv, int gate_mode, const double* q,
                        const double* k, const double* v, const double* g,
                        const double* beta, const double* S0, double* out, double* ST,
                        int nthreads)
 {
-    if (num_seqs < 0 || H <= 0 || dk <= 0 || dv <= 0) return -1;
+    if (num_seqs < 0 || H <= 0 || Hk <= 0 || H % Hk != 0 || dk <= 0 || dv <= 0) return -1;
     if (gate_mode < 0 || gate_mode > 2) return -1;
     if (gate_mode != ORACLE_GATE_NONE && g == NULL) return -1;
     if (!q || !k || !v || !beta || !out || !seq_start || !seq_len) return -1;
@@ -127,13 +130,14 @@ int kda_oracle_forward(int num_seqs, const int64_t* seq_start, const int64_t* se
 #pragma omp parallel for schedule(dynamic, 1) reduction(| : failed)
     for (int64_t p = 0; p < pairs; ++p) {
         const int n = (int)(p / H), h = (int)(p % H);
+        const int hk = h / (H / Hk);
         const size_t soff = (size_t)p * dv * dk;
         double* S = (double*)malloc(sizeof(double) * (size_t)dv * dk);
         double* alpha = (double*)malloc(sizeof(double) * (size_t)dk);
         double* vhat = (double*)malloc(sizeof(double) * (size_t)dv);
         double* e = (double*)malloc(sizeof(double) * (size_t)dv);
         if (S && alpha && vhat && e)
-            oracle_one_pair(seq_start[n], seq_len[n], h, H, dk, dv, gate_mode, q, k, v, g,
+            oracle_one_pair(seq_start[n], seq_len[n], h, H, hk, Hk, dk, dv, gate_mode, q, k, v, g,
                             beta, S0 ? S0 + soff : NULL, out, ST ? ST + soff : NULL, S,
                             alpha, vhat, e);
         else

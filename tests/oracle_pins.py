@@ -326,4 +326,30 @@ def pin_chunkwise_identity(lib=None):
             _close(sc, s, tol=1e-10, what=f"chunk C={C} S_T strong={strong}")
 
 
+def pin_grouped_value_heads(lib=None):
+    """Grouped value heads: G consecutive value heads share one query/key head
+    (the value-head grid axis of the fused recurrent kernel in the GeekNews
+    summary).  Equal, bit for bit, to the one-to-one recurrence with each q/k
+    head repeated for its G value heads; a mapping that pairs value head h with
+    q/k head h mod Hk (or ignores the grouping) differs."""
+    rng = _rng(41)
+    B, T, Hk, G, dk, dv = 2, 6, 2, 3, 4, 5
+    H = Hk * G
+    q = rng.standard_normal((B, T, Hk, dk))
+    k = rng.standard_normal((B, T, Hk, dk))
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.standard_normal((B, T, H, dv))
+    g = -np.log1p(np.exp(rng.standard_normal((B, T, H, dk))))
+    beta = 1.0 / (1.0 + np.exp(-rng.standard_normal((B, T, H))))
+    S0 = 0.1 * rng.standard_normal((B, H, dv, dk))
+    o1, s1 = oracle.forward(q, k, v, g, beta, S0=S0, gate="channel", lib=lib)
+    o2, s2 = oracle.forward(np.repeat(q, G, axis=2), np.repeat(k, G, axis=2), v, g, beta, S0=S0,
+                            gate="channel", lib=lib)
+    assert np.array_equal(o1, o2) and np.array_equal(s1, s2), "grouped value heads != repeated q/k"
+    # value heads of different groups must see different q/k heads
+    o3, _ = oracle.forward(np.repeat(q[:, :, ::-1], G, axis=2), np.repeat(k[:, :, ::-1], G, axis=2), v,
+                           g, beta, S0=S0, gate="channel", lib=lib)
+    assert not np.allclose(o1, o3)
+
+
 ALL_PINS = [v for n, v in sorted(globals().items()) if n.startswith("pin_")]

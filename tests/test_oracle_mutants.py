@@ -25,6 +25,8 @@ MUTANTS = {
     "gate_previous_token": ("alpha[c] = exp(g[(row * H + h) * dk + c]);",
                             "alpha[c] = exp(g[((row > start ? row - 1 : row) * H + h) * dk + c]);"),
     "ignore_S0": ("if (S0) memcpy(S, S0, sizeof(double) * (size_t)dv * dk);", "if (0) (void)S0;"),
+    "value_heads_interleaved": ("const int hk = h / (H / Hk);", "const int hk = h % Hk;"),
+    "value_heads_ignored": ("const int hk = h / (H / Hk);", "const int hk = 0;"),
     "predict_before_decay": (None, None),
     "read_before_write": (None, None),
 }
