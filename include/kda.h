@@ -80,7 +80,19 @@ typedef struct {
     int32_t gate;       /* kda_gate_t */
     int32_t chunk;      /* chunk length C of kda_chunk_fwd; ignored by decode */
     int32_t* dev_status;/* optional device int32, see KDA_DEV_*; may be NULL */
+    int32_t qk_heads;   /* query/key heads Hk; 0 means H.  See "Grouped value heads". */
 } kda_shape_t;
+
+/*
+ * Grouped value heads.  H counts value heads: v, out, g, beta and every
+ * state have H heads.  q and k may have fewer, Hk = qk_heads, with H a
+ * multiple of Hk; value head h then reads query/key head h / (H / Hk), so
+ * consecutive groups of H / Hk value heads share one query/key head (the
+ * value-head grid axis of the fused recurrent kernel, GeekNews summary,
+ * section "fused recurrent kernel for decode").  Below, a q/k layout written
+ * [.., H, d_k] means [.., Hk, d_k].  qk_heads = 0 or H is the one-to-one case;
+ * any other value that does not divide H returns KDA_ERR_INVALID_ARG.
+ */
 
 /*
  * kda_chunk_fwd -- chunkwise-parallel prefill forward.

@@ -34,11 +34,11 @@ class KDAError(RuntimeError):
 
 
 class Shape(ctypes.Structure):
-    """kda_shape_t."""
+    """kda_shape_t (qk_heads = 0: one query/key head per value head)."""
     _fields_ = [("B", ctypes.c_int32), ("T", ctypes.c_int32), ("H", ctypes.c_int32),
                 ("d_k", ctypes.c_int32), ("d_v", ctypes.c_int32), ("num_seqs", ctypes.c_int32),
                 ("dtype", ctypes.c_int32), ("gate", ctypes.c_int32), ("chunk", ctypes.c_int32),
-                ("dev_status", ctypes.c_void_p)]
+                ("dev_status", ctypes.c_void_p), ("qk_heads", ctypes.c_int32)]
 
 
 _lib = None
@@ -108,6 +108,15 @@ def _gate_code(g, q) -> int:
     raise ValueError(f"g has {g.dim()} dims; expected {q.dim()} (per channel) or {q.dim() - 1} (scalar)")
 
 
+def _heads(q, v, lead: int):
+    """(value heads H, query/key heads Hk) from q [.., Hk, d_k] and v [.., H, d_v]
+    (`lead` leading dims before the head axis); H must be a multiple of Hk."""
+    Hk, H = q.shape[lead], v.shape[lead]
+    if v.shape[:lead] != q.shape[:lead] or Hk <= 0 or H % Hk != 0:
+        raise ValueError(f"q/k heads ({Hk}) must divide the value heads of v ({H}) with equal leading dims")
+    return H, Hk
+
+
 def _check_cuda(*ts):
     for t in ts:
         if t is not None:
@@ -121,21 +130,24 @@ def kda_chunk_fwd(q, k, v, g, beta, S0=None, cu_seqlens=None, chunk: int = 64, o
                   S_T=None, want_state: bool = True, dev_status=None, workspace=True, lib=None):
     """Chunkwise KDA prefill (kda_chunk_fwd of include/kda.h).
 
-    q, k [B,T,H,d_k]; v [B,T,H,d_v] (bf16 or fp32, same dtype); g [B,T,H,d_k]
+    q, k [B,T,Hk,d_k]; v [B,T,H,d_v] (bf16 or fp32, same dtype); g [B,T,H,d_k]
     (per channel) | [B,T,H] (scalar) | None (no gate), fp32 log-decay;
     beta [B,T,H] fp32; S0 [N,H,d_v,d_k] fp32 or None; cu_seqlens int32 [N+1]
-    with B == 1 for packed sequences.  Returns (out, S_T); S_T is None when
-    want_state is False and no S_T buffer is given.
+    with B == 1 for packed sequences.  H value heads, Hk query/key heads
+    (H a multiple of Hk; value head h reads q/k head h // (H // Hk)).
+    Returns (out, S_T); S_T is None when want_state is False and no S_T buffer
+    is given.
 
     workspace: True allocates the scratch of the two-kernel schedule with torch
     (when the shape takes a path that uses one), a uint8 CUDA tensor supplies
     it, None / False runs the single fused kernel with no scratch.
     """
     _check_cuda(q, k, v, g, beta, S0, cu_seqlens, out, S_T, dev_status)
-    B, T, H, Dk = q.shape
+    B, T, Hk, Dk = q.shape
+    H, _ = _heads(q, v, 2)
     Dv = v.shape[-1]
     N = B if cu_seqlens is None else cu_seqlens.numel() - 1
-    if k.shape != q.shape or v.shape[:3] != q.shape[:3] or beta.shape != q.shape[:3]:
+    if k.shape != q.shape or beta.shape != v.shape[:3]:
         raise ValueError("shape mismatch among q, k, v, beta")
     if k.dtype != q.dtype or v.dtype != q.dtype:
         raise TypeError("q, k, v must share one dtype")
@@ -148,7 +160,7 @@ def kda_chunk_fwd(q, k, v, g, beta, S0=None, cu_seqlens=None, chunk: int = 64, o
     if S_T is None and want_state:
         S_T = torch.empty(N, H, Dv, Dk, dtype=torch.float32, device=q.device)
     sh = Shape(B, T, H, Dk, Dv, N, _dtype_code(q.dtype), _gate_code(g, q), int(chunk),
-               None if dev_status is None else dev_status.data_ptr())
+               None if dev_status is None else dev_status.data_ptr(), Hk)
     lib = lib or load_library()
     if isinstance(workspace, torch.Tensor):
         _check_cuda(workspace)
@@ -171,7 +183,8 @@ def kda_chunk_fwd_noalloc(q, k, v, g, beta, S0=None, cu_seqlens=None, chunk: int
     """kda_chunk_fwd_noalloc of include/kda.h: the library's own static scratch
     instead of a workspace (arguments and results as kda_chunk_fwd)."""
     _check_cuda(q, k, v, g, beta, S0, cu_seqlens, out, S_T, dev_status)
-    B, T, H, Dk = q.shape
+    B, T, Hk, Dk = q.shape
+    H, _ = _heads(q, v, 2)
     Dv = v.shape[-1]
     N = B if cu_seqlens is None else cu_seqlens.numel() - 1
     if out is None:
@@ -179,7 +192,7 @@ def kda_chunk_fwd_noalloc(q, k, v, g, beta, S0=None, cu_seqlens=None, chunk: int
     if S_T is None and want_state:
         S_T = torch.empty(N, H, Dv, Dk, dtype=torch.float32, device=q.device)
     sh = Shape(B, T, H, Dk, Dv, N, _dtype_code(q.dtype), _gate_code(g, q), int(chunk),
-               None if dev_status is None else dev_status.data_ptr())
+               None if dev_status is None else dev_status.data_ptr(), Hk)
     lib = lib or load_library()
     st = lib.kda_chunk_fwd_noalloc(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
                                    _ptr(S0), _ptr(cu_seqlens), _ptr(out), _ptr(S_T),
@@ -191,9 +204,10 @@ def kda_chunk_fwd_noalloc(q, k, v, g, beta, S0=None, cu_seqlens=None, chunk: int
 
 def kda_chunk_fwd_workspace_size(q, v, g=None, cu_seqlens=None, chunk: int = 64, lib=None) -> int:
     """Bytes of scratch the two-kernel schedule needs for these inputs (0: none)."""
-    B, T, H, Dk = q.shape
+    B, T, Hk, Dk = q.shape
+    H, _ = _heads(q, v, 2)
     N = B if cu_seqlens is None else cu_seqlens.numel() - 1
-    sh = Shape(B, T, H, Dk, v.shape[-1], N, _dtype_code(q.dtype), _gate_code(g, q), int(chunk), None)
+    sh = Shape(B, T, H, Dk, v.shape[-1], N, _dtype_code(q.dtype), _gate_code(g, q), int(chunk), None, Hk)
     lib = lib or load_library()
     return int(lib.kda_chunk_fwd_workspace_size(ctypes.byref(sh), int(cu_seqlens is not None)))
 
@@ -201,17 +215,19 @@ def kda_chunk_fwd_workspace_size(q, v, g=None, cu_seqlens=None, chunk: int = 64,
 def kda_decode_step(q, k, v, g, beta, S, out=None, lib=None):
     """One fused recurrent KDA token (kda_decode_step of include/kda.h).
 
-    q, k [N,H,d_k]; v [N,H,d_v]; g [N,H,d_k] | [N,H] | None (fp32 log-decay);
+    q, k [N,Hk,d_k]; v [N,H,d_v]; g [N,H,d_k] | [N,H] | None (fp32 log-decay);
     beta [N,H] fp32; S [N,H,d_v,d_k] fp32, updated in place.  Returns out [N,H,d_v].
+    H value heads, Hk query/key heads (H a multiple of Hk).
     """
     _check_cuda(q, k, v, g, beta, S, out)
-    N, H, Dk = q.shape
+    N, Hk, Dk = q.shape
+    H, _ = _heads(q, v, 1)
     Dv = v.shape[-1]
     if S.shape != (N, H, Dv, Dk) or S.dtype != torch.float32:
         raise ValueError("S must be float32 [N, H, d_v, d_k]")
     if out is None:
         out = torch.empty_like(v)
-    sh = Shape(N, 1, H, Dk, Dv, N, _dtype_code(q.dtype), _gate_code(g, q), 0, None)
+    sh = Shape(N, 1, H, Dk, Dv, N, _dtype_code(q.dtype), _gate_code(g, q), 0, None, Hk)
     lib = lib or load_library()
     st = lib.kda_decode_step(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
                              _ptr(S), _ptr(out), _stream_handle(q.device))
@@ -223,18 +239,20 @@ def kda_decode_step(q, k, v, g, beta, S, out=None, lib=None):
 def kda_recurrent_fwd(q, k, v, g, beta, S, out=None, lib=None):
     """Fused recurrent KDA over T tokens per sequence (kda_recurrent_fwd of include/kda.h).
 
-    q, k [N,T,H,d_k]; v [N,T,H,d_v]; g [N,T,H,d_k] | [N,T,H] | None (fp32 log-decay);
+    q, k [N,T,Hk,d_k]; v [N,T,H,d_v]; g [N,T,H,d_k] | [N,T,H] | None (fp32 log-decay);
     beta [N,T,H] fp32; S [N,H,d_v,d_k] fp32, read once and overwritten with the state
-    after the T tokens.  Returns out [N,T,H,d_v].
+    after the T tokens.  Returns out [N,T,H,d_v].  H value heads, Hk query/key heads
+    (H a multiple of Hk).
     """
     _check_cuda(q, k, v, g, beta, S, out)
-    N, T, H, Dk = q.shape
+    N, T, Hk, Dk = q.shape
+    H, _ = _heads(q, v, 2)
     Dv = v.shape[-1]
     if S.shape != (N, H, Dv, Dk) or S.dtype != torch.float32:
         raise ValueError("S must be float32 [N, H, d_v, d_k]")
     if out is None:
         out = torch.empty_like(v)
-    sh = Shape(N, T, H, Dk, Dv, N, _dtype_code(q.dtype), _gate_code(g, q), 0, None)
+    sh = Shape(N, T, H, Dk, Dv, N, _dtype_code(q.dtype), _gate_code(g, q), 0, None, Hk)
     lib = lib or load_library()
     st = lib.kda_recurrent_fwd(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
                                _ptr(S), _ptr(out), _stream_handle(q.device))

@@ -28,6 +28,12 @@ bool f32path_supports(int D, int V, int C) {
 
 kda_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA; }
 
+// Query/key heads of a shape (0 means one per value head); -1 if they do not divide H.
+int qk_heads_of(const kda_shape_t* sh) {
+    const int Hk = sh->qk_heads == 0 ? sh->H : sh->qk_heads;
+    return (Hk > 0 && sh->H > 0 && sh->H % Hk == 0) ? Hk : -1;
+}
+
 }  // namespace
 
 extern "C" {
@@ -44,7 +50,7 @@ const char* kda_status_str(kda_status_t s) {
     return "unknown status";
 }
 
-const char* kda_version(void) { return "libkda 0.1 (sm_100a)"; }
+const char* kda_version(void) { return "libkda 0.2 (sm_100a)"; }
 
 size_t kda_chunk_fwd_workspace_size(const kda_shape_t* sh, int varlen) {
     if (sh == nullptr || sh->B < 0 || sh->T < 0 || sh->H <= 0 || sh->num_seqs < 0) return 0;
@@ -59,6 +65,8 @@ kda_status_t kda_chunk_fwd(const kda_shape_t* sh, const void* q, const void* k, 
     if (sh == nullptr) return KDA_ERR_INVALID_ARG;
     const int B = sh->B, T = sh->T, H = sh->H, D = sh->d_k, V = sh->d_v, N = sh->num_seqs;
     if (B < 0 || T < 0 || H <= 0 || D <= 0 || V <= 0 || N < 0) return KDA_ERR_INVALID_ARG;
+    const int Hk = qk_heads_of(sh);
+    if (Hk < 0) return KDA_ERR_INVALID_ARG;
     if (sh->dtype != KDA_F32 && sh->dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
     if (sh->gate != KDA_GATE_CHANNEL && sh->gate != KDA_GATE_SCALAR && sh->gate != KDA_GATE_NONE)
         return KDA_ERR_INVALID_ARG;
@@ -95,6 +103,7 @@ kda_status_t kda_chunk_fwd(const kda_shape_t* sh, const void* q, const void* k, 
     a.out = out; a.S_T = S_T; a.dev_status = sh->dev_status;
     a.B = B; a.T = T; a.H = H; a.d_k = D; a.d_v = V; a.num_seqs = N; a.gate = sh->gate;
     a.chunk = C;
+    a.Hk = Hk;
     a.scale = 1.0f / sqrtf((float)D);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (split) {
@@ -125,6 +134,8 @@ kda_status_t kda_recurrent_fwd(const kda_shape_t* sh, const void* q, const void*
     if (sh == nullptr) return KDA_ERR_INVALID_ARG;
     const int N = sh->B, T = sh->T, H = sh->H, D = sh->d_k, V = sh->d_v;
     if (N < 0 || T < 0 || H <= 0 || D <= 0 || V <= 0 || sh->num_seqs != N) return KDA_ERR_INVALID_ARG;
+    const int Hk = qk_heads_of(sh);
+    if (Hk < 0) return KDA_ERR_INVALID_ARG;
     if (sh->dtype != KDA_F32 && sh->dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
     if (sh->gate != KDA_GATE_CHANNEL && sh->gate != KDA_GATE_SCALAR && sh->gate != KDA_GATE_NONE)
         return KDA_ERR_INVALID_ARG;
@@ -143,6 +154,7 @@ kda_status_t kda_recurrent_fwd(const kda_shape_t* sh, const void* q, const void*
         kda::DecodeArgs d;
         d.q = q; d.k = k; d.v = v; d.g = g; d.beta = beta; d.S = S; d.out = out;
         d.N = N; d.H = H; d.d_k = D; d.d_v = V; d.gate = sh->gate;
+        d.Hk = Hk;
         d.scale = 1.0f / sqrtf((float)D);
         return from_cuda(kda::launch_decode(d, sh->dtype == KDA_BF16, static_cast<cudaStream_t>(stream)));
     }
@@ -150,6 +162,7 @@ kda_status_t kda_recurrent_fwd(const kda_shape_t* sh, const void* q, const void*
     kda::RecurrentArgs a;
     a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.S = S; a.out = out;
     a.N = N; a.T = T; a.H = H; a.d_k = D; a.d_v = V; a.gate = sh->gate;
+    a.Hk = Hk;
     a.scale = 1.0f / sqrtf((float)D);
     return from_cuda(kda::launch_recurrent(a, sh->dtype == KDA_BF16, static_cast<cudaStream_t>(stream)));
 }
@@ -160,6 +173,8 @@ kda_status_t kda_decode_step(const kda_shape_t* sh, const void* q, const void* k
     if (sh == nullptr) return KDA_ERR_INVALID_ARG;
     const int N = sh->B, H = sh->H, D = sh->d_k, V = sh->d_v;
     if (N < 0 || H <= 0 || D <= 0 || V <= 0 || sh->T != 1) return KDA_ERR_INVALID_ARG;
+    const int Hk = qk_heads_of(sh);
+    if (Hk < 0) return KDA_ERR_INVALID_ARG;
     if (sh->dtype != KDA_F32 && sh->dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
     if (sh->gate != KDA_GATE_CHANNEL && sh->gate != KDA_GATE_SCALAR && sh->gate != KDA_GATE_NONE)
         return KDA_ERR_INVALID_ARG;
@@ -176,6 +191,7 @@ kda_status_t kda_decode_step(const kda_shape_t* sh, const void* q, const void* k
     kda::DecodeArgs a;
     a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.S = S; a.out = out;
     a.N = N; a.H = H; a.d_k = D; a.d_v = V; a.gate = sh->gate;
+    a.Hk = Hk;
     a.scale = 1.0f / sqrtf((float)D);
     return from_cuda(kda::launch_decode(a, sh->dtype == KDA_BF16, static_cast<cudaStream_t>(stream)));
 }

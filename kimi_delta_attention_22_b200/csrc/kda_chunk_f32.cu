@@ -42,6 +42,7 @@ __global__ void __launch_bounds__(kThreads) kda_chunk_f32_kernel(ChunkArgs a) {
     extern __shared__ float4 smem_raw[];
     const int C = a.chunk, D = a.d_k, V = a.d_v, H = a.H;
     const int n = blockIdx.x / H, h = blockIdx.x % H;
+    const int hk = h / (H / a.Hk);   // query/key head (grouped value heads share it)
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
     float* base = reinterpret_cast<float*>(smem_raw);
@@ -79,9 +80,9 @@ __global__ void __launch_bounds__(kThreads) kda_chunk_f32_kernel(ChunkArgs a) {
             const int i = idx / D, c = idx % D;
             float kv = 0.f, qv = 0.f, gv = 0.f;
             if (i < L) {
-                const size_t tok = (size_t)(c0 + i) * H + h;
-                kv = ld_in(k + tok * D + c);
-                qv = ld_in(q + tok * D + c) * a.scale;
+                const size_t tok = (size_t)(c0 + i) * H + h, tk = (size_t)(c0 + i) * a.Hk + hk;
+                kv = ld_in(k + tk * D + c);
+                qv = ld_in(q + tk * D + c) * a.scale;
                 if (GATE == KDA_GATE_CHANNEL) gv = a.g[tok * D + c];
                 else if (GATE == KDA_GATE_SCALAR) gv = a.g[tok];
             }

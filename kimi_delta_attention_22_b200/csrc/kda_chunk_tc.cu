@@ -116,6 +116,7 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
     const int vt = blockIdx.x % NVT;
     const int h = (blockIdx.x / NVT) % H;
     const int n = blockIdx.x / (NVT * H);
+    const int hk = h / (H / a.Hk);     // query/key head (grouped value heads share it)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int sp = warp & 3;           // TMEM sub-partition of this warp
     const int vhalf = warp >> 2;       // which 32 of the tile's 64 value columns
@@ -182,8 +183,8 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
     auto issue_kq = [&](long long c1) {
         if (GATE == KDA_GATE_CHANNEL) mbar_expect_tx(full_bar, 32768u);   // g arrives later
         else mbar_arrive_expect_tx(full_bar, 32768u);
-        tma_load_3d(sm + OFF_RK, &p.map_k, full_bar, 0, h, (int)c1);
-        tma_load_3d(sm + OFF_RQ, &p.map_q, full_bar, 0, h, (int)c1);
+        tma_load_3d(sm + OFF_RK, &p.map_k, full_bar, 0, hk, (int)c1);
+        tma_load_3d(sm + OFF_RQ, &p.map_q, full_bar, 0, hk, (int)c1);
     };
     auto issue_g = [&](long long c1) {
         mbar_arrive_expect_tx(full_bar, 32768u);
@@ -819,9 +820,9 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t st) {
     p.a = a;
     const long long tokens = (long long)a.B * a.T;
     if (tokens > 0) {  // with no tokens the kernel only copies S0 to S_T and never issues TMA
-        bool ok = make_map(&p.map_k, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DK, a.H, tokens, DK,
+        bool ok = make_map(&p.map_k, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DK, a.Hk, tokens, DK,
                            C, CU_TENSOR_MAP_SWIZZLE_NONE) &&
-                  make_map(&p.map_q, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DK, a.H, tokens, DK,
+                  make_map(&p.map_q, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DK, a.Hk, tokens, DK,
                            C, CU_TENSOR_MAP_SWIZZLE_NONE) &&
                   make_map(&p.map_v, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DV, a.H, tokens, BV,
                            C, CU_TENSOR_MAP_SWIZZLE_128B);

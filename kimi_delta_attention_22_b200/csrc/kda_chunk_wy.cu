@@ -107,6 +107,7 @@ struct WyParams {
     uint8_t* rec;
     int T, H, num_seqs, nc;   // nc: slots per sequence of a dense batch
     int ahead;                // fast kernel: CTAs resident at once (L2 prefetch distance)
+    int group;                // value heads per query/key head (q/k head of h: h / group)
     float scale;
 };
 
@@ -214,8 +215,8 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
         // K, Q (16 KB each), per-channel g (32 KB); V (two 8 KB tiles) on its own barrier
         const uint32_t bytes = 16384u * 2u + (GATE == KDA_GATE_CHANNEL ? 32768u : 0u);
         mbar_arrive_expect_tx(full_bar, bytes);
-        tma_load_3d(sm + M::RK, &p.map_k, full_bar, 0, h, (int)c0);
-        tma_load_3d(sm + M::RQ, &p.map_q, full_bar, 0, h, (int)c0);
+        tma_load_3d(sm + M::RK, &p.map_k, full_bar, 0, h / p.group, (int)c0);
+        tma_load_3d(sm + M::RQ, &p.map_q, full_bar, 0, h / p.group, (int)c0);
         if (GATE == KDA_GATE_CHANNEL) tma_load_3d(sm + M::RG, &p.map_g, full_bar, 0, h, (int)c0);
         mbar_arrive_expect_tx(v_bar, 16384u);
         tma_load_3d(sm + M::RV, &p.map_v, v_bar, 0, h, (int)c0);
@@ -229,8 +230,8 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
             if (lin < (long long)gridDim.x * gridDim.y &&
                 decode_slot(p, (int)(lin % gridDim.x), c2, L2)) {
                 const int h2 = (int)(lin / gridDim.x);
-                tma_prefetch_l2_3d(&p.map_k, 0, h2, (int)c2);
-                tma_prefetch_l2_3d(&p.map_q, 0, h2, (int)c2);
+                tma_prefetch_l2_3d(&p.map_k, 0, h2 / p.group, (int)c2);
+                tma_prefetch_l2_3d(&p.map_q, 0, h2 / p.group, (int)c2);
                 tma_prefetch_l2_3d(&p.map_v, 0, h2, (int)c2);
                 tma_prefetch_l2_3d(&p.map_v, 64, h2, (int)c2);
                 if (GATE == KDA_GATE_CHANNEL) tma_prefetch_l2_3d(&p.map_g, 0, h2, (int)c2);
@@ -841,9 +842,10 @@ cudaError_t launch_chunk_wy(const ChunkArgs& a, uint8_t* ws, const rec::Layout& 
     p.scale = a.scale;
     const long long tokens = (long long)a.B * a.T;
     if (tokens == 0 || lay.slots == 0) return cudaSuccess;
-    bool ok = make_map(&p.map_k, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DK, a.H, tokens, DK, C,
+    p.group = a.H / a.Hk;
+    bool ok = make_map(&p.map_k, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DK, a.Hk, tokens, DK, C,
                        CU_TENSOR_MAP_SWIZZLE_NONE) &&
-              make_map(&p.map_q, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DK, a.H, tokens, DK, C,
+              make_map(&p.map_q, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DK, a.Hk, tokens, DK, C,
                        CU_TENSOR_MAP_SWIZZLE_NONE) &&
               make_map(&p.map_v, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rec::DV, a.H, tokens, 64, C,
                        CU_TENSOR_MAP_SWIZZLE_128B);

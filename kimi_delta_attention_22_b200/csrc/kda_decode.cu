@@ -46,8 +46,10 @@ __global__ void __launch_bounds__(kThreads, 2) kda_decode_kernel(DecodeArgs a) {
     const int nh = blockIdx.x;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int sub = lane & 7, rsel = lane >> 3;
-    const TI* qp = static_cast<const TI*>(a.q) + (size_t)nh * kDK;
-    const TI* kp = static_cast<const TI*>(a.k) + (size_t)nh * kDK;
+    // query/key head of value head h = nh % H (grouped value heads share it)
+    const size_t nhk = (size_t)(nh / a.H) * a.Hk + (nh % a.H) / (a.H / a.Hk);
+    const TI* qp = static_cast<const TI*>(a.q) + nhk * kDK;
+    const TI* kp = static_cast<const TI*>(a.k) + nhk * kDK;
 
     float kr[16], qr[16], al[16];
 #pragma unroll

@@ -24,6 +24,7 @@ struct ChunkArgs {
     float* S_T;
     int32_t* dev_status;
     int B, T, H, d_k, d_v, num_seqs, gate, chunk;
+    int Hk;       // query/key heads: value head h reads q/k head h / (H / Hk)
     float scale;  // d_k^{-1/2}
 };
 
@@ -36,6 +37,7 @@ struct DecodeArgs {
     float* S;
     void* out;
     int N, H, d_k, d_v, gate;
+    int Hk;       // query/key heads: value head h reads q/k head h / (H / Hk)
     float scale;
 };
 
@@ -49,6 +51,7 @@ struct RecurrentArgs {
     float* S;
     void* out;
     int N, T, H, d_k, d_v, gate;
+    int Hk;       // query/key heads: value head h reads q/k head h / (H / Hk)
     float scale;
 };
 

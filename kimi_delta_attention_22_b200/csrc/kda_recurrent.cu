@@ -45,16 +45,17 @@ __global__ void __launch_bounds__(kThreads, 2) kda_recurrent_kernel(RecurrentArg
 
     // Stage token t into buffer b: threads 0-127 own channel tid, 128-255 row tid - 128.
     const size_t tok0 = (size_t)n * a.T;
+    const int hk = h / (a.H / a.Hk);   // query/key head (grouped value heads share it)
     auto stage = [&](int t, int b) {
-        const size_t th = (tok0 + t) * a.H + h;
+        const size_t th = (tok0 + t) * a.H + h, tk = (tok0 + t) * a.Hk + hk;
         Stage& st = stg[b];
         if (tid < kDK) {
             float gc = 0.f;
             if (GATE == KDA_GATE_CHANNEL) gc = __ldg(a.g + th * kDK + tid);
             else if (GATE == KDA_GATE_SCALAR) gc = __ldg(a.g + th);
             st.al[tid] = (GATE == KDA_GATE_NONE) ? 1.f : expf(gc);
-            st.k[tid] = to_f32(static_cast<const TI*>(a.k)[th * kDK + tid]);
-            st.qs[tid] = to_f32(static_cast<const TI*>(a.q)[th * kDK + tid]) * a.scale;
+            st.k[tid] = to_f32(static_cast<const TI*>(a.k)[tk * kDK + tid]);
+            st.qs[tid] = to_f32(static_cast<const TI*>(a.q)[tk * kDK + tid]) * a.scale;
             if (tid == 0) st.beta = __ldg(a.beta + th);
         } else {
             const int r = rbase + tid - kDK;

@@ -45,6 +45,11 @@ class Workload:
     num_seqs: int = 0   # varlen only
     len_lo: int = 0
     len_hi: int = 0
+    qk_heads: int = 0   # query/key heads (grouped value heads); 0 = one per value head
+
+    @property
+    def Hk(self) -> int:
+        return self.qk_heads or self.H
 
     @property
     def torch_dtype(self):
@@ -71,6 +76,9 @@ _add(Workload("small_f32_t64_d16", 1, 64, 1, 16, 16, "f32", "channel", "sigmoid"
 # bf16 chunkwise prefill: B=4, H=16, T=2048, d=128, chunk 64, S0 ~ N(0, 0.02^2).
 _add(Workload("prefill_b4_h16_t2048", 4, 2048, 16, 128, 128, "bf16", "channel", "sigmoid", 64,
               0.02, 2))
+# the same prefill with grouped value heads: 16 value heads over 4 query/key heads
+_add(Workload("prefill_b4_h16_qk4_t2048", 4, 2048, 16, 128, 128, "bf16", "channel", "sigmoid", 64,
+              0.02, 12, qk_heads=4))
 # varlen prefill: 8 packed sequences, 65536 tokens, lengths in [1024, 15360], state reset.
 _add(Workload("varlen_h32_t65536", 1, 65536, 32, 128, 128, "bf16", "channel", "sigmoid", 64,
               None, 4, varlen=True, num_seqs=8, len_lo=1024, len_hi=15360))
@@ -104,14 +112,16 @@ def _gen(device, seed):
 
 
 def draw(B, T, H, d_k, d_v, *, dtype=torch.bfloat16, gate="channel", beta="sigmoid",
-         s0_std=None, num_states=None, seed=0, device="cpu"):
-    """Draw one input set.  Returns a dict with q, k, v ([B,T,H,d] in dtype),
-    g (fp32 [B,T,H,d_k] | [B,T,H] | None), beta (fp32 [B,T,H]) and S0
-    (fp32 [num_states,H,d_v,d_k] or None; num_states defaults to B)."""
+         s0_std=None, num_states=None, seed=0, device="cpu", qk_heads=None):
+    """Draw one input set.  Returns a dict with q, k ([B,T,Hk,d_k]), v ([B,T,H,d_v])
+    in dtype, g (fp32 [B,T,H,d_k] | [B,T,H] | None), beta (fp32 [B,T,H]) and S0
+    (fp32 [num_states,H,d_v,d_k] or None; num_states defaults to B).  Hk =
+    qk_heads (grouped value heads) or H."""
     gen = _gen(device, seed)
     f32 = dict(dtype=torch.float32, device=device, generator=gen)
-    q = torch.randn(B, T, H, d_k, **f32)
-    k = torch.randn(B, T, H, d_k, **f32)
+    Hk = H if qk_heads is None else qk_heads
+    q = torch.randn(B, T, Hk, d_k, **f32)
+    k = torch.randn(B, T, Hk, d_k, **f32)
     k = k / k.norm(dim=-1, keepdim=True).clamp_min(1e-12)
     v = torch.randn(B, T, H, d_v, **f32)
     if gate == "channel":
@@ -148,7 +158,8 @@ def workload_inputs(w: Workload | str, device="cpu", T: int | None = None, B: in
     B_, T_, H_ = B or w.B, T or w.T, H or w.H
     out = draw(B_, T_, H_, w.d_k, w.d_v, dtype=w.torch_dtype, gate=w.gate, beta=w.beta,
                s0_std=w.s0_std, seed=w.seed, device=device,
-               num_states=(w.num_seqs if w.varlen else None))
+               num_states=(w.num_seqs if w.varlen else None),
+               qk_heads=(H_ * w.qk_heads // w.H if w.qk_heads else None))
     out["cu_seqlens"] = None
     if w.varlen:
         lo = max(1, w.len_lo * T_ // w.T)

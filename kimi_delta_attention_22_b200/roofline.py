@@ -10,13 +10,16 @@ from __future__ import annotations
 
 
 def prefill_bytes(w) -> int:
+    """q and k count once per query/key head (grouped value heads share them)."""
     ht = w.B * w.T * w.H
+    Hk = getattr(w, "Hk", w.H)
     el = 2 if w.dtype == "bf16" else 4
     g = {"channel": 4 * w.d_k, "scalar": 4, "none": 0}[w.gate_mode]
-    per_ht = el * (2 * w.d_k + w.d_v) + g + 4 + el * w.d_v
+    per_ht = el * w.d_v + g + 4 + el * w.d_v
+    qk = w.B * w.T * Hk * el * 2 * w.d_k
     seqs = w.num_seqs if w.varlen else w.B
     states = seqs * w.H * w.d_v * w.d_k * 4 * ((1 if w.s0_std is not None else 0) + 1)
-    return ht * per_ht + states
+    return ht * per_ht + qk + states
 
 
 def prefill_flops(w) -> float:
