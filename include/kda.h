@@ -207,6 +207,38 @@ kda_status_t kda_decode_step(const kda_shape_t* shape, const void* q, const void
  * T = 1 runs the decode step's kernel (the same arithmetic, at the state-copy rate).
  * Else KDA_ERR_UNSUPPORTED.
  */
+/*
+ * kda_recurrent_bwd -- gradients of kda_recurrent_fwd (training).
+ *
+ * For the loss sum(out * d_out) + sum(S_T * d_ST), where (out, S_T) is what
+ * kda_recurrent_fwd returns from the state S0 over the T tokens, writes the
+ * gradients with respect to every input.  It differentiates the five-step
+ * update token by token (the pages give no backward derivation; this is the
+ * chain rule of the recurrence itself), walking the tokens in reverse on CUDA
+ * cores with the state recomputed from checkpoints kept in the workspace.
+ *
+ * Layouts as kda_recurrent_fwd (dense batch, N = shape->B, num_seqs == N):
+ *   q, k [N, T, Hk, d_k], v, d_out [N, T, H, d_v] dtype; g, beta, S0 as there;
+ *   d_ST [N, H, d_v, d_k] fp32 or NULL (zero).
+ * Outputs, all fp32 and caller-owned:
+ *   dq, dk [N, T, Hk, d_k] (summed over the value heads of a group)
+ *   dv     [N, T, H, d_v]
+ *   dg     the shape of g (NULL when the gate is KDA_GATE_NONE, required otherwise)
+ *   dbeta  [N, T, H]
+ *   dS0    [N, H, d_v, d_k], or NULL when not wanted.
+ * S0, d_ST and dS0 are 16-byte aligned; the workspace (>= the size below) 16 bytes.
+ * Support: d_k = 128, d_v from 1 to 65535*16; else KDA_ERR_UNSUPPORTED.
+ */
+kda_status_t kda_recurrent_bwd(const kda_shape_t* shape, const void* q, const void* k,
+                               const void* v, const float* g, const float* beta,
+                               const float* S0, const void* d_out, const float* d_ST, float* dq,
+                               float* dk, float* dv, float* dg, float* dbeta, float* dS0,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace kda_recurrent_bwd needs: the state of every (sequence, head)
+ * every 8 tokens (fp32). */
+size_t kda_recurrent_bwd_workspace_size(const kda_shape_t* shape);
+
 kda_status_t kda_recurrent_fwd(const kda_shape_t* shape, const void* q, const void* k,
                                const void* v, const float* g, const float* beta, float* S,
                                void* out, void* stream);

@@ -13,7 +13,7 @@ import os
 
 import torch
 
-__all__ = ["kda_chunk_fwd", "kda_recurrent_fwd", "kda_chunk_fwd_noalloc", "kda_chunk_fwd_workspace_size", "kda_decode_step", "kda_status_str", "library_path", "load_library",
+__all__ = ["kda_chunk_fwd", "kda_recurrent_fwd", "kda_recurrent_bwd", "kda_chunk_fwd_noalloc", "kda_chunk_fwd_workspace_size", "kda_decode_step", "kda_status_str", "library_path", "load_library",
            "KDAError", "KDA_F32", "KDA_BF16", "KDA_GATE_CHANNEL", "KDA_GATE_SCALAR",
            "KDA_GATE_NONE", "KDA_DEV_BAD_SEQLENS", "KDA_DEV_TIMEOUT", "Shape"]
 
@@ -69,6 +69,10 @@ def load_library(path: str | None = None):
     lib.kda_decode_step.argtypes = [ctypes.POINTER(Shape), P, P, P, P, P, P, P, P]
     lib.kda_recurrent_fwd.argtypes = [ctypes.POINTER(Shape), P, P, P, P, P, P, P, P]
     lib.kda_recurrent_fwd.restype = ctypes.c_int
+    lib.kda_recurrent_bwd.argtypes = [ctypes.POINTER(Shape)] + [P] * 15 + [ctypes.c_size_t, P]
+    lib.kda_recurrent_bwd.restype = ctypes.c_int
+    lib.kda_recurrent_bwd_workspace_size.argtypes = [ctypes.POINTER(Shape)]
+    lib.kda_recurrent_bwd_workspace_size.restype = ctypes.c_size_t
     lib.kda_decode_step.restype = ctypes.c_int
     lib.kda_status_str.argtypes = [ctypes.c_int]
     lib.kda_status_str.restype = ctypes.c_char_p
@@ -259,3 +263,42 @@ def kda_recurrent_fwd(q, k, v, g, beta, S, out=None, lib=None):
     if st != 0:
         raise KDAError(st, "kda_recurrent_fwd")
     return out
+
+
+def kda_recurrent_bwd(q, k, v, g, beta, S0, d_out, d_ST=None, want_dS0: bool = True, workspace=None,
+                      lib=None):
+    """Gradients of kda_recurrent_fwd (kda_recurrent_bwd of include/kda.h).
+
+    Inputs as kda_recurrent_fwd, with S0 [N,H,d_v,d_k] fp32 or None (the state
+    before the tokens; not modified), d_out [N,T,H,d_v] in the input dtype and
+    d_ST [N,H,d_v,d_k] fp32 or None.  Returns a dict of fp32 tensors dq, dk
+    [N,T,Hk,d_k], dv [N,T,H,d_v], dg (shape of g, or None), dbeta [N,T,H] and
+    dS0 [N,H,d_v,d_k] (None unless want_dS0) for the loss
+    sum(out * d_out) + sum(S_T * d_ST).
+    """
+    _check_cuda(q, k, v, g, beta, S0, d_out, d_ST)
+    N, T, Hk, Dk = q.shape
+    H, _ = _heads(q, v, 2)
+    Dv = v.shape[-1]
+    if d_out.shape != v.shape or d_out.dtype != v.dtype:
+        raise ValueError("d_out must match v in shape and dtype")
+    f32 = dict(dtype=torch.float32, device=q.device)
+    dq = torch.empty(N, T, Hk, Dk, **f32)
+    dk = torch.empty(N, T, Hk, Dk, **f32)
+    dv = torch.empty(N, T, H, Dv, **f32)
+    dg = None if g is None else torch.empty(g.shape, **f32)
+    dbeta = torch.empty(N, T, H, **f32)
+    dS0 = torch.empty(N, H, Dv, Dk, **f32) if want_dS0 else None
+    sh = Shape(N, T, H, Dk, Dv, N, _dtype_code(q.dtype), _gate_code(g, q), 0, None, Hk)
+    lib = lib or load_library()
+    if workspace is None:
+        nbytes = lib.kda_recurrent_bwd_workspace_size(ctypes.byref(sh))
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    _check_cuda(workspace)
+    st = lib.kda_recurrent_bwd(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0),
+                               _ptr(d_out), _ptr(d_ST), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), _ptr(dbeta),
+                               _ptr(dS0), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                               _stream_handle(q.device))
+    if st != 0:
+        raise KDAError(st, "kda_recurrent_bwd")
+    return dict(dq=dq, dk=dk, dv=dv, dg=dg, dbeta=dbeta, dS0=dS0)

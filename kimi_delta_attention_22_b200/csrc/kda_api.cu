@@ -167,6 +167,62 @@ kda_status_t kda_recurrent_fwd(const kda_shape_t* sh, const void* q, const void*
     return from_cuda(kda::launch_recurrent(a, sh->dtype == KDA_BF16, static_cast<cudaStream_t>(stream)));
 }
 
+size_t kda_recurrent_bwd_workspace_size(const kda_shape_t* sh) {
+    if (sh == nullptr || sh->B <= 0 || sh->T <= 0 || sh->H <= 0 || sh->d_v <= 0) return 0;
+    return kda::recurrent_bwd_workspace_bytes(sh->B, sh->T, sh->H, sh->d_v);
+}
+
+kda_status_t kda_recurrent_bwd(const kda_shape_t* sh, const void* q, const void* k, const void* v,
+                               const float* g, const float* beta, const float* S0, const void* d_out,
+                               const float* d_ST, float* dq, float* dk, float* dv, float* dg,
+                               float* dbeta, float* dS0, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+    if (sh == nullptr) return KDA_ERR_INVALID_ARG;
+    const int N = sh->B, T = sh->T, H = sh->H, D = sh->d_k, V = sh->d_v;
+    if (N < 0 || T < 0 || H <= 0 || D <= 0 || V <= 0 || sh->num_seqs != N) return KDA_ERR_INVALID_ARG;
+    const int Hk = qk_heads_of(sh);
+    if (Hk < 0) return KDA_ERR_INVALID_ARG;
+    if (sh->dtype != KDA_F32 && sh->dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+    if (sh->gate != KDA_GATE_CHANNEL && sh->gate != KDA_GATE_SCALAR && sh->gate != KDA_GATE_NONE)
+        return KDA_ERR_INVALID_ARG;
+    const bool gated = sh->gate != KDA_GATE_NONE;
+    if (gated != (g != nullptr) || gated != (dg != nullptr)) return KDA_ERR_INVALID_ARG;
+    const bool any = (long long)N * T > 0;
+    if (any && (!q || !k || !v || !beta || !d_out || !dq || !dk || !dv || !dbeta)) return KDA_ERR_INVALID_ARG;
+    if (!aligned4(q) || !aligned4(k) || !aligned4(v) || !aligned4(g) || !aligned4(beta) || !aligned4(d_out) ||
+        !aligned16(S0) || !aligned16(d_ST) || !aligned4(dq) || !aligned4(dk) || !aligned4(dv) ||
+        !aligned4(dg) || !aligned4(dbeta) || !aligned16(dS0) || !aligned16(workspace))
+        return KDA_ERR_MISALIGNED;
+    if (D != 128 || V > 65535 * 16) return KDA_ERR_UNSUPPORTED;
+    if ((long long)N * H > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+    if (N == 0) return KDA_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (T == 0) {   // no tokens: S_T = S0, so dS0 = d_ST
+        if (!dS0) return KDA_OK;
+        const size_t nb = (size_t)N * H * V * D * sizeof(float);
+        return from_cuda(d_ST ? cudaMemcpyAsync(dS0, d_ST, nb, cudaMemcpyDeviceToDevice, st)
+                              : cudaMemsetAsync(dS0, 0, nb, st));
+    }
+    const size_t need = kda::recurrent_bwd_workspace_bytes(N, T, H, V);
+    if (workspace == nullptr || workspace_bytes < need) return KDA_ERR_INVALID_ARG;
+
+    const size_t ntok = (size_t)N * T;
+    cudaError_t e = cudaMemsetAsync(dq, 0, ntok * Hk * D * sizeof(float), st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dk, 0, ntok * Hk * D * sizeof(float), st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dbeta, 0, ntok * H * sizeof(float), st);
+    if (e == cudaSuccess && gated)
+        e = cudaMemsetAsync(dg, 0, ntok * H * (sh->gate == KDA_GATE_CHANNEL ? D : 1) * sizeof(float), st);
+    if (e != cudaSuccess) return KDA_ERR_CUDA;
+
+    kda::RecurrentBwdArgs a;
+    a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.S0 = S0; a.d_out = d_out; a.d_ST = d_ST;
+    a.dq = dq; a.dk = dk; a.dv = dv; a.dg = dg; a.dbeta = dbeta; a.dS0 = dS0;
+    a.ws = static_cast<float*>(workspace);
+    a.N = N; a.T = T; a.H = H; a.Hk = Hk; a.d_k = D; a.d_v = V; a.gate = sh->gate;
+    a.scale = 1.0f / sqrtf((float)D);
+    return from_cuda(kda::launch_recurrent_bwd(a, sh->dtype == KDA_BF16, st));
+}
+
 kda_status_t kda_decode_step(const kda_shape_t* sh, const void* q, const void* k, const void* v,
                              const float* g, const float* beta, float* S, void* out,
                              void* stream) {

@@ -55,7 +55,31 @@ struct RecurrentArgs {
     float scale;
 };
 
+// Gradients of the token loop (dense batch, as RecurrentArgs); dq, dk, dg, dbeta are
+// accumulated with atomics into zeroed buffers, dv and dS0 written.
+struct RecurrentBwdArgs {
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* g;
+    const float* beta;
+    const float* S0;      // may be null (zero state)
+    const void* d_out;
+    const float* d_ST;    // may be null (zero)
+    float* dq;
+    float* dk;
+    float* dv;
+    float* dg;            // null without a gate
+    float* dbeta;
+    float* dS0;           // may be null
+    float* ws;            // recurrent_bwd_workspace_bytes()
+    int N, T, H, Hk, d_k, d_v, gate;
+    float scale;
+};
+
 cudaError_t launch_recurrent(const RecurrentArgs& a, bool bf16, cudaStream_t s);
+cudaError_t launch_recurrent_bwd(const RecurrentBwdArgs& a, bool bf16, cudaStream_t s);
+size_t recurrent_bwd_workspace_bytes(int N, int T, int H, int d_v);
 cudaError_t launch_chunk_f32path(const ChunkArgs& a, bool bf16, cudaStream_t s);
 cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t s);
 // Two-kernel tensor-core prefill over a caller workspace laid out by rec::layout().

@@ -21,6 +21,7 @@ roofline.recurrent_bytes (state read once and written once per call).
 from __future__ import annotations
 
 import argparse
+import ctypes
 import json
 import os
 import statistics
@@ -131,6 +132,39 @@ def measure_recurrent(T: int, iters: int, warmup: int, N: int = 256, H: int = 32
     return res
 
 
+def measure_backward(N: int, T: int, H: int, iters: int, warmup: int) -> dict:
+    """kda_recurrent_bwd on N sequences x T tokens x H heads (d = 128, bf16 inputs,
+    per-channel gate), against the forward pass of the same tokens."""
+    d = inputs.draw(N, T, H, 128, 128, dtype=torch.bfloat16, gate="channel", s0_std=0.05, seed=8,
+                    device="cuda")
+    gen = torch.Generator(device="cuda").manual_seed(9)
+    d_out = torch.randn(N, T, H, 128, device="cuda", generator=gen).to(torch.bfloat16)
+    d_ST = torch.randn(N, H, 128, 128, device="cuda", generator=gen)
+    sh = kda.Shape(N, T, H, 128, 128, N, kda.KDA_BF16, kda.KDA_GATE_CHANNEL, 0, None, H)
+    ws = torch.empty(kda.load_library().kda_recurrent_bwd_workspace_size(ctypes.byref(sh)),
+                     dtype=torch.uint8, device="cuda")
+    S = d["S0"].clone()
+
+    def bwd():
+        kda.kda_recurrent_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], d_out, d_ST, workspace=ws)
+
+    def fwd():
+        S.copy_(d["S0"])
+        kda.kda_recurrent_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], S)
+
+    ms = _time(bwd, iters, warmup)
+    ms_f = _time(fwd, iters, warmup)
+    # fp32 arithmetic per (token, head, state element): the forward twice (decay,
+    # prediction, write: 3 FMA-class ops) and the reverse step (9), FMA counted as 2
+    flops = N * T * H * 128 * 128 * 2 * (2 * 3 + 9)
+    res = {"kernel": "kda_recurrent_bwd", "N": N, "H": H, "T": T, "ms_per_call": ms,
+           "tokens_per_s": N * T / (ms * 1e-3), "fp32_tflops": flops / (ms * 1e-3) / 1e12,
+           "forward_ms": ms_f, "backward_over_forward": ms / ms_f, "iters": iters}
+    del d, d_out, d_ST, ws, S
+    torch.cuda.empty_cache()
+    return res
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--workloads", default=",".join(n for n in inputs.WORKLOADS))
@@ -139,10 +173,17 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--recurrent", action="store_true")
     ap.add_argument("--tokens", default="1,4,16,64")
+    ap.add_argument("--backward", default=None,
+                    help="N,T,H[;N,T,H...]: time kda_recurrent_bwd on these shapes")
     args = ap.parse_args()
     if not torch.cuda.is_available():
         raise SystemExit("measure needs a CUDA device")
     kda.load_library()
+    if args.backward:
+        for spec in args.backward.split(";"):
+            N, T, H = (int(x) for x in spec.split(","))
+            print(json.dumps(measure_backward(N, T, H, args.iters, args.warmup)), flush=True)
+        return
     if args.recurrent:
         for T in (int(x) for x in args.tokens.split(",")):
             print(json.dumps(measure_recurrent(T, args.iters, args.warmup)), flush=True)
