@@ -16,6 +16,7 @@ replica (weak scaling; the path has no exchange step).  The reference arm
 from __future__ import annotations
 
 import argparse
+import ctypes
 import hashlib
 import json
 import os
@@ -340,6 +341,48 @@ def bench_prefill(args, world, rank, peaks, peak_kind):
     return res
 
 
+def bench_backward(args, world):
+    """kda_recurrent_bwd (gradients of the token loop) on the short-run shape:
+    256 sequences x 32 heads x 16 tokens, d = 128, bf16 inputs, per-channel gate."""
+    import kimi_delta_attention_22_b200 as kda
+    from kimi_delta_attention_22_b200 import inputs
+
+    N, T, H = 256, 16, 32
+    dev = torch.device("cuda", torch.cuda.current_device())
+    d = inputs.draw(N, T, H, 128, 128, dtype=torch.bfloat16, gate="channel", s0_std=0.05, seed=8, device=dev)
+    gen = torch.Generator(device=dev).manual_seed(9)
+    d_out = torch.randn(N, T, H, 128, device=dev, generator=gen).to(torch.bfloat16)
+    d_ST = torch.randn(N, H, 128, 128, device=dev, generator=gen)
+    sh = kda.Shape(N, T, H, 128, 128, N, kda.KDA_BF16, kda.KDA_GATE_CHANNEL, 0, None, H)
+    ws = torch.empty(kda.load_library().kda_recurrent_bwd_workspace_size(ctypes.byref(sh)),
+                     dtype=torch.uint8, device=dev)
+
+    def step():
+        kda.kda_recurrent_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], d_out, d_ST, workspace=ws)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    stream = torch.cuda.current_stream(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    iters = 5
+    a.record(stream)
+    for _ in range(iters):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(a.elapsed_time(b), world) / iters
+    del d, d_out, d_ST, ws
+    torch.cuda.empty_cache()
+    return {"metric": "KDA token-loop backward tokens/s", "value": world * N * T / (ms * 1e-3),
+            "unit": "tokens/s", "ms_per_call": ms, "iters": iters,
+            "config": {"workload": "recurrent_bwd_n256_h32_t16", "N": N, "T": T, "H": H, "d_k": 128,
+                       "d_v": 128, "gate": "channel", "dtype": "bf16 inputs, fp32 gradients"},
+            "kernel": "kda_recurrent_bwd_kernel (CUDA cores)"}
+
+
 def bench_decode(args, world, rank, peaks, peak_kind):
     import kimi_delta_attention_22_b200 as kda
     from kimi_delta_attention_22_b200 import inputs
@@ -391,6 +434,7 @@ def run_ours(args, world, rank, local):
     clocks.start()
     pre = bench_prefill(args, world, rank, peaks, peak_kind)
     dec = bench_decode(args, world, rank, peaks, peak_kind)
+    bwd = bench_backward(args, world)
     clk = clocks.stop()
     w = pre["w"]
     cpu = None
@@ -416,7 +460,7 @@ def run_ours(args, world, rank, local):
                            "parallelism": f"replicas x{world}",
                            "l2": "3 rotating input sets (~630 MB) > 126 MB L2"},
                 "roofline": pre["roofline"], "tensor": pre["tensor"], "cpu_baseline": cpu,
-                "e2e": pre["e2e"], "decode": dec, "clocks": clk,
+                "e2e": pre["e2e"], "decode": dec, "backward": bwd, "clocks": clk,
                 # per step, two-kernel schedule: the WY kernel, the (empty when every chunk
                 # takes one reference) sub-block WY kernel and the state scan; fused: one kernel
                 "gpu_launches": (1 if args.schedule == "fused" else 3) * args.steps,
