@@ -20,8 +20,12 @@
 //
 // S_{t-1} is needed in reverse order, so the kernel first runs the forward for
 // its rows and stores the state every kSeg tokens (workspace), then, segment by
-// segment from the end, reloads the segment's starting state, recomputes its
-// kSeg tokens keeping S~_t and vh_t in shared memory, and walks them backwards.
+// segment from the end, walks the segment backwards in windows of kWin tokens:
+// for each window (last first) it reloads the segment's starting state,
+// recomputes the forward up to the window's end keeping S~_t of the window's
+// tokens in shared memory, and walks those tokens backwards.  Windows shorter
+// than the segment trade some recomputation for shared memory, i.e. for more
+// resident warps.
 #include "kda_internal.cuh"
 
 namespace kda {
@@ -32,19 +36,22 @@ constexpr int kRows = 16;              // state rows per CTA
 constexpr int kThreads = 8 * kRows;    // one 8-lane group per row
 constexpr int kSeg = 8;                // tokens per checkpoint segment
 
+// kWin: tokens whose S~ is kept at once -- the whole segment (8) when the grid is
+// small, half of it (4, one more resident CTA per SM) when the grid is large.
+template <int kWin>
 struct Smem {
     float al[kSeg][kDK], kk[kSeg][kDK], qs[kSeg][kDK];   // the segment's token vectors
-    float sb[kSeg][kRows][kDK];                          // S~_t of this CTA's rows
+    float sb[kWin][kRows][kDK];                          // S~_t of this CTA's rows (one window)
     float vr[kSeg][kRows], dor[kSeg][kRows], vh[kSeg][kRows];
     float beta[kSeg];
     float red[3][kRows][kDK];                            // per-row partials of dq~, dk, dg
     float redb[kRows];
 };
 
-template <typename TI, int GATE>
+template <typename TI, int GATE, int kWin>
 __global__ void __launch_bounds__(kThreads, 1) kda_recurrent_bwd_kernel(RecurrentBwdArgs a) {
     extern __shared__ float4 smem_raw[];
-    Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
+    Smem<kWin>& sm = *reinterpret_cast<Smem<kWin>*>(smem_raw);
     const int nh = blockIdx.x;
     const int n = nh / a.H, h = nh - n * a.H;
     const int hk = h / (a.H / a.Hk);
@@ -87,8 +94,9 @@ __global__ void __launch_bounds__(kThreads, 1) kda_recurrent_bwd_kernel(Recurren
         x += __shfl_xor_sync(0xffffffffu, x, 4);
         return x;
     };
-    // one forward token from slot j: S <- S~ + e k^T; keeps S~ and vh when `keep`
-    auto fwd_token = [&](float (&S)[16], int j, bool keep) {
+    // one forward token from slot j: S <- S~ + e k^T; keeps S~ (window slot w) and vh when w >= 0
+    auto fwd_token = [&](float (&S)[16], int j, int w) {
+        const bool keep = w >= 0;
         float pa = 0.f;
 #pragma unroll
         for (int m = 0; m < 4; ++m)
@@ -101,7 +109,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_recurrent_bwd_kernel(Recurren
         if (keep) {
 #pragma unroll
             for (int m = 0; m < 4; ++m)
-                *reinterpret_cast<float4*>(&sm.sb[j][rl][ch(m, 0)]) =
+                *reinterpret_cast<float4*>(&sm.sb[w][rl][ch(m, 0)]) =
                     make_float4(S[4 * m], S[4 * m + 1], S[4 * m + 2], S[4 * m + 3]);
             if (sub == 0) sm.vh[j][rl] = pa;
         }
@@ -137,7 +145,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_recurrent_bwd_kernel(Recurren
         __syncthreads();   // the previous segment's slots are read
         for (int j = 0; j < len; ++j) stage(t0 + j, j);
         __syncthreads();
-        for (int j = 0; j < len; ++j) fwd_token(S, j, false);
+        for (int j = 0; j < len; ++j) fwd_token(S, j, -1);
     }
 
     // ---- backward, segment by segment from the end
@@ -148,17 +156,19 @@ __global__ void __launch_bounds__(kThreads, 1) kda_recurrent_bwd_kernel(Recurren
         __syncthreads();
         for (int j = 0; j < len; ++j) stage(t0 + j, j);
         __syncthreads();
+        for (int w0 = ((len - 1) / kWin) * kWin; w0 >= 0; w0 -= kWin) {
+        const int w1 = min(w0 + kWin, len);
         load_rows(S, ck_at(s));   // this thread's own rows: written by it in the forward
-        for (int j = 0; j < len; ++j) fwd_token(S, j, true);
+        for (int j = 0; j < w1; ++j) fwd_token(S, j, j >= w0 ? j - w0 : -1);
         __syncthreads();
-        for (int j = len - 1; j >= 0; --j) {
+        for (int j = w1 - 1; j >= w0; --j) {
             const int t = t0 + j;
             const float b = sm.beta[j], vhv = sm.vh[j][rl], dov = sm.dor[j][rl];
             const float e = b * (sm.vr[j][rl] - vhv);
             float sb[16], pq[16];
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
-                const float4 x = *reinterpret_cast<const float4*>(&sm.sb[j][rl][ch(m, 0)]);
+                const float4 x = *reinterpret_cast<const float4*>(&sm.sb[j - w0][rl][ch(m, 0)]);
                 sb[4 * m] = x.x; sb[4 * m + 1] = x.y; sb[4 * m + 2] = x.z; sb[4 * m + 3] = x.w;
             }
             // o_t = S_t q~:  G += d_out q~^T,  dq~ += S_t^T d_out
@@ -225,36 +235,42 @@ __global__ void __launch_bounds__(kThreads, 1) kda_recurrent_bwd_kernel(Recurren
                     atomicAdd(a.dbeta + tv, sb2);
                 }
             }
-            __syncthreads();   // red is rewritten by the next token
+            __syncthreads();   // red (and, after the window, sb) is rewritten next
+        }
         }
     }
     if (a.dS0) store_rows(a.dS0 + sg, G);
 }
 
+template <typename TI, int GATE, int kWin>
+cudaError_t launch_one(const RecurrentBwdArgs& a, dim3 grid, cudaStream_t st) {
+    auto kern = kda_recurrent_bwd_kernel<TI, GATE, kWin>;
+    const size_t bytes = sizeof(Smem<kWin>);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kThreads, bytes, st>>>(a);
+    return cudaGetLastError();
+}
+
+template <typename TI, int GATE>
+cudaError_t launch_gate(const RecurrentBwdArgs& a, cudaStream_t st) {
+    const dim3 grid((unsigned)(a.N * a.H), (unsigned)((a.d_v + kRows - 1) / kRows));
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    // many CTAs: residency pays more than the recomputation the half window costs
+    const bool wide = (long long)grid.x * grid.y >= 8LL * sms;
+    return wide ? launch_one<TI, GATE, kSeg / 2>(a, grid, st) : launch_one<TI, GATE, kSeg>(a, grid, st);
+}
+
 template <typename TI>
 cudaError_t launch_typed(const RecurrentBwdArgs& a, cudaStream_t st) {
-    const dim3 grid((unsigned)(a.N * a.H), (unsigned)((a.d_v + kRows - 1) / kRows));
-    const size_t bytes = sizeof(Smem);
-    cudaError_t e = cudaSuccess;
     switch (a.gate) {
-        case KDA_GATE_CHANNEL:
-            e = cudaFuncSetAttribute(kda_recurrent_bwd_kernel<TI, KDA_GATE_CHANNEL>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-            if (e == cudaSuccess) kda_recurrent_bwd_kernel<TI, KDA_GATE_CHANNEL><<<grid, kThreads, bytes, st>>>(a);
-            break;
-        case KDA_GATE_SCALAR:
-            e = cudaFuncSetAttribute(kda_recurrent_bwd_kernel<TI, KDA_GATE_SCALAR>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-            if (e == cudaSuccess) kda_recurrent_bwd_kernel<TI, KDA_GATE_SCALAR><<<grid, kThreads, bytes, st>>>(a);
-            break;
-        default:
-            e = cudaFuncSetAttribute(kda_recurrent_bwd_kernel<TI, KDA_GATE_NONE>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-            if (e == cudaSuccess) kda_recurrent_bwd_kernel<TI, KDA_GATE_NONE><<<grid, kThreads, bytes, st>>>(a);
-            break;
+        case KDA_GATE_CHANNEL: return launch_gate<TI, KDA_GATE_CHANNEL>(a, st);
+        case KDA_GATE_SCALAR: return launch_gate<TI, KDA_GATE_SCALAR>(a, st);
+        default: return launch_gate<TI, KDA_GATE_NONE>(a, st);
     }
-    if (e != cudaSuccess) return e;
-    return cudaGetLastError();
 }
 
 }  // namespace

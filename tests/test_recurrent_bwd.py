@@ -70,6 +70,7 @@ CASES = [
     (2, 5, 3, 1, 40, torch.float32, "scalar"),
     (1, 33, 2, 2, 128, torch.float32, "none"),
     (1, 1, 2, 2, 128, torch.bfloat16, "channel_strong"),
+    (4, 13, 40, 20, 128, torch.bfloat16, "channel"),   # 1280 CTAs: the half-window kernel
 ]
 
 
