@@ -70,14 +70,16 @@ def test_bf16(B, T, H, gate, beta, s0, chunk, schedule):
     check(ST, rs, "bf16", "S_T")
 
 
-@pytest.mark.parametrize("gate", ["channel", "channel_strong"])
-def test_whole_width_scan_matches_oracle(gate):
+@pytest.mark.parametrize("gate,qk_div", [("channel", 1), ("channel_strong", 1), ("channel", 2)])
+def test_whole_width_scan_matches_oracle(gate, qk_div):
     """More (sequence, head) pairs than SMs take the whole-width (N = 128) state
     scan: 2 x 90 heads, ragged 130-token sequences, one- and sub-block-reference
-    chunks; every pair against the oracle."""
+    chunks, and grouped value heads (two per q/k head); every pair against the oracle."""
     props = torch.cuda.get_device_properties(0)
     B, T, H = 2, 130, max(90, props.multi_processor_count // 2 + 1)
-    d = inputs.draw(B, T, H, 128, 128, dtype=torch.bfloat16, gate=gate, s0_std=0.02, seed=4242)
+    H += H % 2
+    d = inputs.draw(B, T, H, 128, 128, dtype=torch.bfloat16, gate=gate, s0_std=0.02, seed=4242,
+                    qk_heads=H // qk_div)
     out, ST = run_chunk(d, 64)
     ro, rs = oracle_chunk(d, "channel")
     check(out, ro, "bf16", "out")

@@ -82,3 +82,16 @@ def test_noalloc_over_capacity_runs_the_fused_kernel():
     for (n, h), (ro, rs) in sampled_pairs_oracle(d, [(0, 31)], "channel").items():
         check(o1[n, :, h], ro, "bf16", f"out ({n},{h})")
         check(s1[n, h], rs, "bf16", f"S_T ({n},{h})")
+
+
+@pytest.mark.gpu
+def test_noalloc_grouped_value_heads_equals_workspace():
+    """Grouped value heads through the static scratch: the same kernels and bits as
+    the caller-workspace call."""
+    d = inputs.draw(2, 200, 8, 128, 128, dtype=torch.bfloat16, s0_std=0.02, seed=2205, qk_heads=2)
+    on = to_dev(d)
+    args = (on["q"], on["k"], on["v"], on["g"], on["beta"])
+    o1, s1 = kda.kda_chunk_fwd_noalloc(*args, S0=on["S0"])
+    o2, s2 = kda.kda_chunk_fwd(*args, S0=on["S0"], workspace=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(s1, s2)
