@@ -227,6 +227,8 @@ kda_status_t kda_decode_step(const kda_shape_t* shape, const void* q, const void
  *   dbeta  [N, T, H]
  *   dS0    [N, H, d_v, d_k], or NULL when not wanted.
  * S0, d_ST and dS0 are 16-byte aligned; the workspace (>= the size below) 16 bytes.
+ * dq, dk, dg and dbeta are sums over state rows accumulated with atomic adds, so
+ * their last bits may differ from run to run; dv and dS0 are written directly.
  * Support: d_k = 128, d_v from 1 to 65535*16; else KDA_ERR_UNSUPPORTED.
  */
 kda_status_t kda_recurrent_bwd(const kda_shape_t* shape, const void* q, const void* k,
