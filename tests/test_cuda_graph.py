@@ -1,0 +1,78 @@
+"""The entry points are stream-ordered, allocate nothing and never synchronise,
+so they can be captured in a CUDA graph and replayed: the two-kernel prefill
+(its memset, programmatic-dependent launches and workspace), the fused prefill,
+the decode step and the recurrent pass, replayed bit-identical to eager calls."""
+import pytest
+import torch
+
+import kimi_delta_attention_22_b200 as kda
+from kimi_delta_attention_22_b200 import inputs
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("workspace", [True, None])
+def test_prefill_graph_replay_equals_eager(workspace):
+    d = inputs.draw(2, 300, 4, 128, 128, dtype=torch.bfloat16, s0_std=0.02, seed=808, device="cuda")
+    args = (d["q"], d["k"], d["v"], d["g"], d["beta"])
+    ws = None
+    if workspace:
+        ws = torch.empty(kda.kda_chunk_fwd_workspace_size(d["q"], d["v"], d["g"]), dtype=torch.uint8,
+                         device="cuda")
+    out = torch.empty_like(d["v"])
+    ST = torch.empty(2, 4, 128, 128, dtype=torch.float32, device="cuda")
+    o_ref, s_ref = kda.kda_chunk_fwd(*args, S0=d["S0"], workspace=ws if workspace else None)
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):   # warm-up on the capture stream
+        kda.kda_chunk_fwd(*args, S0=d["S0"], out=out, S_T=ST, workspace=ws if workspace else None)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    out.zero_()
+    ST.zero_()
+    with torch.cuda.graph(g):
+        kda.kda_chunk_fwd(*args, S0=d["S0"], out=out, S_T=ST, workspace=ws if workspace else None)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, o_ref) and torch.equal(ST, s_ref)
+
+
+@pytest.mark.gpu
+def test_decode_and_recurrent_graph_replay():
+    N, H, T = 8, 4, 3
+    d = inputs.draw(N, T, H, 128, 128, dtype=torch.bfloat16, s0_std=0.05, seed=809, device="cuda")
+    steps = [{n: d[n][:, t].contiguous() for n in ("q", "k", "v", "g", "beta")} for t in range(T)]
+    # eager reference: T decode steps, then a recurrent pass over the same tokens
+    S_ref = d["S0"].clone()
+    outs_ref = [kda.kda_decode_step(st["q"], st["k"], st["v"], st["g"], st["beta"], S_ref) for st in steps]
+    S2_ref = S_ref.clone()
+    o2_ref = kda.kda_recurrent_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], S2_ref)
+    torch.cuda.synchronize()
+
+    S = torch.empty_like(d["S0"])
+    S2 = torch.empty_like(d["S0"])
+    outs = [torch.empty(N, H, 128, dtype=torch.bfloat16, device="cuda") for _ in range(T)]
+    o2 = torch.empty_like(d["v"])
+
+    def body():
+        S.copy_(d["S0"])
+        for st, o in zip(steps, outs):
+            kda.kda_decode_step(st["q"], st["k"], st["v"], st["g"], st["beta"], S, out=o)
+        S2.copy_(S)
+        kda.kda_recurrent_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], S2, out=o2)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        body()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        body()
+    g.replay()
+    torch.cuda.synchronize()
+    assert all(torch.equal(a, b) for a, b in zip(outs, outs_ref))
+    assert torch.equal(S, S_ref) and torch.equal(o2, o2_ref) and torch.equal(S2, S2_ref)
