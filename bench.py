@@ -1,11 +1,15 @@
 """Benchmark of the KDA hot path on B200.
 
-One step = one kda_chunk_fwd over the bf16 prefill workload (B=4, H=16,
+One step = one kda_chunk_fwd call over the bf16 prefill workload (B=4, H=16,
 T=2048, d_k=d_v=128, chunk 64, per-channel gates, S0 ~ N(0, 0.02^2)): every
 chunkwise step (cumulative decay, decay-masked products, triangular solve,
-state scan and outputs) runs inside that one launch.  The decode step
+state scan and outputs) runs inside that one call (the WY, sub-block WY and
+state-scan kernels over a preallocated workspace; --schedule fused: the single
+fused kernel).  After it, reported as extra objects of the same line:
+"e2e" (the same step from pinned host buffers, copies included), "decode"
 (256 x 32 heads, d=128, fp32 state in HBM, 128 one-token calls after a
-512-token prefill) is measured after it and reported under "decode".
+512-token prefill) and "backward" (kda_recurrent_bwd, 256 x 32 heads x 16
+tokens).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
