@@ -136,25 +136,76 @@ __device__ __forceinline__ bool decode_slot(const WyParams& p, int slot, long lo
 }
 
 // Off-diagonal 16x16 blocks of T = (I + L)^{-1} from its diagonal blocks T_II, one
-// block column per warp (forward substitution by blocks, no CTA barrier inside):
+// block column per warp (forward substitution by blocks):
 //   T_IJ = -T_II sum_{K=J}^{I-1} L_IK T_KJ        (I > J),
-// each product a 16x16 warp-level tf32 MMA; P is warp-private scratch.
+// each product a 16x16 warp-level tf32 MMA; P is warp-private scratch.  Column 0
+// is the longest chain (T10 -> T20 -> T30): warp 3, on the fourth sub-partition,
+// takes its terms that wait for nothing or only for T10 (L20 T00, L30 T00 + L31 T10)
+// and hands them over through named barriers, in the summation order of the
+// plain column loop.
+__device__ __forceinline__ void named_sync(int id) {
+    asm volatile("bar.sync %0, 64;" ::"r"(id) : "memory");
+}
+__device__ __forceinline__ void named_arrive(int id) {
+    asm volatile("bar.arrive %0, 64;" ::"r"(id) : "memory");
+}
+// The C-fragment pair that blk_store writes, read back.
+__device__ __forceinline__ void blk_load(float (&acc)[2][4], const float* Cm, int ld, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        acc[nt][0] = Cm[g * ld + 8 * nt + 2 * t];
+        acc[nt][1] = Cm[g * ld + 8 * nt + 2 * t + 1];
+        acc[nt][2] = Cm[(g + 8) * ld + 8 * nt + 2 * t];
+        acc[nt][3] = Cm[(g + 8) * ld + 8 * nt + 2 * t + 1];
+    }
+}
 __device__ __forceinline__ void offdiag_columns(float* TF, const float* Lm, float* NS, int warp,
                                                 int lane) {
     auto tf = [&](int I, int J) { return TF + 16 * I * LDT + 16 * J; };
     auto lb = [&](int I, int J) { return Lm + 16 * I * LDT + 16 * J; };
-    if (warp < 3) {
+    auto finish = [&](float (&acc)[2][4], float* P, int I, int J) {   // T_IJ = -T_II acc
+        blk_store(P, LDX, acc, lane, 1.f);
+        __syncwarp();
+        float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        blk_mma(acc2, tf(I, I), LDT, P, LDX, lane);
+        blk_store(tf(I, J), LDT, acc2, lane, -1.f);
+        __syncwarp();
+    };
+    float* XA = NS + 3 * 16 * LDX;   // L20 T00
+    float* XB = NS + 4 * 16 * LDX;   // L30 T00 + L31 T10
+    if (warp == 0) {
+        float* P = NS;
+        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        blk_mma(acc, lb(1, 0), LDT, tf(0, 0), LDT, lane);
+        finish(acc, P, 1, 0);
+        named_arrive(1);   // T10 ready
+        named_sync(2);     // L20 T00 ready
+        blk_load(acc, XA, LDX, lane);
+        blk_mma(acc, lb(2, 1), LDT, tf(1, 0), LDT, lane);
+        finish(acc, P, 2, 0);
+        named_sync(3);     // L30 T00 + L31 T10 ready
+        blk_load(acc, XB, LDX, lane);
+        blk_mma(acc, lb(3, 2), LDT, tf(2, 0), LDT, lane);
+        finish(acc, P, 3, 0);
+    } else if (warp == 3) {
+        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        blk_mma(acc, lb(2, 0), LDT, tf(0, 0), LDT, lane);
+        blk_store(XA, LDX, acc, lane, 1.f);
+        float accb[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        blk_mma(accb, lb(3, 0), LDT, tf(0, 0), LDT, lane);
+        named_arrive(2);
+        named_sync(1);
+        blk_mma(accb, lb(3, 1), LDT, tf(1, 0), LDT, lane);
+        blk_store(XB, LDX, accb, lane, 1.f);
+        named_arrive(3);
+    } else if (warp < 3) {
         const int J = warp;
         float* P = NS + warp * 16 * LDX;
         for (int I = J + 1; I < 4; ++I) {
             float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
             for (int K = J; K < I; ++K) blk_mma(acc, lb(I, K), LDT, tf(K, J), LDT, lane);
-            blk_store(P, LDX, acc, lane, 1.f);
-            __syncwarp();
-            float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-            blk_mma(acc2, tf(I, I), LDT, P, LDX, lane);
-            blk_store(tf(I, J), LDT, acc2, lane, -1.f);
-            __syncwarp();
+            finish(acc, P, I, J);
         }
     }
     __syncthreads();
