@@ -245,6 +245,22 @@ kda_status_t kda_recurrent_fwd(const kda_shape_t* shape, const void* q, const vo
                                const void* v, const float* g, const float* beta, float* S,
                                void* out, void* stream);
 
+/* Failure-detection self-test.  Every wait of the library's tensor-core kernels is
+ * a bounded mbarrier wait: when it runs out, the kernel ORs KDA_DEV_TIMEOUT into
+ * *dev_status, lets its own copies and MMAs in flight land, frees its tensor memory
+ * and returns, so the context stays usable.  This call launches one 128-thread CTA
+ * that takes the same bounded wait, with a budget of budget_us microseconds, on a
+ * barrier of its own shared memory:
+ *   complete = 0: nothing ever arrives, the wait runs out and KDA_DEV_TIMEOUT is
+ *                 ORed into *dev_status;
+ *   complete != 0: one thread arrives first, the wait succeeds and *dev_status is
+ *                 left as it is.
+ * dev_status: device int32 (required, 4-byte aligned).  budget_us: 1 to 1000000,
+ * else KDA_ERR_INVALID_ARG.  Asynchronous on `stream`; read *dev_status after a
+ * sync.  No other memory is touched. */
+kda_status_t kda_selftest_bounded_wait(int32_t* dev_status, uint32_t budget_us, int32_t complete,
+                                       void* stream);
+
 /* Human-readable text for a status code (static storage). */
 const char* kda_status_str(kda_status_t status);
 

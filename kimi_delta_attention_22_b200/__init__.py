@@ -13,7 +13,7 @@ import os
 
 import torch
 
-__all__ = ["kda_chunk_fwd", "kda_recurrent_fwd", "kda_recurrent_bwd", "kda_chunk_fwd_noalloc", "kda_chunk_fwd_workspace_size", "kda_decode_step", "kda_status_str", "library_path", "load_library",
+__all__ = ["kda_chunk_fwd", "kda_recurrent_fwd", "kda_recurrent_bwd", "kda_chunk_fwd_noalloc", "kda_chunk_fwd_workspace_size", "kda_decode_step", "kda_selftest_bounded_wait", "kda_status_str", "library_path", "load_library",
            "KDAError", "KDA_F32", "KDA_BF16", "KDA_GATE_CHANNEL", "KDA_GATE_SCALAR",
            "KDA_GATE_NONE", "KDA_DEV_BAD_SEQLENS", "KDA_DEV_TIMEOUT", "Shape"]
 
@@ -77,6 +77,8 @@ def load_library(path: str | None = None):
     lib.kda_status_str.argtypes = [ctypes.c_int]
     lib.kda_status_str.restype = ctypes.c_char_p
     lib.kda_version.restype = ctypes.c_char_p
+    lib.kda_selftest_bounded_wait.argtypes = [P, ctypes.c_uint32, ctypes.c_int32, P]
+    lib.kda_selftest_bounded_wait.restype = ctypes.c_int
     if path is None:
         _lib = lib
     return lib
@@ -302,3 +304,19 @@ def kda_recurrent_bwd(q, k, v, g, beta, S0, d_out, d_ST=None, want_dS0: bool = T
     if st != 0:
         raise KDAError(st, "kda_recurrent_bwd")
     return dict(dq=dq, dk=dk, dv=dv, dg=dg, dbeta=dbeta, dS0=dS0)
+
+
+def kda_selftest_bounded_wait(dev_status: torch.Tensor, budget_us: int, complete: bool = False,
+                              lib=None) -> None:
+    """kda_selftest_bounded_wait: one CTA takes the kernels' bounded mbarrier wait
+    (budget_us microseconds) on a barrier that never completes (complete=False;
+    KDA_DEV_TIMEOUT is ORed into dev_status) or completes at once (complete=True;
+    dev_status untouched).  dev_status: int32 device tensor; read it after a sync."""
+    _check_cuda(dev_status)
+    if dev_status.dtype != torch.int32 or dev_status.numel() < 1:
+        raise ValueError("dev_status must be an int32 device tensor")
+    lib = lib or load_library()
+    st = lib.kda_selftest_bounded_wait(_ptr(dev_status), int(budget_us), int(bool(complete)),
+                                       _stream_handle(dev_status.device))
+    if st != 0:
+        raise KDAError(st, "kda_selftest_bounded_wait")

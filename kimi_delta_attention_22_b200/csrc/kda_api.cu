@@ -252,4 +252,12 @@ kda_status_t kda_decode_step(const kda_shape_t* sh, const void* q, const void* k
     return from_cuda(kda::launch_decode(a, sh->dtype == KDA_BF16, static_cast<cudaStream_t>(stream)));
 }
 
+kda_status_t kda_selftest_bounded_wait(int32_t* dev_status, uint32_t budget_us, int32_t complete,
+                                       void* stream) {
+    if (dev_status == nullptr || !aligned4(dev_status)) return KDA_ERR_INVALID_ARG;
+    if (budget_us < 1u || budget_us > 1000000u) return KDA_ERR_INVALID_ARG;
+    return from_cuda(kda::launch_selftest_wait(dev_status, 1000ull * budget_us, complete != 0,
+                                               static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

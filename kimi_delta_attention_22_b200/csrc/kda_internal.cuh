@@ -87,6 +87,9 @@ cudaError_t launch_chunk_wy(const ChunkArgs& a, uint8_t* ws, const rec::Layout& 
 cudaError_t launch_chunk_scan(const ChunkArgs& a, const uint8_t* ws, const rec::Layout& lay,
                               cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs& a, bool bf16, cudaStream_t s);
+// One CTA taking the kernels' bounded mbarrier wait (budget_ns) on a barrier that
+// completes (complete) or never does; on expiry it ORs KDA_DEV_TIMEOUT into *dev_status.
+cudaError_t launch_selftest_wait(int32_t* dev_status, uint64_t budget_ns, bool complete, cudaStream_t s);
 
 // Rows [bos, eos) of the packed token axis that sequence n covers.  Returns
 // false (and flags dev_status) when cu_seqlens is inconsistent.
