@@ -1,7 +1,7 @@
 """Time kda_chunk_fwd on the named synthetic workloads (one GPU).
 
     python -m kimi_delta_attention_22_b200.measure [--workloads a,b,...] [--schedule split|fused]
-                                                   [--iters 10] [--warmup 3]
+                                                   [--iters 10] [--warmup 3] [--shape B,T,H]
     python -m kimi_delta_attention_22_b200.measure --recurrent [--tokens 1,4,16,64]
 
 For each workload: inputs drawn once on the device (kimi_delta_attention_22_b200.inputs),
@@ -22,6 +22,7 @@ from __future__ import annotations
 
 import argparse
 import ctypes
+import dataclasses
 import json
 import os
 import statistics
@@ -43,8 +44,15 @@ def peaks():
         return json.load(f)
 
 
-def measure(name: str, schedule: str, iters: int, warmup: int) -> dict:
+def measure(name: str, schedule: str, iters: int, warmup: int, shape=None) -> dict:
+    """shape = (B, T, H): the workload's recipe at other sizes (dense workloads only)."""
     w = inputs.WORKLOADS[name]
+    if shape is not None:
+        if w.varlen:
+            raise ValueError("--shape applies to dense workloads only")
+        B, T, H = shape
+        w = dataclasses.replace(w, name=f"{name}@B{B}_T{T}_H{H}", B=B, T=T, H=H,
+                                qk_heads=(H * w.qk_heads // w.H if w.qk_heads else 0))
     d = inputs.workload_inputs(w, device="cuda")
     cu = d.get("cu_seqlens")
     ws = None
@@ -73,7 +81,7 @@ def measure(name: str, schedule: str, iters: int, warmup: int) -> dict:
         times.append(a.elapsed_time(b))
     ms = statistics.median(times)
     nbytes, flops = prefill_bytes(w), prefill_flops(w)
-    res = {"workload": name, "schedule": schedule, "ms_per_call": ms,
+    res = {"workload": w.name, "schedule": schedule, "ms_per_call": ms,
            "tokens_per_s": w.tokens / (ms * 1e-3), "hbm_gbs": nbytes / (ms * 1e-3) / 1e9,
            "tflops": flops / (ms * 1e-3) / 1e12, "algorithmic_bytes": nbytes, "flops": flops,
            "iters": iters}
@@ -171,6 +179,7 @@ def main():
     ap.add_argument("--schedule", choices=["split", "fused"], default="split")
     ap.add_argument("--iters", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--shape", default=None, help="B,T,H: run the named dense workloads' recipe at these sizes")
     ap.add_argument("--recurrent", action="store_true")
     ap.add_argument("--tokens", default="1,4,16,64")
     ap.add_argument("--backward", default=None,
@@ -188,8 +197,9 @@ def main():
         for T in (int(x) for x in args.tokens.split(",")):
             print(json.dumps(measure_recurrent(T, args.iters, args.warmup)), flush=True)
         return
+    shape = tuple(int(x) for x in args.shape.split(",")) if args.shape else None
     for name in args.workloads.split(","):
-        print(json.dumps(measure(name, args.schedule, args.iters, args.warmup)), flush=True)
+        print(json.dumps(measure(name, args.schedule, args.iters, args.warmup, shape)), flush=True)
 
 
 if __name__ == "__main__":
