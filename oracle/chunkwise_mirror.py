@@ -230,3 +230,41 @@ def chunk_backward(q, k, v, g, beta, S0, d_out, d_ST=None, chunk=16, gate="chann
     if S0 is None:
         res["dS0"] = None
     return res
+
+
+def chunk_records_one_pair(k, q, g, beta, chunk):
+    """Per chunk of one (sequence, head): the state-independent operands the
+    forward's WY records hold -- W = T diag(beta) (K e^Gamma), Qg = Q~ e^Gamma,
+    Kd = K e^{gamma - Gamma}, lower(Qp) (the inclusive A_qk) and gamma = Gamma_last."""
+    k, q, g, beta = (np.asarray(a, dtype=np.float64) for a in (k, q, g, beta))
+    T, dk = k.shape
+    qs = q / np.sqrt(dk)
+    recs = []
+    for c0 in range(0, T, chunk):
+        sl = slice(c0, min(c0 + chunk, T))
+        K, Q, G, b = k[sl], qs[sl], g[sl], beta[sl]
+        C = K.shape[0]
+        Gam = np.cumsum(G, axis=0)
+        lower = np.tril(np.ones((C, C), dtype=bool))
+        strict = np.tril(np.ones((C, C), dtype=bool), -1)
+        R = np.where(lower[:, :, None],
+                     np.exp(np.where(lower[:, :, None], Gam[:, None, :] - Gam[None, :, :], 0.0)), 0.0)
+        A = np.einsum("jc,ijc,ic->ij", K, R, K)
+        Tinv = np.linalg.inv(np.eye(C) + np.where(strict, b[:, None] * A, 0.0))
+        recs.append(dict(rows=sl, W=Tinv @ (b[:, None] * K * np.exp(Gam)), Qg=Q * np.exp(Gam),
+                         Kd=K * np.exp(Gam[-1][None, :] - Gam),
+                         AQ=np.einsum("jc,ijc,ic->ij", K, R, Q), gamma=Gam[-1]))
+    return recs
+
+
+def reverse_state_scan(recs, d_out, d_ST):
+    """dL/dS0 of one (sequence, head) from the records alone, chunk by chunk in
+    reverse: dE = Kd dS^T + lower(Qp)^T dO, then
+    dS <- dS Diag(e^gamma) + dO^T Qg - dE^T W (using (beta . dEbar)^T K e^Gamma = dE^T W)."""
+    d_out = np.asarray(d_out, dtype=np.float64)
+    dS = np.array(d_ST, dtype=np.float64, copy=True)
+    for r in reversed(recs):
+        dO = d_out[r["rows"]]
+        dE = r["Kd"] @ dS.T + r["AQ"].T @ dO
+        dS = dS * np.exp(r["gamma"])[None, :] + dO.T @ r["Qg"] - dE.T @ r["W"]
+    return dS

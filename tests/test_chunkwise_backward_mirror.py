@@ -58,3 +58,16 @@ def test_chunk_backward_strong_decay():
     d = _inputs(8, T=20)
     d["g"] = -5.0 * np.random.default_rng(9).random(d["g"].shape)
     _compare(d, 8, "channel")
+
+
+@pytest.mark.parametrize("chunk", [1, 8, 16])
+def test_reverse_state_scan_from_records_alone(chunk):
+    """The sequential part of the chunkwise backward needs only the forward's
+    record operands (W, Qg, Kd, lower(Qp), gamma): its dS0 equals autograd's."""
+    d = _inputs(20 + chunk, B=1, T=37, H=1)
+    ref = ob.backward(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], d["d_out"], d["d_ST"])
+    recs = cm.chunk_records_one_pair(d["k"][0, :, 0], d["q"][0, :, 0], d["g"][0, :, 0],
+                                     d["beta"][0, :, 0], chunk)
+    dS0 = cm.reverse_state_scan(recs, d["d_out"][0, :, 0], d["d_ST"][0, 0])
+    r = ref["dS0"].numpy()[0, 0]
+    assert np.max(np.abs(dS0 - r)) <= 1e-12 * max(1.0, np.max(np.abs(r)))
