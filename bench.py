@@ -4,12 +4,15 @@ One step = one kda_chunk_fwd call over the bf16 prefill workload (B=4, H=16,
 T=2048, d_k=d_v=128, chunk 64, per-channel gates, S0 ~ N(0, 0.02^2)): every
 chunkwise step (cumulative decay, decay-masked products, triangular solve,
 state scan and outputs) runs inside that one call (the WY, sub-block WY and
-state-scan kernels over a preallocated workspace; --schedule fused: the single
-fused kernel).  After it, reported as extra objects of the same line:
-"e2e" (the same step from pinned host buffers, copies included), "decode"
-(256 x 32 heads, d=128, fp32 state in HBM, 128 one-token calls after a
-512-token prefill) and "backward" (kda_recurrent_bwd, 256 x 32 heads x 16
-tokens).
+state-scan kernels over a preallocated workspace; --schedule pool: the same
+kernels with no workspace passed, so each call takes its scratch from the
+stream-ordered memory pool).  After it, reported as extra objects of the same
+line: "e2e" (the same step from pinned host buffers, copies included),
+"no_workspace" (the same call without a workspace), "varlen" (8 packed
+sequences, 65,536 tokens, 32 heads) and "sweep" (B=8, H=64, T=8192 in six
+gate / beta regimes), each with its own roofline; "decode" (256 x 32 heads,
+d=128, fp32 state in HBM, 128 one-token calls after a 512-token prefill) and
+"backward" (kda_recurrent_bwd, 256 x 32 heads x 16 tokens).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -40,6 +43,10 @@ from kimi_delta_attention_22_b200.roofline import prefill_bytes, prefill_flops
 METRIC = "KDA prefill tokens/s (% bf16 TC peak); decode step HBM GB/s (% of peak)"
 WORKLOAD = "prefill_b4_h16_t2048"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+SPEC_HBM_GBS = 7700.0   # nominal HBM3e bandwidth of one B200 (context for fractions of the copy peak)
+PREFILL_SRC = ["kimi_delta_attention_22_b200/csrc/kda_chunk_wy.cu",
+               "kimi_delta_attention_22_b200/csrc/kda_chunk_scan.cu",
+               "kimi_delta_attention_22_b200/csrc/kda_chunk_record.cuh"]
 
 
 # ------------------------------------------------------------------ helpers
@@ -230,8 +237,8 @@ def bench_prefill(args, world, rank, peaks, peak_kind):
     outs = [torch.empty_like(s["v"]) for s in sets]
     STs = [torch.empty(w.B, w.H, w.d_v, w.d_k, dtype=torch.float32, device=dev) for _ in sets]
     # scratch of the two-kernel schedule, allocated once outside the timed region
-    # (--schedule fused: no workspace, the single fused kernel)
-    ws = None if args.schedule == "fused" else torch.empty(
+    # (--schedule pool: no workspace, each call draws it from the stream-ordered pool)
+    ws = None if args.schedule == "pool" else torch.empty(
         kda.kda_chunk_fwd_workspace_size(sets[0]["q"], sets[0]["v"], sets[0]["g"], chunk=w.chunk),
         dtype=torch.uint8, device=dev)
 
@@ -264,10 +271,7 @@ def bench_prefill(args, world, rank, peaks, peak_kind):
     flops = prefill_flops(w)
     achieved_gbs = alg_bytes / (launch_ms * 1e-3) / 1e9
     achieved_tf = flops / (launch_ms * 1e-3) / 1e12
-    src = (["kimi_delta_attention_22_b200/csrc/kda_chunk_tc.cu"] if args.schedule == "fused" else
-           ["kimi_delta_attention_22_b200/csrc/kda_chunk_wy.cu",
-            "kimi_delta_attention_22_b200/csrc/kda_chunk_scan.cu"])
-    traffic = dram_traffic("chunk_fwd_" + args.schedule, WORKLOAD, src)
+    traffic = dram_traffic("chunk_fwd", WORKLOAD, PREFILL_SRC)
     res = {
         "w": w, "elapsed_ms": elapsed_ms, "launch_ms": launch_ms,
         "value": world * args.steps * w.tokens / (elapsed_ms * 1e-3),
@@ -275,13 +279,33 @@ def bench_prefill(args, world, rank, peaks, peak_kind):
                      "unit": "GB/s", "frac": achieved_gbs / peaks["hbm_gbs"],
                      "traffic": traffic, "peak_source": f"{peak_kind} hbm_gbs",
                      "algorithmic_bytes_per_launch": alg_bytes,
-                     "kernel": ("kda_chunk_fwd call (fused kernel)" if args.schedule == "fused"
-                                else "kda_chunk_fwd call (WY, sub-block WY and state-scan kernels)")},
+                     "kernel": "kda_chunk_fwd call (WY, sub-block WY and state-scan kernels)"},
         "tensor": {"achieved_tflops": achieved_tf, "flops_per_launch": flops,
                    "peak_tflops": peaks["bf16_tflops"],
                    "frac": achieved_tf / peaks["bf16_tflops"],
                    "peak_source": f"{peak_kind} bf16_tflops (burst)"},
     }
+    # ---- the same call with no workspace: the scratch comes from the stream-ordered
+    #      pool (cudaMallocAsync / cudaFreeAsync on the call's stream) every call
+    nw_iters = max(5, min(args.steps, 20))
+    for i in range(2):
+        s = sets[i % n_sets]
+        kda.kda_chunk_fwd(s["q"], s["k"], s["v"], s["g"], s["beta"], S0=s["S0"], chunk=w.chunk,
+                          out=outs[i % n_sets], S_T=STs[i % n_sets], workspace=None)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(nw_iters):
+        s = sets[i % n_sets]
+        kda.kda_chunk_fwd(s["q"], s["k"], s["v"], s["g"], s["beta"], S0=s["S0"], chunk=w.chunk,
+                          out=outs[i % n_sets], S_T=STs[i % n_sets], workspace=None)
+    b.record(stream)
+    torch.cuda.synchronize()
+    nw_ms = max_over_ranks(a.elapsed_time(b), world) / nw_iters
+    res["no_workspace"] = {"ms_per_call": nw_ms, "iters": nw_iters,
+                           "value": world * w.tokens / (nw_ms * 1e-3), "unit": "tokens/s",
+                           "vs_workspace": nw_ms / (elapsed_ms / args.steps),
+                           "scratch": "cudaMallocAsync / cudaFreeAsync on the call's stream"}
     # ---- end to end through the public API with host buffers: every step copies
     #      its inputs from pinned host memory, runs the call and reads out and S_T
     #      back, all inside the timed region.  Steps are double-buffered on three
@@ -343,6 +367,57 @@ def bench_prefill(args, world, rank, peaks, peak_kind):
     del sets, outs, STs, dbufs, ws
     torch.cuda.empty_cache()
     return res
+
+
+def bench_workload(name, world, peaks, peak_kind, iters=5, warmup=2):
+    """One named workload of the larger configurations: inputs drawn once on the
+    device (larger than L2), the workspace allocated once, `warmup` untimed calls,
+    then `iters` calls back to back between two CUDA events."""
+    import kimi_delta_attention_22_b200 as kda
+    from kimi_delta_attention_22_b200 import inputs
+
+    w = inputs.WORKLOADS[name]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream(dev)
+    d = inputs.workload_inputs(w, device=dev)
+    cu = d.get("cu_seqlens")
+    ws = torch.empty(kda.kda_chunk_fwd_workspace_size(d["q"], d["v"], d["g"], cu_seqlens=cu, chunk=w.chunk),
+                     dtype=torch.uint8, device=dev)
+    out = torch.empty_like(d["v"])
+    N = w.num_seqs if w.varlen else w.B
+    S_T = torch.empty(N, w.H, w.d_v, w.d_k, dtype=torch.float32, device=dev)
+
+    def call():
+        kda.kda_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], S0=d["S0"], cu_seqlens=cu,
+                          chunk=w.chunk, out=out, S_T=S_T, workspace=ws)
+
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(iters):
+        call()
+    b.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(a.elapsed_time(b), world) / iters
+    nbytes, flops = prefill_bytes(w), prefill_flops(w)
+    gbs, tf = nbytes / (ms * 1e-3) / 1e9, flops / (ms * 1e-3) / 1e12
+    del d, ws, out, S_T
+    torch.cuda.empty_cache()
+    return {"workload": name, "ms_per_call": ms, "iters": iters,
+            "value": world * w.tokens / (ms * 1e-3), "unit": "tokens/s",
+            "config": {"B": w.B, "T": w.T, "H": w.H, "gate": w.gate, "beta": w.beta,
+                       "varlen": w.varlen, "num_seqs": N},
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"], "peak_source": f"{peak_kind} hbm_gbs",
+                         "algorithmic_bytes_per_launch": nbytes,
+                         "traffic": dram_traffic("chunk_fwd", name, PREFILL_SRC)},
+            "tensor": {"achieved_tflops": tf, "flops_per_launch": flops, "peak_tflops": peaks["bf16_tflops"],
+                       "frac": tf / peaks["bf16_tflops"], "peak_source": f"{peak_kind} bf16_tflops (burst)"},
+            "gpu_launches": 3 * iters + (1 if w.varlen else 0) * iters}
 
 
 def bench_backward(args, world):
@@ -417,6 +492,9 @@ def bench_decode(args, world, rank, peaks, peak_kind):
     state_bytes = N * H * dv * dk * 4
     per_step = 2 * state_bytes + N * H * (2 * (2 * dk + dv) + 4 * dk + 4)
     gbs = per_step / (us * 1e-6) / 1e9
+    # some state lines are still in the 126 MB L2 from the previous step, so the
+    # algorithmic bytes over the copy peak can exceed 1; frac_spec divides by the nominal
+    # HBM3e bandwidth instead, and the ncu DRAM bytes of the same step sit in "traffic"
     del dec, S
     torch.cuda.empty_cache()
     return {"metric": "decode step HBM GB/s", "value": world * gbs, "unit": "GB/s",
@@ -425,6 +503,8 @@ def bench_decode(args, world, rank, peaks, peak_kind):
                        "state_MB": state_bytes / 1e6, "state_from": f"{D['prefill_T']}-token prefill"},
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / peaks["hbm_gbs"], "peak_source": f"{peak_kind} hbm_gbs",
+                         "frac_spec": gbs / SPEC_HBM_GBS,
+                         "frac_note": "above 1 when state lines stay in L2 between steps",
                          "algorithmic_bytes_per_launch": per_step,
                          "traffic": dram_traffic("decode", D["name"],
                                                  ["kimi_delta_attention_22_b200/csrc/kda_decode.cu"]),
@@ -437,6 +517,11 @@ def run_ours(args, world, rank, local):
     clocks = ClockSampler(local)
     clocks.start()
     pre = bench_prefill(args, world, rank, peaks, peak_kind)
+    big = {}
+    if not args.quick:
+        big["varlen"] = bench_workload("varlen_h32_t65536", world, peaks, peak_kind)
+        big["sweep"] = [bench_workload(f"sweep_b8_h64_t8192_{g}_beta{b}", world, peaks, peak_kind)
+                        for g in ("none", "scalar", "channel_strong") for b in ("one", "sigmoid")]
     dec = bench_decode(args, world, rank, peaks, peak_kind)
     bwd = bench_backward(args, world)
     clk = clocks.stop()
@@ -464,13 +549,14 @@ def run_ours(args, world, rank, local):
                            "parallelism": f"replicas x{world}",
                            "l2": "3 rotating input sets (~630 MB) > 126 MB L2"},
                 "roofline": pre["roofline"], "tensor": pre["tensor"], "cpu_baseline": cpu,
-                "e2e": pre["e2e"], "decode": dec, "backward": bwd, "clocks": clk,
-                # per step, two-kernel schedule: the WY kernel, the (empty when every chunk
-                # takes one reference) sub-block WY kernel and the state scan; fused: one kernel
-                "gpu_launches": (1 if args.schedule == "fused" else 3) * args.steps,
-                "schedule": ("fused (one kernel per sequence, head, value tile)"
-                             if args.schedule == "fused" else
-                             "two-kernel (parallel WY records + sequential state scan)"),
+                "e2e": pre["e2e"], "no_workspace": pre["no_workspace"], **big,
+                "decode": dec, "backward": bwd, "clocks": clk,
+                # per step: the WY kernel, the (empty when every chunk takes one reference)
+                # sub-block WY kernel and the state scan
+                "gpu_launches": 3 * args.steps,
+                "schedule": ("two-kernel (parallel WY records + sequential state scan), "
+                             + ("scratch from the stream-ordered pool" if args.schedule == "pool"
+                                else "preallocated workspace")),
                 "kernel_ms_per_launch": pre["launch_ms"]}
         print(json.dumps(line), flush=True)
 
@@ -481,8 +567,10 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--schedule", choices=["split", "fused"], default="split",
-                    help="prefill schedule: two kernels over a workspace (default) or the fused kernel")
+    ap.add_argument("--schedule", choices=["workspace", "pool"], default="workspace",
+                    help="prefill scratch: a preallocated workspace (default) or none (stream-ordered pool)")
+    ap.add_argument("--quick", action="store_true",
+                    help="skip the varlen and sweep workloads")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -23,9 +23,10 @@
  *   - All tensor pointers are DEVICE pointers owned by the caller, contiguous,
  *     row-major.  q, k, v, out, per-channel g and every state are 16-byte
  *     aligned (TMA and 128-bit loads); beta, scalar g and cu_seqlens need
- *     only their 4-byte element alignment.  The library allocates no memory
- *     (scratch comes from the caller's workspace) and keeps no state between
- *     calls.
+ *     only their 4-byte element alignment.  Scratch comes from the caller's
+ *     workspace; the one exception is kda_chunk_fwd called without one, which
+ *     takes it from the device's stream-ordered memory pool (see there).  No
+ *     state is kept between calls.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
  *     default stream) and never synchronise.  Host-side validation happens
  *     before any launch and returns an error status with nothing launched.
@@ -51,7 +52,9 @@ typedef enum {
     KDA_ERR_UNSUPPORTED = 2,  /* valid but not implemented (head size, chunk, dtype) */
     KDA_ERR_MISALIGNED = 3,   /* a pointer breaks its alignment rule (see above) */
     KDA_ERR_CUDA = 4,         /* a CUDA launch or attribute call failed */
-    KDA_ERR_TIMEOUT = 5       /* reserved: a bounded device wait expired */
+    KDA_ERR_TIMEOUT = 5,      /* reserved: a bounded device wait expired */
+    KDA_ERR_TOO_LARGE = 6     /* kda_chunk_fwd_noalloc: the shape needs more scratch than
+                                 the library's static array holds */
 } kda_status_t;
 
 /* Element type of q, k, v and out.  g, beta and every state are always fp32. */
@@ -123,17 +126,21 @@ typedef struct {
  *             shape the fp32 path takes (CUDA-core path).
  *   KDA_F32:  d_k, d_v multiples of 16 in [16, 128], chunk in {16, 32, 64}.
  *   Anything else returns KDA_ERR_UNSUPPORTED.
- * Workspace (caller-owned device memory, 256-byte aligned, contents need no
- *   initialisation and are garbage afterwards):
- *   workspace_bytes >= kda_chunk_fwd_workspace_size(shape) selects, on the
- *   tensor-core path, the two-kernel schedule: every (chunk, head) computes its
- *   state-independent operands in parallel into the workspace, then one short
- *   sequential scan per (sequence, head) applies the state.  With workspace ==
- *   NULL (workspace_bytes ignored) one fused kernel walks each sequence and
- *   nothing else is needed.  A non-NULL workspace that is too small or
- *   misaligned returns KDA_ERR_INVALID_ARG / KDA_ERR_MISALIGNED.  Both
- *   schedules compute the same result up to rounding order.  The CUDA-core
- *   path ignores the workspace.
+ * Schedule and scratch (tensor-core path): every (chunk, head) first computes
+ *   its state-independent operands in parallel into a scratch buffer of
+ *   kda_chunk_fwd_workspace_size(shape) bytes (about 73 KB per (chunk, head)),
+ *   then one sequential scan per (sequence, head) applies the state.
+ *   workspace != NULL: caller-owned device memory, 256-byte aligned, at least
+ *     that many bytes (else KDA_ERR_MISALIGNED / KDA_ERR_INVALID_ARG); contents
+ *     need no initialisation and are garbage afterwards.
+ *   workspace == NULL (workspace_bytes ignored): the scratch is allocated with
+ *     cudaMallocAsync on `stream` from the current device's default memory pool
+ *     and released with cudaFreeAsync on `stream` after the kernels that read it,
+ *     so the call stays stream-ordered (and can be captured in a CUDA graph).  A
+ *     failed allocation returns KDA_ERR_CUDA with nothing launched.  Callers
+ *     that must not allocate pass a workspace or use kda_chunk_fwd_noalloc.
+ *   The results do not depend on where the scratch lives.  The CUDA-core path
+ *   uses no scratch and ignores the workspace.
  */
 kda_status_t kda_chunk_fwd(const kda_shape_t* shape, const void* q, const void* k,
                            const void* v, const float* g, const float* beta,
@@ -145,20 +152,35 @@ kda_status_t kda_chunk_fwd(const kda_shape_t* shape, const void* q, const void* 
  * Bytes of workspace the two-kernel schedule of kda_chunk_fwd needs for this
  * shape; varlen != 0 for a packed batch (a cu_seqlens array will be passed).
  * Returns 0 for a NULL shape or for shapes whose path uses no workspace (the
- * fp32 CUDA-core path).  About 73 KB per (chunk, head) plus bookkeeping.
+ * fp32 CUDA-core path).  74,240 bytes per (chunk, head) plus bookkeeping.
  */
 size_t kda_chunk_fwd_workspace_size(const kda_shape_t* shape, int varlen);
 
 /*
- * kda_chunk_fwd_noalloc -- kda_chunk_fwd with library-owned scratch.
+ * kda_chunk_fwd_noalloc -- kda_chunk_fwd for callers that cannot allocate.
  *
- * Same operation, layouts, support and errors as kda_chunk_fwd, with no
- * workspace argument: when the shape's workspace fits a 160 MiB scratch
- * array that the library reserves in device memory at load time (module
- * static storage; nothing is allocated per call), the two-kernel schedule
- * runs on it; otherwise the fused kernel runs.  The scratch is shared by
- * every call in the process: calls on different streams that may overlap
- * must be ordered by the caller.
+ * The paper has no counterpart: this is an allocation-free way into the same
+ * prefill.  Some callers may not call cudaMalloc (or cudaMallocAsync) at all:
+ * code running under an allocator that owns all device memory, inside a
+ * region where allocation is forbidden (a CUDA graph being captured by a
+ * framework that does not accept allocation nodes, a real-time loop), or a
+ * plugin whose host forbids it.  This entry point takes no workspace and
+ * allocates nothing: the scratch is a file-scope __device__ array of 160 MiB
+ * (167,772,160 bytes) inside the library, which every GPU that loads the library
+ * holds until the process exits.
+ *
+ * Same operation, layouts, support and errors as kda_chunk_fwd, plus:
+ *   - shapes whose scratch (kda_chunk_fwd_workspace_size) exceeds 160 MiB return
+ *     KDA_ERR_TOO_LARGE with nothing launched (4 sequences x 16 heads x 2048
+ *     tokens fit; split larger batches into calls that fit);
+ *   - the first call on a device resolves the array's device address with
+ *     cudaGetSymbolAddress (this may load the library's module there, which
+ *     reserves the 160 MiB) and caches it; make that first call before any stream
+ *     capture, as module loading cannot happen inside one;
+ *   - every call on a device shares the one array and leaves its contents
+ *     behind (each call overwrites what it reads, so no clearing is needed):
+ *     calls that may overlap on the GPU (different streams, or several host
+ *     threads) race on it and must be ordered by the caller.
  */
 kda_status_t kda_chunk_fwd_noalloc(const kda_shape_t* shape, const void* q, const void* k,
                                    const void* v, const float* g, const float* beta,

@@ -24,7 +24,7 @@ KDA_F32, KDA_BF16 = 0, 1
 KDA_GATE_CHANNEL, KDA_GATE_SCALAR, KDA_GATE_NONE = 0, 1, 2
 KDA_DEV_BAD_SEQLENS, KDA_DEV_TIMEOUT = 1, 2
 _STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED",
-           3: "KDA_ERR_MISALIGNED", 4: "KDA_ERR_CUDA", 5: "KDA_ERR_TIMEOUT"}
+           3: "KDA_ERR_MISALIGNED", 4: "KDA_ERR_CUDA", 5: "KDA_ERR_TIMEOUT", 6: "KDA_ERR_TOO_LARGE"}
 
 
 class KDAError(RuntimeError):
@@ -144,9 +144,10 @@ def kda_chunk_fwd(q, k, v, g, beta, S0=None, cu_seqlens=None, chunk: int = 64, o
     Returns (out, S_T); S_T is None when want_state is False and no S_T buffer
     is given.
 
-    workspace: True allocates the scratch of the two-kernel schedule with torch
-    (when the shape takes a path that uses one), a uint8 CUDA tensor supplies
-    it, None / False runs the single fused kernel with no scratch.
+    workspace: True allocates the tensor-core path's scratch with torch (when the
+    shape takes a path that uses one), a uint8 CUDA tensor supplies it, and None /
+    False passes no workspace, so that the library takes the scratch from the
+    device's stream-ordered memory pool on the current stream.
     """
     _check_cuda(q, k, v, g, beta, S0, cu_seqlens, out, S_T, dev_status)
     B, T, Hk, Dk = q.shape

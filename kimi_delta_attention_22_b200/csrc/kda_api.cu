@@ -1,22 +1,31 @@
 // kda_api.cu -- the C ABI of include/kda.h: host-side validation and kernel
-// selection.  Nothing here allocates memory or synchronises; every check runs
-// before any launch, so a rejected call launches nothing.
+// selection.  Every check runs before any launch, so a rejected call launches
+// nothing, and nothing here synchronises.  The only memory this file obtains is
+// the tensor-core prefill's scratch when the caller passes no workspace: it is
+// taken from the device's stream-ordered pool (cudaMallocAsync) and given back
+// on the same stream after the kernels that use it.
+#include <atomic>
 #include <stdint.h>
 
 #include "kda_internal.cuh"
 
 namespace kda {
 size_t chunk_f32_smem_bytes(int C, int D, int V);
-bool chunk_tc_supported(int D, int V, int C);
 }  // namespace kda
 
 namespace {
 
-// Scratch of kda_chunk_fwd_noalloc: module-static device memory, reserved when
-// the library is loaded; 160 MiB holds the records of 2,200+ (chunk, head)
-// pairs (e.g. 4 sequences x 16 heads x 2048 tokens).
+// Scratch of kda_chunk_fwd_noalloc: a file-scope device array that every device
+// which loads this module holds until the process exits.  160 MiB holds the records
+// of 2,200+ (chunk, head) pairs (e.g. 4 sequences x 16 heads x 2048 tokens).
 constexpr size_t kStaticScratchBytes = (size_t)160 << 20;
 static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
+// Its device address, resolved once per device (host code cannot use the symbol itself).
+constexpr int kMaxDevices = 64;
+std::atomic<void*> g_static_scratch_addr[kMaxDevices];
+
+// The tensor-core prefill: bf16 q/k/v with d_k = d_v = 128 and chunks of 64.
+bool tc_supports(int D, int V, int C) { return D == 128 && V == 128 && C == 64; }
 
 bool aligned16(const void* p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void* p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
@@ -46,6 +55,7 @@ const char* kda_status_str(kda_status_t s) {
         case KDA_ERR_MISALIGNED: return "pointer not 16-byte aligned";
         case KDA_ERR_CUDA: return "CUDA launch error";
         case KDA_ERR_TIMEOUT: return "bounded device wait expired";
+        case KDA_ERR_TOO_LARGE: return "shape needs more scratch than the library's static array holds";
     }
     return "unknown status";
 }
@@ -54,7 +64,7 @@ const char* kda_version(void) { return "libkda 0.2 (sm_100a)"; }
 
 size_t kda_chunk_fwd_workspace_size(const kda_shape_t* sh, int varlen) {
     if (sh == nullptr || sh->B < 0 || sh->T < 0 || sh->H <= 0 || sh->num_seqs < 0) return 0;
-    if (sh->dtype != KDA_BF16 || !kda::chunk_tc_supported(sh->d_k, sh->d_v, sh->chunk)) return 0;
+    if (sh->dtype != KDA_BF16 || !tc_supports(sh->d_k, sh->d_v, sh->chunk)) return 0;
     return kda::rec::layout(sh->B, sh->T, sh->H, sh->num_seqs, varlen != 0).bytes;
 }
 
@@ -86,15 +96,16 @@ kda_status_t kda_chunk_fwd(const kda_shape_t* sh, const void* q, const void* k, 
 
     const bool bf16 = sh->dtype == KDA_BF16;
     const int C = sh->chunk;
-    const bool tc = bf16 && kda::chunk_tc_supported(D, V, C);
+    const bool tc = bf16 && tc_supports(D, V, C);
     if (!tc && !f32path_supports(D, V, C)) return KDA_ERR_UNSUPPORTED;
     kda::rec::Layout lay{};
-    const bool split = tc && workspace != nullptr;
-    if (split) {
-        if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KDA_ERR_MISALIGNED;
+    if (tc) {
         lay = kda::rec::layout(B, T, H, N, cu_seqlens != nullptr);
-        if (workspace_bytes < lay.bytes) return KDA_ERR_INVALID_ARG;
         if (lay.slots * H > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+        if (workspace != nullptr) {
+            if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KDA_ERR_MISALIGNED;
+            if (workspace_bytes < lay.bytes) return KDA_ERR_INVALID_ARG;
+        }
     }
     if (N == 0) return KDA_OK;
 
@@ -106,13 +117,18 @@ kda_status_t kda_chunk_fwd(const kda_shape_t* sh, const void* q, const void* k, 
     a.Hk = Hk;
     a.scale = 1.0f / sqrtf((float)D);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (split) {
-        uint8_t* ws = static_cast<uint8_t*>(workspace);
-        cudaError_t e = kda::launch_chunk_wy(a, ws, lay, st);
-        if (e == cudaSuccess) e = kda::launch_chunk_scan(a, ws, lay, st);
-        return from_cuda(e);
+    if (!tc) return from_cuda(kda::launch_chunk_f32path(a, bf16, st));
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const bool pooled = ws == nullptr;   // scratch from the stream-ordered pool (256-byte aligned)
+    if (pooled && cudaMallocAsync(reinterpret_cast<void**>(&ws), lay.bytes, st) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    cudaError_t e = kda::launch_chunk_wy(a, ws, lay, st);
+    if (e == cudaSuccess) e = kda::launch_chunk_scan(a, ws, lay, st);
+    if (pooled) {
+        const cudaError_t f = cudaFreeAsync(ws, st);
+        if (e == cudaSuccess) e = f;
     }
-    return from_cuda(tc ? kda::launch_chunk_tc(a, st) : kda::launch_chunk_f32path(a, bf16, st));
+    return from_cuda(e);
 }
 
 kda_status_t kda_chunk_fwd_noalloc(const kda_shape_t* sh, const void* q, const void* k,
@@ -120,13 +136,21 @@ kda_status_t kda_chunk_fwd_noalloc(const kda_shape_t* sh, const void* q, const v
                                    const int32_t* cu_seqlens, void* out, float* S_T, void* stream) {
     if (sh == nullptr) return KDA_ERR_INVALID_ARG;
     const size_t need = kda_chunk_fwd_workspace_size(sh, cu_seqlens != nullptr);
-    const bool any = sh->num_seqs > 0 && (long long)sh->B * sh->T > 0;
-    void* ws = nullptr;
-    if (any && need > 0 && need <= kStaticScratchBytes &&
-        cudaGetSymbolAddress(&ws, g_static_scratch) != cudaSuccess)
-        return KDA_ERR_CUDA;
-    return kda_chunk_fwd(sh, q, k, v, g, beta, S0, cu_seqlens, out, S_T, ws,
-                         ws ? kStaticScratchBytes : 0, stream);
+    // Shapes without scratch (the CUDA-core path), empty batches and invalid shapes go
+    // straight through: kda_chunk_fwd validates them and, for them, takes no memory.
+    if (need == 0 || sh->num_seqs <= 0)
+        return kda_chunk_fwd(sh, q, k, v, g, beta, S0, cu_seqlens, out, S_T, nullptr, 0, stream);
+    if (need > kStaticScratchBytes) return KDA_ERR_TOO_LARGE;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KDA_ERR_CUDA;
+    void* ws = g_static_scratch_addr[dev].load(std::memory_order_acquire);
+    if (ws == nullptr) {
+        // set-up on this device's first call: the array's device address (loading the
+        // module and with it the array, if nothing on this device has yet)
+        if (cudaGetSymbolAddress(&ws, g_static_scratch) != cudaSuccess || ws == nullptr) return KDA_ERR_CUDA;
+        g_static_scratch_addr[dev].store(ws, std::memory_order_release);
+    }
+    return kda_chunk_fwd(sh, q, k, v, g, beta, S0, cu_seqlens, out, S_T, ws, kStaticScratchBytes, stream);
 }
 
 kda_status_t kda_recurrent_fwd(const kda_shape_t* sh, const void* q, const void* k, const void* v,

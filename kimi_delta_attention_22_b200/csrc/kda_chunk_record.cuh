@@ -12,14 +12,15 @@
 //   Aqk = lower(Qp) (diagonal included)       dec = e^{Gamma_last}
 //
 // and the state-scan kernel (kda_chunk_scan.cu) walks the chunks of a
-// sequence in order with S in registers:
+// sequence in order with the state S (d_v x d_k, row v = value index):
 //
-//   E = U - W S^T,  O = Qg S^T + Aqk E,  S^T <- Diag(dec) S^T + Kd^T E.
+//   E^T = U^T - S W^T,   O^T = S Qg^T + E^T Aqk^T,   S <- S Diag(dec) + E^T Kd.
 //
-// Every tile is stored as the exact byte image of its tcgen05 shared-memory
-// operand (128-byte swizzle), so the scan kernel moves it with one untiled
-// bulk copy and feeds it to the tensor cores unchanged.  Rows i >= L of a
-// short final chunk are zero in W, U, Qg, Kd and Aqk.
+// Every matrix is stored in fp16 (11 significant bits; every value here is
+// bounded: |K e^{Gamma}|, |Kd| <= |k|, and W, U, Qg, Aqk are products of bounded
+// factors) as the exact byte image of a tcgen05 shared-memory operand of the
+// scan's MMAs (128-byte swizzle), so the scan kernel moves a whole record with
+// one bulk copy.  Rows of a short final chunk beyond its length are zero.
 #pragma once
 
 #include <stddef.h>
@@ -28,14 +29,18 @@
 namespace kda {
 namespace rec {
 
-constexpr int C = 64, DK = 128, DV = 128, BV = 64, NVT = DV / BV;
+constexpr int C = 64, DK = 128, DV = 128;
 
 // Byte offsets inside one record.
 constexpr int WQ = 0;        // 32 KB: rows 0-63 W, rows 64-127 Qg; (row r, channel c) at
-                             //        mnmaj_off(c, r, 128), read as a K-major A operand
-constexpr int KD = 32768;    // 16 KB: Kd, (row i, channel c) at mnmaj_off(c, i, 128)
-constexpr int AQ = 49152;    //  8 KB: Aqk, (row i, column j) at kmaj_off(i, j, 64)
-constexpr int U = 57344;     // 2 x 8 KB: U of value tile t, (row i, v) at mnmaj_off(v - 64 t, i, 64)
+                             //        mnmaj_off(c, r, 128) (K-major over the channel, 8-row
+                             //        groups 2048 bytes apart): B operand of S [W ; Qg]^T
+constexpr int KD = 32768;    // 16 KB: Kd, (token j, channel c) at mnmaj_off(c, j, 128):
+                             //        MN-major B operand of E^T Kd
+constexpr int AQ = 49152;    //  8 KB: Aqk, (token i, token j) at kmaj_off(i, j, 64):
+                             //        K-major B operand of E^T Aqk^T
+constexpr int UT = 57344;    // 16 KB: U^T, (value v, token j) at kmaj_off(v, j, 128): read
+                             //        by the thread that owns value row v
 constexpr int DEC = 73728;   // 512 B: fp32 dec[c]
 constexpr int BYTES = 74240;
 static_assert(BYTES % 256 == 0, "records must keep 256-byte alignment");

@@ -2,7 +2,7 @@
 // tensor-core prefill: one CTA per (chunk, head) computes the log-space
 // cumulative decay, the decay-masked key/key and query/key products (tcgen05
 // MMAs), the unit-lower-triangular inverse T = (I + L)^{-1} and the WY/UT
-// pseudo-value products W and U, and writes them as a record (layout in
+// pseudo-value products W and U^T, and writes them as a record (layout in
 // kda_chunk_record.cuh).  Chunks are independent, so the whole grid runs in
 // parallel; only the state scan that follows is sequential.
 //
@@ -24,6 +24,15 @@
 // The fast kernel takes every chunk; a chunk that needs sub-block references
 // is put on a list that the slow kernel (more shared memory, one CTA per SM)
 // works through afterwards.
+//
+// Precision.  The decay factors span far more than fp16's exponent range, so
+// the Gram operands are bf16; the query rows and the j-side are each carried
+// as a two-term bf16 expansion (hi + lo, about 16 significant bits), and the
+// products hi*hi + hi*lo + lo*hi are summed in the fp32 accumulator, so Qp
+// keeps close to fp32 accuracy (the key rows, which only feed L, use one
+// term).  T diag(beta) is split the same way for the W and U products, whose
+// other operands (K e^{Gamma} in bf16, the raw bf16 values) are used as they
+// are.  Everything the record carries is fp16.
 #include <cudaTypedefs.h>
 
 #include "kda_chunk_record.cuh"
@@ -43,8 +52,9 @@ constexpr float kFastLimit2 = 112.f;          // one reference while max |Gamma_
 constexpr int LDT = 68;                       // fp32 row stride of L and T (bank spread)
 constexpr int LDX = 20;                       // fp32 row stride of 16x16 block scratch
 constexpr uint32_t TMEM_COLS = 256;
-constexpr uint32_t TM_GRAM = 0;               // Gram: 64 (one reference) or 128 columns
-constexpr uint32_t TM_WU = 128;               // W (lanes 0-15 of each sub-partition), U (16-31)
+constexpr uint32_t TM_GRAM = 0;               // Gram: 128 columns (two accumulator regions)
+constexpr uint32_t TM_UT = 0;                 // U^T (M = 128, N = 64), after the Gram is read out
+constexpr uint32_t TM_W = 128;                // W (M = 64: lanes 0-15 of each sub-partition)
 
 // Shared-memory maps (bytes from a 1024-aligned base).
 template <bool SLOW>
@@ -52,44 +62,48 @@ struct WyMap;
 template <>
 struct WyMap<false> {                          // one-reference chunks, two CTAs per SM
     static constexpr int RK = 0, RQ = 16384, RG = 32768, RV = 65536;   // raw K, Q, g, V (2 tiles)
-    static constexpr int KQG = 0;              // after prep: rows 0-63 K e^G, rows 64-127 Q~ e^G
-    static constexpr int KYG = 32768;          //   K e^{-G}
-    static constexpr int KG = KQG;             //   K e^G as the B operand of W
-    static constexpr int KDST = 49152;         //   K e^{G_last - G} record image (over raw g)
+    // after prep: rows 0-63 K e^G, 64-127 Q~ e^G (hi), 128-191 Q~ e^G (lo), each (row r,
+    // channel c) at mnmaj_off(c, r, 128); rows 0-63 are also the B operand of W
+    static constexpr int KQ3 = 0;
+    static constexpr int KY = 49152;           //   K e^{-G} (hi)
+    static constexpr int KYL = 81920;          //   K e^{-G} (lo)
+    static constexpr int KG = KQ3;
+    static constexpr int TOT4 = 98304;         // decay scan scratch (prep only)
+    static constexpr int GREF = TOT4 + 8192, GLAST = GREF + 2048, RED = GLAST + 512;
     static constexpr int L = 16384;            // after the Gram: fp32 L, T, Neumann blocks
     static constexpr int TF = L + 64 * LDT * 4;
     static constexpr int NS = TF + 64 * LDT * 4;
-    static constexpr int TOT4 = 81920;         // decay scan scratch (prep only)
-    static constexpr int GREF = TOT4 + 8192, GLAST = GREF + 2048, RED = GLAST + 512;
-    static constexpr int TB = 81920;           // after prep: T diag(beta) bf16 (K-major, 64 rows)
-    static constexpr int OX = 0, OY = 0, AQS = 0;   // sub-block path only
-    static constexpr int AQST = TB;            // bf16 lower(Qp) staging (before T diag(beta) exists)
-    static constexpr int WST = L, UST = L + 16384;   // after the W/U MMAs: record images of W, U
+    static constexpr int AQST = 81920;         // fp16 lower(Qp) staging
+    static constexpr int TB = 90112, TBL = 98304;   // T diag(beta), hi and lo (bf16, K-major, 64 rows)
+    static constexpr int WST = 16384, UST = 32768;  // after the W/U MMAs: record images of W, U^T
+    static constexpr int OX = 0, OXL = 0, OY = 0, OYL = 0;   // sub-block path only
     static constexpr int DECS = RED + 64, BETA = DECS + 512, BAR = BETA + 256, DQS = BAR + 64;
     static constexpr int END = DQS + 256;
     static_assert(NS + 10 * 16 * LDX * 4 <= RV, "phase-3 scratch overflows into V");
-    static_assert(TB + 8192 <= DECS, "T diag(beta) overlaps live scratch");
+    static_assert(KY + 16384 <= RV && RV + 16384 <= KYL, "operands overlap V");
+    static_assert(TBL + 8192 <= DECS, "T diag(beta) overlaps live scratch");
 };
 template <>
 struct WyMap<true> {                           // sub-block references, one CTA per SM
     static constexpr int RK = 0, RQ = 16384, RG = 32768, RV = 65536;
     static constexpr int OX = 0;               // after prep: Gram i-side rows (K-major, 128 rows)
     static constexpr int KG = 32768;           //   K e^G (MN-major, MN = channel)
-    static constexpr int A = 81920;            // 64 KB, reused: scan scratch, Gram j-side
+    static constexpr int OXL = 49152;          //   Q~ i-side rows (lo), K-major, 64 rows
+    static constexpr int A = 81920;            // 64 KB, reused: scan scratch, Gram j-side (hi)
     static constexpr int TOT4 = A, GREF = TOT4 + 8192, GLAST = GREF + 2048, RED = GLAST + 512;
     static constexpr int OY = A;               //   2 K-major tiles of 128 rows (versions 2g, 2g+1)
+    static constexpr int OYL = A + 65536;      //   the same, lo terms
     static constexpr int L = A;                //   after the Gram: fp32 L, T, Neumann blocks,
     static constexpr int TF = L + 64 * LDT * 4;
     static constexpr int NS = TF + 64 * LDT * 4;
-    static constexpr int AQS = NS + 10 * 16 * LDX * 4;   // bf16 lower(Qp) staging
-    static constexpr int TB = A + 65536;
-    static constexpr int KQG = 0, KYG = 0, KDST = 0;   // one-reference path only
-    static constexpr int AQST = AQS;
-    static constexpr int WST = A, UST = A + 16384;   // after the W/U MMAs: record images of W, U
-    static_assert(UST + 16384 <= AQS, "W/U staging overlaps the lower(Qp) staging");
-    static constexpr int DECS = TB + 8192, BETA = DECS + 512, BAR = BETA + 256, DQS = BAR + 64;
+    static constexpr int AQST = NS + 10 * 16 * LDX * 4;   // fp16 lower(Qp) staging
+    static constexpr int TB = OYL, TBL = OYL + 8192;
+    static constexpr int KQ3 = 0, KY = 0, KYL = 0;   // one-reference path only
+    static constexpr int WST = A, UST = A + 16384;   // after the W/U MMAs: record images of W, U^T
+    static_assert(UST + 16384 <= AQST, "W/U staging overlaps the lower(Qp) staging");
+    static constexpr int DECS = OYL + 65536, BETA = DECS + 512, BAR = BETA + 256, DQS = BAR + 64;
     static constexpr int END = DQS + 256;
-    static_assert(AQS + 8192 <= A + 65536, "phase-3 scratch overflows region A");
+    static_assert(AQST + 8192 <= OYL, "phase-3 scratch overflows region A");
 };
 template <bool SLOW>
 constexpr int wy_smem_bytes() { return WyMap<SLOW>::END + 1024; }
@@ -424,40 +438,13 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
     uint8_t* g_wq = rec_p + rec::WQ;
     uint8_t* g_kd = rec_p + rec::KD;
     // the 16-byte chunks of this thread: (row 4 rg + r, channels c8..c8+7) in the
-    // mnmaj_off(c, row, 128) layout shared by K e^G, Q~ e^G, K e^{-G} and Kd
+    // mnmaj_off(c, row, 128) layout shared by K e^G, Q~ e^G, K e^{-G}, Qg and Kd
     const uint32_t basemn = (uint32_t)((rg >> 1) * 2048 + (cq >> 3) * 1024 + (rg & 1) * 512);
-    if (ROWGATE) {
-        // ================= one reference, one decay per row: factors from the row scan
-        const float dd = dec_s[0];
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            const int i = 4 * rg + r;
-            const uint32_t omn =
-                basemn + (((uint32_t)(cq & 7) ^ (uint32_t)(4 * (rg & 1) + r)) << 4) + (uint32_t)(r * 128);
-            const float eg = (GATE == KDA_GATE_SCALAR) ? rowf[i] : 1.f;
-            const float ey = (GATE == KDA_GATE_SCALAR) ? rowi[i] : 1.f;
-            const float qs = p.scale * eg, kd = dd * ey;
-            float kf[8], qf[8], t1[8], t2[8], t3[8], t4[8];
-            unpack8(kraw[r], kf);
-            unpack8(qraw[r], qf);
-            dqp[r] = 0.f;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                dqp[r] = fmaf(kf[e], qf[e], dqp[r]);
-                t1[e] = kf[e] * eg;
-                t2[e] = qf[e] * qs;
-                t3[e] = kf[e] * ey;
-                t4[e] = kf[e] * kd;
-            }
-            st_shared_v4(sm + M::KQG, omn, pack8(t1));
-            st_shared_v4(sm + M::KQG, omn + 16384, pack8(t2));
-            st_shared_v4(sm + M::KYG, omn, pack8(t3));
-            st_shared_v4(sm + M::KDST, omn, pack8(t4));
-        }
-    } else if (!SLOW) {
-        // ================= one reference: 2^{Gamma_i} <= 1 on the i-side, 2^{-Gamma_j} <= 2^112 on the j-side
+    if (!SLOW) {
+        // ================= one reference: 2^{Gamma_i} <= 1 on the i-side, 2^{-Gamma_j} <= 2^112 on
+        // the j-side; one decay per row when the gate is scalar or absent
         float pre[8], dec[8];
-        {
+        if (!ROWGATE) {
             const float4* pp = reinterpret_cast<const float4*>(tot4 + rg * DK + c8);
             const float4* dp = reinterpret_cast<const float4*>(dec_s + c8);
             const float4 p0 = pp[0], p1 = pp[1], d0 = dp[0], d1 = dp[1];
@@ -468,27 +455,43 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
         }
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
+            const int i = 4 * rg + r;
             const uint32_t omn =
                 basemn + (((uint32_t)(cq & 7) ^ (uint32_t)(4 * (rg & 1) + r)) << 4) + (uint32_t)(r * 128);
-            float kf[8], qf[8], t1[8], t2[8], t3[8], t4[8];
+            float kf[8], qf[8], kx[8], qx[8], ky[8], kd[8];
             unpack8(kraw[r], kf);
             unpack8(qraw[r], qf);
             dqp[r] = 0.f;
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 dqp[r] = fmaf(kf[e], qf[e], dqp[r]);
-                const float gm = pre[e] + g2[r][e];   // Gamma_i (log2), <= 0
-                const float eg = ex2(gm), ey = ex2(-gm);
-                t1[e] = kf[e] * eg;                    // K e^{Gamma}
-                t2[e] = (qf[e] * p.scale) * eg;        // Q~ e^{Gamma}
-                t3[e] = kf[e] * ey;                    // K e^{-Gamma}
-                t4[e] = kf[e] * (dec[e] * ey);         // K e^{Gamma_last - Gamma}
+                float eg, ey, dd;
+                if (ROWGATE) {
+                    eg = (GATE == KDA_GATE_SCALAR) ? rowf[i] : 1.f;
+                    ey = (GATE == KDA_GATE_SCALAR) ? rowi[i] : 1.f;
+                    dd = dec_s[0];
+                } else {
+                    const float gm = pre[e] + g2[r][e];   // Gamma_i (log2), <= 0
+                    eg = ex2(gm);
+                    ey = ex2(-gm);
+                    dd = dec[e];
+                }
+                kx[e] = kf[e] * eg;                    // K e^{Gamma}
+                qx[e] = (qf[e] * p.scale) * eg;        // Q~ e^{Gamma}
+                ky[e] = kf[e] * ey;                    // K e^{-Gamma}
+                kd[e] = kf[e] * (dd * ey);             // K e^{Gamma_last - Gamma}
             }
-            // rows 64-127 of K|Q e^G are also the Qg half of the record image
-            st_shared_v4(sm + M::KQG, omn, pack8(t1));
-            st_shared_v4(sm + M::KQG, omn + 16384, pack8(t2));
-            st_shared_v4(sm + M::KYG, omn, pack8(t3));
-            st_shared_v4(sm + M::KDST, omn, pack8(t4));
+            uint4 hi, lo;
+            st_shared_v4(sm + M::KQ3, omn, pack8(kx));
+            pack8_split(qx, hi, lo);
+            st_shared_v4(sm + M::KQ3, omn + 16384, hi);
+            st_shared_v4(sm + M::KQ3, omn + 32768, lo);
+            pack8_split(ky, hi, lo);
+            st_shared_v4(sm + M::KY, omn, hi);
+            st_shared_v4(sm + M::KYL, omn, lo);
+            // Qg (rows 64-127 of the W|Qg image) and Kd go to the record as they are formed
+            *reinterpret_cast<uint4*>(g_wq + omn + 16384) = pack8_f16(qx);
+            *reinterpret_cast<uint4*>(g_kd + omn) = pack8_f16(kd);
         }
     } else {
         // ================= sub-block references
@@ -525,6 +528,8 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
         // the same rows inside a 128-row K-major tile: K-atom stride 16 KB
         const uint32_t baseY = (uint32_t)((cq >> 3) * 16384 + (rg >> 1) * 1024 + (rg & 1) * 512);
         const uint32_t base128 = (uint32_t)((cq >> 3) * 16384 + ((rg >> 1) + 2 * b) * 1024 + (rg & 1) * 512);
+        // Q~ i-side lo rows: row i of a 64-row K-major tile (K-atom stride 8 KB)
+        const uint32_t base64 = (uint32_t)((cq >> 3) * 8192 + (rg >> 1) * 1024 + (rg & 1) * 512);
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
             const uint32_t swz = ((sw0 ^ (uint32_t)(4 * (rg & 1) + r)) << 4) + (uint32_t)(r * 128);
@@ -542,24 +547,31 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
                 y[e] = ex2(-dl);
                 qf[e] *= p.scale;
             }
-            // Gram i-side: K rows at 32 b + (i - 16 b), Q rows 16 further
+            uint4 hi, lo;
+            // Gram i-side: K rows at 32 b + (i - 16 b), Q rows 16 further (hi); Q lo rows at i
 #pragma unroll
             for (int e = 0; e < 8; ++e) t[e] = kf[e] * x[e];
             st_shared_v4(sm + M::OX, o128, pack8(t));
 #pragma unroll
             for (int e = 0; e < 8; ++e) t[e] = qf[e] * x[e];
-            st_shared_v4(sm + M::OX, o128 + 2048, pack8(t));
-            // Gram j-side for this sub-block and the later ones
+            pack8_split(t, hi, lo);
+            st_shared_v4(sm + M::OX, o128 + 2048, hi);
+            st_shared_v4(sm + M::OXL, base64 + swz, lo);
+            // Gram j-side for this sub-block and the later ones (hi and lo)
             float ky[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) ky[e] = kf[e] * y[e];
-            st_shared_v4(sm + M::OY + (b >> 1) * 32768 + (b & 1) * 8192, oy, pack8(ky));
+            pack8_split(ky, hi, lo);
+            st_shared_v4(sm + M::OY + (b >> 1) * 32768 + (b & 1) * 8192, oy, hi);
+            st_shared_v4(sm + M::OYL + (b >> 1) * 32768 + (b & 1) * 8192, oy, lo);
 #pragma unroll
             for (int I = 1; I < 4; ++I) {
                 if (I > b) {
 #pragma unroll
                     for (int e = 0; e < 8; ++e) t[e] = ky[e] * z[I][e];
-                    st_shared_v4(sm + M::OY + (I >> 1) * 32768 + (I & 1) * 8192, oy, pack8(t));
+                    pack8_split(t, hi, lo);
+                    st_shared_v4(sm + M::OY + (I >> 1) * 32768 + (I & 1) * 8192, oy, hi);
+                    st_shared_v4(sm + M::OYL + (I >> 1) * 32768 + (I & 1) * 8192, oy, lo);
                 }
             }
             // K e^Gamma (shared, MN-major), Q~ e^Gamma and K e^{Gamma_last - Gamma} (record)
@@ -571,10 +583,10 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
                 t2[e] = qf[e] * eg;
             }
             st_shared_v4(sm + M::KG, omn, pack8(t));
-            *reinterpret_cast<uint4*>(g_wq + omn + 16384) = pack8(t2);
+            *reinterpret_cast<uint4*>(g_wq + omn + 16384) = pack8_f16(t2);
 #pragma unroll
             for (int e = 0; e < 8; ++e) t[e] = kf[e] * (Lr[e] * y[e]);
-            *reinterpret_cast<uint4*>(g_kd + omn) = pack8(t);
+            *reinterpret_cast<uint4*>(g_kd + omn) = pack8_f16(t);
         }
     }
     store_dq();
@@ -582,42 +594,59 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    // ================= Gram MMAs
-    // one reference: D[n][j] = [K e^G ; Q~ e^G]_n . (K e^-G)_j   (M = 128, N = 64)
+    // ================= Gram MMAs (hi * hi + hi * lo + lo * hi, fp32 accumulation)
+    // one reference: cols 0-63 = [K e^G ; Q~ e^G]_n . (K e^-G)_j over both j-side terms,
+    // cols 64-127 = [Q~ e^G (hi) ; Q~ e^G (lo)]_n . (K e^-G)_j (hi): lanes 64-127 of it are
+    // the lo * hi term of the Qp rows   (M = 128, N = 64)
     // sub-blocks: group g (M = 128, N = 64): A rows 0-63 are the j-side of version 2g,
-    // rows 64-127 that of version 2g+1; B rows the i-side rows of sub-blocks 2g, 2g+1
+    // rows 64-127 that of version 2g+1 (hi, then lo); B rows the i-side rows of sub-blocks
+    // 2g, 2g+1; cols 128 + 32 g: the same j-side (hi) against their Q~ lo rows (N = 32)
     if (tid == 0) {
         if (!SLOW) {
-            // Qg and Kd images to the record; their shared-memory reads overlap the MMA issue
-            bulk_store(g_wq + 16384, sm + M::KQG + 16384, 16384u);
-            bulk_store(g_kd, sm + M::KDST, 16384u);
-            bulk_commit();
+            const uint32_t kq = sbase + M::KQ3, ky = sbase + M::KY, kyl = sbase + M::KYL;
 #pragma unroll
             for (int s8 = 0; s8 < 8; ++s8)
-                mma_bf16(tm + TM_GRAM, rowview_desc(sbase + M::KQG, s8), rowview_desc(sbase + M::KYG, s8),
+                mma_bf16(tm + TM_GRAM, rowview_desc(kq, s8), rowview_desc(ky, s8),
                          idesc_bf16(128, 64, false, false), s8 > 0);
-        } else {
-            const uint32_t ox = sbase + M::OX, oy = sbase + M::OY;
 #pragma unroll
             for (int s8 = 0; s8 < 8; ++s8)
+                mma_bf16(tm + TM_GRAM + 64, rowview_desc(kq + 16384, s8), rowview_desc(ky, s8),
+                         idesc_bf16(128, 64, false, false), s8 > 0);
 #pragma unroll
-                for (int g = 0; g < 2; ++g)
+            for (int s8 = 0; s8 < 8; ++s8)
+                mma_bf16(tm + TM_GRAM, rowview_desc(kq, s8), rowview_desc(kyl, s8),
+                         idesc_bf16(128, 64, false, false), 1);
+        } else {
+            const uint32_t ox = sbase + M::OX, oxl = sbase + M::OXL, oy = sbase + M::OY, oyl = sbase + M::OYL;
+#pragma unroll
+            for (int g = 0; g < 2; ++g) {
+#pragma unroll
+                for (int s8 = 0; s8 < 8; ++s8)
                     mma_bf16(tm + TM_GRAM + 64 * g, kmaj_desc(oy + g * 32768, 128, s8),
                              kmaj_desc(ox + g * 8192, 128, s8), idesc_bf16(128, 64, false, false), s8 > 0);
+#pragma unroll
+                for (int s8 = 0; s8 < 8; ++s8)
+                    mma_bf16(tm + TM_GRAM + 128 + 32 * g, kmaj_desc(oy + g * 32768, 128, s8),
+                             kmaj_desc(oxl + g * 4096, 64, s8), idesc_bf16(128, 32, false, false), s8 > 0);
+#pragma unroll
+                for (int s8 = 0; s8 < 8; ++s8)
+                    mma_bf16(tm + TM_GRAM + 64 * g, kmaj_desc(oyl + g * 32768, 128, s8),
+                             kmaj_desc(ox + g * 8192, 128, s8), idesc_bf16(128, 64, false, false), 1);
+            }
         }
         mma_commit(mma_bar);
-        if (!SLOW) bulk_wait_read();   // both images are overwritten once the Gram is read out
     }
     if (!wait_all(mma_bar, mma_phase)) return 2;
     tc_fence_after();
-    // ================= coupling matrix L (fp32, shared) and lower(Qp) (bf16, record)
+    // ================= coupling matrix L (fp32, shared) and lower(Qp) (fp16, record)
     float* Lm = reinterpret_cast<float*>(sm + M::L);
     float* TF = reinterpret_cast<float*>(sm + M::TF);
     if (!SLOW) {
         // lane n = 32 sp + lane: row i of P (n < 64) or of Qp (n >= 64); columns 32 half ..
         const int n = 32 * sp + lane, j0 = 32 * half;
-        float v[32];
+        float v[32], w[32];
         tmem_ld32(tm + lane_base + TM_GRAM + j0, v);
+        tmem_ld32(tm + lane_base + TM_GRAM + 64 + j0, w);   // lanes 64-127: the lo * hi term
         if (n < 64) {
             const int i = n;
             const float bi = beta_s[i];
@@ -639,9 +668,9 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const int j = j0 + 8 * q + e;
-                    t8[e] = (j < i) ? v[8 * q + e] : ((j == i) ? dii : 0.f);
+                    t8[e] = (j < i) ? v[8 * q + e] + w[8 * q + e] : ((j == i) ? dii : 0.f);
                 }
-                st_shared_v4(sm + M::AQST, kmaj_off(i, j0 + 8 * q, 64), pack8(t8));
+                st_shared_v4(sm + M::AQST, kmaj_off(i, j0 + 8 * q, 64), pack8_f16(t8));
             }
         }
     } else {
@@ -649,14 +678,16 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
         // sub-block 2g's version, those of 2-3 rows j of sub-block 2g+1's version
         const int g = half, hi = sp >> 1;
         const int I = 2 * g + hi, j = 32 * (sp & 1) + lane;
-        __nv_bfloat16* aqs = reinterpret_cast<__nv_bfloat16*>(sm + M::AQS);
-        float v[32];
+        __half* aqs = reinterpret_cast<__half*>(sm + M::AQST);
+        float v[32], w[16];
         tmem_ld32(tm + lane_base + TM_GRAM + 64 * g + 32 * hi, v);
+        tmem_ld16(tm + lane_base + TM_GRAM + 128 + 32 * g + 16 * hi, w);
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
             const int i = 16 * I + u;
             Lm[i * LDT + j] = (j < i) ? beta_s[i] * v[u] : 0.f;
-            aqs[kmaj_off(i, j, 64) >> 1] = __float2bfloat16_rn((j < i) ? v[16 + u] : ((j == i) ? dq_s[i] : 0.f));
+            aqs[kmaj_off(i, j, 64) >> 1] =
+                __float2half_rn((j < i) ? v[16 + u] + w[u] : ((j == i) ? dq_s[i] : 0.f));
         }
     }
     fence_async_smem();
@@ -688,7 +719,7 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
     if (tid == 0) bulk_wait_read();   // the staging is overwritten from here on
     __syncthreads();
     offdiag_columns(TF, Lm, reinterpret_cast<float*>(sm + M::NS), warp, lane);
-    // T diag(beta) -> bf16 (K-major, K = j), 8 columns per step
+    // T diag(beta) -> two-term bf16 expansion (K-major, K = j), 8 columns per step
     for (int e = tid; e < C * 8; e += NT) {
         const int i = e >> 3, j0 = 8 * (e & 7);
         const float4 a0 = *reinterpret_cast<const float4*>(TF + i * LDT + j0);
@@ -700,55 +731,65 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
         float t8[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) t8[k] = (j0 + k <= i) ? tv[k] * bv[k] : 0.f;
-        st_shared_v4(sm + M::TB, kmaj_off(i, j0, 64), pack8(t8));
+        uint4 hi, lo;
+        pack8_split(t8, hi, lo);
+        st_shared_v4(sm + M::TB, kmaj_off(i, j0, 64), hi);
+        st_shared_v4(sm + M::TBL, kmaj_off(i, j0, 64), lo);
     }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    // ================= W = T diag(beta) K e^G (M = 64, N = 128, lanes 0-15 of each
-    // sub-partition) and U = T diag(beta) V (two M = 64, N = 64 tiles, lanes 16-31)
+    // ================= W = T diag(beta) K e^G (M = 64, N = 128: lanes 0-15 of each
+    // sub-partition) and U^T = V^T (T diag(beta))^T (M = 128 over the value index, N = 64),
+    // each over both terms of T diag(beta)
     wait_v();   // V landed long ago; every thread observes it before its tiles are MMA operands
     if (tid == 0) {
-        const uint32_t tb = sbase + M::TB;
 #pragma unroll
-        for (int s = 0; s < 4; ++s)
-            mma_bf16(tm + TM_WU, kmaj_desc(tb, 64, s), mnmaj_desc(sbase + M::KG, 128, s),
-                     idesc_bf16(64, 128, false, true), s > 0);
-#pragma unroll
-        for (int t = 0; t < 2; ++t)
+        for (int t = 0; t < 2; ++t) {
+            const uint32_t tb = sbase + (t == 0 ? M::TB : M::TBL);
 #pragma unroll
             for (int s = 0; s < 4; ++s)
-                mma_bf16(tm + TM_WU + (16u << 16) + 64 * t, kmaj_desc(tb, 64, s),
-                         mnmaj_desc(sbase + M::RV + 8192 * t, 64, s), idesc_bf16(64, 64, false, true),
-                         s > 0);
+                mma_bf16(tm + TM_W, kmaj_desc(tb, 64, s), mnmaj_desc(sbase + M::KG, 128, s),
+                         idesc_bf16(64, 128, false, true), t > 0 || s > 0);
+            // V: the two 64-column TMA tiles are the MN halves (8 KB apart) of one MN-major
+            // operand; k-step s covers tokens 16 s .. 16 s + 15
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                mma_bf16(tm + TM_UT, desc_sw128(sbase + M::RV + 2048u * s, 8192u, 1024u), kmaj_desc(tb, 64, s),
+                         idesc_bf16(128, 64, true, false), t > 0 || s > 0);
+        }
         mma_commit(mma_bar);
     }
     if (!wait_all(mma_bar, mma_phase)) return 2;
     tc_fence_after();
     {
-        // lane l < 16: W row 16 sp + l; l >= 16: U row 16 sp + l - 16; columns 64 half ..
-        const bool isw = lane < 16;
+        // W: lane l < 16 of each sub-partition holds row 16 sp + l; columns 64 half ..
         const int i = 16 * sp + (lane & 15);
 #pragma unroll
         for (int hc = 0; hc < 2; ++hc) {
             float v[32];
-            tmem_ld32(tm + lane_base + TM_WU + 64 * half + 32 * hc, v);
+            tmem_ld32(tm + lane_base + TM_W + 64 * half + 32 * hc, v);
+            if (lane < 16) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int c = 64 * half + 32 * hc + 8 * q;
-                const uint32_t off = isw ? (uint32_t)M::WST + mnmaj_off(c, i, 128)
-                                         : (uint32_t)(M::UST + 8192 * half) + mnmaj_off(c - 64 * half, i, 64);
-                st_shared_v4(sm, off, pack8(v + 8 * q));
+                for (int q = 0; q < 4; ++q)
+                    st_shared_v4(sm + M::WST, mnmaj_off(64 * half + 32 * hc + 8 * q, i, 128), pack8_f16(v + 8 * q));
             }
         }
+        // U^T: lane = value row v, columns (tokens) 32 half ..
+        const int vr = 32 * sp + lane;
+        float u[32];
+        tmem_ld32(tm + lane_base + TM_UT + 32 * half, u);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            st_shared_v4(sm + M::UST, kmaj_off(vr, 32 * half + 8 * q, 128), pack8_f16(u + 8 * q));
     }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
-    if (tid == 0) {   // W (rows 0-63 of the W|Qg image) and both U tiles
+    if (tid == 0) {   // W (rows 0-63 of the W|Qg image) and U^T
         bulk_store(rec_p + rec::WQ, sm + M::WST, 16384u);
-        bulk_store(rec_p + rec::U, sm + M::UST, 16384u);
+        bulk_store(rec_p + rec::UT, sm + M::UST, 16384u);
         bulk_commit();
         bulk_wait_read();
     }

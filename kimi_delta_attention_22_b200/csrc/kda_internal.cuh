@@ -81,7 +81,6 @@ cudaError_t launch_recurrent(const RecurrentArgs& a, bool bf16, cudaStream_t s);
 cudaError_t launch_recurrent_bwd(const RecurrentBwdArgs& a, bool bf16, cudaStream_t s);
 size_t recurrent_bwd_workspace_bytes(int N, int T, int H, int d_v);
 cudaError_t launch_chunk_f32path(const ChunkArgs& a, bool bf16, cudaStream_t s);
-cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t s);
 // Two-kernel tensor-core prefill over a caller workspace laid out by rec::layout().
 cudaError_t launch_chunk_wy(const ChunkArgs& a, uint8_t* ws, const rec::Layout& lay, cudaStream_t s);
 cudaError_t launch_chunk_scan(const ChunkArgs& a, const uint8_t* ws, const rec::Layout& lay,

@@ -4,6 +4,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cudaTypedefs.h>
 #include <stdint.h>
 
@@ -21,6 +22,14 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
     __nv_bfloat162 t = *reinterpret_cast<__nv_bfloat162*>(&u);
     return __bfloat1622float2(t);
+}
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+    __half2 t = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&t);
+}
+__device__ __forceinline__ float2 unpack_f16(uint32_t u) {
+    __half2 t = *reinterpret_cast<__half2*>(&u);
+    return __half22float2(t);
 }
 __device__ __forceinline__ void st_shared_v4(uint8_t* base, uint32_t off, uint4 v) {
     *reinterpret_cast<uint4*>(base + off) = v;
@@ -122,6 +131,29 @@ __device__ __forceinline__ void unpack8(uint4 u, float* f) {
 __device__ __forceinline__ uint4 pack8(const float* v) {
     return make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
                       pack_bf16(v[6], v[7]));
+}
+
+// 8 consecutive fp32 values as one 16-byte fp16 chunk, and back.
+__device__ __forceinline__ uint4 pack8_f16(const float* v) {
+    return make_uint4(pack_f16(v[0], v[1]), pack_f16(v[2], v[3]), pack_f16(v[4], v[5]),
+                      pack_f16(v[6], v[7]));
+}
+__device__ __forceinline__ void unpack8_f16(uint4 u, float* f) {
+    const float2 a = unpack_f16(u.x), b = unpack_f16(u.y), c = unpack_f16(u.z), d = unpack_f16(u.w);
+    f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y; f[4] = c.x; f[5] = c.y; f[6] = d.x; f[7] = d.y;
+}
+// Two-term bf16 expansion of 8 fp32 values: hi = bf16(v), lo = bf16(v - hi), so that
+// hi + lo carries about 16 significant bits (products of expansions summed in fp32
+// keep the operand rounding near 2^-17 relative instead of bf16's 2^-9).
+__device__ __forceinline__ void pack8_split(const float* v, uint4& hi, uint4& lo) {
+    float h[8], l[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        h[e] = __bfloat162float(__float2bfloat16_rn(v[e]));
+        l[e] = v[e] - h[e];
+    }
+    hi = pack8(h);
+    lo = pack8(l);
 }
 
 // ------------------------------------------------------------------ host side

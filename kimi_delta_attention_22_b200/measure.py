@@ -1,11 +1,12 @@
 """Time kda_chunk_fwd on the named synthetic workloads (one GPU).
 
-    python -m kimi_delta_attention_22_b200.measure [--workloads a,b,...] [--schedule split|fused]
+    python -m kimi_delta_attention_22_b200.measure [--workloads a,b,...] [--schedule workspace|pool]
                                                    [--iters 10] [--warmup 3] [--shape B,T,H]
     python -m kimi_delta_attention_22_b200.measure --recurrent [--tokens 1,4,16,64]
 
 For each workload: inputs drawn once on the device (kimi_delta_attention_22_b200.inputs),
-the two-kernel schedule's workspace allocated once, `warmup` untimed calls, then `iters`
+the prefill's workspace allocated once (--schedule pool: none, so each call takes its
+scratch from the stream-ordered pool), `warmup` untimed calls, then `iters`
 calls timed one by one with CUDA events on the current stream; the median is reported
 with tokens/s, the algorithmic HBM bytes and FLOPs of kimi_delta_attention_22_b200.roofline
 and their fractions of MEASURED_PEAKS.json (repository root) when that file exists.
@@ -56,7 +57,7 @@ def measure(name: str, schedule: str, iters: int, warmup: int, shape=None) -> di
     d = inputs.workload_inputs(w, device="cuda")
     cu = d.get("cu_seqlens")
     ws = None
-    if schedule == "split":
+    if schedule == "workspace":
         n = kda.kda_chunk_fwd_workspace_size(d["q"], d["v"], d["g"], cu_seqlens=cu, chunk=w.chunk)
         ws = torch.empty(n, dtype=torch.uint8, device="cuda") if n else None
     out = torch.empty_like(d["v"])
@@ -176,7 +177,7 @@ def measure_backward(N: int, T: int, H: int, iters: int, warmup: int) -> dict:
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--workloads", default=",".join(n for n in inputs.WORKLOADS))
-    ap.add_argument("--schedule", choices=["split", "fused"], default="split")
+    ap.add_argument("--schedule", choices=["workspace", "pool"], default="workspace")
     ap.add_argument("--iters", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--shape", default=None, help="B,T,H: run the named dense workloads' recipe at these sizes")

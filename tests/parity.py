@@ -11,19 +11,14 @@ from kimi_delta_attention_22_b200 import inputs
 
 # Tolerances (see the readings of the pages).  fp32 mode: the maximum
 # absolute error, max |gpu - oracle| <= 1e-4.  bf16-input/fp32-state mode:
-# the error relative to the RMS of the oracle's tensor, per tensor:
-#   * rms(gpu - oracle) / rms(oracle) <= 2e-2 (the stated tolerance), and
-#   * element by element, |gpu - oracle| <= 5 * 2e-2 * rms(oracle) + q |oracle|.
-#     Rounding errors summed over many bf16 products are close to Gaussian, and
-#     the largest of 1e5..1e6 such errors sits near 5 sigma, so this bound is
-#     the worst element consistent with the RMS tolerance.  It catches
-#     localised defects (one bad row or chunk) that an RMS could dilute.
-#     q = 2^-8 (half a bf16 ulp, relative) when the library stores that tensor
-#     in bf16, 0 for fp32 tensors: rounding the stored result is not an
-#     arithmetic error of the path.
+# the error relative to the RMS of the oracle's tensor, per tensor, element by
+# element: max |gpu - oracle| / rms(oracle) <= 2e-2, where for a tensor the
+# library stores in bf16 each element may also differ by the rounding of the
+# stored result, q |oracle| with q = 2^-8 (half a bf16 ulp, relative): rounding
+# the returned value is not an arithmetic error of the path.  fp32 tensors
+# (the final state) get no allowance.  The RMS ratio is reported beside it.
 TOL_F32_ABS = 1e-4
 TOL_BF16_REL = 2e-2
-ELEM_FACTOR = 5.0
 BF16_HALF_ULP = 2.0 ** -8
 
 
@@ -32,10 +27,9 @@ def to_dev(d, dev="cuda"):
 
 
 def err(got, ref, mode, stored_bf16=None):
-    """Returns the error figure compared against TOL_F32_ABS (fp32 mode) or
-    TOL_BF16_REL (bf16 mode: the larger of the RMS ratio and the worst
-    element-wise excess over the rounding allowance divided by ELEM_FACTOR,
-    both relative to rms(oracle))."""
+    """Returns the error figure compared against TOL_F32_ABS (fp32 mode: max abs)
+    or TOL_BF16_REL (bf16 mode: the worst element-wise excess over the stored-result
+    rounding allowance, relative to rms(oracle); never below the RMS ratio)."""
     if stored_bf16 is None:
         stored_bf16 = hasattr(got, "dtype") and got.dtype == torch.bfloat16
     got = got.detach().cpu().double().numpy() if hasattr(got, "detach") else np.asarray(got)
@@ -52,7 +46,7 @@ def err(got, ref, mode, stored_bf16=None):
     q = 2 * BF16_HALF_ULP if stored_bf16 == "both" else (BF16_HALF_ULP if stored_bf16 else 0.0)
     elem = float(np.max(d - q * np.abs(ref))) / rms
     rel_rms = float(np.sqrt(np.mean(d ** 2))) / rms
-    return max(rel_rms, elem / ELEM_FACTOR)
+    return max(rel_rms, elem)
 
 
 # Every check's figure, for the optional per-test error report (conftest.py).
@@ -68,8 +62,9 @@ def check(got, ref, mode, what, stored_bf16=None):
 
 
 def run_chunk(d, chunk, want_state=True, cu=None, workspace=True):
-    """kda_chunk_fwd on the GPU copies of d.  workspace=True takes the two-kernel
-    schedule on the tensor-core path, False the single fused kernel."""
+    """kda_chunk_fwd on the GPU copies of d.  workspace=True passes a torch-allocated
+    workspace; None / False passes none, so the library draws its scratch from the
+    stream-ordered pool (the same kernels either way)."""
     on = to_dev(d)
     out, ST = kda.kda_chunk_fwd(on["q"], on["k"], on["v"], on["g"], on["beta"], S0=on["S0"],
                                 cu_seqlens=on.get("cu_seqlens") if cu is None else cu.cuda(),

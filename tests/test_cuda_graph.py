@@ -1,7 +1,9 @@
-"""The entry points are stream-ordered, allocate nothing and never synchronise,
-so they can be captured in a CUDA graph and replayed: the two-kernel prefill
-(its memset, programmatic-dependent launches and workspace), the fused prefill,
-the decode step and the recurrent pass, replayed bit-identical to eager calls."""
+"""The entry points are stream-ordered and never synchronise, so they can be
+captured in a CUDA graph and replayed: the prefill with a caller workspace (its
+memset and programmatic-dependent launches), with pool scratch (stream-ordered
+allocation and release inside the graph), through the static scratch of the
+no-alloc entry point (after a first call outside the capture), the decode step
+and the recurrent pass, each replayed bit-identical to eager calls."""
 import pytest
 import torch
 
@@ -10,29 +12,34 @@ from kimi_delta_attention_22_b200 import inputs
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("workspace", [True, None])
+@pytest.mark.parametrize("workspace", [True, None, "noalloc"])
 def test_prefill_graph_replay_equals_eager(workspace):
     d = inputs.draw(2, 300, 4, 128, 128, dtype=torch.bfloat16, s0_std=0.02, seed=808, device="cuda")
     args = (d["q"], d["k"], d["v"], d["g"], d["beta"])
     ws = None
-    if workspace:
+    if workspace is True:
         ws = torch.empty(kda.kda_chunk_fwd_workspace_size(d["q"], d["v"], d["g"]), dtype=torch.uint8,
                          device="cuda")
     out = torch.empty_like(d["v"])
     ST = torch.empty(2, 4, 128, 128, dtype=torch.float32, device="cuda")
-    o_ref, s_ref = kda.kda_chunk_fwd(*args, S0=d["S0"], workspace=ws if workspace else None)
+    def call(**kw):
+        if workspace == "noalloc":
+            return kda.kda_chunk_fwd_noalloc(*args, S0=d["S0"], **kw)
+        return kda.kda_chunk_fwd(*args, S0=d["S0"], workspace=ws, **kw)
+
+    o_ref, s_ref = call()
     torch.cuda.synchronize()
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(side):   # warm-up on the capture stream
-        kda.kda_chunk_fwd(*args, S0=d["S0"], out=out, S_T=ST, workspace=ws if workspace else None)
+        call(out=out, S_T=ST)
     torch.cuda.current_stream().wait_stream(side)
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
     out.zero_()
     ST.zero_()
     with torch.cuda.graph(g):
-        kda.kda_chunk_fwd(*args, S0=d["S0"], out=out, S_T=ST, workspace=ws if workspace else None)
+        call(out=out, S_T=ST)
     for _ in range(3):
         g.replay()
     torch.cuda.synchronize()

@@ -1,7 +1,9 @@
 """GPU parity: the CUDA path through the C ABI against the float64 oracle on
 the same seeded inputs (element by element), plus equivalences that hold at
-any size.  Tolerances: fp32 mode max |gpu - oracle| <= 1e-4; bf16 mode
-max |gpu - oracle| / rms(oracle) <= 2e-2, per tensor (outputs and states)."""
+any size.  Tolerances: fp32 mode max |gpu - oracle| <= 1e-4; bf16 mode, per
+tensor (outputs and states), max |gpu - oracle| / rms(oracle) <= 2e-2 element by
+element, with half a bf16 ulp of the oracle's value allowed on bf16-stored
+outputs for the rounding of the stored result (tests/parity.py)."""
 import numpy as np
 import pytest
 import torch
@@ -59,12 +61,12 @@ BF16_CASES = [
 ]
 
 
-@pytest.mark.parametrize("schedule", ["split", "fused"])
+@pytest.mark.parametrize("schedule", ["workspace", "pool"])
 @pytest.mark.parametrize("B,T,H,gate,beta,s0,chunk", BF16_CASES)
 def test_bf16(B, T, H, gate, beta, s0, chunk, schedule):
     d = inputs.draw(B, T, H, 128, 128, dtype=torch.bfloat16, gate=gate, beta=beta,
                     s0_std=0.02 if s0 else None, seed=B * 1000 + T + H)
-    out, ST = run_chunk(d, chunk, workspace=schedule == "split")
+    out, ST = run_chunk(d, chunk, workspace=schedule == "workspace")
     ro, rs = oracle_chunk(d, gate_of(d))
     check(out, ro, "bf16", "out")
     check(ST, rs, "bf16", "S_T")
@@ -86,7 +88,7 @@ def test_whole_width_scan_matches_oracle(gate, qk_div):
     check(ST, rs, "bf16", "S_T")
 
 
-@pytest.mark.parametrize("schedule", ["split", "fused"])
+@pytest.mark.parametrize("schedule", ["workspace", "pool"])
 def test_varlen_small_ragged_and_empty(schedule):
     """Packed sequences of lengths 0, 1, 64, 65, 127, 200 (state restarts per
     sequence; the empty one returns S0)."""
@@ -95,7 +97,7 @@ def test_varlen_small_ragged_and_empty(schedule):
     d = inputs.draw(1, int(cu[-1]), 2, 128, 128, dtype=torch.bfloat16, s0_std=0.02,
                     num_states=len(lens), seed=77)
     d["cu_seqlens"] = cu
-    out, ST = run_chunk(d, 64, workspace=schedule == "split")
+    out, ST = run_chunk(d, 64, workspace=schedule == "workspace")
     ro, rs = oracle_chunk(d, "channel")
     check(out, ro, "bf16", "out")
     check(ST, rs, "bf16", "S_T")

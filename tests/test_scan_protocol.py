@@ -1,4 +1,4 @@
-"""Model check of the state scan's MMA-warp schedule (the 64-column form in
+"""Model check of the state scan's barrier protocol (the MMA-warp schedule of
 kimi_delta_attention_22_b200/csrc/kda_chunk_scan.cu), on the CPU.
 
 The kernel's correctness rests on its barrier protocol, which one GPU run only
@@ -12,8 +12,9 @@ copies a random speed, so that any of them can lag far behind).  It checks that
   * no barrier ever runs two phases ahead of a thread waiting on it (a parity
     wait would then stall: the hardware sees the same parity again);
   * every pair of conflicting accesses (at least one a write) to a shared
-    buffer -- the two TMEM column sets [W ; Qg] S^T / O, the Kd^T E columns,
-    the bf16 state copy and each part of each record stage -- happens in the
+    buffer -- the two halves of each of the two TMEM column sets S [W ; Qg]^T /
+    O^T, the E^T Kd columns, the fp16 copies of S and E^T that are MMA operands
+    in tensor memory, and each part of each record stage -- happens in the
     order the algorithm needs.
 
 Mbarrier semantics: a wait for the k-th completion (parity k & 1) passes when
@@ -35,23 +36,20 @@ class Barrier:
 
 
 class Model:
-    def __init__(self, nch, nstage, n_e=4, n_o=4, seed=0):
+    def __init__(self, nch, nstage, nw=8, seed=0):
         self.rng = random.Random(seed)
         self.nch, self.ns = nch, nstage
-        nw = n_e + n_o
         B = Barrier
         self.bars = {"bar1": B("bar1", 1), "bar2": B("bar2", 1), "bar3": B("bar3", 1),
-                     "eready": B("eready", n_e), "oread": B("oread", n_o), "sready": B("sready", nw)}
+                     "eready": B("eready", nw), "sready": B("sready", nw)}
         for s in range(nstage):
             self.bars[f"full{s}"] = B(f"full{s}", 1)
         self.log = {}          # buffer -> [(key, is_write, who)]
         self.pipe = []         # issued tcgen05 work, executed in order
         self.copies = []       # record copies in flight
         self.actors = {"mma": self.issuer()}
-        for w in range(n_e):
-            self.actors[f"e{w}"] = self.state_warp(True)
-        for w in range(n_o):
-            self.actors[f"o{w}"] = self.state_warp(False)
+        for w in range(nw):
+            self.actors[f"w{w}"] = self.state_warp(f"w{w}")
         self.blocked = {}      # actor -> (barrier, k)
         # per-run speeds, so that some warps, the MMA pipe or the copies lag far behind
         speeds = (0.02, 0.2, 1.0, 5.0)
@@ -66,23 +64,24 @@ class Model:
 
     def execute(self, op):
         kind, m = op
-        if kind == "mma1":         # [W ; Qg] S^T -> d1[m & 1]
-            self.touch(f"d1_{m & 1}", (m // 2, 0), True, "mma1")
-            self.touch("scopy", (m, 0), False, "mma1")
+        if kind == "mma1":         # S [W ; Qg]^T -> both halves of d1[m & 1]
+            self.touch(f"d1lo_{m & 1}", (m // 2, 0), True, "mma1")
+            self.touch(f"d1hi_{m & 1}", (m // 2, 0), True, "mma1")
+            self.touch("as", (m, 1), False, "mma1")
             self.stage_touch("WQ", m, 1, False, "mma1")
-        elif kind == "mma2":       # Kd^T E -> ds
-            self.touch("ds", (m, 0), True, "mma2")
-            self.stage_touch("KA", m, 1, False, "mma2")
-            self.stage_touch("U", m, 2, False, "mma2")
-        elif kind == "mma3":       # [* ; Aqk] E accumulated onto d1[m & 1]
-            self.touch(f"d1_{m & 1}", (m // 2, 2), True, "mma3")
-            self.stage_touch("KA", m, 1, False, "mma3")
-            self.stage_touch("U", m, 2, False, "mma3")
+        elif kind == "mma2":       # E^T Kd -> d2
+            self.touch("d2", (m, 0), True, "mma2")
+            self.touch("ae", (m, 1), False, "mma2")
+            self.stage_touch("KD", m, 1, False, "mma2")
+        elif kind == "mma3":       # E^T Aqk^T accumulated onto the upper half of d1[m & 1]
+            self.touch(f"d1hi_{m & 1}", (m // 2, 1), True, "mma3")
+            self.touch("ae", (m, 1), False, "mma3")
+            self.stage_touch("AQ", m, 1, False, "mma3")
         elif kind == "commit":
             self.bars[m].arrive()
 
     def land(self, m):
-        for part in ("WQ", "KA", "U", "dec"):
+        for part in ("WQ", "KD", "AQ", "UT", "DEC"):
             self.stage_touch(part, m, 0, True, "copy")
         self.bars[f"full{m % self.ns}"].arrive()
 
@@ -92,9 +91,8 @@ class Model:
         for m in range(min(nch, ns - 1)):
             self.copies.append(m)
         yield
-        if nch:
-            yield ("wait", "full0", 0)
         for m in range(nch):
+            yield ("wait", f"full{m % ns}", m // ns)
             if m > 0:
                 yield ("wait", "sready", m - 1)
             self.pipe += [("mma1", m), ("commit", "bar1")]
@@ -104,38 +102,26 @@ class Model:
                     yield ("wait", "bar3", m - 1)
                 self.copies.append(m + ns - 1)
             yield ("wait", "eready", m)
-            self.pipe += [("mma2", m), ("commit", "bar2")]
+            self.pipe += [("mma2", m), ("commit", "bar2"), ("mma3", m), ("commit", "bar3")]
             yield
-            if m > 0:
-                yield ("wait", "oread", m - 1)
-            self.pipe += [("mma3", m), ("commit", "bar3")]
-            yield
-            if m + 1 < nch:
-                yield ("wait", f"full{(m + 1) % ns}", (m + 1) // ns)
 
-    def state_warp(self, e_warp):
-        who = "E" if e_warp else "O"
+    def state_warp(self, who):
         for m in range(self.nch):
-            if e_warp:
-                yield ("wait", "bar1", m)
-                self.touch(f"d1_{m & 1}", (m // 2, 1), False, who)      # W S^T read-out
-                self.stage_touch("U", m, 1, True, who)                  # E written over U
-                yield
-                self.bars["eready"].arrive()
-            elif m > 0:
-                yield ("wait", "bar3", m - 1)
-                self.touch(f"d1_{(m - 1) & 1}", ((m - 1) // 2, 3), False, who)   # outputs
-                yield
-                self.bars["oread"].arrive()
+            yield ("wait", "bar1", m)
+            self.touch(f"d1lo_{m & 1}", (m // 2, 1), False, who)   # S W^T read out
+            self.stage_touch("UT", m, 1, False, who)
+            self.touch("ae", (m, 0), True, who)                     # E^T stored
+            yield
+            self.bars["eready"].arrive()
             yield ("wait", "bar2", m)
-            self.touch("ds", (m, 1), False, who)
-            self.stage_touch("dec", m, 1, False, who)
-            self.touch("scopy", (m, 1), True, who)
+            self.touch("d2", (m, 1), False, who)
+            self.stage_touch("DEC", m, 1, False, who)
+            self.touch("as", (m + 1, 0), True, who)                 # S of the next chunk stored
             yield
             self.bars["sready"].arrive()
-        if not e_warp and self.nch:
-            yield ("wait", "bar3", self.nch - 1)
-            self.touch(f"d1_{(self.nch - 1) & 1}", ((self.nch - 1) // 2, 3), False, who)
+            yield ("wait", "bar3", m)
+            self.touch(f"d1hi_{m & 1}", (m // 2, 2), False, who)   # outputs read out
+            yield
 
     # ---- scheduler
     def check_alias(self):
@@ -188,12 +174,12 @@ class Model:
 @pytest.mark.parametrize("nch", [0, 1, 2, 3, 5, 9])
 def test_mma_warp_schedule_protocol(nch, nstage):
     for seed in range(150):
-        m = Model(nch, nstage, seed=seed)
+        m = Model(nch, nstage, nw=4, seed=seed)
         m.run()
         m.check_order()
 
 
-@pytest.mark.parametrize("dropped", ["oread", "sready", "eready", "bar3", "full"])
+@pytest.mark.parametrize("dropped", ["sready", "eready", "bar3", "full"])
 def test_protocol_check_catches_a_missing_wait(dropped):
     """The check has teeth: drop any one of the MMA thread's waits and some
     interleaving breaks an ordering or runs a barrier two phases ahead."""
@@ -206,7 +192,7 @@ def test_protocol_check_catches_a_missing_wait(dropped):
 
     caught = 0
     for seed in range(300):
-        m = Dropped(6, 3, seed=seed)
+        m = Dropped(6, 3, nw=4, seed=seed)
         try:
             m.run()
             m.check_order()
