@@ -53,7 +53,7 @@ constexpr int LDT = 68;                       // fp32 row stride of L and T (ban
 constexpr int LDX = 20;                       // fp32 row stride of 16x16 block scratch
 constexpr uint32_t TMEM_COLS = 256;
 constexpr uint32_t TM_GRAM = 0;               // Gram: 128 columns (two accumulator regions)
-constexpr uint32_t TM_UT = 0;                 // U^T (M = 128, N = 64), after the Gram is read out
+constexpr uint32_t TM_UT = 0;                 // U^T hi and lo terms (M = 128, N = 128), after the Gram is read out
 constexpr uint32_t TM_W = 128;                // W (M = 64: lanes 0-15 of each sub-partition)
 
 // Shared-memory maps (bytes from a 1024-aligned base).
@@ -61,27 +61,28 @@ template <bool SLOW>
 struct WyMap;
 template <>
 struct WyMap<false> {                          // one-reference chunks, two CTAs per SM
-    static constexpr int RK = 0, RQ = 16384, RG = 32768, RV = 65536;   // raw K, Q, g, V (2 tiles)
+    static constexpr int RK = 0, RQ = 16384, RG = 32768, RV = 81920;   // raw K, Q, g, V (2 tiles)
     // after prep: rows 0-63 K e^G, 64-127 Q~ e^G (hi), 128-191 Q~ e^G (lo), each (row r,
     // channel c) at mnmaj_off(c, r, 128); rows 0-63 are also the B operand of W
     static constexpr int KQ3 = 0;
-    static constexpr int KY = 49152;           //   K e^{-G} (hi)
-    static constexpr int KYL = 81920;          //   K e^{-G} (lo)
+    static constexpr int KY = 49152;           //   rows 0-63 K e^{-G} (hi), rows 64-127 its lo term
     static constexpr int KG = KQ3;
     static constexpr int TOT4 = 98304;         // decay scan scratch (prep only)
     static constexpr int GREF = TOT4 + 8192, GLAST = GREF + 2048, RED = GLAST + 512;
     static constexpr int L = 16384;            // after the Gram: fp32 L, T, Neumann blocks
     static constexpr int TF = L + 64 * LDT * 4;
     static constexpr int NS = TF + 64 * LDT * 4;
-    static constexpr int AQST = 81920;         // fp16 lower(Qp) staging
-    static constexpr int TB = 90112, TBL = 98304;   // T diag(beta), hi and lo (bf16, K-major, 64 rows)
+    static constexpr int AQST = 65536;         // fp16 lower(Qp) staging (over the lo j-side)
+    // T diag(beta), hi then lo (bf16, K-major, 64 rows each: one 128-row tile), over the
+    // lower(Qp) staging once its bulk store has read it
+    static constexpr int TB = 65536, TBL = TB + 8192;
     static constexpr int WST = 16384, UST = 32768;  // after the W/U MMAs: record images of W, U^T
     static constexpr int OX = 0, OXL = 0, OY = 0, OYL = 0;   // sub-block path only
     static constexpr int DECS = RED + 64, BETA = DECS + 512, BAR = BETA + 256, DQS = BAR + 64;
     static constexpr int END = DQS + 256;
-    static_assert(NS + 10 * 16 * LDX * 4 <= RV, "phase-3 scratch overflows into V");
-    static_assert(KY + 16384 <= RV && RV + 16384 <= KYL, "operands overlap V");
-    static_assert(TBL + 8192 <= DECS, "T diag(beta) overlaps live scratch");
+    static_assert(NS + 10 * 16 * LDX * 4 <= KY + 16384, "phase-3 scratch overflows into the lo j-side");
+    static_assert(KY + 32768 <= RV && RV + 16384 <= TOT4, "operands overlap V");
+    static_assert(TBL + 8192 <= RV, "T diag(beta) overlaps V");
 };
 template <>
 struct WyMap<true> {                           // sub-block references, one CTA per SM
@@ -97,8 +98,8 @@ struct WyMap<true> {                           // sub-block references, one CTA 
     static constexpr int TF = L + 64 * LDT * 4;
     static constexpr int NS = TF + 64 * LDT * 4;
     static constexpr int AQST = NS + 10 * 16 * LDX * 4;   // fp16 lower(Qp) staging
-    static constexpr int TB = OYL, TBL = OYL + 8192;
-    static constexpr int KQ3 = 0, KY = 0, KYL = 0;   // one-reference path only
+    static constexpr int TB = OYL, TBL = TB + 8192;
+    static constexpr int KQ3 = 0, KY = 0;      // one-reference path only
     static constexpr int WST = A, UST = A + 16384;   // after the W/U MMAs: record images of W, U^T
     static_assert(UST + 16384 <= AQST, "W/U staging overlaps the lower(Qp) staging");
     static constexpr int DECS = OYL + 65536, BETA = DECS + 512, BAR = BETA + 256, DQS = BAR + 64;
@@ -488,7 +489,7 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
             st_shared_v4(sm + M::KQ3, omn + 32768, lo);
             pack8_split(ky, hi, lo);
             st_shared_v4(sm + M::KY, omn, hi);
-            st_shared_v4(sm + M::KYL, omn, lo);
+            st_shared_v4(sm + M::KY, omn + 16384, lo);
             // Qg (rows 64-127 of the W|Qg image) and Kd go to the record as they are formed
             *reinterpret_cast<uint4*>(g_wq + omn + 16384) = pack8_f16(qx);
             *reinterpret_cast<uint4*>(g_kd + omn) = pack8_f16(kd);
@@ -595,27 +596,24 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
     __syncthreads();
     tc_fence_after();
     // ================= Gram MMAs (hi * hi + hi * lo + lo * hi, fp32 accumulation)
-    // one reference: cols 0-63 = [K e^G ; Q~ e^G]_n . (K e^-G)_j over both j-side terms,
-    // cols 64-127 = [Q~ e^G (hi) ; Q~ e^G (lo)]_n . (K e^-G)_j (hi): lanes 64-127 of it are
-    // the lo * hi term of the Qp rows   (M = 128, N = 64)
+    // one reference: cols 0-127 = [K e^G ; Q~ e^G]_n . [(K e^-G) hi ; (K e^-G) lo]_j
+    // (M = 128, N = 128: the two j-side terms side by side), cols 128-191 =
+    // [Q~ e^G (hi) ; Q~ e^G (lo)]_n . (K e^-G)_j (hi) (N = 64): lanes 64-127 of it are the
+    // lo * hi term of the Qp rows
     // sub-blocks: group g (M = 128, N = 64): A rows 0-63 are the j-side of version 2g,
     // rows 64-127 that of version 2g+1 (hi, then lo); B rows the i-side rows of sub-blocks
     // 2g, 2g+1; cols 128 + 32 g: the same j-side (hi) against their Q~ lo rows (N = 32)
     if (tid == 0) {
         if (!SLOW) {
-            const uint32_t kq = sbase + M::KQ3, ky = sbase + M::KY, kyl = sbase + M::KYL;
+            const uint32_t kq = sbase + M::KQ3, ky = sbase + M::KY;
 #pragma unroll
             for (int s8 = 0; s8 < 8; ++s8)
                 mma_bf16(tm + TM_GRAM, rowview_desc(kq, s8), rowview_desc(ky, s8),
-                         idesc_bf16(128, 64, false, false), s8 > 0);
+                         idesc_bf16(128, 128, false, false), s8 > 0);
 #pragma unroll
             for (int s8 = 0; s8 < 8; ++s8)
-                mma_bf16(tm + TM_GRAM + 64, rowview_desc(kq + 16384, s8), rowview_desc(ky, s8),
+                mma_bf16(tm + TM_GRAM + 128, rowview_desc(kq + 16384, s8), rowview_desc(ky, s8),
                          idesc_bf16(128, 64, false, false), s8 > 0);
-#pragma unroll
-            for (int s8 = 0; s8 < 8; ++s8)
-                mma_bf16(tm + TM_GRAM, rowview_desc(kq, s8), rowview_desc(kyl, s8),
-                         idesc_bf16(128, 64, false, false), 1);
         } else {
             const uint32_t ox = sbase + M::OX, oxl = sbase + M::OXL, oy = sbase + M::OY, oyl = sbase + M::OYL;
 #pragma unroll
@@ -646,7 +644,10 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
         const int n = 32 * sp + lane, j0 = 32 * half;
         float v[32], w[32];
         tmem_ld32(tm + lane_base + TM_GRAM + j0, v);
-        tmem_ld32(tm + lane_base + TM_GRAM + 64 + j0, w);   // lanes 64-127: the lo * hi term
+        tmem_ld32(tm + lane_base + TM_GRAM + 64 + j0, w);   // the hi * lo term
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] += w[e];
+        tmem_ld32(tm + lane_base + TM_GRAM + 128 + j0, w);  // lanes 64-127: the lo * hi term
         if (n < 64) {
             const int i = n;
             const float bi = beta_s[i];
@@ -741,8 +742,8 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
     __syncthreads();
     tc_fence_after();
     // ================= W = T diag(beta) K e^G (M = 64, N = 128: lanes 0-15 of each
-    // sub-partition) and U^T = V^T (T diag(beta))^T (M = 128 over the value index, N = 64),
-    // each over both terms of T diag(beta)
+    // sub-partition), over both terms of T diag(beta), and U^T = V^T [hi ; lo]^T
+    // (M = 128 over the value index, N = 128: the two terms side by side)
     wait_v();   // V landed long ago; every thread observes it before its tiles are MMA operands
     if (tid == 0) {
 #pragma unroll
@@ -752,13 +753,13 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
             for (int s = 0; s < 4; ++s)
                 mma_bf16(tm + TM_W, kmaj_desc(tb, 64, s), mnmaj_desc(sbase + M::KG, 128, s),
                          idesc_bf16(64, 128, false, true), t > 0 || s > 0);
-            // V: the two 64-column TMA tiles are the MN halves (8 KB apart) of one MN-major
-            // operand; k-step s covers tokens 16 s .. 16 s + 15
-#pragma unroll
-            for (int s = 0; s < 4; ++s)
-                mma_bf16(tm + TM_UT, desc_sw128(sbase + M::RV + 2048u * s, 8192u, 1024u), kmaj_desc(tb, 64, s),
-                         idesc_bf16(128, 64, true, false), t > 0 || s > 0);
         }
+        // V: the two 64-column TMA tiles are the MN halves (8 KB apart) of one MN-major
+        // operand; k-step s covers tokens 16 s .. 16 s + 15
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+            mma_bf16(tm + TM_UT, desc_sw128(sbase + M::RV + 2048u * s, 8192u, 1024u),
+                     kmaj_desc(sbase + M::TB, 128, s), idesc_bf16(128, 128, true, false), s > 0);
         mma_commit(mma_bar);
     }
     if (!wait_all(mma_bar, mma_phase)) return 2;
@@ -776,10 +777,13 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
                     st_shared_v4(sm + M::WST, mnmaj_off(64 * half + 32 * hc + 8 * q, i, 128), pack8_f16(v + 8 * q));
             }
         }
-        // U^T: lane = value row v, columns (tokens) 32 half ..
+        // U^T: lane = value row v, columns (tokens) 32 half .., hi term + lo term
         const int vr = 32 * sp + lane;
-        float u[32];
+        float u[32], ul[32];
         tmem_ld32(tm + lane_base + TM_UT + 32 * half, u);
+        tmem_ld32(tm + lane_base + TM_UT + 64 + 32 * half, ul);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) u[e] += ul[e];
 #pragma unroll
         for (int q = 0; q < 4; ++q)
             st_shared_v4(sm + M::UST, kmaj_off(vr, 32 * half + 8 * q, 128), pack8_f16(u + 8 * q));

@@ -146,14 +146,15 @@ __device__ __forceinline__ void unpack8_f16(uint4 u, float* f) {
 // hi + lo carries about 16 significant bits (products of expansions summed in fp32
 // keep the operand rounding near 2^-17 relative instead of bf16's 2^-9).
 __device__ __forceinline__ void pack8_split(const float* v, uint4& hi, uint4& lo) {
-    float h[8], l[8];
+    uint32_t h[4], l[4];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        h[e] = __bfloat162float(__float2bfloat16_rn(v[e]));
-        l[e] = v[e] - h[e];
+    for (int e = 0; e < 4; ++e) {
+        h[e] = pack_bf16(v[2 * e], v[2 * e + 1]);
+        const float2 r = unpack_bf16(h[e]);   // exact: the rounded pair back in fp32
+        l[e] = pack_bf16(v[2 * e] - r.x, v[2 * e + 1] - r.y);
     }
-    hi = pack8(h);
-    lo = pack8(l);
+    hi = make_uint4(h[0], h[1], h[2], h[3]);
+    lo = make_uint4(l[0], l[1], l[2], l[3]);
 }
 
 // ------------------------------------------------------------------ host side

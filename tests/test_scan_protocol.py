@@ -12,10 +12,10 @@ copies a random speed, so that any of them can lag far behind).  It checks that
   * no barrier ever runs two phases ahead of a thread waiting on it (a parity
     wait would then stall: the hardware sees the same parity again);
   * every pair of conflicting accesses (at least one a write) to a shared
-    buffer -- the two halves of each of the two TMEM column sets S [W ; Qg]^T /
-    O^T, the E^T Kd columns, the fp16 copies of S and E^T that are MMA operands
-    in tensor memory, and each part of each record stage -- happens in the
-    order the algorithm needs.
+    buffer -- the halves of the two S [W ; Qg]^T / O^T column sets, the fp32 S
+    (scaled by the threads, accumulated by E^T Kd, read for its fp16 copy), the
+    fp16 copies of S and E^T that are MMA operands in tensor memory, and each
+    part of each record stage -- happens in the order the algorithm needs.
 
 Mbarrier semantics: a wait for the k-th completion (parity k & 1) passes when
 exactly k + 1 completions have happened."""
@@ -44,12 +44,14 @@ class Model:
                      "eready": B("eready", nw), "sready": B("sready", nw)}
         for s in range(nstage):
             self.bars[f"full{s}"] = B(f"full{s}", 1)
+            self.bars[f"empty{s}"] = B(f"empty{s}", 1)
         self.log = {}          # buffer -> [(key, is_write, who)]
         self.pipe = []         # issued tcgen05 work, executed in order
         self.copies = []       # record copies in flight
-        self.actors = {"mma": self.issuer()}
-        for w in range(nw):
-            self.actors[f"w{w}"] = self.state_warp(f"w{w}")
+        self.actors = {"mma": self.issuer(), "copy": self.copier()}
+        self.warps = [f"w{w}" for w in range(nw)]
+        for w in self.warps:
+            self.actors[w] = self.state_warp(w)
         self.blocked = {}      # actor -> (barrier, k)
         # per-run speeds, so that some warps, the MMA pipe or the copies lag far behind
         speeds = (0.02, 0.2, 1.0, 5.0)
@@ -59,23 +61,29 @@ class Model:
     def touch(self, buf, key, write, who):
         self.log.setdefault(buf, []).append((key, write, who))
 
+    def touch_slices(self, buf, key, write, who):
+        """An MMA reads or accumulates every state warp's slice (lanes x columns) of a
+        tensor-memory operand; each warp touches only its own slice."""
+        for w in self.warps:
+            self.touch(f"{buf}.{w}", key, write, who)
+
     def stage_touch(self, part, m, rank, write, who):
         self.touch(f"stage{m % self.ns}.{part}", (m // self.ns, rank), write, who)
 
     def execute(self, op):
         kind, m = op
-        if kind == "mma1":         # S [W ; Qg]^T -> both halves of d1[m & 1]
+        if kind == "mma1":         # S_m [W ; Qg]^T -> both halves of d1[m & 1]
             self.touch(f"d1lo_{m & 1}", (m // 2, 0), True, "mma1")
             self.touch(f"d1hi_{m & 1}", (m // 2, 0), True, "mma1")
-            self.touch("as", (m, 1), False, "mma1")
+            self.touch_slices("as", (m, 1), False, "mma1")
             self.stage_touch("WQ", m, 1, False, "mma1")
-        elif kind == "mma2":       # E^T Kd -> d2
-            self.touch("d2", (m, 0), True, "mma2")
-            self.touch("ae", (m, 1), False, "mma2")
+        elif kind == "mma2":       # E^T Kd accumulated onto the decayed fp32 S
+            self.touch_slices("s32", (m, 1), True, "mma2")
+            self.touch_slices("ae", (m, 1), False, "mma2")
             self.stage_touch("KD", m, 1, False, "mma2")
         elif kind == "mma3":       # E^T Aqk^T accumulated onto the upper half of d1[m & 1]
             self.touch(f"d1hi_{m & 1}", (m // 2, 1), True, "mma3")
-            self.touch("ae", (m, 1), False, "mma3")
+            self.touch_slices("ae", (m, 1), False, "mma3")
             self.stage_touch("AQ", m, 1, False, "mma3")
         elif kind == "commit":
             self.bars[m].arrive()
@@ -86,37 +94,44 @@ class Model:
         self.bars[f"full{m % self.ns}"].arrive()
 
     # ---- programs (generators yielding ("wait", bar, k) or nothing)
-    def issuer(self):
+    def copier(self):
         nch, ns = self.nch, self.ns
-        for m in range(min(nch, ns - 1)):
+        for m in range(min(nch, ns)):
             self.copies.append(m)
         yield
+        for m in range(ns, nch):
+            # stage m % ns takes chunk m once chunk m - ns's MMAs are done
+            yield ("wait", f"empty{m % ns}", m // ns - 1)
+            self.copies.append(m)
+            yield
+
+    def issuer(self):
+        nch, ns = self.nch, self.ns
         for m in range(nch):
-            yield ("wait", f"full{m % ns}", m // ns)
             if m > 0:
                 yield ("wait", "sready", m - 1)
+            yield ("wait", f"full{m % ns}", m // ns)
             self.pipe += [("mma1", m), ("commit", "bar1")]
             yield
-            if m + ns - 1 < nch:
-                if m > 0:
-                    yield ("wait", "bar3", m - 1)
-                self.copies.append(m + ns - 1)
             yield ("wait", "eready", m)
-            self.pipe += [("mma2", m), ("commit", "bar2"), ("mma3", m), ("commit", "bar3")]
+            self.pipe += [("mma2", m), ("commit", "bar2"), ("mma3", m), ("commit", "bar3"),
+                          ("commit", f"empty{m % ns}")]
             yield
 
     def state_warp(self, who):
         for m in range(self.nch):
+            yield ("wait", f"full{m % self.ns}", m // self.ns)
+            self.stage_touch("UT", m, 1, False, who)                # U^T read ahead of S W^T
+            self.stage_touch("DEC", m, 1, False, who)
+            self.touch(f"s32.{who}", (m, 0), True, who)             # S <- S Diag(dec)
             yield ("wait", "bar1", m)
             self.touch(f"d1lo_{m & 1}", (m // 2, 1), False, who)   # S W^T read out
-            self.stage_touch("UT", m, 1, False, who)
-            self.touch("ae", (m, 0), True, who)                     # E^T stored
+            self.touch(f"ae.{who}", (m, 0), True, who)              # E^T stored
             yield
             self.bars["eready"].arrive()
             yield ("wait", "bar2", m)
-            self.touch("d2", (m, 1), False, who)
-            self.stage_touch("DEC", m, 1, False, who)
-            self.touch("as", (m + 1, 0), True, who)                 # S of the next chunk stored
+            self.touch(f"s32.{who}", (m, 2), False, who)            # S_{m+1} read for its copy
+            self.touch(f"as.{who}", (m + 1, 0), True, who)          # fp16 S_{m+1} stored
             yield
             self.bars["sready"].arrive()
             yield ("wait", "bar3", m)
@@ -179,14 +194,20 @@ def test_mma_warp_schedule_protocol(nch, nstage):
         m.check_order()
 
 
-@pytest.mark.parametrize("dropped", ["sready", "eready", "bar3", "full"])
+@pytest.mark.parametrize("dropped", ["sready", "eready", "full", "empty"])
 def test_protocol_check_catches_a_missing_wait(dropped):
-    """The check has teeth: drop any one of the MMA thread's waits and some
+    """The check has teeth: drop any one of the MMA or copy thread's waits and some
     interleaving breaks an ordering or runs a barrier two phases ahead."""
     class Dropped(Model):
         def issuer(self):
             for step in super().issuer():
                 if step is not None and step[1].startswith(dropped) and step[2] > 0:
+                    continue
+                yield step
+
+        def copier(self):
+            for step in super().copier():
+                if step is not None and step[1].startswith(dropped):
                     continue
                 yield step
 
