@@ -263,6 +263,57 @@ kda_status_t kda_recurrent_bwd(const kda_shape_t* shape, const void* q, const vo
  * every 8 tokens (fp32). */
 size_t kda_recurrent_bwd_workspace_size(const kda_shape_t* shape);
 
+/*
+ * kda_chunk_bwd -- gradients of kda_chunk_fwd (training), chunkwise.
+ *
+ * For the loss sum(out * d_out) + sum(S_T * d_ST), where (out, S_T) is what
+ * kda_chunk_fwd returns for the same arguments, writes the gradients with
+ * respect to q, k, v, g, beta and S0.  The GeekNews summary of "You could have
+ * come up with Kimi Delta Attention" (section "fused recurrent Triton kernel for
+ * decode") names the chunkwise schedule as the one for training; the pages give
+ * no backward derivation, so this is the chain rule of the chunk map that
+ * kda_chunk_fwd computes (cumulative decay, decay-masked Gram products, the
+ * triangular solve, the state and output products), undone chunk by chunk:
+ *   1. the forward's records and, from a forward state scan, every chunk's
+ *      incoming state (fp32, in the workspace);
+ *   2. a reverse state scan on the tensor cores: with dS = d_ST, per chunk from
+ *      the last, dE^T = dS Kd^T + dO^T Aqk and dS <- dS Diag(e^gamma) + dO^T Qg -
+ *      dE^T W (the records' operands, fp16, fp32 accumulation); the final dS is dS0;
+ *   3. per (chunk, head) in parallel, on CUDA cores in fp32: the triangular
+ *      solve's gradient, dv and dbeta, then dq, dk and dg.
+ * Arguments as kda_chunk_fwd (dense or varlen through cu_seqlens, grouped value
+ * heads through shape->qk_heads), plus:
+ *   d_out  [B, T, H, d_v] bf16, 16-byte aligned
+ *   d_ST   [num_seqs, H, d_v, d_k] fp32 or NULL (zero)
+ * Outputs, all fp32 and caller-owned, 16-byte aligned unless stated:
+ *   dq, dk [B, T, Hk, d_k] (summed over the value heads of a group)
+ *   dv     [B, T, H, d_v]
+ *   dg     the shape of g (NULL exactly when the gate is KDA_GATE_NONE; a scalar
+ *          gate's dg is 4-byte aligned)
+ *   dbeta  [B, T, H], 4-byte aligned
+ *   dS0    [num_seqs, H, d_v, d_k], or NULL when not wanted.
+ * Rows of a packed batch that no sequence covers are left untouched.  With
+ * grouped value heads (Hk < H) dq and dk are first zeroed and then summed with
+ * atomic adds (their last bits may vary from run to run); otherwise every output
+ * is written once and the result is deterministic.
+ * Workspace: kda_chunk_bwd_workspace_size(shape, varlen) bytes, 256-byte aligned,
+ *   or NULL: the scratch is then taken from the device's stream-ordered pool
+ *   (cudaMallocAsync) and returned on `stream` after the last kernel.
+ * Support: KDA_BF16 with d_k = d_v = 128 and chunk = 64; else KDA_ERR_UNSUPPORTED.
+ * Errors as kda_chunk_fwd; a too-small workspace is KDA_ERR_INVALID_ARG.
+ */
+kda_status_t kda_chunk_bwd(const kda_shape_t* shape, const void* q, const void* k, const void* v,
+                           const float* g, const float* beta, const float* S0,
+                           const int32_t* cu_seqlens, const void* d_out, const float* d_ST, float* dq,
+                           float* dk, float* dv, float* dg, float* dbeta, float* dS0, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace kda_chunk_bwd needs (0 for unsupported shapes): the forward's
+ * records plus, per (chunk, head), two fp32 states (the incoming state and the
+ * outgoing state's gradient), two fp32 d_v x C tiles and one fp32 C x C tile:
+ * 74,240 + 131,072 + 65,536 + 16,384 = 287,232 bytes. */
+size_t kda_chunk_bwd_workspace_size(const kda_shape_t* shape, int varlen);
+
 kda_status_t kda_recurrent_fwd(const kda_shape_t* shape, const void* q, const void* k,
                                const void* v, const float* g, const float* beta, float* S,
                                void* out, void* stream);

@@ -71,6 +71,10 @@ def load_library(path: str | None = None):
     lib.kda_recurrent_fwd.restype = ctypes.c_int
     lib.kda_recurrent_bwd.argtypes = [ctypes.POINTER(Shape)] + [P] * 15 + [ctypes.c_size_t, P]
     lib.kda_recurrent_bwd.restype = ctypes.c_int
+    lib.kda_chunk_bwd.argtypes = [ctypes.POINTER(Shape)] + [P] * 16 + [ctypes.c_size_t, P]
+    lib.kda_chunk_bwd.restype = ctypes.c_int
+    lib.kda_chunk_bwd_workspace_size.argtypes = [ctypes.POINTER(Shape), ctypes.c_int]
+    lib.kda_chunk_bwd_workspace_size.restype = ctypes.c_size_t
     lib.kda_recurrent_bwd_workspace_size.argtypes = [ctypes.POINTER(Shape)]
     lib.kda_recurrent_bwd_workspace_size.restype = ctypes.c_size_t
     lib.kda_decode_step.restype = ctypes.c_int
@@ -304,6 +308,54 @@ def kda_recurrent_bwd(q, k, v, g, beta, S0, d_out, d_ST=None, want_dS0: bool = T
                                _stream_handle(q.device))
     if st != 0:
         raise KDAError(st, "kda_recurrent_bwd")
+    return dict(dq=dq, dk=dk, dv=dv, dg=dg, dbeta=dbeta, dS0=dS0)
+
+
+def kda_chunk_bwd(q, k, v, g, beta, S0, d_out, d_ST=None, cu_seqlens=None, chunk: int = 64,
+                  want_dS0: bool = True, dev_status=None, workspace=True, lib=None):
+    """Gradients of kda_chunk_fwd (kda_chunk_bwd of include/kda.h), chunkwise.
+
+    Inputs as kda_chunk_fwd (bf16 q, k, v with d_k = d_v = 128, chunk 64; dense or
+    packed through cu_seqlens), with d_out [B,T,H,d_v] bf16 and d_ST [N,H,d_v,d_k]
+    fp32 or None.  Returns a dict of fp32 tensors dq, dk [B,T,Hk,d_k], dv
+    [B,T,H,d_v], dg (shape of g, or None), dbeta [B,T,H] and dS0 [N,H,d_v,d_k]
+    (None unless want_dS0) for the loss sum(out * d_out) + sum(S_T * d_ST).
+
+    workspace: True allocates the scratch with torch, a uint8 CUDA tensor supplies
+    it, None / False lets the library take it from the stream-ordered pool.
+    """
+    _check_cuda(q, k, v, g, beta, S0, d_out, d_ST, cu_seqlens, dev_status)
+    B, T, Hk, Dk = q.shape
+    H, _ = _heads(q, v, 2)
+    Dv = v.shape[-1]
+    N = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    if d_out.shape != v.shape or d_out.dtype != v.dtype:
+        raise ValueError("d_out must match v in shape and dtype")
+    if cu_seqlens is not None and cu_seqlens.dtype != torch.int32:
+        raise TypeError("cu_seqlens is int32")
+    f32 = dict(dtype=torch.float32, device=q.device)
+    dq = torch.empty(B, T, Hk, Dk, **f32)
+    dk = torch.empty(B, T, Hk, Dk, **f32)
+    dv = torch.empty(B, T, H, Dv, **f32)
+    dg = None if g is None else torch.empty(g.shape, **f32)
+    dbeta = torch.empty(B, T, H, **f32)
+    dS0 = torch.empty(N, H, Dv, Dk, **f32) if want_dS0 else None
+    sh = Shape(B, T, H, Dk, Dv, N, _dtype_code(q.dtype), _gate_code(g, q), int(chunk),
+               None if dev_status is None else dev_status.data_ptr(), Hk)
+    lib = lib or load_library()
+    if isinstance(workspace, torch.Tensor):
+        _check_cuda(workspace)
+    if workspace is True:
+        nbytes = lib.kda_chunk_bwd_workspace_size(ctypes.byref(sh), int(cu_seqlens is not None))
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device) if nbytes else None
+    elif workspace is False:
+        workspace = None
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.kda_chunk_bwd(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0),
+                           _ptr(cu_seqlens), _ptr(d_out), _ptr(d_ST), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg),
+                           _ptr(dbeta), _ptr(dS0), _ptr(workspace), ws_bytes, _stream_handle(q.device))
+    if st != 0:
+        raise KDAError(st, "kda_chunk_bwd")
     return dict(dq=dq, dk=dk, dv=dv, dg=dg, dbeta=dbeta, dS0=dS0)
 
 

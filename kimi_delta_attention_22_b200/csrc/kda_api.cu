@@ -7,6 +7,7 @@
 #include <atomic>
 #include <stdint.h>
 
+#include "kda_chunk_bwd.cuh"
 #include "kda_internal.cuh"
 
 namespace kda {
@@ -245,6 +246,81 @@ kda_status_t kda_recurrent_bwd(const kda_shape_t* sh, const void* q, const void*
     a.N = N; a.T = T; a.H = H; a.Hk = Hk; a.d_k = D; a.d_v = V; a.gate = sh->gate;
     a.scale = 1.0f / sqrtf((float)D);
     return from_cuda(kda::launch_recurrent_bwd(a, sh->dtype == KDA_BF16, st));
+}
+
+size_t kda_chunk_bwd_workspace_size(const kda_shape_t* sh, int varlen) {
+    if (sh == nullptr || sh->B < 0 || sh->T < 0 || sh->H <= 0 || sh->num_seqs < 0) return 0;
+    if (sh->dtype != KDA_BF16 || !tc_supports(sh->d_k, sh->d_v, sh->chunk)) return 0;
+    return kda::bwd_layout(sh->B, sh->T, sh->H, sh->num_seqs, varlen != 0).bytes;
+}
+
+kda_status_t kda_chunk_bwd(const kda_shape_t* sh, const void* q, const void* k, const void* v,
+                           const float* g, const float* beta, const float* S0,
+                           const int32_t* cu_seqlens, const void* d_out, const float* d_ST, float* dq,
+                           float* dk, float* dv, float* dg, float* dbeta, float* dS0, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+    if (sh == nullptr) return KDA_ERR_INVALID_ARG;
+    const int B = sh->B, T = sh->T, H = sh->H, N = sh->num_seqs;
+    if (B < 0 || T < 0 || H <= 0 || sh->d_k <= 0 || sh->d_v <= 0 || N < 0) return KDA_ERR_INVALID_ARG;
+    const int Hk = qk_heads_of(sh);
+    if (Hk < 0) return KDA_ERR_INVALID_ARG;
+    if (sh->dtype != KDA_F32 && sh->dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+    if (sh->gate != KDA_GATE_CHANNEL && sh->gate != KDA_GATE_SCALAR && sh->gate != KDA_GATE_NONE)
+        return KDA_ERR_INVALID_ARG;
+    const bool gated = sh->gate != KDA_GATE_NONE;
+    if (cu_seqlens == nullptr) {
+        if (N != B) return KDA_ERR_INVALID_ARG;
+    } else if (B != 1) {
+        return KDA_ERR_INVALID_ARG;
+    }
+    const long long tok = (long long)B * T;
+    // without tokens, the per-token tensors are empty (and their pointers may be null)
+    if (!gated && (g != nullptr || dg != nullptr)) return KDA_ERR_INVALID_ARG;
+    if (tok > 0 && (!q || !k || !v || !beta || !d_out || !dq || !dk || !dv || !dbeta || (gated && (!g || !dg))))
+        return KDA_ERR_INVALID_ARG;
+    const bool g_vec = sh->gate == KDA_GATE_CHANNEL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !(g_vec ? aligned16(g) : aligned4(g)) ||
+        !aligned4(beta) || !aligned16(S0) || !aligned4(cu_seqlens) || !aligned16(d_out) ||
+        !aligned16(d_ST) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+        !(g_vec ? aligned16(dg) : aligned4(dg)) || !aligned4(dbeta) || !aligned16(dS0))
+        return KDA_ERR_MISALIGNED;
+    if (sh->dtype != KDA_BF16 || !tc_supports(sh->d_k, sh->d_v, sh->chunk)) return KDA_ERR_UNSUPPORTED;
+    if ((long long)N * H * 2 > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+    const kda::BwdLayout bl = kda::bwd_layout(B, T, H, N, cu_seqlens != nullptr);
+    if (bl.fwd.slots * H > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+    if (workspace != nullptr) {
+        if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KDA_ERR_MISALIGNED;
+        if (workspace_bytes < bl.bytes) return KDA_ERR_INVALID_ARG;
+    }
+    if (N == 0) return KDA_OK;
+
+    kda::ChunkBwdArgs a;
+    a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.S0 = S0; a.cu_seqlens = cu_seqlens;
+    a.d_out = d_out; a.d_ST = d_ST;
+    a.dq = dq; a.dk = dk; a.dv = dv; a.dg = dg; a.dbeta = dbeta; a.dS0 = dS0;
+    a.dev_status = sh->dev_status;
+    a.B = B; a.T = T; a.H = H; a.Hk = Hk; a.num_seqs = N; a.gate = sh->gate;
+    a.scale = 1.0f / sqrtf((float)sh->d_k);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaSuccess;
+    if (Hk != H && tok > 0) {   // query/key heads shared by several value heads: summed with atomics
+        e = cudaMemsetAsync(dq, 0, (size_t)tok * Hk * sh->d_k * sizeof(float), st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(dk, 0, (size_t)tok * Hk * sh->d_k * sizeof(float), st);
+        if (e != cudaSuccess) return KDA_ERR_CUDA;
+    }
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const bool pooled = ws == nullptr;
+    if (pooled && cudaMallocAsync(reinterpret_cast<void**>(&ws), bl.bytes, st) != cudaSuccess) return KDA_ERR_CUDA;
+    const kda::ChunkArgs fa = kda::forward_args(a);
+    e = kda::launch_chunk_wy(fa, ws, bl.fwd, st);
+    if (e == cudaSuccess) e = kda::launch_chunk_scan(fa, ws, bl.fwd, st, reinterpret_cast<float*>(ws + bl.chk_off));
+    if (e == cudaSuccess) e = kda::launch_chunk_bwd_scan(a, ws, bl, st);
+    if (e == cudaSuccess) e = kda::launch_chunk_bwd_grad(a, ws, bl, st);
+    if (pooled) {
+        const cudaError_t f = cudaFreeAsync(ws, st);
+        if (e == cudaSuccess) e = f;
+    }
+    return from_cuda(e);
 }
 
 kda_status_t kda_decode_step(const kda_shape_t* sh, const void* q, const void* k, const void* v,

@@ -74,7 +74,8 @@ struct ScanParams {
     const int32_t* cu_seqlens;
     const float* S0;
     float* S_T;
-    __nv_bfloat16* out;
+    __nv_bfloat16* out;   // null: outputs not written (state checkpoints only)
+    float* S_chk;         // null, or [slot][H][d_v][d_k]: the incoming state of every chunk
     int32_t* dev_status;
     int T, H, num_seqs, nc;
 };
@@ -94,10 +95,7 @@ __device__ __forceinline__ void tmem_ld_n(uint32_t taddr, float* v) {
 template <int N>
 __device__ __forceinline__ void tmem_st_n(uint32_t taddr, const uint32_t* r) {
     if constexpr (N == 8) {
-        asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(
-                         taddr),
-                     "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
-                     : "memory");
+        tmem_st8(taddr, r);
     } else if constexpr (N == 16) {
         tmem_st16(taddr, r);
     } else {
@@ -177,14 +175,21 @@ struct Tile {
         for (int q = 0; q < G::EC / 8; ++q)
             u[q] = *reinterpret_cast<const uint4*>(stg + rec::UT + kmaj_off(v, G::EC * part + 8 * q, 128));
     }
-    // S <- S Diag(dec of chunk m), ahead of the accumulation of E^T Kd
-    __device__ __forceinline__ void decay(int m) const {
+    // S <- S Diag(dec of chunk m), ahead of the accumulation of E^T Kd; with chk set,
+    // S (the incoming state of chunk m) is first copied there (row v of this thread)
+    __device__ __forceinline__ void decay(int m, float* chk) const {
         const float4* dec = reinterpret_cast<const float4*>(sm + (m % G::NSTAGE) * G::STAGE + rec::DEC) +
                             (G::SC / 4) * part;
 #pragma unroll
         for (int c32 = 0; c32 < G::SC / 32; ++c32) {
             float x[32];
             tmem_ld32(tm + lane_base + G::TM_S + G::SC * part + 32 * c32, x);
+            if (chk) {
+                float4* dst = reinterpret_cast<float4*>(chk + (size_t)v * DK + G::SC * part + 32 * c32);
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    dst[q] = make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
+            }
             uint32_t r[32];
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
@@ -231,6 +236,7 @@ struct Tile {
     // tokens goes token-major into the warp's staging block (one 64-byte row of 32 values
     // per token), which the warp then writes out as 16-byte vectors
     __device__ __forceinline__ void read_out(const ScanParams& p, int m, long long c0, int L, int warp) const {
+        if (p.out == nullptr) return;
         float o[G::EC];
         tmem_ld_n<G::EC>(tm + lane_base + G::TM_D1 + 128u * (uint32_t)(m & 1) + 64u + G::EC * part, o);
         __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(sm + G::OFF_OUT + warp * G::OUT_WARP);
@@ -414,7 +420,7 @@ __global__ void __launch_bounds__(Cfg<NW>::NT, 1) kda_chunk_scan_kernel(const __
             uint4 ut[G::EC / 8];
             if (!(ok = warp_wait(b.full + m % NSTAGE, (uint32_t)((m / NSTAGE) & 1)))) break;
             t.load_ut(m, ut);
-            t.decay(m);
+            t.decay(m, p.S_chk ? p.S_chk + ((size_t)(first + m) * p.H + t.h) * DV * DK : nullptr);
             if (!(ok = warp_wait(b.bar1, (uint32_t)(m & 1)))) break;
             tc_fence_after();
             t.e_step(m, ut);
@@ -469,8 +475,10 @@ cudaError_t launch_scan(const ScanParams& p, long long pairs, cudaStream_t st) {
 
 }  // namespace
 
-cudaError_t launch_chunk_scan(const ChunkArgs& a, const uint8_t* ws, const rec::Layout& lay, cudaStream_t st) {
+cudaError_t launch_chunk_scan(const ChunkArgs& a, const uint8_t* ws, const rec::Layout& lay, cudaStream_t st,
+                              float* S_chk) {
     ScanParams p;
+    p.S_chk = S_chk;
     p.rec = ws + lay.rec_off;
     p.coff = a.cu_seqlens ? reinterpret_cast<const int32_t*>(ws + lay.coff_off) : nullptr;
     p.cu_seqlens = a.cu_seqlens;

@@ -83,8 +83,10 @@ size_t recurrent_bwd_workspace_bytes(int N, int T, int H, int d_v);
 cudaError_t launch_chunk_f32path(const ChunkArgs& a, bool bf16, cudaStream_t s);
 // Two-kernel tensor-core prefill over a caller workspace laid out by rec::layout().
 cudaError_t launch_chunk_wy(const ChunkArgs& a, uint8_t* ws, const rec::Layout& lay, cudaStream_t s);
+// S_chk: null, or [slot][H][d_v][d_k] fp32 to receive the incoming state of every chunk
+// (the backward's checkpoints); a.out may then be null (no outputs written).
 cudaError_t launch_chunk_scan(const ChunkArgs& a, const uint8_t* ws, const rec::Layout& lay,
-                              cudaStream_t s);
+                              cudaStream_t s, float* S_chk = nullptr);
 cudaError_t launch_decode(const DecodeArgs& a, bool bf16, cudaStream_t s);
 // One CTA taking the kernels' bounded mbarrier wait (budget_ns) on a barrier that
 // completes (complete) or never does; on expiry it ORs KDA_DEV_TIMEOUT into *dev_status.
