@@ -310,8 +310,9 @@ kda_status_t kda_chunk_bwd(const kda_shape_t* shape, const void* q, const void* 
 
 /* Bytes of workspace kda_chunk_bwd needs (0 for unsupported shapes): the forward's
  * records plus, per (chunk, head), two fp32 states (the incoming state and the
- * outgoing state's gradient), two fp32 d_v x C tiles and one fp32 C x C tile:
- * 74,240 + 131,072 + 65,536 + 16,384 = 287,232 bytes. */
+ * outgoing state's gradient), one fp32 C x d_v tile, three fp16 C x d_v operand
+ * images and one fp32 C x C tile: 74,240 + 131,072 + 32,768 + 49,152 + 16,384 =
+ * 303,616 bytes, and a small header. */
 size_t kda_chunk_bwd_workspace_size(const kda_shape_t* shape, int varlen);
 
 kda_status_t kda_recurrent_fwd(const kda_shape_t* shape, const void* q, const void* k,

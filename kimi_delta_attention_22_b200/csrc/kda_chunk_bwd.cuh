@@ -6,10 +6,11 @@
 //   2. the forward's state scan with outputs off, keeping every chunk's incoming
 //      state S_c (fp32) in the workspace;
 //   3. the reverse state scan (kda_chunk_bwd_scan.cu): dS0, and per chunk the
-//      gradient of its outgoing state dS' and dE^T;
+//      gradient of its outgoing state dS' and dE;
 //   4. and 5. the chunk-parallel gradient kernels (kda_chunk_bwd_grad.cu): per
 //      (chunk, head), the triangular-solve half (E, the solve's gradient, dv,
-//      dbeta) and then the rest (dq, dk, dg).
+//      dbeta) and then the rest (dq, dk, dg); their dense products run on the
+//      tensor cores, the decay-weighted Gram parts on CUDA cores.
 #pragma once
 
 #include "kda_chunk_record.cuh"
@@ -41,14 +42,17 @@ struct ChunkBwdArgs {
 // Workspace: the forward's records (rec::layout), then per (slot, head):
 //   chk  fp32 [d_v][d_k]  incoming state of the chunk
 //   dsp  fp32 [d_v][d_k]  gradient of the chunk's outgoing state
-//   de   fp32 [d_v][C]    dE^T from the reverse scan; the first gradient kernel
-//                         overwrites it with dPr^T = -(diag(beta) dEbar)^T
-//   et   fp32 [d_v][C]    E^T
+//   de   fp32 [C][d_v]    dE from the reverse scan
+//   e16  2 x 16 KB        E as a two-term fp16 expansion (hi, then lo = E - hi), each the
+//                         byte image of a K-major 64 x 128 MMA operand tile
+//   pr16 16 KB            dPr = -diag(beta) dEbar, one such image (fp16)
 //   da   fp32 [C][C]      dA = diag(beta) dL (strictly lower)
 struct BwdLayout {
     rec::Layout fwd;
-    size_t chk_off, dsp_off, de_off, et_off, da_off, bytes;
+    size_t chk_off, dsp_off, de_off, e16_off, pr16_off, da_off, bytes;
 };
+
+constexpr size_t kTile16 = (size_t)rec::C * rec::DV * 2;   // one fp16 64 x 128 operand image
 
 inline BwdLayout bwd_layout(int B, int T, int H, int num_seqs, bool varlen) {
     BwdLayout b;
@@ -60,8 +64,9 @@ inline BwdLayout bwd_layout(int B, int T, int H, int num_seqs, bool varlen) {
     b.chk_off = rec::round256(b.fwd.bytes);
     b.dsp_off = b.chk_off + units * st;
     b.de_off = b.dsp_off + units * st;
-    b.et_off = b.de_off + units * vc;
-    b.da_off = b.et_off + units * vc;
+    b.e16_off = b.de_off + units * vc;
+    b.pr16_off = b.e16_off + units * 2 * kTile16;
+    b.da_off = b.pr16_off + units * kTile16;
     b.bytes = b.da_off + units * cc;
     return b;
 }

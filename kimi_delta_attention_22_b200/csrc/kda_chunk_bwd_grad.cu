@@ -1,36 +1,47 @@
 // kda_chunk_bwd_grad.cu -- the chunk-parallel half of the chunkwise backward.
 //
 // With every chunk's incoming state S (checkpointed by the forward scan), the
-// gradient of its outgoing state dS' and dE^T (both from the reverse scan), the
+// gradient of its outgoing state dS' and dE (both from the reverse scan), the
 // gradients of a chunk's inputs depend on that chunk alone, so one CTA per
 // (chunk, head) forms them.  The chunk map is the forward's (the GeekNews summary
 // of "You could have come up with Kimi Delta Attention", section "Chunkwise KDA";
 // the triangular solve the curriculum page names):
 //
 //   Gamma = cumsum(g),  A_ij = sum_c K_ic K_jc e^{Gamma_ic - Gamma_jc} (j < i),
-//   M = I + strict_lower(diag(beta) A),  resid = V - (K e^Gamma) S^T,
-//   E = M^{-1} diag(beta) resid,  Aqk_ij = sum_c Q~_ic K_jc e^{Gamma_ic - Gamma_jc} (j <= i),
+//   M = I + strict_lower(diag(beta) A),  T = M^{-1},  resid = V - (K e^Gamma) S^T,
+//   E = T diag(beta) resid,  Aqk_ij = sum_c Q~_ic K_jc e^{Gamma_ic - Gamma_jc} (j <= i),
 //   O = (Q~ e^Gamma) S^T + Aqk E,  S' = S Diag(e^gamma) + E^T (K e^{gamma - Gamma}),
 //
 // and the gradients below are its chain rule, step by step in reverse (the pages
 // give no backward derivation):
 //
-//   solve kernel (one CTA per (chunk, head)):
-//     dEbar = M^{-T} dE (back substitution),  dbeta = rowsum(dEbar . resid) + rowsum(dL . A),
-//     dL = strict_lower(-dEbar E^T),  dv = diag(beta) dEbar,
-//     and for the next kernel E^T, dPr^T = -(diag(beta) dEbar)^T and dA = diag(beta) dL;
+//   solve kernel:
+//     dEbar = T^T dE,  dL = strict_lower(-dEbar E^T),  dv = diag(beta) dEbar,
+//     dbeta = rowsum(dEbar . resid) + rowsum(dL . A),
+//     and for the dqk kernel E, dPr = -diag(beta) dEbar and dA = diag(beta) dL;
 //   dqk kernel:
-//     dKd = E dS',  dQg = dO S,  dKg = dPr S  (one fused pass over the state rows),
-//     dAqk = lower(dO E^T), the two decay-weighted Gram products' own gradients,
+//     dKd = E dS',  dQg = dO S,  dKg = dPr S,  dAqk = lower(dO E^T),
+//     the two decay-weighted Gram products' own gradients,
 //     dgamma = colsum(S . dS') e^gamma + colsum(dKd . Kd), dg = reverse cumsum of dGamma.
 //
-// The decay factor e^{Gamma_ic - Gamma_jc} of a Gram entry is split over 16-token
-// sub-blocks I (of i) and J (of j), with r(I) the sub-block's first row:
+// The dense products (the ones with S, dS', T, E, dEbar and dO) are tcgen05 MMAs
+// with M = 64 token rows (row i in lane 16 (i / 16) + i % 16 of the tensor memory),
+// fp16 operands and fp32 accumulators; every operand here is a bounded value, not a
+// decay factor.  The gradients of the decay (dg) sum products of the state with
+// other terms that largely cancel, so the operands whose rounding reaches them --
+// S, dS', E, and T, diag(beta) resid, dE on the way to E and dEbar -- are carried
+// as two-term fp16 expansions x = hi + lo (lo = fp16(x - hi), about 22 significant
+// bits), with the products hi*hi + hi*lo + lo*hi summed in the fp32 accumulator;
+// dO is exact in fp16, and dPr, dEbar in dEbar E^T and the residual product's
+// operands are single fp16 (float64 emulation of the chunk: each adds < 5e-4).
+// The decay-weighted Gram products stay on CUDA cores in fp32, because their
+// factors span far more than fp16's range: the factor e^{Gamma_ic - Gamma_jc} is
+// split over 16-token sub-blocks I (of i) and J (of j), r(I) the first row of I:
 //   a_ic = 2^{G_ic - G_r(I)c} <= 1,  b_jc = 2^{G_r(J)c - G_jc} (its own sub-block only),
 //   d^{IJ}_c = 2^{G_r(I)c - G_r(J)c} <= 1 (J < I),   (G = Gamma in log2 units)
 // so every Gram product and its gradient becomes a plain product of row-scaled
 // operands with a per-column factor per sub-block pair; b stays bounded by the decay
-// of 15 tokens.  Everything here is fp32 on CUDA cores.
+// of 15 tokens.
 #include <cuda_bf16.h>
 
 #include "kda_chunk_bwd.cuh"
@@ -41,20 +52,65 @@ namespace kda {
 namespace {
 
 using namespace tc;
-using sm100::pdl_wait;
+using namespace sm100;
 
 constexpr int C = rec::C, DK = rec::DK, DV = rec::DV, NT = 256;
 constexpr int LD = 132;          // fp32 row stride of [64][128] tiles
-constexpr int LT = 68;           // fp32 row stride of [128][64] and [64][64] tiles
-constexpr int REG = 128 * LT;    // floats per shared-memory region
-static_assert(REG >= 64 * LD, "a region holds either tile shape");
-constexpr float kLog2e = 1.4426950408889634f;
+constexpr int LT = 68;           // fp32 row stride of [64][64] tiles
+constexpr uint64_t kWaitNs = 1000000000ull;   // 1 s bound on every wait
+constexpr uint32_t TMEM_COLS = 512;
 
-constexpr int SOLVE_FLOATS = 5 * REG + C * LT + 6 * DK + C;
-constexpr int DQK_FLOATS = 4 * REG + 2 * C * LT + 2 * C * LT + 6 * DK + 16 * C;
-constexpr int SOLVE_SMEM = SOLVE_FLOATS * 4;
-constexpr int DQK_SMEM = DQK_FLOATS * 4;
-static_assert(SOLVE_SMEM <= 232448 && DQK_SMEM <= 232448, "shared memory over the sm_100 per-block limit");
+// Solve kernel: shared-memory map (bytes from a 1024-aligned base).
+namespace s1 {
+constexpr int G = 0;               // fp32 [64][LD]  G (log2 units)
+constexpr int A = 33792;           // fp32 [64][LT]  A, strictly lower
+constexpr int TF = 51200;          // fp32 [64][LT]  T = M^{-1}
+constexpr int RES = 68608;         // fp32 [64][LD]  resid
+constexpr int TH = 102400;         // fp16 T (hi), K-major 64 x 64 (read MN-major it is T^T)
+constexpr int TL = 110592;         // its lo term
+constexpr int U = 118784;          // 67584-byte union:
+constexpr int KA = U, KB = U + 33792;              //   Gram: fp32 [64][LD] K a, K b
+constexpr int KG16 = U, S16 = U + 16384;           //   product 1: K e^Gamma (64 rows), S (128 rows), K-major
+constexpr int EBH = U, EBL = U + 16384;            //   products 2, 3: diag(beta) resid (hi, lo) and
+constexpr int DEH = U + 32768, DEL = U + 49152;    //   dE (hi, lo), MN-major over v
+constexpr int DB16 = U, E16 = U + 16384;           //   product 4: dEbar, E (hi) (K-major, 64 rows)
+constexpr int DFAC = U + 67584;    // fp32 [6][128]
+constexpr int SB = DFAC + 3072;    // fp32 [64] beta
+constexpr int RED = SB + 256;      // fp32 [4][64] dbeta partial sums
+constexpr int PS = RED + 1024;     // fp32 [3][16][16] inverse scratch
+constexpr int BAR = PS + 3072;     // 5 mbarriers, TMEM base
+constexpr int BYTES = BAR + 64 + 1024;
+static_assert(U % 1024 == 0 && TH % 1024 == 0 && TL % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+static_assert(BYTES <= 232448, "shared memory over the sm_100 per-block limit");
+constexpr uint32_t TM_R = 0, TM_E = 128, TM_DB = 256, TM_DL = 384;
+}  // namespace s1
+
+// dqk kernel: shared-memory map.
+namespace s2 {
+constexpr int G = 0;               // fp32 [64][LD]  G
+constexpr int OPS = 33792;         // 101376-byte union: the MMA operands of one half of the
+                                   // value axis (v = 64 h .. +63), then the per-element
+                                   // partial results P, then K a, Q~ a, K b
+constexpr int SH = OPS, SL = OPS + 16384;            // S (hi, lo), MN-major over the channel
+constexpr int DH = OPS + 32768, DL = OPS + 49152;    // dS' (hi, lo), the same
+constexpr int EH = OPS + 65536, EL = OPS + 73728;    // E (hi, lo), K-major 64 rows
+constexpr int DO16 = OPS + 81920, PR16 = OPS + 90112;  // dO, dPr, K-major 64 rows
+constexpr int P = OPS;             // fp32 3 x [64][LD]: dK, dQ, dGamma partials
+constexpr int AQK = OPS + 101376;  // fp32 [64][LT] dAqk (lower, diagonal included)
+constexpr int DA = AQK + 17408;    // fp32 [64][LT] dA (strictly lower)
+constexpr int AQT = DA + 17408;    // fp32 [64][LT] dAqk^T
+constexpr int DAT = AQT + 17408;   // fp32 [64][LT] dA^T
+constexpr int SRED = AQT;          // fp32 [16][64] scalar-gate row sums (after the Gram loops)
+constexpr int DFAC = DAT + 17408;  // fp32 [6][128]
+constexpr int UCOL = DFAC + 3072;  // fp32 [4][128] colsum(dKd . Kd) partials
+constexpr int SGS = UCOL + 2048;   // fp32 [8][128] colsum(S . dS') partials
+constexpr int BAR = SGS + 4096;    // 5 mbarriers, TMEM base
+constexpr int BYTES = BAR + 64 + 1024;
+static_assert(OPS % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+static_assert(PR16 + 8192 - OPS <= 101376 && 3 * 64 * LD * 4 <= 101376, "operands and partials fit the union");
+static_assert(BYTES <= 232448, "shared memory over the sm_100 per-block limit");
+constexpr uint32_t TM_KD = 0, TM_QG = 128, TM_KG = 256, TM_AQ = 384;
+}  // namespace s2
 
 struct GradParams {
     const __nv_bfloat16* q;
@@ -67,14 +123,16 @@ struct GradParams {
     const int32_t* coff;
     const float* chk;     // [slot][H][d_v][d_k]
     const float* dsp;     // [slot][H][d_v][d_k]
-    float* de;            // [slot][H][d_v][C]: dE^T in, dPr^T out
-    float* et;            // [slot][H][d_v][C]
+    const float* de;      // [slot][H][C][d_v]
+    uint8_t* e16;         // [slot][H] 2 x 16 KB: the hi and lo images of E
+    uint8_t* pr16;        // [slot][H] 16 KB: the image of dPr
     float* da;            // [slot][H][C][C]
     float* dq;
     float* dk;
     float* dv;
     float* dg;
     float* dbeta;
+    int32_t* dev_status;
     int T, H, num_seqs, nc, group;
     float scale;
 };
@@ -101,22 +159,40 @@ __device__ __forceinline__ bool slot_rows(const GradParams& p, int slot, long lo
 
 __device__ __forceinline__ int pair_index(int I, int J) { return I * (I - 1) / 2 + J; }   // J < I
 
-// G = cumulative log2 decay of the chunk (rows past L carry no decay), threads 0..127.
+// G = cumulative log2 decay of the chunk (rows past L carry no decay).  The raw g
+// tile goes into sG with every load in flight at once; the column prefix sums then
+// run in shared memory, two threads per channel (rows 0-31 and 32-63).  Every thread
+// of the CTA calls this; the caller synchronises before reading sG.
 template <int GATE>
 __device__ __forceinline__ void load_gamma(const GradParams& p, long long c0, int L, int h, float* sG) {
-    const int c = threadIdx.x;
-    if (c >= DK) return;
+    const int tid = threadIdx.x;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+        const int x = tid + NT * r, i = x >> 5, c4 = x & 31;
+        float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (i < L) {
+            if (GATE == KDA_GATE_CHANNEL) {
+                f = __ldg(reinterpret_cast<const float4*>(p.g + ((c0 + i) * p.H + h) * DK) + c4);
+            } else if (GATE == KDA_GATE_SCALAR) {
+                const float gv = __ldg(p.g + (c0 + i) * p.H + h);
+                f = make_float4(gv, gv, gv, gv);
+            }
+        }
+        *reinterpret_cast<float4*>(sG + i * LD + 4 * c4) = f;
+    }
+    __syncthreads();
+    const int c = tid & (DK - 1), half = tid >> 7;
     float acc = 0.f;
 #pragma unroll 8
-    for (int i = 0; i < C; ++i) {
-        float gv = 0.f;
-        if (GATE == KDA_GATE_CHANNEL) {
-            if (i < L) gv = p.g[((c0 + i) * p.H + h) * DK + c];
-        } else if (GATE == KDA_GATE_SCALAR) {
-            if (i < L) gv = p.g[(c0 + i) * p.H + h];
-        }
-        acc += gv * kLog2e;
+    for (int i = 32 * half; i < 32 * half + 32; ++i) {
+        acc = fmaf(sG[i * LD + c], kLog2e, acc);
         sG[i * LD + c] = acc;
+    }
+    __syncthreads();
+    if (half == 1) {
+        const float base = sG[31 * LD + c];
+#pragma unroll 8
+        for (int i = 32; i < C; ++i) sG[i * LD + c] += base;
     }
 }
 
@@ -129,13 +205,17 @@ __device__ __forceinline__ void load_dfac(const float* sG, float* dfac) {
     }
 }
 
-// 8 bf16 values of row `row` (or zeros past the chunk).
-__device__ __forceinline__ void load8(const __nv_bfloat16* base, bool valid, float* f) {
-    if (valid) {
-        unpack8(__ldg(reinterpret_cast<const uint4*>(base)), f);
-    } else {
+// n bf16 values (n = 8 or 32) of one row, or zeros past the chunk.
+template <int N>
+__device__ __forceinline__ void loadn(const __nv_bfloat16* base, bool valid, float* f) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) f[e] = 0.f;
+    for (int q = 0; q < N / 8; ++q) {
+        if (valid) {
+            unpack8(__ldg(reinterpret_cast<const uint4*>(base) + q), f + 8 * q);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[8 * q + e] = 0.f;
+        }
     }
 }
 
@@ -146,48 +226,99 @@ __device__ __forceinline__ void st4(float* p, float a, float b, float c, float d
 __device__ __forceinline__ float comp(const float4& x, int e) {
     return e == 0 ? x.x : (e == 1 ? x.y : (e == 2 ? x.z : x.w));
 }
-
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sm100::smem_u32(dst)), "l"(src) : "memory");
+__device__ __forceinline__ void ld8(const float* p, float* f) {
+    const float4 a = ld4(p), b = ld4(p + 4);
+    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void ld8g(const float* p, float* f) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(p)), b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+
+// Every thread waits for the MMA group behind `bar` (bounded); all agree on the outcome.
+__device__ __forceinline__ bool wait_mma(uint64_t* bar) {
+    const bool ok = mbar_wait(bar, 0, kWaitNs);
+    return __syncthreads_and(ok) != 0;
+}
+// Generic-proxy shared-memory writes become visible to the tensor cores' reads.
+__device__ __forceinline__ void operands_ready() {
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+}
+
+// T = (I + strict_lower(diag(beta) A))^{-1} in fp32: diagonal 16 x 16 blocks by
+// forward substitution (one thread per column), then the off-diagonal blocks by
+// distance from the diagonal: T_IJ = -T_II sum_{K=J}^{I-1} L_IK T_KJ.
+__device__ __forceinline__ void invert_unit_lower(const float* sA, const float* sb, float* sT, float* ps) {
+    const int tid = threadIdx.x;
+    for (int x = tid; x < C * C; x += NT) sT[(x >> 6) * LT + (x & 63)] = 0.f;
+    __syncthreads();
+    if (tid < C) {
+        const int I = tid >> 4, c = tid & 15, o = 16 * I;
+        float x[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            float s = r == c ? 1.f : 0.f;
+            const float br = sb[o + r];
+#pragma unroll
+            for (int q = 0; q < r; ++q) s = fmaf(-br * sA[(o + r) * LT + o + q], x[q], s);
+            x[r] = s;
+            sT[(o + r) * LT + o + c] = s;
+        }
+    }
+    __syncthreads();
+    for (int dist = 1; dist < 4; ++dist) {
+        const int npair = 4 - dist;
+        for (int x = tid; x < npair * 256; x += NT) {   // P = sum_K L_IK T_KJ
+            const int pr = x >> 8, r = (x >> 4) & 15, c = x & 15, J = pr, I = J + dist;
+            const float br = sb[16 * I + r];
+            float s = 0.f;
+            for (int K = J; K < I; ++K)
+#pragma unroll
+                for (int q = 0; q < 16; ++q)
+                    s = fmaf(br * sA[(16 * I + r) * LT + 16 * K + q], sT[(16 * K + q) * LT + 16 * J + c], s);
+            ps[x] = s;
+        }
+        __syncthreads();
+        for (int x = tid; x < npair * 256; x += NT) {   // T_IJ = -T_II P
+            const int pr = x >> 8, r = (x >> 4) & 15, c = x & 15, J = pr, I = J + dist;
+            float s = 0.f;
+#pragma unroll
+            for (int q = 0; q < 16; ++q) s = fmaf(sT[(16 * I + r) * LT + 16 * I + q], ps[(pr << 8) + q * 16 + c], s);
+            sT[(16 * I + r) * LT + 16 * J + c] = -s;
+        }
+        __syncthreads();
+    }
+}
 
 // ---------------------------------------------------------------- solve kernel
 template <int GATE>
-__global__ void __launch_bounds__(NT, 1) kda_chunk_bwd_solve_kernel(const __grid_constant__ GradParams p) {
-    extern __shared__ float4 smem4[];
-    float* sG = reinterpret_cast<float*>(smem4);   // [64][LD] G (log2 units)
-    float* R1 = sG + REG;                          // K a  -> (K e^Gamma)^T [128][LT]
-    float* R2 = R1 + REG;                          // K b  -> resid^T [128][LT]
-    float* R3 = R2 + REG;                          // E^T [128][LT]
-    float* R4 = R3 + REG;                          // dE^T -> dEbar^T [128][LT]
-    float* sA = R4 + REG;                          // [64][LT] A, strictly lower
-    float* dfac = sA + C * LT;                     // [6][128]
-    float* sb = dfac + 6 * DK;                     // [64] beta
-    float* red = R1;                               // after the resid product: dbeta partial sums
-                                                   // [4 + 16][64], summed in a fixed order
-    const int tid = threadIdx.x;
-    const int slot = blockIdx.x / p.H, h = blockIdx.x % p.H, hk = h / p.group;
-    pdl_wait();
-    long long c0;
-    int L;
-    if (!slot_rows(p, slot, c0, L)) return;
-    const size_t sh = (size_t)slot * p.H + h;
+__device__ __forceinline__ bool solve_body(const GradParams& p, uint8_t* sm, uint32_t tm, uint64_t* bars,
+                                           long long c0, int L, int h, int hk, size_t sh) {
+    using namespace s1;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, sp = warp & 3, hc = warp >> 2;
+    const uint32_t sbase = smem_u32(sm), lane_base = (uint32_t)(32 * sp) << 16;
+    float* sG = reinterpret_cast<float*>(sm + G);
+    float* sA = reinterpret_cast<float*>(sm + A);
+    float* sT = reinterpret_cast<float*>(sm + TF);
+    float* sRes = reinterpret_cast<float*>(sm + RES);
+    float* dfac = reinterpret_cast<float*>(sm + DFAC);
+    float* sb = reinterpret_cast<float*>(sm + SB);
+    float* red = reinterpret_cast<float*>(sm + RED);
+    float* Ka = reinterpret_cast<float*>(sm + KA);
+    float* Kb = reinterpret_cast<float*>(sm + KB);
+    const int Hk = p.H / p.group;
 
     load_gamma<GATE>(p, c0, L, h, sG);
     if (tid < C) sb[tid] = tid < L ? p.beta[(c0 + tid) * p.H + h] : 0.f;
-    {
-        const float4* src = reinterpret_cast<const float4*>(p.de + sh * DV * C);
-        for (int x = tid; x < DV * C / 4; x += NT) *reinterpret_cast<float4*>(R4 + (x >> 4) * LT + 4 * (x & 15)) = src[x];
-    }
-    // this thread's K: rows i = x & 63, 8-channel chunk x >> 6, for x = tid + 256 r
+    // this thread's K: row i = x & 63, 8-channel chunk x >> 6, for x = tid + 256 r
     float kr[4][8];
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
         const int x = tid + NT * r, i = x & 63, cc = x >> 6;
-        load8(p.k + ((c0 + i) * (p.H / p.group) + hk) * DK + 8 * cc, i < L, kr[r]);
+        loadn<8>(p.k + ((c0 + i) * Hk + hk) * DK + 8 * cc, i < L, kr[r]);
     }
     __syncthreads();
     load_dfac(sG, dfac);
@@ -202,25 +333,26 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_bwd_solve_kernel(const __grid
             ka[e] = kr[r][e] * ex2(Gi[e] - Gr[e]);
             kb[e] = kr[r][e] * ex2(Gr[e] - Gi[e]);
         }
-        st4(R1 + i * LD + 8 * cc, ka[0], ka[1], ka[2], ka[3]);
-        st4(R1 + i * LD + 8 * cc + 4, ka[4], ka[5], ka[6], ka[7]);
-        st4(R2 + i * LD + 8 * cc, kb[0], kb[1], kb[2], kb[3]);
-        st4(R2 + i * LD + 8 * cc + 4, kb[4], kb[5], kb[6], kb[7]);
+        st4(Ka + i * LD + 8 * cc, ka[0], ka[1], ka[2], ka[3]);
+        st4(Ka + i * LD + 8 * cc + 4, ka[4], ka[5], ka[6], ka[7]);
+        st4(Kb + i * LD + 8 * cc, kb[0], kb[1], kb[2], kb[3]);
+        st4(Kb + i * LD + 8 * cc + 4, kb[4], kb[5], kb[6], kb[7]);
     }
     __syncthreads();
 
-    // ---- A (strictly lower): tiles of 4 rows x 4 columns
+    // ---- A (strictly lower), CUDA cores: tiles of 4 rows x 4 columns
     {
         const int ig = tid & 15, jg = tid >> 4, I = ig >> 2, J = jg >> 2;
         float acc[4][4] = {};
         if (J <= I) {
             const float* dv = dfac + (J < I ? pair_index(I, J) : 0) * DK;
+#pragma unroll 2
             for (int c = 0; c < DK; c += 4) {
                 float4 a[4], b[4];
 #pragma unroll
                 for (int r = 0; r < 4; ++r) {
-                    a[r] = ld4(R1 + (4 * ig + r) * LD + c);
-                    b[r] = ld4(R2 + (4 * jg + r) * LD + c);
+                    a[r] = ld4(Ka + (4 * ig + r) * LD + c);
+                    b[r] = ld4(Kb + (4 * jg + r) * LD + c);
                 }
                 if (J < I) {
                     const float4 d = ld4(dv + c);
@@ -248,308 +380,448 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_bwd_solve_kernel(const __grid
         }
     }
     __syncthreads();
-    // (K e^Gamma)^T into R1
+
+    // ---- product 1 (tensor cores): (K e^Gamma) S^T; operands K e^Gamma and S in fp16
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
         const int x = tid + NT * r, i = x & 63, cc = x >> 6;
+        float kg[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) R1[(8 * cc + e) * LT + i] = kr[r][e] * ex2(sG[i * LD + 8 * cc + e]);
+        for (int e = 0; e < 8; ++e) kg[e] = kr[r][e] * ex2(sG[i * LD + 8 * cc + e]);
+        st_shared_v4(sm + KG16, kmaj_off(i, 8 * cc, 64), pack8_f16(kg));
     }
-    __syncthreads();
+    {
+        const float* S = p.chk + sh * DV * DK;
+#pragma unroll
+        for (int x = tid; x < DV * 16; x += NT) {
+            const int v = x >> 4, cc = x & 15;
+            float f[8];
+            ld8g(S + (size_t)v * DK + 8 * cc, f);
+            st_shared_v4(sm + S16, kmaj_off(v, 8 * cc, 128), pack8_f16(f));
+        }
+    }
+    operands_ready();
+    if (tid == 0) {
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
+            mma_bf16(tm + TM_R, kmaj_desc(sbase + KG16, 64, s), kmaj_desc(sbase + S16, 128, s),
+                     idesc_f16(64, 128, false, false), s > 0);
+        mma_commit(bars + 0);
+    }
+    // meanwhile on the CUDA cores: T, and its two-term fp16 image
+    invert_unit_lower(sA, sb, sT, reinterpret_cast<float*>(sm + PS));
+    for (int x = tid; x < C * 8; x += NT) {
+        const int i = x >> 3, jc = x & 7;
+        float t[8];
+        ld8(sT + i * LT + 8 * jc, t);
+        uint4 hi, lo;
+        pack8_split16(t, hi, lo);
+        st_shared_v4(sm + TH, kmaj_off(i, 8 * jc, 64), hi);
+        st_shared_v4(sm + TL, kmaj_off(i, 8 * jc, 64), lo);
+    }
+    if (!wait_mma(bars + 0)) return false;
+    tc_fence_after();
 
-    // ---- resid^T = V^T - S (K e^Gamma)^T: rows v = 8 vg .. +7, columns i = 4 ig .. +3
+    // ---- resid = V - product 1 (row i = 16 sp + lane, values 64 hc ..); diag(beta) resid
+    // and dE as the MN-major operands of products 2 and 3
     {
-        const int vg = tid >> 4, ig = tid & 15;
-        const float* S = p.chk + sh * DV * DK + (size_t)(8 * vg) * DK;
-        float acc[8][4] = {};
-        float4 cur[8], nxt[8];
+        const int i = 16 * sp + (lane & 15);
+        const bool own = lane < 16;
+        const float b = sb[i];
 #pragma unroll
-        for (int r = 0; r < 8; ++r) cur[r] = __ldg(reinterpret_cast<const float4*>(S + r * DK));
-#pragma unroll 2
-        for (int c = 0; c < DK; c += 4) {
-            if (c + 4 < DK) {
+        for (int q = 0; q < 2; ++q) {
+            const int v0 = 64 * hc + 32 * q;
+            float d[32], vv[32];
+            tmem_ld32(tm + lane_base + TM_R + v0, d);
+            if (own) {
+                loadn<32>(p.v + ((c0 + i) * p.H + h) * DV + v0, i < L, vv);
 #pragma unroll
-                for (int r = 0; r < 8; ++r) nxt[r] = __ldg(reinterpret_cast<const float4*>(S + r * DK + c + 4));
-            }
+                for (int e = 0; e < 32; ++e) d[e] = vv[e] - d[e];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float4 kg = ld4(R1 + (c + e) * LT + 4 * ig);
+                for (int u = 0; u < 8; ++u) st4(sRes + i * LD + v0 + 4 * u, d[4 * u], d[4 * u + 1], d[4 * u + 2], d[4 * u + 3]);
 #pragma unroll
-                for (int r = 0; r < 8; ++r) {
-                    const float s = comp(cur[r], e);
-                    acc[r][0] = fmaf(s, kg.x, acc[r][0]);
-                    acc[r][1] = fmaf(s, kg.y, acc[r][1]);
-                    acc[r][2] = fmaf(s, kg.z, acc[r][2]);
-                    acc[r][3] = fmaf(s, kg.w, acc[r][3]);
-                }
-            }
+                for (int e = 0; e < 32; ++e) d[e] *= b;
 #pragma unroll
-            for (int r = 0; r < 8; ++r) cur[r] = nxt[r];
-        }
-        float vv[4][8];
-#pragma unroll
-        for (int s = 0; s < 4; ++s) {
-            const int i = 4 * ig + s;
-            load8(p.v + ((c0 + i) * p.H + h) * DV + 8 * vg, i < L, vv[s]);
-        }
-#pragma unroll
-        for (int r = 0; r < 8; ++r)
-            st4(R2 + (8 * vg + r) * LT + 4 * ig, vv[0][r] - acc[r][0], vv[1][r] - acc[r][1], vv[2][r] - acc[r][2],
-                vv[3][r] - acc[r][3]);
-    }
-    __syncthreads();
-
-    // ---- E = M^{-1} diag(beta) resid and dEbar = M^{-T} dE, per value row v: two
-    // threads per row split every sum by the parity of its index (each keeps the
-    // entries of its own parity) and meet through one shuffle.
-    {
-        const int v = tid >> 1, par = tid & 1;
-        const float* rs = R2 + v * LT;
-        float* er = R3 + v * LT;
-        for (int i = 0; i < C; ++i) {
-            float part = 0.f;
-            for (int j = par; j < i; j += 2) part = fmaf(sA[i * LT + j], er[j], part);
-            const float tot = part + __shfl_xor_sync(0xffffffffu, part, 1);
-            if ((i & 1) == par) er[i] = sb[i] * (rs[i] - tot);
-        }
-        float* dr = R4 + v * LT;
-        for (int j = C - 1; j >= 0; --j) {
-            float part = 0.f;
-            int i0 = j + 1;
-            if ((i0 & 1) != par) ++i0;
-            for (int i = i0; i < C; i += 2) part = fmaf(sb[i] * sA[i * LT + j], dr[i], part);
-            const float tot = part + __shfl_xor_sync(0xffffffffu, part, 1);
-            if ((j & 1) == par) dr[j] -= tot;
-        }
-    }
-    __syncthreads();
-
-    // ---- dbeta: rowsum(dEbar . resid) + rowsum(dL . A);  dL = -dEbar E^T, dA = diag(beta) dL
-    {
-        const int i = tid & 63, vq = tid >> 6;
-        float s = 0.f;
-        for (int v = 32 * vq; v < 32 * vq + 32; ++v) s = fmaf(R4[v * LT + i], R2[v * LT + i], s);
-        red[vq * C + i] = s;
-    }
-    {
-        const int ig = tid & 15, jg = tid >> 4;
-        float acc[4][4] = {};
-        if (jg <= ig) {
-            for (int v = 0; v < DV; ++v) {
-                const float4 a = ld4(R4 + v * LT + 4 * ig), e = ld4(R3 + v * LT + 4 * jg);
-#pragma unroll
-                for (int r = 0; r < 4; ++r) {
-                    const float ar = comp(a, r);
-                    acc[r][0] = fmaf(ar, e.x, acc[r][0]);
-                    acc[r][1] = fmaf(ar, e.y, acc[r][1]);
-                    acc[r][2] = fmaf(ar, e.z, acc[r][2]);
-                    acc[r][3] = fmaf(ar, e.w, acc[r][3]);
+                for (int u = 0; u < 4; ++u) {
+                    uint4 hi, lo;
+                    pack8_split16(d + 8 * u, hi, lo);
+                    st_shared_v4(sm + EBH, mnmaj_off(v0 + 8 * u, i, 128), hi);
+                    st_shared_v4(sm + EBL, mnmaj_off(v0 + 8 * u, i, 128), lo);
                 }
             }
         }
-        float* da = p.da + sh * C * C;
+    }
+    {
+        const float* dE = p.de + sh * C * DV;
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            const int i = 4 * ig + r;
-            float o[4], dbp = 0.f;
+        for (int x = tid; x < C * 16; x += NT) {
+            const int i = x >> 4, vc = x & 15;
+            float f[8];
+            ld8g(dE + (size_t)i * DV + 8 * vc, f);
+            uint4 hi, lo;
+            pack8_split16(f, hi, lo);
+            st_shared_v4(sm + DEH, mnmaj_off(8 * vc, i, 128), hi);
+            st_shared_v4(sm + DEL, mnmaj_off(8 * vc, i, 128), lo);
+        }
+    }
+    operands_ready();
+    if (tid == 0) {
+        // E = T (diag(beta) resid);  dEbar = T^T dE (the T images read MN-major are T^T);
+        // each over the expansions: hi*hi + hi*lo + lo*hi
+        const uint32_t ta[3] = {sbase + TH, sbase + TH, sbase + TL};
+        const uint32_t eb[3] = {sbase + EBH, sbase + EBL, sbase + EBH};
+        const uint32_t de[3] = {sbase + DEH, sbase + DEL, sbase + DEH};
 #pragma unroll
-            for (int s = 0; s < 4; ++s) {
-                const int j = 4 * jg + s;
-                const float dl = j < i ? -acc[r][s] : 0.f;
-                dbp = fmaf(dl, sA[i * LT + j], dbp);
-                o[s] = sb[i] * dl;
+        for (int t = 0; t < 3; ++t)
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                mma_bf16(tm + TM_E, kmaj_desc(ta[t], 64, s), mnmaj_desc(eb[t], 128, s),
+                         idesc_f16(64, 128, false, true), t > 0 || s > 0);
+#pragma unroll
+        for (int t = 0; t < 3; ++t)
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                mma_bf16(tm + TM_DB, mnmaj_desc(ta[t], 64, s), mnmaj_desc(de[t], 128, s),
+                         idesc_f16(64, 128, true, true), t > 0 || s > 0);
+        mma_commit(bars + 1);
+    }
+    if (!wait_mma(bars + 1)) return false;
+    tc_fence_after();
+
+    // ---- E and dEbar out of tensor memory: the K-major operands of product 4, the
+    // images for the dqk kernel, dv = diag(beta) dEbar, and rowsum(dEbar . resid)
+    {
+        const int i = 16 * sp + (lane & 15);
+        const bool own = lane < 16;
+        const float b = sb[i];
+        uint8_t* e_img = p.e16 + sh * 2 * kTile16;
+        uint8_t* pr_img = p.pr16 + sh * kTile16;
+        float* dv = p.dv + ((c0 + i) * p.H + h) * DV;
+        float db1 = 0.f;
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const int v0 = 64 * hc + 32 * q;
+            float e[32], d[32];
+            tmem_ld32(tm + lane_base + TM_E + v0, e);
+            tmem_ld32(tm + lane_base + TM_DB + v0, d);
+            if (own) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const uint32_t off = kmaj_off(i, v0 + 8 * u, 64);
+                    uint4 e8, el;
+                    pack8_split16(e + 8 * u, e8, el);
+                    st_shared_v4(sm + E16, off, e8);
+                    *reinterpret_cast<uint4*>(e_img + off) = e8;
+                    *reinterpret_cast<uint4*>(e_img + kTile16 + off) = el;
+                    st_shared_v4(sm + DB16, off, pack8_f16(d + 8 * u));
+                    float pr[8];
+#pragma unroll
+                    for (int t = 0; t < 8; ++t) pr[t] = -b * d[8 * u + t];
+                    *reinterpret_cast<uint4*>(pr_img + off) = pack8_f16(pr);
+                }
+#pragma unroll
+                for (int t = 0; t < 32; ++t) db1 = fmaf(d[t], sRes[i * LD + v0 + t], db1);
+                if (i < L) {
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        st4(dv + v0 + 4 * u, b * d[4 * u], b * d[4 * u + 1], b * d[4 * u + 2], b * d[4 * u + 3]);
+                }
             }
-            st4(da + i * C + 4 * jg, o[0], o[1], o[2], o[3]);
-            red[(4 + jg) * C + i] = dbp;
+        }
+        if (own) red[hc * C + i] = db1;
+    }
+    operands_ready();
+    if (tid == 0) {   // dEbar E^T
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
+            mma_bf16(tm + TM_DL, kmaj_desc(sbase + DB16, 64, s), kmaj_desc(sbase + E16, 64, s),
+                     idesc_f16(64, 64, false, false), s > 0);
+        mma_commit(bars + 2);
+    }
+    if (!wait_mma(bars + 2)) return false;
+    tc_fence_after();
+    // ---- dL = -strict_lower(dEbar E^T): rowsum(dL . A), dA = diag(beta) dL
+    {
+        const int i = 16 * sp + (lane & 15);
+        float d[32];
+        tmem_ld32(tm + lane_base + TM_DL + 32 * hc, d);
+        if (lane < 16) {
+            const float b = sb[i];
+            float db2 = 0.f, o[32];
+#pragma unroll
+            for (int t = 0; t < 32; ++t) {
+                const int j = 32 * hc + t;
+                const float dl = j < i ? -d[t] : 0.f;
+                db2 = fmaf(dl, sA[i * LT + j], db2);
+                o[t] = b * dl;
+            }
+            float* da = p.da + sh * C * C + (size_t)i * C + 32 * hc;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) st4(da + 4 * u, o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
+            red[(2 + hc) * C + i] = db2;
         }
     }
     __syncthreads();
+    if (tid < L) p.dbeta[(c0 + tid) * p.H + h] = (red[tid] + red[C + tid]) + (red[2 * C + tid] + red[3 * C + tid]);
+    return true;
+}
 
-    if (tid < L) {
-        float s = 0.f;
-#pragma unroll
-        for (int q = 0; q < 20; ++q) s += red[q * C + tid];
-        p.dbeta[(c0 + tid) * p.H + h] = s;
+template <int GATE>
+__global__ void __launch_bounds__(NT, 1) kda_chunk_bwd_solve_kernel(const __grid_constant__ GradParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int slot = blockIdx.x / p.H, h = blockIdx.x % p.H, hk = h / p.group;
+    pdl_wait();
+    long long c0;
+    int L;
+    if (!slot_rows(p, slot, c0, L)) return;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + s1::BAR);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
+    if (tid == 0) {
+        for (int b = 0; b < 4; ++b) mbar_init(bars + b, 1);
+        fence_mbar_init();
     }
-    {
-        const int v = tid & 127;
-        for (int i = tid >> 7; i < L; i += 2) p.dv[((c0 + i) * p.H + h) * DV + v] = sb[i] * R4[v * LT + i];
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, TMEM_COLS);
+        tmem_relinquish();
     }
-    {
-        float4* de = reinterpret_cast<float4*>(p.de + sh * DV * C);
-        float4* et = reinterpret_cast<float4*>(p.et + sh * DV * C);
-        for (int x = tid; x < DV * C / 4; x += NT) {
-            const int v = x >> 4, i = 4 * (x & 15);
-            const float4 d = ld4(R4 + v * LT + i);
-            de[x] = make_float4(-sb[i] * d.x, -sb[i + 1] * d.y, -sb[i + 2] * d.z, -sb[i + 3] * d.w);
-            et[x] = ld4(R3 + v * LT + i);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = *tmem_slot;
+    const bool ok = solve_body<GATE>(p, sm, tm, bars, c0, L, h, hk, (size_t)slot * p.H + h);
+    if (!ok) {
+        // a bounded wait expired: record it and let every MMA in flight complete
+        if (tid == 0) {
+            if (p.dev_status) atomicOr(p.dev_status, KDA_DEV_TIMEOUT);
+            mma_commit(bars + 3);
+            (void)mbar_wait(bars + 3, 0, kWaitNs);
         }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tm, TMEM_COLS);
     }
 }
 
 // ---------------------------------------------------------------- dqk kernel
 template <int GATE>
-__global__ void __launch_bounds__(NT, 1) kda_chunk_bwd_dqk_kernel(const __grid_constant__ GradParams p) {
-    extern __shared__ float4 smem4[];
-    float* sG = reinterpret_cast<float*>(smem4);   // [64][LD] G (log2 units)
-    float* R1 = sG + REG;                          // E^T [128][LT]   -> K a [64][LD]
-    float* R2 = R1 + REG;                          // dO^T [128][LT]  -> Q~ a
-    float* R3 = R2 + REG;                          // dPr^T [128][LT] -> K b
-    float* sAqk = R3 + REG;                        // [64][LT] dAqk (lower, diagonal included)
-    float* sDA = sAqk + C * LT;                    // [64][LT] dA (strictly lower)
-    float* R4 = sDA + C * LT;                      // state-row ring, then dAqk^T and dA^T
-    float* dfac = R4 + 2 * C * LT;                 // [6][128]
-    float* sred = dfac + 6 * DK;                   // [16][64] scalar-gate partial row sums
-    const int tid = threadIdx.x;
-    const int slot = blockIdx.x / p.H, h = blockIdx.x % p.H, hk = h / p.group, Hk = p.H / p.group;
-    pdl_wait();
-    long long c0;
-    int L;
-    if (!slot_rows(p, slot, c0, L)) return;
-    const size_t sh = (size_t)slot * p.H + h;
-    const float* S = p.chk + sh * DV * DK;
-    const float* dS = p.dsp + sh * DV * DK;
-    // ring of 3 stages, each 8 state rows of S then 8 of dS' (2048 floats)
-    auto issue = [&](int b) {
-        float* stg = R4 + (b % 3) * 2048;
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-            const int x = tid + NT * q, which = x >> 8, rr = (x >> 5) & 7, c4 = x & 31;
-            const float* src = (which ? dS : S) + (size_t)(8 * b + rr) * DK + 4 * c4;
-            cp_async16(stg + which * 1024 + rr * 128 + 4 * c4, src);
-        }
-        cp_async_commit();
-    };
-    issue(0);
-    issue(1);
+__device__ __forceinline__ bool dqk_body(const GradParams& p, uint8_t* sm, uint32_t tm, uint64_t* bars,
+                                         long long c0, int L, int h, int hk, size_t sh, int& fetched) {
+    using namespace s2;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, sp = warp & 3, hc = warp >> 2;
+    const uint32_t sbase = smem_u32(sm), lane_base = (uint32_t)(32 * sp) << 16;
+    float* sG = reinterpret_cast<float*>(sm + G);
+    float* sAqk = reinterpret_cast<float*>(sm + AQK);
+    float* sDA = reinterpret_cast<float*>(sm + DA);
+    float* dAT = reinterpret_cast<float*>(sm + AQT);
+    float* dDT = reinterpret_cast<float*>(sm + DAT);
+    float* dfac = reinterpret_cast<float*>(sm + DFAC);
+    float* ucol = reinterpret_cast<float*>(sm + UCOL);
+    float* sgs = reinterpret_cast<float*>(sm + SGS);
+    float* sred = reinterpret_cast<float*>(sm + SRED);
+    float* Pk = reinterpret_cast<float*>(sm + P);
+    float* Pq = Pk + 64 * LD;
+    float* Pg = Pq + 64 * LD;
+    const int Hk = p.H / p.group;
 
-    load_gamma<GATE>(p, c0, L, h, sG);
-    {
-        const float4* e4 = reinterpret_cast<const float4*>(p.et + sh * DV * C);
-        const float4* p4 = reinterpret_cast<const float4*>(p.de + sh * DV * C);
-        for (int x = tid; x < DV * C / 4; x += NT) {
-            const int off = (x >> 4) * LT + 4 * (x & 15);
-            *reinterpret_cast<float4*>(R1 + off) = e4[x];
-            *reinterpret_cast<float4*>(R3 + off) = p4[x];
+    // The products run in two passes over halves hv of the value axis (the operand
+    // tiles of one half fill the union).  E (hi, lo) and dPr of half hv are the second
+    // 8 KB of their K-major images when hv = 1: one bulk copy each.
+    auto fetch = [&](int hv, uint64_t* bar) {
+        if (tid == 0) {
+            mbar_arrive_expect_tx(bar, 3u * 8192u);
+            const uint8_t* e = p.e16 + sh * 2 * kTile16 + 8192 * hv;
+            bulk_load(sm + EH, e, 8192u, bar);
+            bulk_load(sm + EL, e + kTile16, 8192u, bar);
+            bulk_load(sm + PR16, p.pr16 + sh * kTile16 + 8192 * hv, 8192u, bar);
+            fetched = hv + 1;
         }
+    };
+    // dO (bf16 -> fp16, exact), S and dS' (fp32 -> two-term fp16, MN-major over the
+    // channel) of half hv; colsum(S . dS') partials of this thread's channels
+    float sgs_acc[8] = {};
+    auto build = [&](int hv) {
+#pragma unroll
+        for (int x = tid; x < C * 8; x += NT) {
+            const int i = x >> 3, vc = x & 7;
+            float f[8];
+            loadn<8>(p.d_out + ((c0 + i) * p.H + h) * DV + 64 * hv + 8 * vc, i < L, f);
+            st_shared_v4(sm + DO16, kmaj_off(i, 8 * vc, 64), pack8_f16(f));
+        }
+        const float* S = p.chk + sh * DV * DK;
+        const float* dS = p.dsp + sh * DV * DK;
+        const int cc = tid & 15;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const int vl = (tid >> 4) + 16 * r, v = 64 * hv + vl;
+            float s8[8], d8[8];
+            ld8g(S + (size_t)v * DK + 8 * cc, s8);
+            ld8g(dS + (size_t)v * DK + 8 * cc, d8);
+            uint4 hi, lo;
+            pack8_split16(s8, hi, lo);
+            st_shared_v4(sm + SH, mnmaj_off(8 * cc, vl, 128), hi);
+            st_shared_v4(sm + SL, mnmaj_off(8 * cc, vl, 128), lo);
+            pack8_split16(d8, hi, lo);
+            st_shared_v4(sm + DH, mnmaj_off(8 * cc, vl, 128), hi);
+            st_shared_v4(sm + DL, mnmaj_off(8 * cc, vl, 128), lo);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) sgs_acc[e] = fmaf(s8[e], d8[e], sgs_acc[e]);
+        }
+    };
+    // dKd = E dS' (hi*hi + hi*lo + lo*hi), dQg = dO S, dKg = dPr S, dO E^T (over S's and E's
+    // two terms); the first product of half 0 starts each accumulator
+    auto issue = [&](int hv) {
+        const uint32_t xa[3] = {sbase + EH, sbase + EH, sbase + EL};
+        const uint32_t xb[3] = {sbase + DH, sbase + DL, sbase + DH};
+        const uint32_t st2[2] = {sbase + SH, sbase + SL};
+        const uint32_t et2[2] = {sbase + EH, sbase + EL};
+#pragma unroll
+        for (int t = 0; t < 3; ++t)
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                mma_bf16(tm + TM_KD, kmaj_desc(xa[t], 64, s), mnmaj_desc(xb[t], 128, s),
+                         idesc_f16(64, 128, false, true), hv > 0 || t > 0 || s > 0);
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+            for (int s = 0; s < 4; ++s) {
+                mma_bf16(tm + TM_QG, kmaj_desc(sbase + DO16, 64, s), mnmaj_desc(st2[t], 128, s),
+                         idesc_f16(64, 128, false, true), hv > 0 || t > 0 || s > 0);
+                mma_bf16(tm + TM_KG, kmaj_desc(sbase + PR16, 64, s), mnmaj_desc(st2[t], 128, s),
+                         idesc_f16(64, 128, false, true), hv > 0 || t > 0 || s > 0);
+                mma_bf16(tm + TM_AQ, kmaj_desc(sbase + DO16, 64, s), kmaj_desc(et2[t], 64, s),
+                         idesc_f16(64, 64, false, false), hv > 0 || t > 0 || s > 0);
+            }
+    };
+
+    fetch(0, bars + 0);
+    load_gamma<GATE>(p, c0, L, h, sG);
+    build(0);
+    {
         const float4* a4 = reinterpret_cast<const float4*>(p.da + sh * C * C);
+#pragma unroll
         for (int x = tid; x < C * C / 4; x += NT) *reinterpret_cast<float4*>(sDA + (x >> 4) * LT + 4 * (x & 15)) = a4[x];
     }
+    if (!__syncthreads_and(mbar_wait(bars + 0, 0, kWaitNs))) return false;
+    operands_ready();
+    if (tid == 0) {
+        issue(0);
+        mma_commit(bars + 1);
+    }
+    load_dfac(sG, dfac);
+    if (!wait_mma(bars + 1)) return false;
+    fetch(1, bars + 2);
+    build(1);
+    if (!__syncthreads_and(mbar_wait(bars + 2, 0, kWaitNs))) return false;
+    operands_ready();
+    if (tid == 0) {
+        issue(1);
+        mma_commit(bars + 3);
+    }
+    {
+        const int cc = tid & 15;
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {   // dO^T
-        const int x = tid + NT * r, i = x & 63, cc = x >> 6;
-        float o[8];
-        load8(p.d_out + ((c0 + i) * p.H + h) * DV + 8 * cc, i < L, o);
+        for (int e = 0; e < 8; ++e) sgs_acc[e] += __shfl_xor_sync(0xffffffffu, sgs_acc[e], 16);
+        if (lane < 16) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) R2[(8 * cc + e) * LT + i] = o[e];
+            for (int e = 0; e < 8; ++e) sgs[warp * DK + 8 * cc + e] = sgs_acc[e];
+        }
+    }
+    if (!wait_mma(bars + 3)) return false;
+    tc_fence_after();
+
+    // ---- per element (row i = 16 sp + lane, channels 64 hc ..): dK, dQ, dGamma so far,
+    // colsum(dKd . Kd) partials, and dAqk (and its transpose)
+    {
+        const int i = 16 * sp + (lane & 15);
+        const bool own = lane < 16;
+#pragma unroll 1
+        for (int q = 0; q < 2; ++q) {
+            const int cb = 64 * hc + 32 * q;
+            float xk[32], xq[32], xg[32];
+            tmem_ld32(tm + lane_base + TM_KD + cb, xk);
+            tmem_ld32(tm + lane_base + TM_QG + cb, xq);
+            tmem_ld32(tm + lane_base + TM_KG + cb, xg);
+            float kx[32], qx[32];
+            loadn<32>(p.k + ((c0 + i) * Hk + hk) * DK + cb, own && i < L, kx);
+            loadn<32>(p.q + ((c0 + i) * Hk + hk) * DK + cb, own && i < L, qx);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const int c = cb + e;
+                const float Gv = sG[i * LD + c], gam = sG[(C - 1) * LD + c];
+                const float eG = ex2(Gv), eD = ex2(gam - Gv);
+                const float Kd = kx[e] * eD, Kg = kx[e] * eG, Qg = qx[e] * p.scale * eG;
+                const float dKd = xk[e], dQg = xq[e], dKg = xg[e];
+                float u = own ? dKd * Kd : 0.f;
+                xk[e] = dKd * eD + dKg * eG;
+                xq[e] = dQg * eG;
+                xg[e] = -dKd * Kd + dQg * Qg + dKg * Kg;
+                u += __shfl_xor_sync(0xffffffffu, u, 1);
+                u += __shfl_xor_sync(0xffffffffu, u, 2);
+                u += __shfl_xor_sync(0xffffffffu, u, 4);
+                u += __shfl_xor_sync(0xffffffffu, u, 8);
+                if (lane == 0) ucol[sp * DK + c] = u;
+            }
+            if (own) {
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    st4(Pk + i * LD + cb + 4 * u, xk[4 * u], xk[4 * u + 1], xk[4 * u + 2], xk[4 * u + 3]);
+                    st4(Pq + i * LD + cb + 4 * u, xq[4 * u], xq[4 * u + 1], xq[4 * u + 2], xq[4 * u + 3]);
+                    st4(Pg + i * LD + cb + 4 * u, xg[4 * u], xg[4 * u + 1], xg[4 * u + 2], xg[4 * u + 3]);
+                }
+            }
+        }
+        float z[32];
+        tmem_ld32(tm + lane_base + TM_AQ + 32 * hc, z);
+        if (own) {
+#pragma unroll
+            for (int t = 0; t < 32; ++t) {
+                const int j = 32 * hc + t;
+                const float x = j <= i ? z[t] : 0.f;
+                sAqk[i * LT + j] = x;
+                dAT[j * LT + i] = x;
+            }
+        }
+    }
+    for (int x = tid; x < C * C; x += NT) {
+        const int i = x & 63, j = x >> 6;
+        dDT[j * LT + i] = sDA[i * LT + j];
     }
     __syncthreads();
-    load_dfac(sG, dfac);
 
-    // ---- dAqk = lower(dO E^T), diagonal included
-    {
-        const int ig = tid & 15, jg = tid >> 4;
-        float acc[4][4] = {};
-        if (jg <= ig) {
-            for (int v = 0; v < DV; ++v) {
-                const float4 a = ld4(R2 + v * LT + 4 * ig), e = ld4(R1 + v * LT + 4 * jg);
-#pragma unroll
-                for (int r = 0; r < 4; ++r) {
-                    const float ar = comp(a, r);
-                    acc[r][0] = fmaf(ar, e.x, acc[r][0]);
-                    acc[r][1] = fmaf(ar, e.y, acc[r][1]);
-                    acc[r][2] = fmaf(ar, e.z, acc[r][2]);
-                    acc[r][3] = fmaf(ar, e.w, acc[r][3]);
-                }
-            }
-        }
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            const int i = 4 * ig + r;
-            float o[4];
-#pragma unroll
-            for (int s = 0; s < 4; ++s) o[s] = (4 * jg + s <= i) ? acc[r][s] : 0.f;
-            st4(sAqk + i * LT + 4 * jg, o[0], o[1], o[2], o[3]);
-        }
-    }
-
-    // ---- one pass over the state rows v: dKd = E dS', dQg = dO S, dKg = dPr S and
-    // colsum(S . dS'); thread: rows i = 4 ig .. +3, channels c = 8 cg .. +7
+    // ---- from here on: thread rows i = 4 ig .. +3, channels c = 8 cg .. +7
     const int cg = tid >> 4, ig = tid & 15, I = ig >> 2;
-    float xk[4][8] = {}, xq[4][8] = {}, xg[4][8] = {}, dgs[8] = {};
-    for (int b = 0; b < DV / 8; ++b) {
-        cp_async_wait1();
-        __syncthreads();
-        if (b + 2 < DV / 8) issue(b + 2); else cp_async_commit();
-        const float* stg = R4 + (b % 3) * 2048;
-#pragma unroll 2
-        for (int rr = 0; rr < 8; ++rr) {
-            const int v = 8 * b + rr;
-            const float4 e = ld4(R1 + v * LT + 4 * ig), o = ld4(R2 + v * LT + 4 * ig), pr = ld4(R3 + v * LT + 4 * ig);
-            const float4 s0 = ld4(stg + rr * 128 + 8 * cg), s1 = ld4(stg + rr * 128 + 8 * cg + 4);
-            const float4 d0 = ld4(stg + 1024 + rr * 128 + 8 * cg), d1 = ld4(stg + 1024 + rr * 128 + 8 * cg + 4);
-            const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-            const float dv[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+    float xk[4][8], xq[4][8], xg[4][8], dgam[8];
 #pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const float er = comp(e, r), orr = comp(o, r), pp = comp(pr, r);
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    xk[r][c] = fmaf(er, dv[c], xk[r][c]);
-                    xq[r][c] = fmaf(orr, sv[c], xq[r][c]);
-                    xg[r][c] = fmaf(pp, sv[c], xg[r][c]);
-                }
-            }
-#pragma unroll
-            for (int c = 0; c < 8; ++c) dgs[c] = fmaf(sv[c], dv[c], dgs[c]);
-        }
+    for (int r = 0; r < 4; ++r) {
+        const int i = 4 * ig + r;
+        ld8(Pk + i * LD + 8 * cg, xk[r]);
+        ld8(Pq + i * LD + 8 * cg, xq[r]);
+        ld8(Pg + i * LD + 8 * cg, xg[r]);
     }
-    cp_async_wait0();
-
-    // ---- element-wise: xk <- dK, xq <- dQ, xg <- dGamma (so far); dgam per channel
-    float gam[8], dgam[8];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) gam[c] = sG[(C - 1) * LD + 8 * cg + c];
-    {
-        float dgp[8] = {};
+    for (int c = 0; c < 8; ++c) {
+        const int cc = 8 * cg + c;
+        float s = 0.f;
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            const int i = 4 * ig + r;
-            float kx[8], qx[8];
-            load8(p.k + ((c0 + i) * Hk + hk) * DK + 8 * cg, i < L, kx);
-            load8(p.q + ((c0 + i) * Hk + hk) * DK + 8 * cg, i < L, qx);
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const float G = sG[i * LD + 8 * cg + c];
-                const float eG = ex2(G), eD = ex2(gam[c] - G);
-                const float Kd = kx[c] * eD, Kg = kx[c] * eG, Qg = qx[c] * p.scale * eG;
-                const float dKd = xk[r][c], dQg = xq[r][c], dKg = xg[r][c];
-                dgp[c] = fmaf(dKd, Kd, dgp[c]);
-                xk[r][c] = dKd * eD + dKg * eG;
-                xq[r][c] = dQg * eG;
-                xg[r][c] = -dKd * Kd + dQg * Qg + dKg * Kg;
-            }
-        }
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            float x = dgp[c];
-            x += __shfl_xor_sync(0xffffffffu, x, 1);
-            x += __shfl_xor_sync(0xffffffffu, x, 2);
-            x += __shfl_xor_sync(0xffffffffu, x, 4);
-            x += __shfl_xor_sync(0xffffffffu, x, 8);
-            dgam[c] = dgs[c] * ex2(gam[c]) + x;
-        }
+        for (int w = 0; w < 8; ++w) s += sgs[w * DK + cc];
+        dgam[c] = s * ex2(sG[(C - 1) * LD + cc]) + ((ucol[cc] + ucol[DK + cc]) + (ucol[2 * DK + cc] + ucol[3 * DK + cc]));
     }
-    __syncthreads();   // E^T, dO^T, dPr^T and the ring are dead from here on
-
-    // K a, Q~ a, K b; dAqk^T and dA^T
-    float* dAT = R4;
-    float* dDT = R4 + C * LT;
+    __syncthreads();   // the partials are in registers; their region takes K a, Q~ a, K b
+    float* Ka = reinterpret_cast<float*>(sm + OPS);
+    float* Qa = Ka + 64 * LD;
+    float* Kb = Qa + 64 * LD;
+#pragma unroll
     for (int x = tid; x < C * 16; x += NT) {
         const int i = x >> 4, cc = x & 15;
         float kx[8], qx[8];
-        load8(p.k + ((c0 + i) * Hk + hk) * DK + 8 * cc, i < L, kx);
-        load8(p.q + ((c0 + i) * Hk + hk) * DK + 8 * cc, i < L, qx);
+        loadn<8>(p.k + ((c0 + i) * Hk + hk) * DK + 8 * cc, i < L, kx);
+        loadn<8>(p.q + ((c0 + i) * Hk + hk) * DK + 8 * cc, i < L, qx);
         const float* Gi = sG + i * LD + 8 * cc;
         const float* Gr = sG + (i & ~15) * LD + 8 * cc;
         float ka[8], qa[8], kb[8];
@@ -560,20 +832,15 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_bwd_dqk_kernel(const __grid_c
             qa[e] = qx[e] * p.scale * a;
             kb[e] = kx[e] * bb;
         }
-        float* o1 = R1 + i * LD + 8 * cc;
-        float* o2 = R2 + i * LD + 8 * cc;
-        float* o3 = R3 + i * LD + 8 * cc;
+        float* o1 = Ka + i * LD + 8 * cc;
+        float* o2 = Qa + i * LD + 8 * cc;
+        float* o3 = Kb + i * LD + 8 * cc;
         st4(o1, ka[0], ka[1], ka[2], ka[3]);
         st4(o1 + 4, ka[4], ka[5], ka[6], ka[7]);
         st4(o2, qa[0], qa[1], qa[2], qa[3]);
         st4(o2 + 4, qa[4], qa[5], qa[6], qa[7]);
         st4(o3, kb[0], kb[1], kb[2], kb[3]);
         st4(o3 + 4, kb[4], kb[5], kb[6], kb[7]);
-    }
-    for (int x = tid; x < C * C; x += NT) {
-        const int i = x & 63, j = x >> 6;
-        dAT[j * LT + i] = sAqk[i * LT + j];
-        dDT[j * LT + i] = sDA[i * LT + j];
     }
     __syncthreads();
 
@@ -585,9 +852,10 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_bwd_dqk_kernel(const __grid_c
             float dv[8];
 #pragma unroll
             for (int c = 0; c < 8; ++c) dv[c] = J < I ? dfac[pair_index(I, J) * DK + 8 * cg + c] : 1.f;
+#pragma unroll 2
             for (int j = 16 * J; j < 16 * J + 16; ++j) {
                 const float4 aq = ld4(dAT + j * LT + 4 * ig), ad = ld4(dDT + j * LT + 4 * ig);
-                const float4 b0 = ld4(R3 + j * LD + 8 * cg), b1 = ld4(R3 + j * LD + 8 * cg + 4);
+                const float4 b0 = ld4(Kb + j * LD + 8 * cg), b1 = ld4(Kb + j * LD + 8 * cg + 4);
                 const float kb[8] = {b0.x * dv[0], b0.y * dv[1], b0.z * dv[2], b0.w * dv[3],
                                      b1.x * dv[4], b1.y * dv[5], b1.z * dv[6], b1.w * dv[7]};
 #pragma unroll
@@ -610,7 +878,7 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_bwd_dqk_kernel(const __grid_c
                 const float a = ex2(sG[i * LD + cc] - sG[16 * I * LD + cc]);
                 xq[r][c] = fmaf(a, x1[r][c], xq[r][c]);
                 xk[r][c] = fmaf(a, x2[r][c], xk[r][c]);
-                xg[r][c] += R2[i * LD + cc] * x1[r][c] + R1[i * LD + cc] * x2[r][c];
+                xg[r][c] += Qa[i * LD + cc] * x1[r][c] + Ka[i * LD + cc] * x2[r][c];
             }
         }
     }
@@ -622,10 +890,11 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_bwd_dqk_kernel(const __grid_c
             float dv[8];
 #pragma unroll
             for (int c = 0; c < 8; ++c) dv[c] = Ip > I ? dfac[pair_index(Ip, I) * DK + 8 * cg + c] : 1.f;
+#pragma unroll 2
             for (int i = 16 * Ip; i < 16 * Ip + 16; ++i) {
                 const float4 aq = ld4(sAqk + i * LT + 4 * ig), ad = ld4(sDA + i * LT + 4 * ig);
-                const float4 q0 = ld4(R2 + i * LD + 8 * cg), q1 = ld4(R2 + i * LD + 8 * cg + 4);
-                const float4 k0 = ld4(R1 + i * LD + 8 * cg), k1 = ld4(R1 + i * LD + 8 * cg + 4);
+                const float4 q0 = ld4(Qa + i * LD + 8 * cg), q1 = ld4(Qa + i * LD + 8 * cg + 4);
+                const float4 k0 = ld4(Ka + i * LD + 8 * cg), k1 = ld4(Ka + i * LD + 8 * cg + 4);
                 const float qa[8] = {q0.x * dv[0], q0.y * dv[1], q0.z * dv[2], q0.w * dv[3],
                                      q1.x * dv[4], q1.y * dv[5], q1.z * dv[6], q1.w * dv[7]};
                 const float ka[8] = {k0.x * dv[0], k0.y * dv[1], k0.z * dv[2], k0.w * dv[3],
@@ -646,7 +915,7 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_bwd_dqk_kernel(const __grid_c
                 const int cc = 8 * cg + c;
                 const float b = ex2(sG[16 * I * LD + cc] - sG[j * LD + cc]);
                 xk[r][c] = fmaf(b, y[r][c], xk[r][c]);
-                xg[r][c] -= R3[j * LD + cc] * y[r][c];
+                xg[r][c] -= Kb[j * LD + cc] * y[r][c];
             }
         }
     }
@@ -671,6 +940,7 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_bwd_dqk_kernel(const __grid_c
         xg[2][c] = s2 + excl;
         xg[3][c] = s3 + excl;
     }
+    if (GATE == KDA_GATE_SCALAR) __syncthreads();   // the row sums reuse the transposes' space
 
     // ---- outputs
 #pragma unroll
@@ -712,16 +982,62 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_bwd_dqk_kernel(const __grid_c
             p.dg[(c0 + tid) * p.H + h] = s;
         }
     }
+    return true;
+}
+
+template <int GATE>
+__global__ void __launch_bounds__(NT, 1) kda_chunk_bwd_dqk_kernel(const __grid_constant__ GradParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int slot = blockIdx.x / p.H, h = blockIdx.x % p.H, hk = h / p.group;
+    pdl_wait();
+    long long c0;
+    int L;
+    if (!slot_rows(p, slot, c0, L)) return;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + s2::BAR);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 5);
+    if (tid == 0) {
+        for (int b = 0; b < 5; ++b) mbar_init(bars + b, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = *tmem_slot;
+    int fetched = 0;   // thread 0: bulk copies issued (halves)
+    const bool ok = dqk_body<GATE>(p, sm, tm, bars, c0, L, h, hk, (size_t)slot * p.H + h, fetched);
+    if (!ok) {
+        if (tid == 0) {
+            if (p.dev_status) atomicOr(p.dev_status, KDA_DEV_TIMEOUT);
+            // the bulk copies and every MMA issued so far land before the memory goes away
+            if (fetched > 0) (void)mbar_wait(bars + 0, 0, kWaitNs);
+            if (fetched > 1) (void)mbar_wait(bars + 2, 0, kWaitNs);
+            mma_commit(bars + 4);
+            (void)mbar_wait(bars + 4, 0, kWaitNs);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tm, TMEM_COLS);
+    }
 }
 
 template <int GATE>
 cudaError_t launch_grad_gate(const GradParams& p, unsigned grid, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(kda_chunk_bwd_solve_kernel<GATE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         SOLVE_SMEM);
+                                         s1::BYTES);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(kda_chunk_bwd_dqk_kernel<GATE>, cudaFuncAttributeMaxDynamicSharedMemorySize, DQK_SMEM);
-    if (e == cudaSuccess) e = launch_after(kda_chunk_bwd_solve_kernel<GATE>, dim3(grid), NT, SOLVE_SMEM, st, p);
-    if (e == cudaSuccess) e = launch_after(kda_chunk_bwd_dqk_kernel<GATE>, dim3(grid), NT, DQK_SMEM, st, p);
+        e = cudaFuncSetAttribute(kda_chunk_bwd_dqk_kernel<GATE>, cudaFuncAttributeMaxDynamicSharedMemorySize, s2::BYTES);
+    if (e == cudaSuccess) e = launch_after(kda_chunk_bwd_solve_kernel<GATE>, dim3(grid), NT, s1::BYTES, st, p);
+    if (e == cudaSuccess) e = launch_after(kda_chunk_bwd_dqk_kernel<GATE>, dim3(grid), NT, s2::BYTES, st, p);
     return e;
 }
 
@@ -739,14 +1055,16 @@ cudaError_t launch_chunk_bwd_grad(const ChunkBwdArgs& a, uint8_t* ws, const BwdL
     p.coff = a.cu_seqlens ? reinterpret_cast<const int32_t*>(ws + bl.fwd.coff_off) : nullptr;
     p.chk = reinterpret_cast<const float*>(ws + bl.chk_off);
     p.dsp = reinterpret_cast<const float*>(ws + bl.dsp_off);
-    p.de = reinterpret_cast<float*>(ws + bl.de_off);
-    p.et = reinterpret_cast<float*>(ws + bl.et_off);
+    p.de = reinterpret_cast<const float*>(ws + bl.de_off);
+    p.e16 = ws + bl.e16_off;
+    p.pr16 = ws + bl.pr16_off;
     p.da = reinterpret_cast<float*>(ws + bl.da_off);
     p.dq = a.dq;
     p.dk = a.dk;
     p.dv = a.dv;
     p.dg = a.dg;
     p.dbeta = a.dbeta;
+    p.dev_status = a.dev_status;
     p.T = a.T;
     p.H = a.H;
     p.num_seqs = a.num_seqs;

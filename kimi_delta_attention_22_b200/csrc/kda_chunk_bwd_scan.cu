@@ -17,7 +17,7 @@
 // the way the forward scan holds S: one value row per tensor-memory lane, the
 // fp32 dS the accumulator of its own update and its fp16 copy the A operand of
 // the next (earlier) chunk's first product, as are dO^T and dE^T.  For every chunk
-// it leaves dS' (the gradient of the chunk's outgoing state) and dE^T in the
+// it leaves dS' (the gradient of the chunk's outgoing state) and dE in the
 // workspace for the chunk-parallel gradient kernels, and writes dS0 at the end.
 // dE^T enters the dS update negated (its fp16 copy is stored as -dE^T), so every
 // product accumulates.
@@ -63,7 +63,7 @@ struct BwdScanParams {
     const float* d_ST;
     float* dS0;
     float* dsp;      // [slot][H][d_v][d_k] fp32: gradient of each chunk's outgoing state
-    float* de;       // [slot][H][d_v][C] fp32: dE^T of each chunk
+    float* de;       // [slot][H][C][d_v] fp32: dE of each chunk
     int32_t* dev_status;
     int T, H, num_seqs, nc;
 };
@@ -239,6 +239,9 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_bwd_scan_kernel(const __grid_
             const size_t slot_h = (size_t)(first + m) * p.H + h;
             if (!(ok = warp_wait(b.full + r % NSTAGE, (uint32_t)((r / NSTAGE) & 1)))) break;
             const uint8_t* st = stage_of(r);
+            // the global writes of dS' and dE come after the arrive that releases the
+            // MMA thread: they leave the chunk's critical path
+            float x[32];
             {
                 // dO^T of this thread's tokens (rows past the chunk's length are zero)
                 const __nv_bfloat16* dot = reinterpret_cast<const __nv_bfloat16*>(st + REC_STAGE);
@@ -251,15 +254,12 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_bwd_scan_kernel(const __grid_
                     o[e] = pack_f16(a, c);
                 }
                 tmem_st8(tm + lane_base + TM_AO + (EC / 2) * part, o);
-                // dS' of this chunk to the workspace, then dS' Diag(dec)
+                // dS' Diag(dec)
                 const float4* dec = reinterpret_cast<const float4*>(st + rec::DEC) + (SC / 4) * part;
-                float x[32];
                 tmem_ld32(tm + lane_base + TM_DS + SC * part, x);
-                float4* out = reinterpret_cast<float4*>(p.dsp + slot_h * DV * DK + (size_t)v * DK + SC * part);
                 uint32_t y[32];
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
-                    out[q] = make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
                     const float4 g = dec[q];
                     y[4 * q] = __float_as_uint(x[4 * q] * g.x);
                     y[4 * q + 1] = __float_as_uint(x[4 * q + 1] * g.y);
@@ -272,16 +272,18 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_bwd_scan_kernel(const __grid_
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(b.oready);
+            {
+                float4* out = reinterpret_cast<float4*>(p.dsp + slot_h * DV * DK + (size_t)v * DK + SC * part);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) out[q] = make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
+            }
             if (!(ok = warp_wait(b.bar1, (uint32_t)(r & 1)))) break;
             tc_fence_after();
+            float d[EC];
             {
-                // dE^T of this thread's tokens to the workspace, and fp16 -dE^T
-                float d[EC];
+                // fp16 -dE^T of this thread's tokens
                 tmem_ld16(tm + lane_base + TM_DE + EC * part, d);
-                float4* de = reinterpret_cast<float4*>(p.de + (slot_h * DV + v) * C + EC * part);
                 uint32_t r16[EC / 2];
-#pragma unroll
-                for (int q = 0; q < EC / 4; ++q) de[q] = make_float4(d[4 * q], d[4 * q + 1], d[4 * q + 2], d[4 * q + 3]);
 #pragma unroll
                 for (int e = 0; e < EC / 2; ++e) r16[e] = pack_f16(-d[2 * e], -d[2 * e + 1]);
                 tmem_st8(tm + lane_base + TM_AE + (EC / 2) * part, r16);
@@ -290,6 +292,13 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_bwd_scan_kernel(const __grid_
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(b.eready);
+            {
+                // dE to the workspace, token-major: one coalesced row of the warp's 32
+                // values per token
+                float* de = p.de + (slot_h * C + EC * part) * DV + v;
+#pragma unroll
+                for (int e = 0; e < EC; ++e) de[(size_t)e * DV] = d[e];
+            }
             if (!(ok = warp_wait(b.bar2, (uint32_t)(r & 1)))) break;
             tc_fence_after();
             {

@@ -175,21 +175,15 @@ struct Tile {
         for (int q = 0; q < G::EC / 8; ++q)
             u[q] = *reinterpret_cast<const uint4*>(stg + rec::UT + kmaj_off(v, G::EC * part + 8 * q, 128));
     }
-    // S <- S Diag(dec of chunk m), ahead of the accumulation of E^T Kd; with chk set,
-    // S (the incoming state of chunk m) is first copied there (row v of this thread)
-    __device__ __forceinline__ void decay(int m, float* chk) const {
+    // S <- S Diag(dec of chunk m), ahead of the accumulation of E^T Kd; S (the incoming
+    // state of chunk m, this thread's SC columns of row v) is also left in keep
+    __device__ __forceinline__ void decay(int m, float (&keep)[G::SC]) const {
         const float4* dec = reinterpret_cast<const float4*>(sm + (m % G::NSTAGE) * G::STAGE + rec::DEC) +
                             (G::SC / 4) * part;
 #pragma unroll
         for (int c32 = 0; c32 < G::SC / 32; ++c32) {
-            float x[32];
+            float* x = keep + 32 * c32;
             tmem_ld32(tm + lane_base + G::TM_S + G::SC * part + 32 * c32, x);
-            if (chk) {
-                float4* dst = reinterpret_cast<float4*>(chk + (size_t)v * DK + G::SC * part + 32 * c32);
-#pragma unroll
-                for (int q = 0; q < 8; ++q)
-                    dst[q] = make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
-            }
             uint32_t r[32];
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
@@ -420,13 +414,21 @@ __global__ void __launch_bounds__(Cfg<NW>::NT, 1) kda_chunk_scan_kernel(const __
             uint4 ut[G::EC / 8];
             if (!(ok = warp_wait(b.full + m % NSTAGE, (uint32_t)((m / NSTAGE) & 1)))) break;
             t.load_ut(m, ut);
-            t.decay(m, p.S_chk ? p.S_chk + ((size_t)(first + m) * p.H + t.h) * DV * DK : nullptr);
+            float s_in[G::SC];
+            t.decay(m, s_in);
             if (!(ok = warp_wait(b.bar1, (uint32_t)(m & 1)))) break;
             tc_fence_after();
             t.e_step(m, ut);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(b.eready);
+            if (p.S_chk) {   // the checkpoint, off the chunk's critical path
+                float4* dst = reinterpret_cast<float4*>(p.S_chk + ((size_t)(first + m) * p.H + t.h) * DV * DK +
+                                                        (size_t)t.v * DK + G::SC * t.part);
+#pragma unroll
+                for (int q = 0; q < G::SC / 4; ++q)
+                    dst[q] = make_float4(s_in[4 * q], s_in[4 * q + 1], s_in[4 * q + 2], s_in[4 * q + 3]);
+            }
             if (!(ok = warp_wait(b.bar2, (uint32_t)(m & 1)))) break;
             tc_fence_after();
             t.s_copy();

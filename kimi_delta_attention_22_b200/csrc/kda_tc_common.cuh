@@ -157,6 +157,21 @@ __device__ __forceinline__ void pack8_split(const float* v, uint4& hi, uint4& lo
     lo = make_uint4(l[0], l[1], l[2], l[3]);
 }
 
+// Two-term fp16 expansion of 8 fp32 values: hi = fp16(v), lo = fp16(v - hi); hi + lo
+// carries about 22 significant bits (lo's own rounding, or its underflow below fp16's
+// normal range, bounds the rest).
+__device__ __forceinline__ void pack8_split16(const float* v, uint4& hi, uint4& lo) {
+    uint32_t h[4], l[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        h[e] = pack_f16(v[2 * e], v[2 * e + 1]);
+        const float2 r = unpack_f16(h[e]);   // exact: the rounded pair back in fp32
+        l[e] = pack_f16(v[2 * e] - r.x, v[2 * e + 1] - r.y);
+    }
+    hi = make_uint4(h[0], h[1], h[2], h[3]);
+    lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
 // ------------------------------------------------------------------ host side
 
 // Launch `kern` after the previous work of `st` with programmatic serialization:

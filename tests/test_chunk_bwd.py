@@ -61,7 +61,7 @@ def test_chunk_bwd_validation(lib):
 def test_chunk_bwd_workspace_size(lib):
     sh = kda.Shape(4, 2048, 16, 128, 128, 4, kda.KDA_BF16, kda.KDA_GATE_CHANNEL, 64, None, 0)
     units = 4 * 32 * 16
-    per = 74240 + 2 * 65536 + 2 * 32768 + 16384
+    per = 74240 + 2 * 65536 + 32768 + 3 * 16384 + 16384
     nbytes = lib.kda_chunk_bwd_workspace_size(ctypes.byref(sh), 0)
     # plus the forward's header: the slow-chunk list (one int32 per unit, and a count)
     assert units * per <= nbytes <= units * per + 4 * (units + 1) + 1024
