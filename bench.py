@@ -11,8 +11,10 @@ line: "e2e" (the same step from pinned host buffers, copies included),
 "no_workspace" (the same call without a workspace), "varlen" (8 packed
 sequences, 65,536 tokens, 32 heads) and "sweep" (B=8, H=64, T=8192 in six
 gate / beta regimes), each with its own roofline; "decode" (256 x 32 heads,
-d=128, fp32 state in HBM, 128 one-token calls after a 512-token prefill) and
-"backward" (kda_recurrent_bwd, 256 x 32 heads x 16 tokens).
+d=128, fp32 state in HBM, 128 one-token calls after a 512-token prefill),
+"backward" (kda_chunk_bwd, the chunkwise gradients of the prefill workload,
+with its own roofline) and "backward_recurrent" (kda_recurrent_bwd, 256 x 32
+heads x 16 tokens).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -38,7 +40,7 @@ if ROOT not in sys.path:
 
 import torch
 
-from kimi_delta_attention_22_b200.roofline import prefill_bytes, prefill_flops
+from kimi_delta_attention_22_b200.roofline import backward_bytes, backward_flops, prefill_bytes, prefill_flops
 
 METRIC = "KDA prefill tokens/s (% bf16 TC peak); decode step HBM GB/s (% of peak)"
 WORKLOAD = "prefill_b4_h16_t2048"
@@ -420,6 +422,66 @@ def bench_workload(name, world, peaks, peak_kind, iters=5, warmup=2):
             "gpu_launches": 3 * iters + (1 if w.varlen else 0) * iters}
 
 
+def bench_chunk_backward(args, world, peaks, peak_kind):
+    """kda_chunk_bwd (the chunkwise gradients) on the prefill workload: 4 x 16 heads
+    x 2048 tokens, d = 128, chunk 64, per-channel gate; seeded N(0, 1) d_out and d_ST.
+    Three rotating input sets (each ~500 MB with its gradients) keep steps out of L2."""
+    import kimi_delta_attention_22_b200 as kda
+    from kimi_delta_attention_22_b200 import inputs
+
+    w = inputs.WORKLOADS[WORKLOAD]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream(dev)
+    sets = []
+    for i in range(3):
+        d = inputs.draw(w.B, w.T, w.H, w.d_k, w.d_v, dtype=w.torch_dtype, gate=w.gate, beta=w.beta,
+                        s0_std=w.s0_std, seed=w.seed + 200 + i, device=dev)
+        gen = torch.Generator(device=dev).manual_seed(300 + i)
+        d["d_out"] = torch.randn(w.B, w.T, w.H, w.d_v, device=dev, generator=gen).to(w.torch_dtype)
+        d["d_ST"] = torch.randn(w.B, w.H, w.d_v, w.d_k, device=dev, generator=gen)
+        sets.append(d)
+    sh = kda.Shape(w.B, w.T, w.H, w.d_k, w.d_v, w.B, kda.KDA_BF16, kda.KDA_GATE_CHANNEL, w.chunk, None, 0)
+    ws = torch.empty(kda.load_library().kda_chunk_bwd_workspace_size(ctypes.byref(sh), 0),
+                     dtype=torch.uint8, device=dev)
+
+    def step(i):
+        s = sets[i % 3]
+        return kda.kda_chunk_bwd(s["q"], s["k"], s["v"], s["g"], s["beta"], s["S0"], s["d_out"],
+                                 d_ST=s["d_ST"], chunk=w.chunk, workspace=ws)
+
+    for i in range(3):
+        step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    iters = 6
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(iters):
+        step(i)
+    b.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(a.elapsed_time(b), world) / iters
+    del sets, ws
+    torch.cuda.empty_cache()
+    nbytes, flops = backward_bytes(w), backward_flops(w)
+    gbs, tf = nbytes / (ms * 1e-3) / 1e9, flops / (ms * 1e-3) / 1e12
+    return {"metric": "KDA chunkwise backward tokens/s", "value": world * w.tokens / (ms * 1e-3),
+            "unit": "tokens/s", "ms_per_call": ms, "iters": iters,
+            "config": {"workload": WORKLOAD, "B": w.B, "T": w.T, "H": w.H, "d_k": w.d_k, "d_v": w.d_v,
+                       "chunk": w.chunk, "gate": w.gate, "dtype": "bf16 inputs, fp32 gradients",
+                       "l2": "3 rotating input sets > 126 MB L2"},
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"], "peak_source": f"{peak_kind} hbm_gbs",
+                         "algorithmic_bytes_per_launch": nbytes, "traffic": None,
+                         "kernel": "kda_chunk_bwd call (WY, forward scan with checkpoints, reverse "
+                                   "state scan, solve and dq/dk kernels)"},
+            "tensor": {"achieved_tflops": tf, "flops_per_launch": flops, "peak_tflops": peaks["bf16_tflops"],
+                       "frac": tf / peaks["bf16_tflops"], "peak_source": f"{peak_kind} bf16_tflops (burst)"},
+            "kernels": "kda_chunk_wy_kernel, kda_chunk_scan_kernel, kda_chunk_bwd_scan_kernel, "
+                       "kda_chunk_bwd_solve_kernel, kda_chunk_bwd_dqk_kernel"}
+
+
 def bench_backward(args, world):
     """kda_recurrent_bwd (gradients of the token loop) on the short-run shape:
     256 sequences x 32 heads x 16 tokens, d = 128, bf16 inputs, per-channel gate."""
@@ -523,6 +585,7 @@ def run_ours(args, world, rank, local):
         big["sweep"] = [bench_workload(f"sweep_b8_h64_t8192_{g}_beta{b}", world, peaks, peak_kind)
                         for g in ("none", "scalar", "channel_strong") for b in ("one", "sigmoid")]
     dec = bench_decode(args, world, rank, peaks, peak_kind)
+    cbwd = bench_chunk_backward(args, world, peaks, peak_kind)
     bwd = bench_backward(args, world)
     clk = clocks.stop()
     w = pre["w"]
@@ -550,7 +613,7 @@ def run_ours(args, world, rank, local):
                            "l2": "3 rotating input sets (~630 MB) > 126 MB L2"},
                 "roofline": pre["roofline"], "tensor": pre["tensor"], "cpu_baseline": cpu,
                 "e2e": pre["e2e"], "no_workspace": pre["no_workspace"], **big,
-                "decode": dec, "backward": bwd, "clocks": clk,
+                "decode": dec, "backward": cbwd, "backward_recurrent": bwd, "clocks": clk,
                 # per step: the WY kernel, the (empty when every chunk takes one reference)
                 # sub-block WY kernel and the state scan
                 "gpu_launches": 3 * args.steps,

@@ -38,3 +38,31 @@ def recurrent_bytes(N: int, T: int, H: int, d_k: int, d_v: int, el: int = 2, gat
     g = {"channel": 4 * d_k, "scalar": 4, "none": 0}[gate]
     per_ht = el * (2 * d_k + 2 * d_v) + g + 4
     return 2 * N * H * d_v * d_k * 4 + N * T * H * per_ht
+
+
+def backward_bytes(w) -> int:
+    """Algorithmic HBM bytes of one kda_chunk_bwd call: every input read once
+    (q, k, v, d_out at the input element size, g, beta, S0 and d_ST) and every
+    gradient written once in fp32 (dq, dk per query/key head; dv, dg, dbeta per
+    value head; dS0 per sequence and head)."""
+    ht = w.B * w.T * w.H
+    Hk = getattr(w, "Hk", w.H)
+    el = 2 if w.dtype == "bf16" else 4
+    g = {"channel": 4 * w.d_k, "scalar": 4, "none": 0}[w.gate_mode]
+    per_ht = 2 * el * w.d_v + 2 * g + 4 + 4 + 4 * w.d_v          # v, d_out, g + dg, beta + dbeta, dv
+    qk = w.B * w.T * Hk * 2 * w.d_k * (el + 4)                    # q, k and dq, dk
+    seqs = w.num_seqs if w.varlen else w.B
+    states = seqs * w.H * w.d_v * w.d_k * 4 * ((1 if w.s0_std is not None else 0) + 2)
+    return ht * per_ht + qk + states
+
+
+def backward_flops(w) -> float:
+    """The forward recomputed (prefill_flops), then per head-token at chunk C:
+    the reverse state scan 6*d_k*d_v + C*d_v (dE = Kd dS'^T + lower(Qp)^T dO and
+    dS <- dS Diag + dO^T Qg - dE^T W); the solve half 2*d_k*d_v + 3*C*d_v + C*d_k
+    (the residual product, E, dEbar and dL over their causal halves, the key Gram);
+    the dq/dk half 6*d_k*d_v + C*d_v + 4*C*d_k (dKd, dQg, dKg, dAqk and the two
+    decay-weighted Grams' gradients)."""
+    C, dk, dv = w.chunk, w.d_k, w.d_v
+    per_ht = 14 * dk * dv + 5 * C * dv + 5 * C * dk
+    return prefill_flops(w) + w.B * w.T * w.H * per_ht
