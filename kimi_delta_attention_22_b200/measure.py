@@ -3,6 +3,7 @@
     python -m kimi_delta_attention_22_b200.measure [--workloads a,b,...] [--schedule workspace|pool]
                                                    [--iters 10] [--warmup 3] [--shape B,T,H]
     python -m kimi_delta_attention_22_b200.measure --recurrent [--tokens 1,4,16,64]
+    python -m kimi_delta_attention_22_b200.measure --chunk-backward workload[,workload...]
 
 For each workload: inputs drawn once on the device (kimi_delta_attention_22_b200.inputs),
 the prefill's workspace allocated once (--schedule pool: none, so each call takes its
@@ -32,7 +33,8 @@ import torch
 
 import kimi_delta_attention_22_b200 as kda
 from kimi_delta_attention_22_b200 import inputs
-from kimi_delta_attention_22_b200.roofline import prefill_bytes, prefill_flops, recurrent_bytes
+from kimi_delta_attention_22_b200.roofline import (backward_bytes, backward_flops, prefill_bytes, prefill_flops,
+                                                   recurrent_bytes)
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -174,6 +176,44 @@ def measure_backward(N: int, T: int, H: int, iters: int, warmup: int) -> dict:
     return res
 
 
+def measure_chunk_backward(name: str, iters: int, warmup: int) -> dict:
+    """kda_chunk_bwd on a named workload (seeded N(0, 1) d_out and d_ST, the workspace
+    allocated once), next to kda_chunk_fwd on the same inputs."""
+    w = inputs.WORKLOADS[name]
+    d = inputs.workload_inputs(w, device="cuda")
+    gen = torch.Generator(device="cuda").manual_seed(w.seed + 1000)
+    nseq = w.num_seqs if w.varlen else w.B
+    d_out = torch.randn(w.B, w.T, w.H, w.d_v, device="cuda", generator=gen).to(w.torch_dtype)
+    d_ST = torch.randn(nseq, w.H, w.d_v, w.d_k, device="cuda", generator=gen)
+    cu = d["cu_seqlens"]
+    gate = {"channel": kda.KDA_GATE_CHANNEL, "scalar": kda.KDA_GATE_SCALAR, "none": kda.KDA_GATE_NONE}[w.gate_mode]
+    sh = kda.Shape(w.B, w.T, w.H, w.d_k, w.d_v, nseq, kda.KDA_BF16, gate, w.chunk, None, w.qk_heads)
+    ws = torch.empty(kda.load_library().kda_chunk_bwd_workspace_size(ctypes.byref(sh), int(cu is not None)),
+                     dtype=torch.uint8, device="cuda")
+
+    def bwd():
+        kda.kda_chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], d_out, d_ST=d_ST, cu_seqlens=cu,
+                          chunk=w.chunk, workspace=ws)
+
+    def fwd():
+        kda.kda_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], S0=d["S0"], cu_seqlens=cu, chunk=w.chunk)
+
+    ms = _time(bwd, iters, warmup)
+    ms_f = _time(fwd, iters, warmup)
+    nbytes, flops = backward_bytes(w), backward_flops(w)
+    res = {"kernel": "kda_chunk_bwd", "workload": name, "ms_per_call": ms, "tokens_per_s": w.tokens / (ms * 1e-3),
+           "hbm_gbs": nbytes / (ms * 1e-3) / 1e9, "tflops": flops / (ms * 1e-3) / 1e12,
+           "algorithmic_bytes": nbytes, "flops": flops, "forward_ms": ms_f,
+           "backward_over_forward": ms / ms_f, "iters": iters}
+    pk = peaks()
+    if pk:
+        res["hbm_frac"] = res["hbm_gbs"] / pk["hbm_gbs"]
+        res["tc_frac"] = res["tflops"] / pk["bf16_tflops"]
+    del d, d_out, d_ST, ws
+    torch.cuda.empty_cache()
+    return res
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--workloads", default=",".join(n for n in inputs.WORKLOADS))
@@ -185,10 +225,16 @@ def main():
     ap.add_argument("--tokens", default="1,4,16,64")
     ap.add_argument("--backward", default=None,
                     help="N,T,H[;N,T,H...]: time kda_recurrent_bwd on these shapes")
+    ap.add_argument("--chunk-backward", default=None,
+                    help="workload[,workload...]: time kda_chunk_bwd (bf16, d = 128 workloads)")
     args = ap.parse_args()
     if not torch.cuda.is_available():
         raise SystemExit("measure needs a CUDA device")
     kda.load_library()
+    if args.chunk_backward:
+        for name in args.chunk_backward.split(","):
+            print(json.dumps(measure_chunk_backward(name, args.iters, args.warmup)), flush=True)
+        return
     if args.backward:
         for spec in args.backward.split(";"):
             N, T, H = (int(x) for x in spec.split(","))
