@@ -36,12 +36,13 @@
 // operands are single fp16 (float64 emulation of the chunk: each adds < 5e-4).
 // The decay-weighted Gram products stay on CUDA cores in fp32, because their
 // factors span far more than fp16's range: the factor e^{Gamma_ic - Gamma_jc} is
-// split over 16-token sub-blocks I (of i) and J (of j), r(I) the first row of I:
-//   a_ic = 2^{G_ic - G_r(I)c} <= 1,  b_jc = 2^{G_r(J)c - G_jc} (its own sub-block only),
+// split over 16-token sub-blocks I (of i) and J (of j), with the reference row
+// r(I) = 16 I + 7 (the forward's sub-block reference):
+//   a_ic = 2^{G_ic - G_r(I)c},  b_jc = 2^{G_r(J)c - G_jc} (each within its own sub-block),
 //   d^{IJ}_c = 2^{G_r(I)c - G_r(J)c} <= 1 (J < I),   (G = Gamma in log2 units)
 // so every Gram product and its gradient becomes a plain product of row-scaled
-// operands with a per-column factor per sub-block pair; b stays bounded by the decay
-// of 15 tokens.
+// operands with a per-column factor per sub-block pair; a and b span at most 8
+// tokens of decay, which fp32 holds while a token's |g| < 10.9 per channel.
 #include <cuda_bf16.h>
 
 #include "kda_chunk_bwd.cuh"
@@ -54,7 +55,9 @@ namespace {
 using namespace tc;
 using namespace sm100;
 
-constexpr int C = rec::C, DK = rec::DK, DV = rec::DV, NT = 256;
+constexpr int C = rec::C, DK = rec::DK, DV = rec::DV;
+constexpr int NT = 256;    // solve kernel: threads per CTA
+constexpr int NT2 = 512;   // dq/dk kernel: threads per CTA (16 warps, at most 128 registers each)
 constexpr int LD = 132;          // fp32 row stride of [64][128] tiles
 constexpr int LT = 68;           // fp32 row stride of [64][64] tiles
 constexpr uint64_t kWaitNs = 1000000000ull;   // 1 s bound on every wait
@@ -100,11 +103,11 @@ constexpr int AQK = OPS + 101376;  // fp32 [64][LT] dAqk (lower, diagonal includ
 constexpr int DA = AQK + 17408;    // fp32 [64][LT] dA (strictly lower)
 constexpr int AQT = DA + 17408;    // fp32 [64][LT] dAqk^T
 constexpr int DAT = AQT + 17408;   // fp32 [64][LT] dA^T
-constexpr int SRED = AQT;          // fp32 [16][64] scalar-gate row sums (after the Gram loops)
+constexpr int SRED = AQT;          // fp32 [32][64] scalar-gate row sums (after the Gram loops)
 constexpr int DFAC = DAT + 17408;  // fp32 [6][128]
 constexpr int UCOL = DFAC + 3072;  // fp32 [4][128] colsum(dKd . Kd) partials
-constexpr int SGS = UCOL + 2048;   // fp32 [8][128] colsum(S . dS') partials
-constexpr int BAR = SGS + 4096;    // 5 mbarriers, TMEM base
+constexpr int SGS = UCOL + 2048;   // fp32 [16][128] colsum(S . dS') partials (one row per warp)
+constexpr int BAR = SGS + 8192;    // 5 mbarriers, TMEM base
 constexpr int BYTES = BAR + 64 + 1024;
 static_assert(OPS % 1024 == 0, "swizzled tiles need 1024-byte alignment");
 static_assert(PR16 + 8192 - OPS <= 101376 && 3 * 64 * LD * 4 <= 101376, "operands and partials fit the union");
@@ -134,6 +137,7 @@ struct GradParams {
     float* dbeta;
     int32_t* dev_status;
     int T, H, num_seqs, nc, group;
+    int ahead;            // L2 prefetch distance in CTAs (one wave: CTAs start in linear order)
     float scale;
 };
 
@@ -157,18 +161,56 @@ __device__ __forceinline__ bool slot_rows(const GradParams& p, int slot, long lo
     return L > 0;
 }
 
+// L2 prefetch of the inputs of the job p.ahead CTAs later, which starts about when
+// this one ends (one CTA per SM, CTAs start in linear order): one bulk prefetch per
+// token row of g, k and v (solve) or g, k, q and d_out (dq/dk), one per workspace tile.
+// Issued in a compute phase, so that a wave's loads do not all queue at its start.
+template <int GATE, bool DQK>
+__device__ __forceinline__ void prefetch_next(const GradParams& p) {
+    const long long job = (long long)blockIdx.x + p.ahead;
+    if (job >= (long long)gridDim.x) return;
+    const int slot = (int)(job / p.H), h = (int)(job % p.H), hk = h / p.group, Hk = p.H / p.group;
+    long long c0;
+    int L;
+    if (!slot_rows(p, slot, c0, L)) return;
+    const size_t sh = (size_t)slot * p.H + h;
+    const int t = threadIdx.x;
+    if (t < L) {
+        const long long row = c0 + t;
+        if (GATE == KDA_GATE_CHANNEL) bulk_prefetch_l2(p.g + (row * p.H + h) * DK, DK * 4);
+        bulk_prefetch_l2(p.k + (row * Hk + hk) * DK, DK * 2);
+        if (DQK) {
+            bulk_prefetch_l2(p.q + (row * Hk + hk) * DK, DK * 2);
+            bulk_prefetch_l2(p.d_out + (row * p.H + h) * DV, DV * 2);
+        } else {
+            bulk_prefetch_l2(p.v + (row * p.H + h) * DV, DV * 2);
+        }
+    } else if (t == C) {
+        bulk_prefetch_l2(p.chk + sh * DV * DK, DV * DK * 4);
+    } else if (t == C + 1) {
+        if (DQK) bulk_prefetch_l2(p.dsp + sh * DV * DK, DV * DK * 4);
+        else bulk_prefetch_l2(p.de + sh * C * DV, C * DV * 4);
+    } else if (DQK && t == C + 2) {
+        bulk_prefetch_l2(p.e16 + sh * 2 * kTile16, 2 * kTile16);
+    } else if (DQK && t == C + 3) {
+        bulk_prefetch_l2(p.pr16 + sh * kTile16, kTile16);
+        bulk_prefetch_l2(p.da + sh * C * C, C * C * 4);
+    }
+}
+
 __device__ __forceinline__ int pair_index(int I, int J) { return I * (I - 1) / 2 + J; }   // J < I
 
 // G = cumulative log2 decay of the chunk (rows past L carry no decay).  The raw g
 // tile goes into sG with every load in flight at once; the column prefix sums then
-// run in shared memory, two threads per channel (rows 0-31 and 32-63).  Every thread
-// of the CTA calls this; the caller synchronises before reading sG.
-template <int GATE>
+// run in shared memory, NTH / 128 threads per channel over consecutive row ranges,
+// each range then offset by the totals of the ranges before it.  Every thread of the
+// CTA (NTH of them) calls this; the caller synchronises before reading sG.
+template <int GATE, int NTH>
 __device__ __forceinline__ void load_gamma(const GradParams& p, long long c0, int L, int h, float* sG) {
     const int tid = threadIdx.x;
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-        const int x = tid + NT * r, i = x >> 5, c4 = x & 31;
+    for (int r = 0; r < C * 32 / NTH; ++r) {
+        const int x = tid + NTH * r, i = x >> 5, c4 = x & 31;
         float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
         if (i < L) {
             if (GATE == KDA_GATE_CHANNEL) {
@@ -181,27 +223,31 @@ __device__ __forceinline__ void load_gamma(const GradParams& p, long long c0, in
         *reinterpret_cast<float4*>(sG + i * LD + 4 * c4) = f;
     }
     __syncthreads();
-    const int c = tid & (DK - 1), half = tid >> 7;
+    constexpr int PARTS = NTH / DK, RP = C / PARTS;
+    const int c = tid & (DK - 1), part = tid >> 7;
     float acc = 0.f;
 #pragma unroll 8
-    for (int i = 32 * half; i < 32 * half + 32; ++i) {
+    for (int i = RP * part; i < RP * part + RP; ++i) {
         acc = fmaf(sG[i * LD + c], kLog2e, acc);
         sG[i * LD + c] = acc;
     }
     __syncthreads();
-    if (half == 1) {
-        const float base = sG[31 * LD + c];
+    float carry = 0.f;
+    for (int q = 0; q < part; ++q) carry += sG[(RP * q + RP - 1) * LD + c];
+    __syncthreads();
+    if (part > 0) {
 #pragma unroll 8
-        for (int i = 32; i < C; ++i) sG[i * LD + c] += base;
+        for (int i = RP * part; i < RP * part + RP; ++i) sG[i * LD + c] += carry;
     }
 }
 
-// d^{IJ}_c for the six sub-block pairs J < I.
+// d^{IJ}_c for the six sub-block pairs J < I (NTH threads).
+template <int NTH>
 __device__ __forceinline__ void load_dfac(const float* sG, float* dfac) {
-    for (int x = threadIdx.x; x < 6 * DK; x += NT) {
+    for (int x = threadIdx.x; x < 6 * DK; x += NTH) {
         const int pi = x / DK, c = x % DK;
         const int I = pi < 1 ? 1 : (pi < 3 ? 2 : 3), J = pi - I * (I - 1) / 2;
-        dfac[x] = ex2(sG[16 * I * LD + c] - sG[16 * J * LD + c]);
+        dfac[x] = ex2(sG[(16 * I + 7) * LD + c] - sG[(16 * J + 7) * LD + c]);
     }
 }
 
@@ -311,7 +357,7 @@ __device__ __forceinline__ bool solve_body(const GradParams& p, uint8_t* sm, uin
     float* Kb = reinterpret_cast<float*>(sm + KB);
     const int Hk = p.H / p.group;
 
-    load_gamma<GATE>(p, c0, L, h, sG);
+    load_gamma<GATE, NT>(p, c0, L, h, sG);
     if (tid < C) sb[tid] = tid < L ? p.beta[(c0 + tid) * p.H + h] : 0.f;
     // this thread's K: row i = x & 63, 8-channel chunk x >> 6, for x = tid + 256 r
     float kr[4][8];
@@ -321,12 +367,12 @@ __device__ __forceinline__ bool solve_body(const GradParams& p, uint8_t* sm, uin
         loadn<8>(p.k + ((c0 + i) * Hk + hk) * DK + 8 * cc, i < L, kr[r]);
     }
     __syncthreads();
-    load_dfac(sG, dfac);
+    load_dfac<NT>(sG, dfac);
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
         const int x = tid + NT * r, i = x & 63, cc = x >> 6;
         const float* Gi = sG + i * LD + 8 * cc;
-        const float* Gr = sG + (i & ~15) * LD + 8 * cc;
+        const float* Gr = sG + ((i & ~15) + 7) * LD + 8 * cc;
         float ka[8], kb[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -408,7 +454,9 @@ __device__ __forceinline__ bool solve_body(const GradParams& p, uint8_t* sm, uin
                      idesc_f16(64, 128, false, false), s > 0);
         mma_commit(bars + 0);
     }
-    // meanwhile on the CUDA cores: T, and its two-term fp16 image
+    // meanwhile on the CUDA cores: T, and its two-term fp16 image; the next wave's
+    // inputs go to L2 while this CTA computes rather than while it loads
+    prefetch_next<GATE, false>(p);
     invert_unit_lower(sA, sb, sT, reinterpret_cast<float*>(sm + PS));
     for (int x = tid; x < C * 8; x += NT) {
         const int i = x >> 3, jc = x & 7;
@@ -613,7 +661,7 @@ template <int GATE>
 __device__ __forceinline__ bool dqk_body(const GradParams& p, uint8_t* sm, uint32_t tm, uint64_t* bars,
                                          long long c0, int L, int h, int hk, size_t sh, int& fetched) {
     using namespace s2;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, sp = warp & 3, hc = warp >> 2;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, sp = warp & 3, qt = warp >> 2;
     const uint32_t sbase = smem_u32(sm), lane_base = (uint32_t)(32 * sp) << 16;
     float* sG = reinterpret_cast<float*>(sm + G);
     float* sAqk = reinterpret_cast<float*>(sm + AQK);
@@ -646,9 +694,8 @@ __device__ __forceinline__ bool dqk_body(const GradParams& p, uint8_t* sm, uint3
     // channel) of half hv; colsum(S . dS') partials of this thread's channels
     float sgs_acc[8] = {};
     auto build = [&](int hv) {
-#pragma unroll
-        for (int x = tid; x < C * 8; x += NT) {
-            const int i = x >> 3, vc = x & 7;
+        {
+            const int i = tid >> 3, vc = tid & 7;   // 64 rows x 8 chunks of 8 values
             float f[8];
             loadn<8>(p.d_out + ((c0 + i) * p.H + h) * DV + 64 * hv + 8 * vc, i < L, f);
             st_shared_v4(sm + DO16, kmaj_off(i, 8 * vc, 64), pack8_f16(f));
@@ -657,8 +704,8 @@ __device__ __forceinline__ bool dqk_body(const GradParams& p, uint8_t* sm, uint3
         const float* dS = p.dsp + sh * DV * DK;
         const int cc = tid & 15;
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            const int vl = (tid >> 4) + 16 * r, v = 64 * hv + vl;
+        for (int r = 0; r < 2; ++r) {
+            const int vl = (tid >> 4) + 32 * r, v = 64 * hv + vl;
             float s8[8], d8[8];
             ld8g(S + (size_t)v * DK + 8 * cc, s8);
             ld8g(dS + (size_t)v * DK + 8 * cc, d8);
@@ -700,12 +747,12 @@ __device__ __forceinline__ bool dqk_body(const GradParams& p, uint8_t* sm, uint3
     };
 
     fetch(0, bars + 0);
-    load_gamma<GATE>(p, c0, L, h, sG);
+    load_gamma<GATE, NT2>(p, c0, L, h, sG);
     build(0);
     {
         const float4* a4 = reinterpret_cast<const float4*>(p.da + sh * C * C);
 #pragma unroll
-        for (int x = tid; x < C * C / 4; x += NT) *reinterpret_cast<float4*>(sDA + (x >> 4) * LT + 4 * (x & 15)) = a4[x];
+        for (int x = tid; x < C * C / 4; x += NT2) *reinterpret_cast<float4*>(sDA + (x >> 4) * LT + 4 * (x & 15)) = a4[x];
     }
     if (!__syncthreads_and(mbar_wait(bars + 0, 0, kWaitNs))) return false;
     operands_ready();
@@ -713,7 +760,7 @@ __device__ __forceinline__ bool dqk_body(const GradParams& p, uint8_t* sm, uint3
         issue(0);
         mma_commit(bars + 1);
     }
-    load_dfac(sG, dfac);
+    load_dfac<NT2>(sG, dfac);
     if (!wait_mma(bars + 1)) return false;
     fetch(1, bars + 2);
     build(1);
@@ -735,23 +782,23 @@ __device__ __forceinline__ bool dqk_body(const GradParams& p, uint8_t* sm, uint3
     if (!wait_mma(bars + 3)) return false;
     tc_fence_after();
 
-    // ---- per element (row i = 16 sp + lane, channels 64 hc ..): dK, dQ, dGamma so far,
-    // colsum(dKd . Kd) partials, and dAqk (and its transpose)
+    // ---- per element (row i = 16 sp + lane, channels 32 qt .. +31 in four steps of 8):
+    // dK, dQ, dGamma so far, colsum(dKd . Kd) partials, and dAqk (and its transpose)
     {
         const int i = 16 * sp + (lane & 15);
         const bool own = lane < 16;
 #pragma unroll 1
-        for (int q = 0; q < 2; ++q) {
-            const int cb = 64 * hc + 32 * q;
-            float xk[32], xq[32], xg[32];
-            tmem_ld32(tm + lane_base + TM_KD + cb, xk);
-            tmem_ld32(tm + lane_base + TM_QG + cb, xq);
-            tmem_ld32(tm + lane_base + TM_KG + cb, xg);
-            float kx[32], qx[32];
-            loadn<32>(p.k + ((c0 + i) * Hk + hk) * DK + cb, own && i < L, kx);
-            loadn<32>(p.q + ((c0 + i) * Hk + hk) * DK + cb, own && i < L, qx);
+        for (int q = 0; q < 4; ++q) {
+            const int cb = 32 * qt + 8 * q;
+            float xk[8], xq[8], xg[8];
+            tmem_ld8(tm + lane_base + TM_KD + cb, xk);
+            tmem_ld8(tm + lane_base + TM_QG + cb, xq);
+            tmem_ld8(tm + lane_base + TM_KG + cb, xg);
+            float kx[8], qx[8];
+            loadn<8>(p.k + ((c0 + i) * Hk + hk) * DK + cb, own && i < L, kx);
+            loadn<8>(p.q + ((c0 + i) * Hk + hk) * DK + cb, own && i < L, qx);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
+            for (int e = 0; e < 8; ++e) {
                 const int c = cb + e;
                 const float Gv = sG[i * LD + c], gam = sG[(C - 1) * LD + c];
                 const float eG = ex2(Gv), eD = ex2(gam - Gv);
@@ -769,47 +816,49 @@ __device__ __forceinline__ bool dqk_body(const GradParams& p, uint8_t* sm, uint3
             }
             if (own) {
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
+                for (int u = 0; u < 2; ++u) {
                     st4(Pk + i * LD + cb + 4 * u, xk[4 * u], xk[4 * u + 1], xk[4 * u + 2], xk[4 * u + 3]);
                     st4(Pq + i * LD + cb + 4 * u, xq[4 * u], xq[4 * u + 1], xq[4 * u + 2], xq[4 * u + 3]);
                     st4(Pg + i * LD + cb + 4 * u, xg[4 * u], xg[4 * u + 1], xg[4 * u + 2], xg[4 * u + 3]);
                 }
             }
         }
-        float z[32];
-        tmem_ld32(tm + lane_base + TM_AQ + 32 * hc, z);
+        float z[16];
+        tmem_ld16(tm + lane_base + TM_AQ + 16 * qt, z);
         if (own) {
 #pragma unroll
-            for (int t = 0; t < 32; ++t) {
-                const int j = 32 * hc + t;
+            for (int t = 0; t < 16; ++t) {
+                const int j = 16 * qt + t;
                 const float x = j <= i ? z[t] : 0.f;
                 sAqk[i * LT + j] = x;
                 dAT[j * LT + i] = x;
             }
         }
     }
-    for (int x = tid; x < C * C; x += NT) {
+    for (int x = tid; x < C * C; x += NT2) {
         const int i = x & 63, j = x >> 6;
         dDT[j * LT + i] = sDA[i * LT + j];
     }
     __syncthreads();
 
-    // ---- from here on: thread rows i = 4 ig .. +3, channels c = 8 cg .. +7
+    prefetch_next<GATE, true>(p);   // the next wave's inputs, while this CTA computes
+    // ---- from here on: thread rows i = 4 ig .. +3, channels c = 4 cg .. +3
     const int cg = tid >> 4, ig = tid & 15, I = ig >> 2;
-    float xk[4][8], xq[4][8], xg[4][8], dgam[8];
+    float xk[4][4], xq[4][4], xg[4][4], dgam[4];
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
         const int i = 4 * ig + r;
-        ld8(Pk + i * LD + 8 * cg, xk[r]);
-        ld8(Pq + i * LD + 8 * cg, xq[r]);
-        ld8(Pg + i * LD + 8 * cg, xg[r]);
+        const float4 a = ld4(Pk + i * LD + 4 * cg), b = ld4(Pq + i * LD + 4 * cg), c = ld4(Pg + i * LD + 4 * cg);
+        xk[r][0] = a.x; xk[r][1] = a.y; xk[r][2] = a.z; xk[r][3] = a.w;
+        xq[r][0] = b.x; xq[r][1] = b.y; xq[r][2] = b.z; xq[r][3] = b.w;
+        xg[r][0] = c.x; xg[r][1] = c.y; xg[r][2] = c.z; xg[r][3] = c.w;
     }
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        const int cc = 8 * cg + c;
+    for (int c = 0; c < 4; ++c) {
+        const int cc = 4 * cg + c;
         float s = 0.f;
 #pragma unroll
-        for (int w = 0; w < 8; ++w) s += sgs[w * DK + cc];
+        for (int w = 0; w < NT2 / 32; ++w) s += sgs[w * DK + cc];
         dgam[c] = s * ex2(sG[(C - 1) * LD + cc]) + ((ucol[cc] + ucol[DK + cc]) + (ucol[2 * DK + cc] + ucol[3 * DK + cc]));
     }
     __syncthreads();   // the partials are in registers; their region takes K a, Q~ a, K b
@@ -817,13 +866,13 @@ __device__ __forceinline__ bool dqk_body(const GradParams& p, uint8_t* sm, uint3
     float* Qa = Ka + 64 * LD;
     float* Kb = Qa + 64 * LD;
 #pragma unroll
-    for (int x = tid; x < C * 16; x += NT) {
+    for (int x = tid; x < C * 16; x += NT2) {
         const int i = x >> 4, cc = x & 15;
         float kx[8], qx[8];
         loadn<8>(p.k + ((c0 + i) * Hk + hk) * DK + 8 * cc, i < L, kx);
         loadn<8>(p.q + ((c0 + i) * Hk + hk) * DK + 8 * cc, i < L, qx);
         const float* Gi = sG + i * LD + 8 * cc;
-        const float* Gr = sG + (i & ~15) * LD + 8 * cc;
+        const float* Gr = sG + ((i & ~15) + 7) * LD + 8 * cc;
         float ka[8], qa[8], kb[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -847,22 +896,20 @@ __device__ __forceinline__ bool dqk_body(const GradParams& p, uint8_t* sm, uint3
     // ---- the Gram gradients, i side: dP1 = a . sum_J d^{IJ} (dAqk_{I,J} K b_J), dP2 likewise
     // with dA; dQ += dP1, dK += dP2, dGamma += Q~ . dP1 + K . dP2
     {
-        float x1[4][8] = {}, x2[4][8] = {};
+        float x1[4][4] = {}, x2[4][4] = {};
         for (int J = 0; J <= I; ++J) {
-            float dv[8];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) dv[c] = J < I ? dfac[pair_index(I, J) * DK + 8 * cg + c] : 1.f;
-#pragma unroll 2
+            float4 dv = make_float4(1.f, 1.f, 1.f, 1.f);
+            if (J < I) dv = ld4(dfac + pair_index(I, J) * DK + 4 * cg);
+#pragma unroll 4
             for (int j = 16 * J; j < 16 * J + 16; ++j) {
                 const float4 aq = ld4(dAT + j * LT + 4 * ig), ad = ld4(dDT + j * LT + 4 * ig);
-                const float4 b0 = ld4(Kb + j * LD + 8 * cg), b1 = ld4(Kb + j * LD + 8 * cg + 4);
-                const float kb[8] = {b0.x * dv[0], b0.y * dv[1], b0.z * dv[2], b0.w * dv[3],
-                                     b1.x * dv[4], b1.y * dv[5], b1.z * dv[6], b1.w * dv[7]};
+                const float4 b0 = ld4(Kb + j * LD + 4 * cg);
+                const float kb[4] = {b0.x * dv.x, b0.y * dv.y, b0.z * dv.z, b0.w * dv.w};
 #pragma unroll
                 for (int r = 0; r < 4; ++r) {
                     const float q1 = comp(aq, r), q2 = comp(ad, r);
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
+                    for (int c = 0; c < 4; ++c) {
                         x1[r][c] = fmaf(q1, kb[c], x1[r][c]);
                         x2[r][c] = fmaf(q2, kb[c], x2[r][c]);
                     }
@@ -873,9 +920,9 @@ __device__ __forceinline__ bool dqk_body(const GradParams& p, uint8_t* sm, uint3
         for (int r = 0; r < 4; ++r) {
             const int i = 4 * ig + r;
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const int cc = 8 * cg + c;
-                const float a = ex2(sG[i * LD + cc] - sG[16 * I * LD + cc]);
+            for (int c = 0; c < 4; ++c) {
+                const int cc = 4 * cg + c;
+                const float a = ex2(sG[i * LD + cc] - sG[(16 * I + 7) * LD + cc]);
                 xq[r][c] = fmaf(a, x1[r][c], xq[r][c]);
                 xk[r][c] = fmaf(a, x2[r][c], xk[r][c]);
                 xg[r][c] += Qa[i * LD + cc] * x1[r][c] + Ka[i * LD + cc] * x2[r][c];
@@ -885,25 +932,21 @@ __device__ __forceinline__ bool dqk_body(const GradParams& p, uint8_t* sm, uint3
     // ---- j side: Y = sum_{I' >= J} d^{I'J} (dAqk_{I',J}^T Q~a_I' + dA_{I',J}^T K a_I');
     // dK += b . Y, dGamma -= K b . Y   (this thread's rows are j, in sub-block J = I)
     {
-        float y[4][8] = {};
+        float y[4][4] = {};
         for (int Ip = I; Ip < 4; ++Ip) {
-            float dv[8];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) dv[c] = Ip > I ? dfac[pair_index(Ip, I) * DK + 8 * cg + c] : 1.f;
-#pragma unroll 2
+            float4 dv = make_float4(1.f, 1.f, 1.f, 1.f);
+            if (Ip > I) dv = ld4(dfac + pair_index(Ip, I) * DK + 4 * cg);
+#pragma unroll 4
             for (int i = 16 * Ip; i < 16 * Ip + 16; ++i) {
                 const float4 aq = ld4(sAqk + i * LT + 4 * ig), ad = ld4(sDA + i * LT + 4 * ig);
-                const float4 q0 = ld4(Qa + i * LD + 8 * cg), q1 = ld4(Qa + i * LD + 8 * cg + 4);
-                const float4 k0 = ld4(Ka + i * LD + 8 * cg), k1 = ld4(Ka + i * LD + 8 * cg + 4);
-                const float qa[8] = {q0.x * dv[0], q0.y * dv[1], q0.z * dv[2], q0.w * dv[3],
-                                     q1.x * dv[4], q1.y * dv[5], q1.z * dv[6], q1.w * dv[7]};
-                const float ka[8] = {k0.x * dv[0], k0.y * dv[1], k0.z * dv[2], k0.w * dv[3],
-                                     k1.x * dv[4], k1.y * dv[5], k1.z * dv[6], k1.w * dv[7]};
+                const float4 q0 = ld4(Qa + i * LD + 4 * cg), k0 = ld4(Ka + i * LD + 4 * cg);
+                const float qa[4] = {q0.x * dv.x, q0.y * dv.y, q0.z * dv.z, q0.w * dv.w};
+                const float ka[4] = {k0.x * dv.x, k0.y * dv.y, k0.z * dv.z, k0.w * dv.w};
 #pragma unroll
                 for (int r = 0; r < 4; ++r) {
                     const float w1 = comp(aq, r), w2 = comp(ad, r);
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) y[r][c] = fmaf(w1, qa[c], fmaf(w2, ka[c], y[r][c]));
+                    for (int c = 0; c < 4; ++c) y[r][c] = fmaf(w1, qa[c], fmaf(w2, ka[c], y[r][c]));
                 }
             }
         }
@@ -911,9 +954,9 @@ __device__ __forceinline__ bool dqk_body(const GradParams& p, uint8_t* sm, uint3
         for (int r = 0; r < 4; ++r) {
             const int j = 4 * ig + r;
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const int cc = 8 * cg + c;
-                const float b = ex2(sG[16 * I * LD + cc] - sG[j * LD + cc]);
+            for (int c = 0; c < 4; ++c) {
+                const int cc = 4 * cg + c;
+                const float b = ex2(sG[(16 * I + 7) * LD + cc] - sG[j * LD + cc]);
                 xk[r][c] = fmaf(b, y[r][c], xk[r][c]);
                 xg[r][c] -= Kb[j * LD + cc] * y[r][c];
             }
@@ -923,10 +966,10 @@ __device__ __forceinline__ bool dqk_body(const GradParams& p, uint8_t* sm, uint3
     // ---- dg = reverse cumulative sum of dGamma (gamma = Gamma of the last row)
     if (ig == 15) {
 #pragma unroll
-        for (int c = 0; c < 8; ++c) xg[3][c] += dgam[c];
+        for (int c = 0; c < 4; ++c) xg[3][c] += dgam[c];
     }
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
+    for (int c = 0; c < 4; ++c) {
         const float s3 = xg[3][c], s2 = xg[2][c] + s3, s1 = xg[1][c] + s2, s0 = xg[0][c] + s1;
         float incl = s0;
 #pragma unroll
@@ -948,29 +991,22 @@ __device__ __forceinline__ bool dqk_body(const GradParams& p, uint8_t* sm, uint3
         const int i = 4 * ig + r;
         if (i >= L) continue;
         const long long row = c0 + i;
-        float* dq = p.dq + (row * Hk + hk) * DK + 8 * cg;
-        float* dk = p.dk + (row * Hk + hk) * DK + 8 * cg;
+        float* dq = p.dq + (row * Hk + hk) * DK + 4 * cg;
+        float* dk = p.dk + (row * Hk + hk) * DK + 4 * cg;
         if (p.group == 1) {
             st4(dq, xq[r][0] * p.scale, xq[r][1] * p.scale, xq[r][2] * p.scale, xq[r][3] * p.scale);
-            st4(dq + 4, xq[r][4] * p.scale, xq[r][5] * p.scale, xq[r][6] * p.scale, xq[r][7] * p.scale);
             st4(dk, xk[r][0], xk[r][1], xk[r][2], xk[r][3]);
-            st4(dk + 4, xk[r][4], xk[r][5], xk[r][6], xk[r][7]);
         } else {
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
+            for (int c = 0; c < 4; ++c) {
                 atomicAdd(dq + c, xq[r][c] * p.scale);
                 atomicAdd(dk + c, xk[r][c]);
             }
         }
         if (GATE == KDA_GATE_CHANNEL) {
-            float* dg = p.dg + (row * p.H + h) * DK + 8 * cg;
-            st4(dg, xg[r][0], xg[r][1], xg[r][2], xg[r][3]);
-            st4(dg + 4, xg[r][4], xg[r][5], xg[r][6], xg[r][7]);
+            st4(p.dg + (row * p.H + h) * DK + 4 * cg, xg[r][0], xg[r][1], xg[r][2], xg[r][3]);
         } else if (GATE == KDA_GATE_SCALAR) {
-            float s = 0.f;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) s += xg[r][c];
-            sred[cg * C + i] = s;
+            sred[cg * C + i] = (xg[r][0] + xg[r][1]) + (xg[r][2] + xg[r][3]);
         }
     }
     if (GATE == KDA_GATE_SCALAR) {
@@ -978,7 +1014,7 @@ __device__ __forceinline__ bool dqk_body(const GradParams& p, uint8_t* sm, uint3
         if (tid < L) {
             float s = 0.f;
 #pragma unroll
-            for (int q = 0; q < 16; ++q) s += sred[q * C + tid];
+            for (int q = 0; q < NT2 / 16; ++q) s += sred[q * C + tid];
             p.dg[(c0 + tid) * p.H + h] = s;
         }
     }
@@ -986,7 +1022,7 @@ __device__ __forceinline__ bool dqk_body(const GradParams& p, uint8_t* sm, uint3
 }
 
 template <int GATE>
-__global__ void __launch_bounds__(NT, 1) kda_chunk_bwd_dqk_kernel(const __grid_constant__ GradParams p) {
+__global__ void __launch_bounds__(NT2, 1) kda_chunk_bwd_dqk_kernel(const __grid_constant__ GradParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -1037,7 +1073,7 @@ cudaError_t launch_grad_gate(const GradParams& p, unsigned grid, cudaStream_t st
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(kda_chunk_bwd_dqk_kernel<GATE>, cudaFuncAttributeMaxDynamicSharedMemorySize, s2::BYTES);
     if (e == cudaSuccess) e = launch_after(kda_chunk_bwd_solve_kernel<GATE>, dim3(grid), NT, s1::BYTES, st, p);
-    if (e == cudaSuccess) e = launch_after(kda_chunk_bwd_dqk_kernel<GATE>, dim3(grid), NT, s2::BYTES, st, p);
+    if (e == cudaSuccess) e = launch_after(kda_chunk_bwd_dqk_kernel<GATE>, dim3(grid), NT2, s2::BYTES, st, p);
     return e;
 }
 
@@ -1071,6 +1107,9 @@ cudaError_t launch_chunk_bwd_grad(const ChunkBwdArgs& a, uint8_t* ws, const BwdL
     p.nc = (a.T + C - 1) / C;
     p.group = a.H / a.Hk;
     p.scale = a.scale;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) (void)cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    p.ahead = sms;
     const long long grid = bl.fwd.slots * a.H;
     if (grid <= 0) return cudaSuccess;
     switch (a.gate) {
