@@ -842,16 +842,41 @@ __device__ __forceinline__ bool dqk_body(const GradParams& p, uint8_t* sm, uint3
     __syncthreads();
 
     prefetch_next<GATE, true>(p);   // the next wave's inputs, while this CTA computes
-    // ---- from here on: thread rows i = 4 ig .. +3, channels c = 4 cg .. +3
-    const int cg = tid >> 4, ig = tid & 15, I = ig >> 2;
-    float xk[4][4], xq[4][4], xg[4][4], dgam[4];
+    // ---- from here on: thread rows i = 4 ig .. +3, channels c = 4 cg .. +3, with the
+    // rows of one warp in one 16-row sub-block I (warp / 4), so that the block-triangular
+    // Gram loops below take the same trip count on every lane (5 sub-blocks per warp).
+    // The thread's 48 partial sums (dK, dQ, dGamma) wait in its own tensor-memory lane
+    // (columns 48 (warp / 4) ..; the products are read out, so the columns are free)
+    // while the Gram loops run, which keeps those loops within the 128-register budget.
+    const int I = warp >> 2, ig = 4 * I + (lane >> 3), cg = 8 * (warp & 3) + (lane & 7);
+    const uint32_t stash = tm + lane_base + 48u * (uint32_t)qt;
+    auto put16 = [&](uint32_t col, const float (&x)[4][4]) {
+        uint32_t r[16];
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-        const int i = 4 * ig + r;
-        const float4 a = ld4(Pk + i * LD + 4 * cg), b = ld4(Pq + i * LD + 4 * cg), c = ld4(Pg + i * LD + 4 * cg);
-        xk[r][0] = a.x; xk[r][1] = a.y; xk[r][2] = a.z; xk[r][3] = a.w;
-        xq[r][0] = b.x; xq[r][1] = b.y; xq[r][2] = b.z; xq[r][3] = b.w;
-        xg[r][0] = c.x; xg[r][1] = c.y; xg[r][2] = c.z; xg[r][3] = c.w;
+        for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(x[e >> 2][e & 3]);
+        tmem_st16(stash + col, r);
+    };
+    auto get16 = [&](uint32_t col, float (&x)[4][4]) {
+        float r[16];
+        tmem_ld16(stash + col, r);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) x[e >> 2][e & 3] = r[e];
+    };
+    float dgam[4];
+    {
+        float xk[4][4], xq[4][4], xg[4][4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const int i = 4 * ig + r;
+            const float4 a = ld4(Pk + i * LD + 4 * cg), b = ld4(Pq + i * LD + 4 * cg), c = ld4(Pg + i * LD + 4 * cg);
+            xk[r][0] = a.x; xk[r][1] = a.y; xk[r][2] = a.z; xk[r][3] = a.w;
+            xq[r][0] = b.x; xq[r][1] = b.y; xq[r][2] = b.z; xq[r][3] = b.w;
+            xg[r][0] = c.x; xg[r][1] = c.y; xg[r][2] = c.z; xg[r][3] = c.w;
+        }
+        put16(0, xk);
+        put16(16, xq);
+        put16(32, xg);
+        tmem_wait_st();
     }
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
@@ -861,7 +886,7 @@ __device__ __forceinline__ bool dqk_body(const GradParams& p, uint8_t* sm, uint3
         for (int w = 0; w < NT2 / 32; ++w) s += sgs[w * DK + cc];
         dgam[c] = s * ex2(sG[(C - 1) * LD + cc]) + ((ucol[cc] + ucol[DK + cc]) + (ucol[2 * DK + cc] + ucol[3 * DK + cc]));
     }
-    __syncthreads();   // the partials are in registers; their region takes K a, Q~ a, K b
+    __syncthreads();   // the partials are stashed; their region takes K a, Q~ a, K b
     float* Ka = reinterpret_cast<float*>(sm + OPS);
     float* Qa = Ka + 64 * LD;
     float* Kb = Qa + 64 * LD;
@@ -894,28 +919,41 @@ __device__ __forceinline__ bool dqk_body(const GradParams& p, uint8_t* sm, uint3
     __syncthreads();
 
     // ---- the Gram gradients, i side: dP1 = a . sum_J d^{IJ} (dAqk_{I,J} K b_J), dP2 likewise
-    // with dA; dQ += dP1, dK += dP2, dGamma += Q~ . dP1 + K . dP2
+    // with dA (per sub-block J a partial sum, then scaled by d^{IJ}); dQ += dP1, dK += dP2,
+    // dGamma += Q~ . dP1 + K . dP2
     {
         float x1[4][4] = {}, x2[4][4] = {};
         for (int J = 0; J <= I; ++J) {
-            float4 dv = make_float4(1.f, 1.f, 1.f, 1.f);
-            if (J < I) dv = ld4(dfac + pair_index(I, J) * DK + 4 * cg);
-#pragma unroll 4
+            float t1[4][4] = {}, t2[4][4] = {};
+#pragma unroll 2
             for (int j = 16 * J; j < 16 * J + 16; ++j) {
                 const float4 aq = ld4(dAT + j * LT + 4 * ig), ad = ld4(dDT + j * LT + 4 * ig);
                 const float4 b0 = ld4(Kb + j * LD + 4 * cg);
-                const float kb[4] = {b0.x * dv.x, b0.y * dv.y, b0.z * dv.z, b0.w * dv.w};
+                const float kb[4] = {b0.x, b0.y, b0.z, b0.w};
 #pragma unroll
                 for (int r = 0; r < 4; ++r) {
                     const float q1 = comp(aq, r), q2 = comp(ad, r);
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
-                        x1[r][c] = fmaf(q1, kb[c], x1[r][c]);
-                        x2[r][c] = fmaf(q2, kb[c], x2[r][c]);
+                        t1[r][c] = fmaf(q1, kb[c], t1[r][c]);
+                        t2[r][c] = fmaf(q2, kb[c], t2[r][c]);
                     }
                 }
             }
+            float4 dv = make_float4(1.f, 1.f, 1.f, 1.f);
+            if (J < I) dv = ld4(dfac + pair_index(I, J) * DK + 4 * cg);
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    x1[r][c] = fmaf(comp(dv, c), t1[r][c], x1[r][c]);
+                    x2[r][c] = fmaf(comp(dv, c), t2[r][c], x2[r][c]);
+                }
         }
+        float xk[4][4], xq[4][4], xg[4][4];
+        get16(0, xk);
+        get16(16, xq);
+        get16(32, xg);
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
             const int i = 4 * ig + r;
@@ -928,28 +966,41 @@ __device__ __forceinline__ bool dqk_body(const GradParams& p, uint8_t* sm, uint3
                 xg[r][c] += Qa[i * LD + cc] * x1[r][c] + Ka[i * LD + cc] * x2[r][c];
             }
         }
+        put16(0, xk);
+        put16(16, xq);
+        put16(32, xg);
+        tmem_wait_st();
     }
     // ---- j side: Y = sum_{I' >= J} d^{I'J} (dAqk_{I',J}^T Q~a_I' + dA_{I',J}^T K a_I');
     // dK += b . Y, dGamma -= K b . Y   (this thread's rows are j, in sub-block J = I)
+    float xk[4][4], xq[4][4], xg[4][4];
     {
         float y[4][4] = {};
         for (int Ip = I; Ip < 4; ++Ip) {
-            float4 dv = make_float4(1.f, 1.f, 1.f, 1.f);
-            if (Ip > I) dv = ld4(dfac + pair_index(Ip, I) * DK + 4 * cg);
+            float t[4][4] = {};
 #pragma unroll 4
             for (int i = 16 * Ip; i < 16 * Ip + 16; ++i) {
                 const float4 aq = ld4(sAqk + i * LT + 4 * ig), ad = ld4(sDA + i * LT + 4 * ig);
                 const float4 q0 = ld4(Qa + i * LD + 4 * cg), k0 = ld4(Ka + i * LD + 4 * cg);
-                const float qa[4] = {q0.x * dv.x, q0.y * dv.y, q0.z * dv.z, q0.w * dv.w};
-                const float ka[4] = {k0.x * dv.x, k0.y * dv.y, k0.z * dv.z, k0.w * dv.w};
+                const float qa[4] = {q0.x, q0.y, q0.z, q0.w};
+                const float ka[4] = {k0.x, k0.y, k0.z, k0.w};
 #pragma unroll
                 for (int r = 0; r < 4; ++r) {
                     const float w1 = comp(aq, r), w2 = comp(ad, r);
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) y[r][c] = fmaf(w1, qa[c], fmaf(w2, ka[c], y[r][c]));
+                    for (int c = 0; c < 4; ++c) t[r][c] = fmaf(w1, qa[c], fmaf(w2, ka[c], t[r][c]));
                 }
             }
+            float4 dv = make_float4(1.f, 1.f, 1.f, 1.f);
+            if (Ip > I) dv = ld4(dfac + pair_index(Ip, I) * DK + 4 * cg);
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) y[r][c] = fmaf(comp(dv, c), t[r][c], y[r][c]);
         }
+        get16(0, xk);
+        get16(16, xq);
+        get16(32, xg);
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
             const int j = 4 * ig + r;
@@ -963,25 +1014,38 @@ __device__ __forceinline__ bool dqk_body(const GradParams& p, uint8_t* sm, uint3
         }
     }
 
-    // ---- dg = reverse cumulative sum of dGamma (gamma = Gamma of the last row)
+    // ---- dg = reverse cumulative sum of dGamma (gamma = Gamma of the last row): within the
+    // warp's 16 rows by shuffles (the four row groups of a channel are lanes 8 apart), then
+    // across the sub-blocks through their totals (the dgam partials' space, consumed)
     if (ig == 15) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) xg[3][c] += dgam[c];
     }
+    float* btot = ucol;   // [4 sub-blocks][128 channels]
+    const int gl = lane >> 3;
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
         const float s3 = xg[3][c], s2 = xg[2][c] + s3, s1 = xg[1][c] + s2, s0 = xg[0][c] + s1;
         float incl = s0;
 #pragma unroll
-        for (int off = 1; off < 16; off <<= 1) {
-            const float y = __shfl_down_sync(0xffffffffu, incl, off, 16);
-            if (ig + off < 16) incl += y;
+        for (int off = 1; off < 4; off <<= 1) {
+            const float y = __shfl_down_sync(0xffffffffu, incl, 8 * off);
+            if (gl + off < 4) incl += y;
         }
         const float excl = incl - s0;
         xg[0][c] = s0 + excl;
         xg[1][c] = s1 + excl;
         xg[2][c] = s2 + excl;
         xg[3][c] = s3 + excl;
+        if (gl == 0) btot[I * DK + 4 * cg + c] = incl;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        float later = 0.f;
+        for (int Ip = I + 1; Ip < 4; ++Ip) later += btot[Ip * DK + 4 * cg + c];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) xg[r][c] += later;
     }
     if (GATE == KDA_GATE_SCALAR) __syncthreads();   // the row sums reuse the transposes' space
 
