@@ -73,7 +73,7 @@ constexpr int TH = 102400;         // fp16 T (hi), K-major 64 x 64 (read MN-majo
 constexpr int TL = 110592;         // its lo term
 constexpr int U = 118784;          // 67584-byte union:
 constexpr int KA = U, KB = U + 33792;              //   Gram: fp32 [64][LD] K a, K b
-constexpr int KG16 = U, S16 = U + 16384;           //   product 1: K e^Gamma (64 rows), S (128 rows), K-major
+constexpr int KG16 = U;                            //   product 1: K e^Gamma (64 rows, K-major)
 constexpr int EBH = U, EBL = U + 16384;            //   products 2, 3: diag(beta) resid (hi, lo) and
 constexpr int DEH = U + 32768, DEL = U + 49152;    //   dE (hi, lo), MN-major over v
 constexpr int DB16 = U, E16 = U + 16384;           //   product 4: dEbar, E (hi) (K-major, 64 rows)
@@ -82,8 +82,11 @@ constexpr int SB = DFAC + 3072;    // fp32 [64] beta
 constexpr int RED = SB + 256;      // fp32 [4][64] dbeta partial sums
 constexpr int PS = RED + 1024;     // fp32 [3][16][16] inverse scratch
 constexpr int BAR = PS + 3072;     // 5 mbarriers, TMEM base
-constexpr int BYTES = BAR + 64 + 1024;
-static_assert(U % 1024 == 0 && TH % 1024 == 0 && TL % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+constexpr int S16 = (BAR + 64 + 1023) / 1024 * 1024;   // fp16 S, K-major 128 rows: product 1, built
+                                                       // while the Gram A runs (Ka, Kb still live)
+constexpr int BYTES = S16 + 32768 + 1024;
+static_assert(U % 1024 == 0 && TH % 1024 == 0 && TL % 1024 == 0 && S16 % 1024 == 0,
+              "swizzled tiles need 1024-byte alignment");
 static_assert(BYTES <= 232448, "shared memory over the sm_100 per-block limit");
 constexpr uint32_t TM_R = 0, TM_E = 128, TM_DB = 256, TM_DL = 384;
 }  // namespace s1
@@ -384,37 +387,43 @@ __device__ __forceinline__ bool solve_body(const GradParams& p, uint8_t* sm, uin
         st4(Kb + i * LD + 8 * cc, kb[0], kb[1], kb[2], kb[3]);
         st4(Kb + i * LD + 8 * cc + 4, kb[4], kb[5], kb[6], kb[7]);
     }
+    for (int x = tid; x < C * C / 4; x += NT) {   // A's tiles above the diagonal stay zero
+        const int i = x >> 4, j4 = 4 * (x & 15);
+        if (j4 > (i | 3)) st4(sA + i * LT + j4, 0.f, 0.f, 0.f, 0.f);
+    }
     __syncthreads();
 
-    // ---- A (strictly lower), CUDA cores: tiles of 4 rows x 4 columns
-    {
-        const int ig = tid & 15, jg = tid >> 4, I = ig >> 2, J = jg >> 2;
+    // ---- A (strictly lower), CUDA cores: the 136 tiles of 4 rows x 4 columns on or below
+    // the diagonal go to threads 0-135 (warps 0-4), so no warp walks an empty tile; warps
+    // 5-7 meanwhile turn S into the fp16 operand of product 1 (its own region)
+    if (tid < 136) {
+        int ig = 0;
+        while ((ig + 1) * (ig + 2) / 2 <= tid) ++ig;   // tile tid = ig (ig + 1) / 2 + jg
+        const int jg = tid - ig * (ig + 1) / 2, I = ig >> 2, J = jg >> 2;
         float acc[4][4] = {};
-        if (J <= I) {
-            const float* dv = dfac + (J < I ? pair_index(I, J) : 0) * DK;
+        const float* dv = dfac + (J < I ? pair_index(I, J) : 0) * DK;
 #pragma unroll 2
-            for (int c = 0; c < DK; c += 4) {
-                float4 a[4], b[4];
+        for (int c = 0; c < DK; c += 4) {
+            float4 a[4], b[4];
 #pragma unroll
-                for (int r = 0; r < 4; ++r) {
-                    a[r] = ld4(Ka + (4 * ig + r) * LD + c);
-                    b[r] = ld4(Kb + (4 * jg + r) * LD + c);
-                }
-                if (J < I) {
-                    const float4 d = ld4(dv + c);
-#pragma unroll
-                    for (int r = 0; r < 4; ++r) b[r].x *= d.x, b[r].y *= d.y, b[r].z *= d.z, b[r].w *= d.w;
-                }
-#pragma unroll
-                for (int r = 0; r < 4; ++r)
-#pragma unroll
-                    for (int s = 0; s < 4; ++s) {
-                        acc[r][s] = fmaf(a[r].x, b[s].x, acc[r][s]);
-                        acc[r][s] = fmaf(a[r].y, b[s].y, acc[r][s]);
-                        acc[r][s] = fmaf(a[r].z, b[s].z, acc[r][s]);
-                        acc[r][s] = fmaf(a[r].w, b[s].w, acc[r][s]);
-                    }
+            for (int r = 0; r < 4; ++r) {
+                a[r] = ld4(Ka + (4 * ig + r) * LD + c);
+                b[r] = ld4(Kb + (4 * jg + r) * LD + c);
             }
+            if (J < I) {
+                const float4 d = ld4(dv + c);
+#pragma unroll
+                for (int r = 0; r < 4; ++r) b[r].x *= d.x, b[r].y *= d.y, b[r].z *= d.z, b[r].w *= d.w;
+            }
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+                for (int s = 0; s < 4; ++s) {
+                    acc[r][s] = fmaf(a[r].x, b[s].x, acc[r][s]);
+                    acc[r][s] = fmaf(a[r].y, b[s].y, acc[r][s]);
+                    acc[r][s] = fmaf(a[r].z, b[s].z, acc[r][s]);
+                    acc[r][s] = fmaf(a[r].w, b[s].w, acc[r][s]);
+                }
         }
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
@@ -423,6 +432,15 @@ __device__ __forceinline__ bool solve_body(const GradParams& p, uint8_t* sm, uin
 #pragma unroll
             for (int s = 0; s < 4; ++s) o[s] = (4 * jg + s < i) ? acc[r][s] : 0.f;
             st4(sA + i * LT + 4 * jg, o[0], o[1], o[2], o[3]);
+        }
+    } else if (tid >= 160) {
+        const float* S = p.chk + sh * DV * DK;
+#pragma unroll 4
+        for (int x = tid - 160; x < DV * 16; x += NT - 160) {
+            const int v = x >> 4, cc = x & 15;
+            float f[8];
+            ld8g(S + (size_t)v * DK + 8 * cc, f);
+            st_shared_v4(sm + S16, kmaj_off(v, 8 * cc, 128), pack8_f16(f));
         }
     }
     __syncthreads();
@@ -435,16 +453,6 @@ __device__ __forceinline__ bool solve_body(const GradParams& p, uint8_t* sm, uin
 #pragma unroll
         for (int e = 0; e < 8; ++e) kg[e] = kr[r][e] * ex2(sG[i * LD + 8 * cc + e]);
         st_shared_v4(sm + KG16, kmaj_off(i, 8 * cc, 64), pack8_f16(kg));
-    }
-    {
-        const float* S = p.chk + sh * DV * DK;
-#pragma unroll
-        for (int x = tid; x < DV * 16; x += NT) {
-            const int v = x >> 4, cc = x & 15;
-            float f[8];
-            ld8g(S + (size_t)v * DK + 8 * cc, f);
-            st_shared_v4(sm + S16, kmaj_off(v, 8 * cc, 128), pack8_f16(f));
-        }
     }
     operands_ready();
     if (tid == 0) {
