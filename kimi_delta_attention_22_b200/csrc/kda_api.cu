@@ -313,8 +313,7 @@ kda_status_t kda_chunk_bwd(const kda_shape_t* sh, const void* q, const void* k, 
     if (pooled && cudaMallocAsync(reinterpret_cast<void**>(&ws), bl.bytes, st) != cudaSuccess) return KDA_ERR_CUDA;
     const kda::ChunkArgs fa = kda::forward_args(a);
     e = kda::launch_chunk_wy(fa, ws, bl.fwd, st);
-    if (e == cudaSuccess) e = kda::launch_chunk_scan(fa, ws, bl.fwd, st, reinterpret_cast<float*>(ws + bl.chk_off));
-    if (e == cudaSuccess) e = kda::launch_chunk_bwd_scan(a, ws, bl, st);
+    if (e == cudaSuccess) e = kda::launch_chunk_scans_bwd(a, ws, bl, st);
     if (e == cudaSuccess) e = kda::launch_chunk_bwd_grad(a, ws, bl, st);
     if (pooled) {
         const cudaError_t f = cudaFreeAsync(ws, st);

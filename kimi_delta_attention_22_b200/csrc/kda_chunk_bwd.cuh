@@ -1,13 +1,13 @@
 // kda_chunk_bwd.cuh -- launch interfaces and workspace layout of the chunkwise
 // backward (gradients of the tensor-core prefill; d_k = d_v = 128, chunk 64).
 //
-// The backward runs five kernels on one stream:
+// The backward runs four launches on one stream:
 //   1. the forward's WY kernel: every chunk's record (kda_chunk_record.cuh);
-//   2. the forward's state scan with outputs off, keeping every chunk's incoming
-//      state S_c (fp32) in the workspace;
-//   3. the reverse state scan (kda_chunk_bwd_scan.cu): dS0, and per chunk the
-//      gradient of its outgoing state dS' and dE;
-//   4. and 5. the chunk-parallel gradient kernels (kda_chunk_bwd_grad.cu): per
+//   2. one launch of two independent scans side by side (kda_chunk_bwd_scan.cu): the
+//      forward's state scan with outputs off, keeping every chunk's incoming state
+//      S_c (fp32) in the workspace, and the reverse state scan: dS0, and per chunk
+//      the gradient of its outgoing state dS' and dE;
+//   3. and 4. the chunk-parallel gradient kernels (kda_chunk_bwd_grad.cu): per
 //      (chunk, head), the triangular-solve half (E, the solve's gradient, dv,
 //      dbeta) and then the rest (dq, dk, dg); their dense products run on the
 //      tensor cores, the decay-weighted Gram parts on CUDA cores.
@@ -96,7 +96,8 @@ inline ChunkArgs forward_args(const ChunkBwdArgs& a) {
     return f;
 }
 
-cudaError_t launch_chunk_bwd_scan(const ChunkBwdArgs& a, const uint8_t* ws, const BwdLayout& bl, cudaStream_t st);
+// The forward scan with checkpoints (no outputs) and the reverse scan, in one launch.
+cudaError_t launch_chunk_scans_bwd(const ChunkBwdArgs& a, const uint8_t* ws, const BwdLayout& bl, cudaStream_t st);
 cudaError_t launch_chunk_bwd_grad(const ChunkBwdArgs& a, uint8_t* ws, const BwdLayout& bl, cudaStream_t st);
 
 }  // namespace kda

@@ -26,12 +26,14 @@
 // one copy thread; each barrier completes once per chunk step.
 #include "kda_chunk_bwd.cuh"
 #include "kda_chunk_record.cuh"
+#include "kda_chunk_scan.cuh"
 #include "kda_internal.cuh"
 #include "kda_tc_common.cuh"
 #include "sm100.cuh"
 
 namespace kda {
 namespace {
+namespace rv {   // the reverse scan (the forward scan's device code comes from kda_chunk_scan.cuh)
 
 using namespace sm100;
 using namespace tc;
@@ -106,12 +108,13 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
 // The state warps read a stage (dO tile, dec) before oready, and everything they
 // write to tensor memory in step r is read by MMAs of step r that complete before
 // the warps' next write (bar1 / bar2 of step r precede it in their program order).
-__global__ void __launch_bounds__(NT, 1) kda_chunk_bwd_scan_kernel(const __grid_constant__ BwdScanParams p) {
+// One CTA's reverse scan: sequence and head of block index bid.
+__device__ __forceinline__ void bwd_scan_cta(const BwdScanParams& p, int bid) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int h = blockIdx.x % p.H, n = blockIdx.x / p.H;
+    const int h = bid % p.H, n = bid / p.H;
     const int sp = warp & 3, part = (warp >> 2) % NPART;
     const int v = 32 * sp + lane;
     const uint32_t lane_base = (uint32_t)(32 * sp) << 16;
@@ -343,14 +346,52 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_bwd_scan_kernel(const __grid_
     }
 }
 
+}  // namespace rv
+
+// The backward's two scans in one launch: CTAs [0, fwd_ctas) run the forward scan
+// (checkpoints, no outputs), the rest the reverse scan.  The reverse scan needs only
+// the records, dO and d_ST, so the two are independent and share the GPU, each
+// having one CTA per (sequence, head).
+struct DualScanParams {
+    ScanParams f;
+    rv::BwdScanParams b;
+    int fwd_ctas;
+};
+static_assert(Cfg<16>::NT == rv::NT, "the two scans run the same block shape");
+constexpr int kDualSmem = Cfg<16>::SMEM_BYTES > rv::SMEM_BYTES ? Cfg<16>::SMEM_BYTES : rv::SMEM_BYTES;
+
+__global__ void __launch_bounds__(rv::NT, 1) kda_chunk_fwdbwd_scan_kernel(const __grid_constant__ DualScanParams p) {
+    if ((int)blockIdx.x < p.fwd_ctas) {
+        scan_cta<16>(p.f, (int)blockIdx.x);
+    } else {
+        rv::bwd_scan_cta(p.b, (int)blockIdx.x - p.fwd_ctas);
+    }
+}
+
 }  // namespace
 
-cudaError_t launch_chunk_bwd_scan(const ChunkBwdArgs& a, const uint8_t* ws, const BwdLayout& bl, cudaStream_t st) {
+cudaError_t launch_chunk_scans_bwd(const ChunkBwdArgs& a, const uint8_t* ws, const BwdLayout& bl, cudaStream_t st) {
+    using rv::BwdScanParams;
+    using rv::NT;
     const rec::Layout& lay = bl.fwd;
-    BwdScanParams p;
-    memset(&p, 0, sizeof(p));
+    DualScanParams d;
+    memset(&d, 0, sizeof(d));
+    ScanParams& f = d.f;
+    f.rec = ws + lay.rec_off;
+    f.coff = a.cu_seqlens ? reinterpret_cast<const int32_t*>(ws + lay.coff_off) : nullptr;
+    f.cu_seqlens = a.cu_seqlens;
+    f.S0 = a.S0;
+    f.S_T = nullptr;
+    f.out = nullptr;
+    f.S_chk = reinterpret_cast<float*>(const_cast<uint8_t*>(ws) + bl.chk_off);
+    f.dev_status = a.dev_status;
+    f.T = a.T;
+    f.H = a.H;
+    f.num_seqs = a.num_seqs;
+    f.nc = (a.T + rec::C - 1) / rec::C;
+    BwdScanParams& p = d.b;
     p.rec = ws + lay.rec_off;
-    p.coff = a.cu_seqlens ? reinterpret_cast<const int32_t*>(ws + lay.coff_off) : nullptr;
+    p.coff = f.coff;
     p.cu_seqlens = a.cu_seqlens;
     p.d_ST = a.d_ST;
     p.dS0 = a.dS0;
@@ -360,16 +401,17 @@ cudaError_t launch_chunk_bwd_scan(const ChunkBwdArgs& a, const uint8_t* ws, cons
     p.T = a.T;
     p.H = a.H;
     p.num_seqs = a.num_seqs;
-    p.nc = (a.T + C - 1) / C;
+    p.nc = f.nc;
     const long long tokens = (long long)a.B * a.T;
-    if (tokens > 0 && !make_map(&p.map_do, a.d_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DV, a.H, tokens, DV, C,
+    if (tokens > 0 && !make_map(&p.map_do, a.d_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rec::DV, a.H, tokens, rec::DV, rec::C,
                                 CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(kda_chunk_bwd_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         SMEM_BYTES);
+    const long long pairs = (long long)a.num_seqs * a.H;
+    d.fwd_ctas = (int)pairs;
+    cudaError_t e = cudaFuncSetAttribute(kda_chunk_fwdbwd_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kDualSmem);
     if (e != cudaSuccess) return e;
-    return launch_after(kda_chunk_bwd_scan_kernel, dim3((unsigned)((long long)a.num_seqs * a.H)), NT, SMEM_BYTES,
-                        st, p);
+    return launch_after(kda_chunk_fwdbwd_scan_kernel, dim3((unsigned)(2 * pairs)), NT, kDualSmem, st, d);
 }
 
 }  // namespace kda
