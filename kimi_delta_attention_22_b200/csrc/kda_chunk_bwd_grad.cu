@@ -72,7 +72,9 @@ constexpr int RES = 68608;         // fp32 [64][LD]  resid
 constexpr int TH = 102400;         // fp16 T (hi), K-major 64 x 64 (read MN-major it is T^T)
 constexpr int TL = 110592;         // its lo term
 constexpr int U = 118784;          // 67584-byte union:
-constexpr int KA = U, KB = U + 33792;              //   Gram: fp32 [64][LD] K a, K b
+constexpr int KA = U, KB = U + 33792;              //   Gram, sub-block form: fp32 [64][LD] K a, K b
+constexpr int KXH = U, KXL = U + 16384;            //   Gram, one reference: K 2^G and K 2^-G as
+constexpr int KYH = U + 32768, KYL = U + 49152;    //   two-term bf16 (K-major, 64 rows)
 constexpr int KG16 = U;                            //   product 1: K e^Gamma (64 rows, K-major)
 constexpr int EBH = U, EBL = U + 16384;            //   products 2, 3: diag(beta) resid (hi, lo) and
 constexpr int DEH = U + 32768, DEL = U + 49152;    //   dE (hi, lo), MN-major over v
@@ -165,10 +167,15 @@ __device__ __forceinline__ bool slot_rows(const GradParams& p, int slot, long lo
 }
 
 // L2 prefetch of the inputs of the job p.ahead CTAs later, which starts about when
-// this one ends (one CTA per SM, CTAs start in linear order): one bulk prefetch per
-// token row of g, k and v (solve) or g, k, q and d_out (dq/dk), one per workspace tile.
-// Issued in a compute phase, so that a wave's loads do not all queue at its start.
-template <int GATE, bool DQK>
+// this one ends (one CTA per SM, CTAs start in linear order).  The strided token rows
+// (g, k and v for the solve kernel; g, k, q and d_out for dq/dk) are prefetched line
+// by line from every thread (one plain prefetch instruction per 128-byte line); each
+// contiguous workspace tile takes one bulk prefetch.  Issued in a compute phase, so
+// that a wave's loads do not all queue at its start.
+__device__ __forceinline__ void prefetch_line(const void* p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+template <int GATE, bool DQK, int NTH>
 __device__ __forceinline__ void prefetch_next(const GradParams& p) {
     const long long job = (long long)blockIdx.x + p.ahead;
     if (job >= (long long)gridDim.x) return;
@@ -178,26 +185,35 @@ __device__ __forceinline__ void prefetch_next(const GradParams& p) {
     if (!slot_rows(p, slot, c0, L)) return;
     const size_t sh = (size_t)slot * p.H + h;
     const int t = threadIdx.x;
-    if (t < L) {
-        const long long row = c0 + t;
-        if (GATE == KDA_GATE_CHANNEL) bulk_prefetch_l2(p.g + (row * p.H + h) * DK, DK * 4);
-        bulk_prefetch_l2(p.k + (row * Hk + hk) * DK, DK * 2);
-        if (DQK) {
-            bulk_prefetch_l2(p.q + (row * Hk + hk) * DK, DK * 2);
-            bulk_prefetch_l2(p.d_out + (row * p.H + h) * DV, DV * 2);
+    // per row: g 4 lines (channel gate), k 2, v 2 or q 2 + d_out 2
+    constexpr int G4 = GATE == KDA_GATE_CHANNEL ? 4 : 0, PER = G4 + (DQK ? 6 : 4);
+    for (int x = t; x < L * PER; x += NTH) {
+        const int i = x / PER, u = x % PER;
+        const long long row = c0 + i;
+        const char* a;
+        if (u < G4) {
+            a = reinterpret_cast<const char*>(p.g + (row * p.H + h) * DK) + 128 * u;
+        } else if (u < G4 + 2) {
+            a = reinterpret_cast<const char*>(p.k + (row * Hk + hk) * DK) + 128 * (u - G4);
+        } else if (!DQK) {
+            a = reinterpret_cast<const char*>(p.v + (row * p.H + h) * DV) + 128 * (u - G4 - 2);
+        } else if (u < G4 + 4) {
+            a = reinterpret_cast<const char*>(p.q + (row * Hk + hk) * DK) + 128 * (u - G4 - 2);
         } else {
-            bulk_prefetch_l2(p.v + (row * p.H + h) * DV, DV * 2);
+            a = reinterpret_cast<const char*>(p.d_out + (row * p.H + h) * DV) + 128 * (u - G4 - 4);
         }
-    } else if (t == C) {
+        prefetch_line(a);
+    }
+    if (t == 0) {
         bulk_prefetch_l2(p.chk + sh * DV * DK, DV * DK * 4);
-    } else if (t == C + 1) {
-        if (DQK) bulk_prefetch_l2(p.dsp + sh * DV * DK, DV * DK * 4);
-        else bulk_prefetch_l2(p.de + sh * C * DV, C * DV * 4);
-    } else if (DQK && t == C + 2) {
-        bulk_prefetch_l2(p.e16 + sh * 2 * kTile16, 2 * kTile16);
-    } else if (DQK && t == C + 3) {
-        bulk_prefetch_l2(p.pr16 + sh * kTile16, kTile16);
-        bulk_prefetch_l2(p.da + sh * C * C, C * C * 4);
+        if (DQK) {
+            bulk_prefetch_l2(p.dsp + sh * DV * DK, DV * DK * 4);
+            bulk_prefetch_l2(p.e16 + sh * 2 * kTile16, 2 * kTile16);
+            bulk_prefetch_l2(p.pr16 + sh * kTile16, kTile16);
+            bulk_prefetch_l2(p.da + sh * C * C, C * C * 4);
+        } else {
+            bulk_prefetch_l2(p.de + sh * C * DV, C * DV * 4);
+        }
     }
 }
 
@@ -369,7 +385,69 @@ __device__ __forceinline__ bool solve_body(const GradParams& p, uint8_t* sm, uin
         const int x = tid + NT * r, i = x & 63, cc = x >> 6;
         loadn<8>(p.k + ((c0 + i) * Hk + hk) * DK + 8 * cc, i < L, kr[r]);
     }
-    __syncthreads();
+    // One decay reference for the whole chunk while its decay stays inside bf16's range
+    // (max_c |G_last| <= 112): A = (K 2^G)(K 2^-G)^T as one tensor-core product over
+    // two-term bf16 operands; otherwise the sub-block form on the CUDA cores in fp32.
+    const bool fast = __syncthreads_and(tid >= DK || sG[(C - 1) * LD + tid] >= -112.f) != 0;
+    if (fast) {
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const int x = tid + NT * r, i = x & 63, cc = x >> 6;
+            float kx[8], ky[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float Gv = sG[i * LD + 8 * cc + e];
+                kx[e] = kr[r][e] * ex2(Gv);
+                ky[e] = kr[r][e] * ex2(-Gv);
+            }
+            uint4 hi, lo;
+            pack8_split(kx, hi, lo);
+            st_shared_v4(sm + KXH, kmaj_off(i, 8 * cc, 64), hi);
+            st_shared_v4(sm + KXL, kmaj_off(i, 8 * cc, 64), lo);
+            pack8_split(ky, hi, lo);
+            st_shared_v4(sm + KYH, kmaj_off(i, 8 * cc, 64), hi);
+            st_shared_v4(sm + KYL, kmaj_off(i, 8 * cc, 64), lo);
+        }
+        operands_ready();
+        if (tid == 0) {
+            const uint32_t xa[3] = {sbase + KXH, sbase + KXH, sbase + KXL};
+            const uint32_t ya[3] = {sbase + KYH, sbase + KYL, sbase + KYH};
+#pragma unroll
+            for (int t = 0; t < 3; ++t)
+#pragma unroll
+                for (int s = 0; s < 8; ++s)
+                    mma_bf16(tm + TM_DL, kmaj_desc(xa[t], 64, s), kmaj_desc(ya[t], 64, s),
+                             idesc_bf16(64, 64, false, false), t > 0 || s > 0);
+            mma_commit(bars + 4);
+        }
+        {   // meanwhile: S as the fp16 operand of product 1
+            const float* S = p.chk + sh * DV * DK;
+#pragma unroll 4
+            for (int x = tid; x < DV * 16; x += NT) {
+                const int v = x >> 4, cc = x & 15;
+                float f[8];
+                ld8g(S + (size_t)v * DK + 8 * cc, f);
+                st_shared_v4(sm + S16, kmaj_off(v, 8 * cc, 128), pack8_f16(f));
+            }
+        }
+        if (!wait_mma(bars + 4)) return false;
+        tc_fence_after();
+        {
+            const int i = 16 * sp + (lane & 15);
+            float d[32];
+            tmem_ld32(tm + lane_base + TM_DL + 32 * hc, d);
+            if (lane < 16) {
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int j = 32 * hc + 4 * u;
+                    st4(sA + i * LT + j, j < i ? d[4 * u] : 0.f, j + 1 < i ? d[4 * u + 1] : 0.f,
+                        j + 2 < i ? d[4 * u + 2] : 0.f, j + 3 < i ? d[4 * u + 3] : 0.f);
+                }
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+    } else {
     load_dfac<NT>(sG, dfac);
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
@@ -444,6 +522,7 @@ __device__ __forceinline__ bool solve_body(const GradParams& p, uint8_t* sm, uin
         }
     }
     __syncthreads();
+    }
 
     // ---- product 1 (tensor cores): (K e^Gamma) S^T; operands K e^Gamma and S in fp16
 #pragma unroll
@@ -464,7 +543,7 @@ __device__ __forceinline__ bool solve_body(const GradParams& p, uint8_t* sm, uin
     }
     // meanwhile on the CUDA cores: T, and its two-term fp16 image; the next wave's
     // inputs go to L2 while this CTA computes rather than while it loads
-    prefetch_next<GATE, false>(p);
+    prefetch_next<GATE, false, NT>(p);
     invert_unit_lower(sA, sb, sT, reinterpret_cast<float*>(sm + PS));
     for (int x = tid; x < C * 8; x += NT) {
         const int i = x >> 3, jc = x & 7;
@@ -634,9 +713,9 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_bwd_solve_kernel(const __grid
     int L;
     if (!slot_rows(p, slot, c0, L)) return;
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + s1::BAR);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 5);
     if (tid == 0) {
-        for (int b = 0; b < 4; ++b) mbar_init(bars + b, 1);
+        for (int b = 0; b < 5; ++b) mbar_init(bars + b, 1);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -795,7 +874,17 @@ __device__ __forceinline__ bool dqk_body(const GradParams& p, uint8_t* sm, uint3
     {
         const int i = 16 * sp + (lane & 15);
         const bool own = lane < 16;
-#pragma unroll 1
+        // this thread's 32 channels of K and Q, all loads in flight before the loop
+        uint4 kraw[4], qraw[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            kraw[q] = qraw[q] = make_uint4(0u, 0u, 0u, 0u);
+            if (own && i < L) {
+                kraw[q] = __ldg(reinterpret_cast<const uint4*>(p.k + ((c0 + i) * Hk + hk) * DK + 32 * qt) + q);
+                qraw[q] = __ldg(reinterpret_cast<const uint4*>(p.q + ((c0 + i) * Hk + hk) * DK + 32 * qt) + q);
+            }
+        }
+#pragma unroll
         for (int q = 0; q < 4; ++q) {
             const int cb = 32 * qt + 8 * q;
             float xk[8], xq[8], xg[8];
@@ -803,8 +892,8 @@ __device__ __forceinline__ bool dqk_body(const GradParams& p, uint8_t* sm, uint3
             tmem_ld8(tm + lane_base + TM_QG + cb, xq);
             tmem_ld8(tm + lane_base + TM_KG + cb, xg);
             float kx[8], qx[8];
-            loadn<8>(p.k + ((c0 + i) * Hk + hk) * DK + cb, own && i < L, kx);
-            loadn<8>(p.q + ((c0 + i) * Hk + hk) * DK + cb, own && i < L, qx);
+            unpack8(kraw[q], kx);
+            unpack8(qraw[q], qx);
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 const int c = cb + e;
@@ -849,7 +938,7 @@ __device__ __forceinline__ bool dqk_body(const GradParams& p, uint8_t* sm, uint3
     }
     __syncthreads();
 
-    prefetch_next<GATE, true>(p);   // the next wave's inputs, while this CTA computes
+    prefetch_next<GATE, true, NT2>(p);   // the next wave's inputs, while this CTA computes
     // ---- from here on: thread rows i = 4 ig .. +3, channels c = 4 cg .. +3, with the
     // rows of one warp in one 16-row sub-block I (warp / 4), so that the block-triangular
     // Gram loops below take the same trip count on every lane (5 sub-blocks per warp).
