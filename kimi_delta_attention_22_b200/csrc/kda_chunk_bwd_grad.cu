@@ -109,12 +109,20 @@ constexpr int DA = AQK + 17408;    // fp32 [64][LT] dA (strictly lower)
 constexpr int AQT = DA + 17408;    // fp32 [64][LT] dAqk^T
 constexpr int DAT = AQT + 17408;   // fp32 [64][LT] dA^T
 constexpr int SRED = AQT;          // fp32 [32][64] scalar-gate row sums (after the Gram loops)
+// one-reference chunks: the Gram gradients as tensor-core products over two-term bf16 tiles
+constexpr int DXQH = AQT, DXQL = AQT + 8192;          // dAqk (hi, lo), K-major 64 x 64 (the
+constexpr int DXAH = AQT + 16384, DXAL = AQT + 24576; // transposes' space), and dA
+constexpr int KBH = OPS, KBL = OPS + 16384;           // K 2^-G, MN-major over the channel (K = token)
+constexpr int QAH = OPS + 32768, QAL = OPS + 49152;   // Q~ 2^G
+constexpr int KAH = OPS + 65536, KAL = OPS + 81920;   // K 2^G
+constexpr uint32_t TM_X1 = 0, TM_X2 = 128, TM_Y = 256;
 constexpr int DFAC = DAT + 17408;  // fp32 [6][128]
 constexpr int UCOL = DFAC + 3072;  // fp32 [4][128] colsum(dKd . Kd) partials
 constexpr int SGS = UCOL + 2048;   // fp32 [16][128] colsum(S . dS') partials (one row per warp)
-constexpr int BAR = SGS + 8192;    // 5 mbarriers, TMEM base
+constexpr int BAR = SGS + 8192;    // 6 mbarriers, TMEM base
 constexpr int BYTES = BAR + 64 + 1024;
-static_assert(OPS % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+static_assert(OPS % 1024 == 0 && AQT % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+static_assert(DXAL + 8192 <= DAT + 64 * LT * 4 && KAL + 16384 - OPS <= 101376, "fast-path tiles fit");
 static_assert(PR16 + 8192 - OPS <= 101376 && 3 * 64 * LD * 4 <= 101376, "operands and partials fit the union");
 static_assert(BYTES <= 232448, "shared memory over the sm_100 per-block limit");
 constexpr uint32_t TM_KD = 0, TM_QG = 128, TM_KG = 256, TM_AQ = 384;
@@ -842,6 +850,8 @@ __device__ __forceinline__ bool dqk_body(const GradParams& p, uint8_t* sm, uint3
         for (int x = tid; x < C * C / 4; x += NT2) *reinterpret_cast<float4*>(sDA + (x >> 4) * LT + 4 * (x & 15)) = a4[x];
     }
     if (!__syncthreads_and(mbar_wait(bars + 0, 0, kWaitNs))) return false;
+    // one decay reference for the whole chunk while its decay stays inside bf16's range
+    const bool fast = __syncthreads_and(tid >= DK || sG[(C - 1) * LD + tid] >= -112.f) != 0;
     operands_ready();
     if (tid == 0) {
         issue(0);
@@ -928,24 +938,153 @@ __device__ __forceinline__ bool dqk_body(const GradParams& p, uint8_t* sm, uint3
                 const int j = 16 * qt + t;
                 const float x = j <= i ? z[t] : 0.f;
                 sAqk[i * LT + j] = x;
-                dAT[j * LT + i] = x;
+                if (!fast) dAT[j * LT + i] = x;
             }
         }
     }
-    for (int x = tid; x < C * C; x += NT2) {
-        const int i = x & 63, j = x >> 6;
-        dDT[j * LT + i] = sDA[i * LT + j];
+    if (!fast) {
+        for (int x = tid; x < C * C; x += NT2) {
+            const int i = x & 63, j = x >> 6;
+            dDT[j * LT + i] = sDA[i * LT + j];
+        }
     }
     __syncthreads();
 
     prefetch_next<GATE, true, NT2>(p);   // the next wave's inputs, while this CTA computes
     // ---- from here on: thread rows i = 4 ig .. +3, channels c = 4 cg .. +3, with the
     // rows of one warp in one 16-row sub-block I (warp / 4), so that the block-triangular
-    // Gram loops below take the same trip count on every lane (5 sub-blocks per warp).
-    // The thread's 48 partial sums (dK, dQ, dGamma) wait in its own tensor-memory lane
-    // (columns 48 (warp / 4) ..; the products are read out, so the columns are free)
-    // while the Gram loops run, which keeps those loops within the 128-register budget.
+    // Gram loops of the sub-block form take the same trip count on every lane (5
+    // sub-blocks per warp).
     const int I = warp >> 2, ig = 4 * I + (lane >> 3), cg = 8 * (warp & 3) + (lane & 7);
+    float dgam[4];
+    float xk[4][4], xq[4][4], xg[4][4];
+    if (fast) {
+        // ---- the Gram gradients on the tensor cores.  With a_i = 2^{G_i}, b_j = 2^{-G_j}:
+        // X1 = dAqk (K b), X2 = dA (K b), Y = dAqk^T (Q~ a) + dA^T (K a) (M = 64, N = 128,
+        // K = 64 tokens, each over two-term bf16 operands); then per element dQ += a X1,
+        // dK += a X2 + b Y, dGamma += Q~ a X1 + K a X2 - K b Y.
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const int i = 4 * ig + r;
+            const float4 a = ld4(Pk + i * LD + 4 * cg), b = ld4(Pq + i * LD + 4 * cg), c = ld4(Pg + i * LD + 4 * cg);
+            xk[r][0] = a.x; xk[r][1] = a.y; xk[r][2] = a.z; xk[r][3] = a.w;
+            xq[r][0] = b.x; xq[r][1] = b.y; xq[r][2] = b.z; xq[r][3] = b.w;
+            xg[r][0] = c.x; xg[r][1] = c.y; xg[r][2] = c.z; xg[r][3] = c.w;
+        }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const int cc = 4 * cg + c;
+        float s = 0.f;
+#pragma unroll
+        for (int w = 0; w < NT2 / 32; ++w) s += sgs[w * DK + cc];
+        dgam[c] = s * ex2(sG[(C - 1) * LD + cc]) + ((ucol[cc] + ucol[DK + cc]) + (ucol[2 * DK + cc] + ucol[3 * DK + cc]));
+    }
+        __syncthreads();   // the partials are in registers; the union takes the operand tiles
+        for (int x = tid; x < C * 8; x += NT2) {   // dAqk, dA: rows i, 8 tokens j per chunk
+            const int i = x >> 3, jc = x & 7;
+            float a8[8], d8[8];
+            ld8(sAqk + i * LT + 8 * jc, a8);
+            ld8(sDA + i * LT + 8 * jc, d8);
+            uint4 hi, lo;
+            pack8_split(a8, hi, lo);
+            st_shared_v4(sm + DXQH, kmaj_off(i, 8 * jc, 64), hi);
+            st_shared_v4(sm + DXQL, kmaj_off(i, 8 * jc, 64), lo);
+            pack8_split(d8, hi, lo);
+            st_shared_v4(sm + DXAH, kmaj_off(i, 8 * jc, 64), hi);
+            st_shared_v4(sm + DXAL, kmaj_off(i, 8 * jc, 64), lo);
+        }
+#pragma unroll
+        for (int x = tid; x < C * 16; x += NT2) {   // K b, Q~ a, K a: token i, 8 channels
+            const int i = x >> 4, cc = x & 15;
+            float kx[8], qx[8];
+            loadn<8>(p.k + ((c0 + i) * Hk + hk) * DK + 8 * cc, i < L, kx);
+            loadn<8>(p.q + ((c0 + i) * Hk + hk) * DK + 8 * cc, i < L, qx);
+            float kb[8], qa[8], ka[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float Gv = sG[i * LD + 8 * cc + e], a = ex2(Gv), bb = ex2(-Gv);
+                kb[e] = kx[e] * bb;
+                qa[e] = qx[e] * p.scale * a;
+                ka[e] = kx[e] * a;
+            }
+            const uint32_t off = mnmaj_off(8 * cc, i, 128);
+            uint4 hi, lo;
+            pack8_split(kb, hi, lo);
+            st_shared_v4(sm + KBH, off, hi);
+            st_shared_v4(sm + KBL, off, lo);
+            pack8_split(qa, hi, lo);
+            st_shared_v4(sm + QAH, off, hi);
+            st_shared_v4(sm + QAL, off, lo);
+            pack8_split(ka, hi, lo);
+            st_shared_v4(sm + KAH, off, hi);
+            st_shared_v4(sm + KAL, off, lo);
+        }
+        operands_ready();
+        if (tid == 0) {
+            const uint32_t xq3[3] = {sbase + DXQH, sbase + DXQH, sbase + DXQL};
+            const uint32_t xa3[3] = {sbase + DXAH, sbase + DXAH, sbase + DXAL};
+            const uint32_t kb3[3] = {sbase + KBH, sbase + KBL, sbase + KBH};
+            const uint32_t qa3[3] = {sbase + QAH, sbase + QAL, sbase + QAH};
+            const uint32_t ka3[3] = {sbase + KAH, sbase + KAL, sbase + KAH};
+#pragma unroll
+            for (int t = 0; t < 3; ++t)
+#pragma unroll
+                for (int s4 = 0; s4 < 4; ++s4) {
+                    const bool acc = t > 0 || s4 > 0;
+                    mma_bf16(tm + TM_X1, kmaj_desc(xq3[t], 64, s4), mnmaj_desc(kb3[t], 128, s4),
+                             idesc_bf16(64, 128, false, true), acc);
+                    mma_bf16(tm + TM_X2, kmaj_desc(xa3[t], 64, s4), mnmaj_desc(kb3[t], 128, s4),
+                             idesc_bf16(64, 128, false, true), acc);
+                    mma_bf16(tm + TM_Y, mnmaj_desc(xq3[t], 64, s4), mnmaj_desc(qa3[t], 128, s4),
+                             idesc_bf16(64, 128, true, true), acc);
+                    mma_bf16(tm + TM_Y, mnmaj_desc(xa3[t], 64, s4), mnmaj_desc(ka3[t], 128, s4),
+                             idesc_bf16(64, 128, true, true), 1);
+                }
+            mma_commit(bars + 4);
+        }
+        if (!wait_mma(bars + 4)) return false;
+        tc_fence_after();
+        {   // X1 | X2 | Y to fp32 [64][LD] each in the union (the operand tiles are spent)
+            const int i = 16 * sp + (lane & 15);
+#pragma unroll 1
+            for (int q = 0; q < 3; ++q) {
+                float d[32];
+                tmem_ld32(tm + lane_base + 128u * (uint32_t)q + 32u * (uint32_t)qt, d);
+                if (lane < 16) {
+                    float* o = Pk + q * 64 * LD + i * LD + 32 * qt;
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) st4(o + 4 * u, d[4 * u], d[4 * u + 1], d[4 * u + 2], d[4 * u + 3]);
+                }
+            }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const int i = 4 * ig + r;
+            const float4 x1 = ld4(Pk + i * LD + 4 * cg), x2 = ld4(Pq + i * LD + 4 * cg), y4 = ld4(Pg + i * LD + 4 * cg);
+            float kx[4] = {0.f, 0.f, 0.f, 0.f}, qx[4] = {0.f, 0.f, 0.f, 0.f};
+            if (i < L) {
+                const uint2 kr2 = __ldg(reinterpret_cast<const uint2*>(p.k + ((c0 + i) * Hk + hk) * DK + 4 * cg));
+                const uint2 qr2 = __ldg(reinterpret_cast<const uint2*>(p.q + ((c0 + i) * Hk + hk) * DK + 4 * cg));
+                const float2 k01 = unpack_bf16(kr2.x), k23 = unpack_bf16(kr2.y);
+                const float2 q01 = unpack_bf16(qr2.x), q23 = unpack_bf16(qr2.y);
+                kx[0] = k01.x; kx[1] = k01.y; kx[2] = k23.x; kx[3] = k23.y;
+                qx[0] = q01.x; qx[1] = q01.y; qx[2] = q23.x; qx[3] = q23.y;
+            }
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const float Gv = sG[i * LD + 4 * cg + c], a = ex2(Gv), bb = ex2(-Gv);
+                const float dP1 = a * comp(x1, c), dP2 = a * comp(x2, c), dKy = bb * comp(y4, c);
+                xq[r][c] += dP1;
+                xk[r][c] += dP2 + dKy;
+                xg[r][c] += qx[c] * p.scale * dP1 + kx[c] * (dP2 - dKy);
+            }
+        }
+    } else {
+    // ---- sub-block form on the CUDA cores.  The thread's 48 partial sums (dK, dQ, dGamma)
+    // wait in its own tensor-memory lane (columns 48 (warp / 4) ..; the products are read
+    // out, so the columns are free) while the Gram loops run, which keeps those loops
+    // within the 128-register budget.
     const uint32_t stash = tm + lane_base + 48u * (uint32_t)qt;
     auto put16 = [&](uint32_t col, const float (&x)[4][4]) {
         uint32_t r[16];
@@ -959,8 +1098,7 @@ __device__ __forceinline__ bool dqk_body(const GradParams& p, uint8_t* sm, uint3
 #pragma unroll
         for (int e = 0; e < 16; ++e) x[e >> 2][e & 3] = r[e];
     };
-    float dgam[4];
-    {
+    {   // the partials to the stash (names shadow the outer ones)
         float xk[4][4], xq[4][4], xg[4][4];
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
@@ -1070,7 +1208,6 @@ __device__ __forceinline__ bool dqk_body(const GradParams& p, uint8_t* sm, uint3
     }
     // ---- j side: Y = sum_{I' >= J} d^{I'J} (dAqk_{I',J}^T Q~a_I' + dA_{I',J}^T K a_I');
     // dK += b . Y, dGamma -= K b . Y   (this thread's rows are j, in sub-block J = I)
-    float xk[4][4], xq[4][4], xg[4][4];
     {
         float y[4][4] = {};
         for (int Ip = I; Ip < 4; ++Ip) {
@@ -1111,6 +1248,7 @@ __device__ __forceinline__ bool dqk_body(const GradParams& p, uint8_t* sm, uint3
         }
     }
 
+    }
     // ---- dg = reverse cumulative sum of dGamma (gamma = Gamma of the last row): within the
     // warp's 16 rows by shuffles (the four row groups of a channel are lanes 8 apart), then
     // across the sub-blocks through their totals (the dgam partials' space, consumed)
@@ -1194,9 +1332,9 @@ __global__ void __launch_bounds__(NT2, 1) kda_chunk_bwd_dqk_kernel(const __grid_
     int L;
     if (!slot_rows(p, slot, c0, L)) return;
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + s2::BAR);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 5);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 6);
     if (tid == 0) {
-        for (int b = 0; b < 5; ++b) mbar_init(bars + b, 1);
+        for (int b = 0; b < 6; ++b) mbar_init(bars + b, 1);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -1215,8 +1353,8 @@ __global__ void __launch_bounds__(NT2, 1) kda_chunk_bwd_dqk_kernel(const __grid_
             // the bulk copies and every MMA issued so far land before the memory goes away
             if (fetched > 0) (void)mbar_wait(bars + 0, 0, kWaitNs);
             if (fetched > 1) (void)mbar_wait(bars + 2, 0, kWaitNs);
-            mma_commit(bars + 4);
-            (void)mbar_wait(bars + 4, 0, kWaitNs);
+            mma_commit(bars + 5);
+            (void)mbar_wait(bars + 5, 0, kWaitNs);
         }
     }
     tc_fence_before();
