@@ -46,9 +46,11 @@ METRIC = "KDA prefill tokens/s (% bf16 TC peak); decode step HBM GB/s (% of peak
 WORKLOAD = "prefill_b4_h16_t2048"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 SPEC_HBM_GBS = 7700.0   # nominal HBM3e bandwidth of one B200 (context for fractions of the copy peak)
-PREFILL_SRC = ["kimi_delta_attention_22_b200/csrc/kda_chunk_wy.cu",
-               "kimi_delta_attention_22_b200/csrc/kda_chunk_scan.cu",
-               "kimi_delta_attention_22_b200/csrc/kda_chunk_record.cuh"]
+_CSRC = "kimi_delta_attention_22_b200/csrc/"
+PREFILL_SRC = [_CSRC + f for f in ("kda_chunk_wy.cu", "kda_chunk_scan.cu", "kda_chunk_scan.cuh",
+                                   "kda_chunk_record.cuh", "kda_tc_common.cuh", "sm100.cuh")]
+CHUNK_BWD_SRC = PREFILL_SRC + [_CSRC + f for f in ("kda_chunk_bwd.cuh", "kda_chunk_bwd_scan.cu",
+                                                   "kda_chunk_bwd_grad.cu")]
 
 
 # ------------------------------------------------------------------ helpers
@@ -473,13 +475,16 @@ def bench_chunk_backward(args, world, peaks, peak_kind):
                        "l2": "3 rotating input sets > 126 MB L2"},
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / peaks["hbm_gbs"], "peak_source": f"{peak_kind} hbm_gbs",
-                         "algorithmic_bytes_per_launch": nbytes, "traffic": None,
-                         "kernel": "kda_chunk_bwd call (WY, forward scan with checkpoints, reverse "
-                                   "state scan, solve and dq/dk kernels)"},
+                         "algorithmic_bytes_per_launch": nbytes,
+                         "traffic": dram_traffic("chunk_bwd", WORKLOAD, CHUNK_BWD_SRC),
+                         "kernel": "kda_chunk_bwd call (WY, forward scan with checkpoints beside the "
+                                   "reverse state scan, solve and dq/dk kernels)"},
             "tensor": {"achieved_tflops": tf, "flops_per_launch": flops, "peak_tflops": peaks["bf16_tflops"],
                        "frac": tf / peaks["bf16_tflops"], "peak_source": f"{peak_kind} bf16_tflops (burst)"},
-            "kernels": "kda_chunk_wy_kernel, kda_chunk_scan_kernel, kda_chunk_bwd_scan_kernel, "
-                       "kda_chunk_bwd_solve_kernel, kda_chunk_bwd_dqk_kernel"}
+            "kernels": "kda_chunk_wy_kernel, kda_chunk_fwdbwd_scan_kernel, kda_chunk_bwd_solve_kernel, "
+                       "kda_chunk_bwd_dqk_kernel",
+            # per call: the two WY kernels, the paired scans, the solve and dq/dk kernels
+            "gpu_launches": 5 * iters}
 
 
 def bench_backward(args, world):

@@ -9,8 +9,9 @@
 //      the gradient of its outgoing state dS' and dE;
 //   3. and 4. the chunk-parallel gradient kernels (kda_chunk_bwd_grad.cu): per
 //      (chunk, head), the triangular-solve half (E, the solve's gradient, dv,
-//      dbeta) and then the rest (dq, dk, dg); their dense products run on the
-//      tensor cores, the decay-weighted Gram parts on CUDA cores.
+//      dbeta) and then the rest (dq, dk, dg); their products run on the tensor
+//      cores, the decay-weighted Gram parts too where one decay reference holds
+//      the chunk (on CUDA cores in fp32 otherwise).
 #pragma once
 
 #include "kda_chunk_record.cuh"

@@ -34,15 +34,25 @@
 // bits), with the products hi*hi + hi*lo + lo*hi summed in the fp32 accumulator;
 // dO is exact in fp16, and dPr, dEbar in dEbar E^T and the residual product's
 // operands are single fp16 (float64 emulation of the chunk: each adds < 5e-4).
-// The decay-weighted Gram products stay on CUDA cores in fp32, because their
-// factors span far more than fp16's range: the factor e^{Gamma_ic - Gamma_jc} is
+// The decay-weighted Gram products (A in the solve kernel, the two Grams' gradients
+// in the dqk kernel) have factors that span far more than fp16's range.  Where one
+// decay reference holds the chunk (max_c |G_last| <= 112, G = Gamma in log2 units)
+// they are tensor-core products over two-term bf16 operands K 2^G, K 2^-G, Q~ 2^G.
+// Otherwise they run on CUDA cores in fp32, with the factor e^{Gamma_ic - Gamma_jc}
 // split over 16-token sub-blocks I (of i) and J (of j), with the reference row
 // r(I) = 16 I + 7 (the forward's sub-block reference):
 //   a_ic = 2^{G_ic - G_r(I)c},  b_jc = 2^{G_r(J)c - G_jc} (each within its own sub-block),
-//   d^{IJ}_c = 2^{G_r(I)c - G_r(J)c} <= 1 (J < I),   (G = Gamma in log2 units)
+//   d^{IJ}_c = 2^{G_r(I)c - G_r(J)c} <= 1 (J < I),
 // so every Gram product and its gradient becomes a plain product of row-scaled
 // operands with a per-column factor per sub-block pair; a and b span at most 8
-// tokens of decay, which fp32 holds while a token's |g| < 10.9 per channel.
+// tokens of decay, which fp32 holds while a token's |g| < 10.9 per channel.  The
+// pair factor is applied in two steps split at the last row m(J) = 16 J + 15 of
+// sub-block J: first f1^J = 2^{G_m(J) - G_r(J)} (at most 8 tokens of decay, never
+// underflows), which brings the j-side to 2^{G_m(J) - G_j} <= 1, then
+// f2^{IJ} = 2^{G_r(I) - G_m(J)}.  Where f2 underflows, the term it drops is below
+// 2^-126 times an i-side factor of at most 2^101; a single factor d^{IJ} could
+// underflow against a j-side factor of up to 2^115 and drop a term as large as
+// 2^-11 (16 tokens of decay beyond 2^-126, some 5.5 nats per token).
 #include <cuda_bf16.h>
 
 #include "kda_chunk_bwd.cuh"
@@ -79,8 +89,8 @@ constexpr int KG16 = U;                            //   product 1: K e^Gamma (64
 constexpr int EBH = U, EBL = U + 16384;            //   products 2, 3: diag(beta) resid (hi, lo) and
 constexpr int DEH = U + 32768, DEL = U + 49152;    //   dE (hi, lo), MN-major over v
 constexpr int DB16 = U, E16 = U + 16384;           //   product 4: dEbar, E (hi) (K-major, 64 rows)
-constexpr int DFAC = U + 67584;    // fp32 [6][128]
-constexpr int SB = DFAC + 3072;    // fp32 [64] beta
+constexpr int DFAC = U + 67584;    // fp32 [9][128] pair factors f2, f1
+constexpr int SB = DFAC + 4608;    // fp32 [64] beta
 constexpr int RED = SB + 256;      // fp32 [4][64] dbeta partial sums
 constexpr int PS = RED + 1024;     // fp32 [3][16][16] inverse scratch
 constexpr int BAR = PS + 3072;     // 5 mbarriers, TMEM base
@@ -116,8 +126,8 @@ constexpr int KBH = OPS, KBL = OPS + 16384;           // K 2^-G, MN-major over t
 constexpr int QAH = OPS + 32768, QAL = OPS + 49152;   // Q~ 2^G
 constexpr int KAH = OPS + 65536, KAL = OPS + 81920;   // K 2^G
 constexpr uint32_t TM_X1 = 0, TM_X2 = 128, TM_Y = 256;
-constexpr int DFAC = DAT + 17408;  // fp32 [6][128]
-constexpr int UCOL = DFAC + 3072;  // fp32 [4][128] colsum(dKd . Kd) partials
+constexpr int DFAC = DAT + 17408;  // fp32 [9][128] pair factors f2, f1
+constexpr int UCOL = DFAC + 4608;  // fp32 [4][128] colsum(dKd . Kd) partials
 constexpr int SGS = UCOL + 2048;   // fp32 [16][128] colsum(S . dS') partials (one row per warp)
 constexpr int BAR = SGS + 8192;    // 6 mbarriers, TMEM base
 constexpr int BYTES = BAR + 64 + 1024;
@@ -268,15 +278,22 @@ __device__ __forceinline__ void load_gamma(const GradParams& p, long long c0, in
     }
 }
 
-// d^{IJ}_c for the six sub-block pairs J < I (NTH threads).
+// The pair factors (NTH threads): f2^{IJ}_c = 2^{G_r(I) - G_m(J)} for the six sub-block
+// pairs J < I (rows 0-5 of dfac), then f1^J_c = 2^{G_m(J) - G_r(J)} for J = 0..2 (rows 6-8).
 template <int NTH>
 __device__ __forceinline__ void load_dfac(const float* sG, float* dfac) {
-    for (int x = threadIdx.x; x < 6 * DK; x += NTH) {
+    for (int x = threadIdx.x; x < 9 * DK; x += NTH) {
         const int pi = x / DK, c = x % DK;
-        const int I = pi < 1 ? 1 : (pi < 3 ? 2 : 3), J = pi - I * (I - 1) / 2;
-        dfac[x] = ex2(sG[(16 * I + 7) * LD + c] - sG[(16 * J + 7) * LD + c]);
+        if (pi < 6) {
+            const int I = pi < 1 ? 1 : (pi < 3 ? 2 : 3), J = pi - I * (I - 1) / 2;
+            dfac[x] = ex2(sG[(16 * I + 7) * LD + c] - sG[(16 * J + 15) * LD + c]);
+        } else {
+            const int J = pi - 6;
+            dfac[x] = ex2(sG[(16 * J + 15) * LD + c] - sG[(16 * J + 7) * LD + c]);
+        }
     }
 }
+constexpr int F1 = 6;   // first dfac row of f1
 
 // n bf16 values (n = 8 or 32) of one row, or zeros past the chunk.
 template <int N>
@@ -487,7 +504,8 @@ __device__ __forceinline__ bool solve_body(const GradParams& p, uint8_t* sm, uin
         while ((ig + 1) * (ig + 2) / 2 <= tid) ++ig;   // tile tid = ig (ig + 1) / 2 + jg
         const int jg = tid - ig * (ig + 1) / 2, I = ig >> 2, J = jg >> 2;
         float acc[4][4] = {};
-        const float* dv = dfac + (J < I ? pair_index(I, J) : 0) * DK;
+        const float* dv = dfac + (J < I ? pair_index(I, J) : 0) * DK;   // f2
+        const float* d1 = dfac + (F1 + (J < 3 ? J : 0)) * DK;            // f1
 #pragma unroll 2
         for (int c = 0; c < DK; c += 4) {
             float4 a[4], b[4];
@@ -496,10 +514,15 @@ __device__ __forceinline__ bool solve_body(const GradParams& p, uint8_t* sm, uin
                 a[r] = ld4(Ka + (4 * ig + r) * LD + c);
                 b[r] = ld4(Kb + (4 * jg + r) * LD + c);
             }
-            if (J < I) {
-                const float4 d = ld4(dv + c);
+            if (J < I) {   // (b f1) f2, in this order
+                const float4 d = ld4(dv + c), e = ld4(d1 + c);
 #pragma unroll
-                for (int r = 0; r < 4; ++r) b[r].x *= d.x, b[r].y *= d.y, b[r].z *= d.z, b[r].w *= d.w;
+                for (int r = 0; r < 4; ++r) {
+                    b[r].x = (b[r].x * e.x) * d.x;
+                    b[r].y = (b[r].y * e.y) * d.y;
+                    b[r].z = (b[r].z * e.z) * d.z;
+                    b[r].w = (b[r].w * e.w) * d.w;
+                }
             }
 #pragma unroll
             for (int r = 0; r < 4; ++r)
@@ -1175,15 +1198,25 @@ __device__ __forceinline__ bool dqk_body(const GradParams& p, uint8_t* sm, uint3
                     }
                 }
             }
-            float4 dv = make_float4(1.f, 1.f, 1.f, 1.f);
-            if (J < I) dv = ld4(dfac + pair_index(I, J) * DK + 4 * cg);
+            if (J < I) {   // (t f1) f2, in this order
+                const float4 dv = ld4(dfac + pair_index(I, J) * DK + 4 * cg);
+                const float4 d1 = ld4(dfac + (F1 + J) * DK + 4 * cg);
 #pragma unroll
-            for (int r = 0; r < 4; ++r)
+                for (int r = 0; r < 4; ++r)
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    x1[r][c] = fmaf(comp(dv, c), t1[r][c], x1[r][c]);
-                    x2[r][c] = fmaf(comp(dv, c), t2[r][c], x2[r][c]);
-                }
+                    for (int c = 0; c < 4; ++c) {
+                        x1[r][c] = fmaf(comp(dv, c), t1[r][c] * comp(d1, c), x1[r][c]);
+                        x2[r][c] = fmaf(comp(dv, c), t2[r][c] * comp(d1, c), x2[r][c]);
+                    }
+            } else {
+#pragma unroll
+                for (int r = 0; r < 4; ++r)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        x1[r][c] += t1[r][c];
+                        x2[r][c] += t2[r][c];
+                    }
+            }
         }
         float xk[4][4], xq[4][4], xg[4][4];
         get16(0, xk);
@@ -1207,9 +1240,11 @@ __device__ __forceinline__ bool dqk_body(const GradParams& p, uint8_t* sm, uint3
         tmem_wait_st();
     }
     // ---- j side: Y = sum_{I' >= J} d^{I'J} (dAqk_{I',J}^T Q~a_I' + dA_{I',J}^T K a_I');
-    // dK += b . Y, dGamma -= K b . Y   (this thread's rows are j, in sub-block J = I)
+    // dK += b . Y, dGamma -= K b . Y   (this thread's rows are j, in sub-block J = I).  The
+    // diagonal sub-block's part goes in with b = 2^{G_r(J) - G_j}; the later ones' with
+    // f2 on the partial sums and b f1 = 2^{G_m(J) - G_j} <= 1 on the j side.
     {
-        float y[4][4] = {};
+        float y[4][4];
         for (int Ip = I; Ip < 4; ++Ip) {
             float t[4][4] = {};
 #pragma unroll 4
@@ -1225,25 +1260,47 @@ __device__ __forceinline__ bool dqk_body(const GradParams& p, uint8_t* sm, uint3
                     for (int c = 0; c < 4; ++c) t[r][c] = fmaf(w1, qa[c], fmaf(w2, ka[c], t[r][c]));
                 }
             }
-            float4 dv = make_float4(1.f, 1.f, 1.f, 1.f);
-            if (Ip > I) dv = ld4(dfac + pair_index(Ip, I) * DK + 4 * cg);
+            if (Ip == I) {
+                get16(0, xk);
+                get16(32, xg);
 #pragma unroll
-            for (int r = 0; r < 4; ++r)
+                for (int r = 0; r < 4; ++r) {
+                    const int j = 4 * ig + r;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) y[r][c] = fmaf(comp(dv, c), t[r][c], y[r][c]);
+                    for (int c = 0; c < 4; ++c) {
+                        const int cc = 4 * cg + c;
+                        const float b = ex2(sG[(16 * I + 7) * LD + cc] - sG[j * LD + cc]);
+                        xk[r][c] = fmaf(b, t[r][c], xk[r][c]);
+                        xg[r][c] -= Kb[j * LD + cc] * t[r][c];
+                        y[r][c] = 0.f;
+                    }
+                }
+                put16(0, xk);
+                put16(32, xg);
+                tmem_wait_st();
+            } else {
+                const float4 dv = ld4(dfac + pair_index(Ip, I) * DK + 4 * cg);
+#pragma unroll
+                for (int r = 0; r < 4; ++r)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) y[r][c] = fmaf(comp(dv, c), t[r][c], y[r][c]);
+            }
         }
         get16(0, xk);
         get16(16, xq);
         get16(32, xg);
+        if (I < 3) {
+            const float4 d1 = ld4(dfac + (F1 + I) * DK + 4 * cg);
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            const int j = 4 * ig + r;
+            for (int r = 0; r < 4; ++r) {
+                const int j = 4 * ig + r;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const int cc = 4 * cg + c;
-                const float b = ex2(sG[(16 * I + 7) * LD + cc] - sG[j * LD + cc]);
-                xk[r][c] = fmaf(b, y[r][c], xk[r][c]);
-                xg[r][c] -= Kb[j * LD + cc] * y[r][c];
+                for (int c = 0; c < 4; ++c) {
+                    const int cc = 4 * cg + c;
+                    const float bf = ex2(sG[(16 * I + 15) * LD + cc] - sG[j * LD + cc]);   // b f1
+                    xk[r][c] = fmaf(bf, y[r][c], xk[r][c]);
+                    xg[r][c] -= (Kb[j * LD + cc] * comp(d1, c)) * y[r][c];
+                }
             }
         }
     }

@@ -48,7 +48,11 @@ using namespace tc;
 
 constexpr int C = rec::C, DK = rec::DK, NT = 256;
 constexpr uint64_t kWaitNs = 1000000000ull;   // 1 s bound on every wait
-constexpr float kFastLimit2 = 112.f;          // one reference while max |Gamma_last| <= 2^112
+constexpr float kFastLimit2 = 112.f;          // one reference while max |Gamma_last| <= 112 (log2)
+// Two references while every 16-row sub-block's decay is <= 100 (log2): an i-side factor of
+// a row of half 1 over row 15 that underflows then meets a j-side factor <= 2^100, so the
+// product it drops is below 2^-26.
+constexpr float kTwoLimit2 = 100.f;
 constexpr int LDT = 68;                       // fp32 row stride of L and T (bank spread)
 constexpr int LDX = 20;                       // fp32 row stride of 16x16 block scratch
 constexpr uint32_t TMEM_COLS = 256;
@@ -68,7 +72,9 @@ struct WyMap<false> {                          // one-reference chunks, two CTAs
     static constexpr int KY = 49152;           //   rows 0-63 K e^{-G} (hi), rows 64-127 its lo term
     static constexpr int KG = KQ3;
     static constexpr int TOT4 = 98304;         // decay scan scratch (prep only)
-    static constexpr int GREF = TOT4 + 8192, GLAST = GREF + 2048, RED = GLAST + 512;
+    // GREF: the two-reference terms per channel, rows G_r0, G_r1, 2^{G_r0}, 2^{G_r1},
+    // 2^{G_last - G_r0}, 2^{G_last - G_r1}
+    static constexpr int GREF = TOT4 + 8192, GLAST = GREF + 3072, RED = GLAST + 512;
     static constexpr int L = 16384;            // after the Gram: fp32 L, T, Neumann blocks
     static constexpr int TF = L + 64 * LDT * 4;
     static constexpr int NS = TF + 64 * LDT * 4;
@@ -400,8 +406,10 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
             reinterpret_cast<float*>(rec_p + rec::DEC)[tid] = d;
         }
     }
-    // exclusive prefix over the 16 row groups, one thread per channel; the reference
-    // row of sub-block b is row 16 b + 7 (prefix before group 4 b + 2)
+    // exclusive prefix over the 16 row groups, one thread per channel.  Sub-block
+    // kernel: the reference row of sub-block b is row 16 b + 7 (prefix before group
+    // 4 b + 2).  One-reference kernel: the two-reference form's rows 15 and 47 (prefix
+    // before groups 4 and 12) and 2^{Gamma_15}.
     if (!ROWGATE && tid < DK) {
         float tv[16];
 #pragma unroll
@@ -409,7 +417,7 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
         float acc = 0.f;
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
-            if ((q & 3) == 2) gref_s[(q >> 2) * DK + tid] = acc;
+            if (SLOW && (q & 3) == 2) gref_s[(q >> 2) * DK + tid] = acc;
             const float t = tv[q];
             tv[q] = acc;
             acc += t;
@@ -417,17 +425,43 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
 #pragma unroll
         for (int q = 0; q < 16; ++q) tot4[q * DK + tid] = tv[q];
         glast_s[tid] = acc;
+        if (!SLOW) {
+            gref_s[tid] = tv[4];
+            gref_s[DK + tid] = tv[12];
+            gref_s[2 * DK + tid] = ex2(tv[4]);
+            gref_s[3 * DK + tid] = ex2(tv[12]);
+            gref_s[4 * DK + tid] = ex2(acc - tv[4]);
+            gref_s[5 * DK + tid] = ex2(acc - tv[12]);
+        }
         const float d = ex2(acc);
         dec_s[tid] = d;
         reinterpret_cast<float*>(rec_p + rec::DEC)[tid] = d;
-        float m = -acc;
+        // the chunk's decay, and the largest decay of one 16-row sub-block
+        float m = -acc, mb = fmaxf(fmaxf(-tv[4], tv[4] - tv[8]), fmaxf(tv[8] - tv[12], tv[12] - acc));
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        if (lane == 0) reinterpret_cast<float*>(sm + M::RED)[warp] = m;
+        for (int o = 16; o > 0; o >>= 1) {
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, o));
+        }
+        if (lane == 0) {
+            reinterpret_cast<float*>(sm + M::RED)[warp] = m;
+            reinterpret_cast<float*>(sm + M::RED)[4 + warp] = mb;
+        }
     }
     __syncthreads();
+    // Two references (one-reference kernel, per-channel gate): rows 15 and 47, each the
+    // reference of its 32-row half, for chunks whose decay is too large for one reference
+    // but within bounds over every 16-row sub-block.
+    // (re-read from shared memory where it is needed again: no register carries it)
+    auto two_ref = [&]() -> bool {
+        if (ROWGATE || SLOW) return false;
+        const volatile float* rv = red;
+        return fmaxf(fmaxf(rv[0], rv[1]), fmaxf(rv[2], rv[3])) > kFastLimit2 &&
+               fmaxf(fmaxf(rv[4], rv[5]), fmaxf(rv[6], rv[7])) <= kTwoLimit2;
+    };
+    const bool two = two_ref();
     if (!ROWGATE) fast = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3])) <= kFastLimit2;
-    if (!SLOW && !fast) {
+    if (!SLOW && !fast && !two) {
         if (tid == 0) {
             const int pos = atomicAdd(p.slow, 1);
             p.slow[1 + pos] = slot * H + h;
@@ -441,7 +475,7 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
     // the 16-byte chunks of this thread: (row 4 rg + r, channels c8..c8+7) in the
     // mnmaj_off(c, row, 128) layout shared by K e^G, Q~ e^G, K e^{-G}, Qg and Kd
     const uint32_t basemn = (uint32_t)((rg >> 1) * 2048 + (cq >> 3) * 1024 + (rg & 1) * 512);
-    if (!SLOW) {
+    if (!SLOW && !two) {
         // ================= one reference: 2^{Gamma_i} <= 1 on the i-side, 2^{-Gamma_j} <= 2^112 on
         // the j-side; one decay per row when the gate is scalar or absent
         float pre[8], dec[8];
@@ -494,6 +528,72 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
             *reinterpret_cast<uint4*>(g_wq + omn + 16384) = pack8_f16(qx);
             *reinterpret_cast<uint4*>(g_kd + omn) = pack8_f16(kd);
         }
+    } else if (!SLOW) {
+        // ================= two references: row r_h = 32 h + 15 for the rows of half h, so
+        // that each factor spans at most 16 rows of decay.  Columns j of half h take
+        // 2^{G_rh - G_j} (rows 32 h .. 32 h + 31 of K e^{-G}'s space: hi, then lo); rows i
+        // take 2^{G_i - G_rh} for h = 0 (every row) and h = 1 (rows of half 1).  The Gram
+        // runs column half 1 first with the rows of half 1 over r_1, then column half 0
+        // with those rows rebuilt over r_0, so rows 0-63 end as K 2^{G - G_r0}: the B
+        // operand of W, whose columns are scaled by 2^{G_r0} when read out.  Rows of half
+        // 1 park (G_i - G_r1, raw k, raw q) in tensor memory columns 192-255 meanwhile.
+        const int hh = rg >> 3;   // warp-uniform: warps 4-7 hold the rows of half 1
+        // per-channel terms come from shared memory row by row (register pressure):
+        // G_r (gref_s row hh), 2^{G_r} (row 2 + hh), 2^{G_last - G_r} (row 4 + hh), and this
+        // row group's prefix
+        auto ld8 = [](const float* src, float (&d)[8]) {
+            const float4 a = *reinterpret_cast<const float4*>(src), b = *reinterpret_cast<const float4*>(src + 4);
+            d[0] = a.x; d[1] = a.y; d[2] = a.z; d[3] = a.w; d[4] = b.x; d[5] = b.y; d[6] = b.z; d[7] = b.w;
+        };
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const uint32_t omn =
+                basemn + (((uint32_t)(cq & 7) ^ (uint32_t)(4 * (rg & 1) + r)) << 4) + (uint32_t)(r * 128);
+            float kf[8], qf[8], kx[8], qx[8], ky[8], t[8], dl[8], u[8];
+            ld8(tot4 + rg * DK + c8, dl);
+            ld8(gref_s + hh * DK + c8, u);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) dl[e] = (dl[e] + g2[r][e]) - u[e];   // G_i - G_r
+            if (hh) {   // parked for the rebuild over r_0: G_i - G_r1, raw k, raw q
+                uint32_t park[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) park[e] = __float_as_uint(dl[e]);
+                tmem_st8(tm + lane_base + 192u + 16u * r, park);
+                park[0] = kraw[r].x; park[1] = kraw[r].y; park[2] = kraw[r].z; park[3] = kraw[r].w;
+                park[4] = qraw[r].x; park[5] = qraw[r].y; park[6] = qraw[r].z; park[7] = qraw[r].w;
+                tmem_st8(tm + lane_base + 200u + 16u * r, park);
+            }
+            unpack8(kraw[r], kf);
+            unpack8(qraw[r], qf);
+            dqp[r] = 0.f;
+            ld8(gref_s + (4 + hh) * DK + c8, t);   // 2^{G_last - G_r}
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                dqp[r] = fmaf(kf[e], qf[e], dqp[r]);
+                const float x = ex2(dl[e]), y = ex2(-dl[e]);
+                qf[e] *= p.scale;
+                kx[e] = kf[e] * x;
+                qx[e] = qf[e] * x;
+                ky[e] = kf[e] * y;
+                // K e^{Gamma_last - Gamma}: where the first factor underflows, y <= 2^100 and the
+                // dropped value is below 2^-26
+                t[e] = kf[e] * (t[e] * y);
+            }
+            uint4 hi, lo;
+            st_shared_v4(sm + M::KQ3, omn, pack8(kx));
+            pack8_split(qx, hi, lo);
+            st_shared_v4(sm + M::KQ3, omn + 16384, hi);
+            st_shared_v4(sm + M::KQ3, omn + 32768, lo);
+            pack8_split(ky, hi, lo);
+            st_shared_v4(sm + M::KY, omn + 8192u * hh, hi);
+            st_shared_v4(sm + M::KY, omn + 8192u * hh + 8192u, lo);
+            *reinterpret_cast<uint4*>(g_kd + omn) = pack8_f16(t);
+            ld8(gref_s + (2 + hh) * DK + c8, u);   // 2^{G_r}
+#pragma unroll
+            for (int e = 0; e < 8; ++e) t[e] = qx[e] * u[e];   // Q~ e^{Gamma}
+            *reinterpret_cast<uint4*>(g_wq + omn + 16384) = pack8_f16(t);
+        }
+        if (hh) tmem_wait_st();
     } else {
         // ================= sub-block references
         const int b = rg >> 2;
@@ -511,7 +611,7 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
                 pre[e] = pv[e];
                 gr[e] = rv[e];
                 Er[e] = ex2(rv[e]);            // e^{Gamma_r}
-                Lr[e] = ex2(lv[e] - rv[e]);    // e^{Gamma_last - Gamma_r}
+                Lr[e] = lv[e] - rv[e];         // Gamma_last - Gamma_r (log2)
             }
 #pragma unroll
             for (int I = 1; I < 4; ++I) {
@@ -520,7 +620,7 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
                     const float4 i0 = ip[0], i1 = ip[1];
                     const float iv[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) z[I][e] = ex2(iv[e] - rv[e]);   // e^{Gamma_rI - Gamma_r} <= 1
+                    for (int e = 0; e < 8; ++e) z[I][e] = iv[e] - rv[e];   // Gamma_rI - Gamma_r (log2)
                 }
             }
         }
@@ -536,16 +636,16 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
             const uint32_t swz = ((sw0 ^ (uint32_t)(4 * (rg & 1) + r)) << 4) + (uint32_t)(r * 128);
             const uint32_t o128 = base128 + swz, omn = basemn + swz;
             const uint32_t oy = baseY + swz;   // + (I >> 1) * 32768 + (I & 1) * 8192 for version I
-            float kf[8], qf[8], x[8], y[8], t[8];
+            float kf[8], qf[8], x[8], y[8], t[8], dl[8];
             unpack8(kraw[r], kf);
             unpack8(qraw[r], qf);
             dqp[r] = 0.f;
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 dqp[r] = fmaf(kf[e], qf[e], dqp[r]);
-                const float dl = (pre[e] + g2[r][e]) - gr[e];   // Gamma_i - Gamma_r (log2)
-                x[e] = ex2(dl);
-                y[e] = ex2(-dl);
+                dl[e] = (pre[e] + g2[r][e]) - gr[e];   // Gamma_i - Gamma_r (log2)
+                x[e] = ex2(dl[e]);
+                y[e] = ex2(-dl[e]);
                 qf[e] *= p.scale;
             }
             uint4 hi, lo;
@@ -558,7 +658,10 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
             pack8_split(t, hi, lo);
             st_shared_v4(sm + M::OX, o128 + 2048, hi);
             st_shared_v4(sm + M::OXL, base64 + swz, lo);
-            // Gram j-side for this sub-block and the later ones (hi and lo)
+            // Gram j-side for this sub-block and the later ones (hi and lo); a later
+            // sub-block I's factor 2^{Gamma_rI - Gamma_j} <= 1 is one power, not the product
+            // of 2^{Gamma_r - Gamma_j} and 2^{Gamma_rI - Gamma_r}: the second can underflow
+            // where the product does not
             float ky[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) ky[e] = kf[e] * y[e];
@@ -569,7 +672,7 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
             for (int I = 1; I < 4; ++I) {
                 if (I > b) {
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) t[e] = ky[e] * z[I][e];
+                    for (int e = 0; e < 8; ++e) t[e] = kf[e] * ex2(z[I][e] - dl[e]);
                     pack8_split(t, hi, lo);
                     st_shared_v4(sm + M::OY + (I >> 1) * 32768 + (I & 1) * 8192, oy, hi);
                     st_shared_v4(sm + M::OYL + (I >> 1) * 32768 + (I & 1) * 8192, oy, lo);
@@ -586,7 +689,7 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
             st_shared_v4(sm + M::KG, omn, pack8(t));
             *reinterpret_cast<uint4*>(g_wq + omn + 16384) = pack8_f16(t2);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) t[e] = kf[e] * (Lr[e] * y[e]);
+            for (int e = 0; e < 8; ++e) t[e] = kf[e] * ex2(Lr[e] - dl[e]);   // one power, as above
             *reinterpret_cast<uint4*>(g_kd + omn) = pack8_f16(t);
         }
     }
@@ -603,7 +706,65 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
     // sub-blocks: group g (M = 128, N = 64): A rows 0-63 are the j-side of version 2g,
     // rows 64-127 that of version 2g+1 (hi, then lo); B rows the i-side rows of sub-blocks
     // 2g, 2g+1; cols 128 + 32 g: the same j-side (hi) against their Q~ lo rows (N = 32)
-    if (tid == 0) {
+    // two references: per column half h, cols 96 h + (0-31 hi, 32-63 lo) = the same
+    // products against the 32 j-side rows of half h, cols 96 h + 64 the lo * hi term
+    auto gram_half = [&](int h) {
+        const uint32_t kq = sbase + M::KQ3, ky = sbase + M::KY + 16384u * h;
+#pragma unroll
+        for (int s8 = 0; s8 < 8; ++s8)
+            mma_bf16(tm + TM_GRAM + 96 * h, rowview_desc(kq, s8), rowview_desc(ky, s8),
+                     idesc_bf16(128, 64, false, false), s8 > 0);
+#pragma unroll
+        for (int s8 = 0; s8 < 8; ++s8)
+            mma_bf16(tm + TM_GRAM + 96 * h + 64, rowview_desc(kq + 16384, s8), rowview_desc(ky, s8),
+                     idesc_bf16(128, 32, false, false), s8 > 0);
+        mma_commit(mma_bar);
+    };
+    if (!SLOW && two) {
+        if (tid == 0) gram_half(1);
+        if (!wait_all(mma_bar, mma_phase)) return 2;
+        tc_fence_after();
+        if (rg >= 8) {   // rows of half 1: the i-side over r_0 for column half 0
+            float d10[8];
+            {
+                const float4* a = reinterpret_cast<const float4*>(gref_s + c8);
+                const float4* b = reinterpret_cast<const float4*>(gref_s + DK + c8);
+                const float4 a0 = a[0], a1 = a[1], b0 = b[0], b1 = b[1];
+                d10[0] = b0.x - a0.x; d10[1] = b0.y - a0.y; d10[2] = b0.z - a0.z; d10[3] = b0.w - a0.w;
+                d10[4] = b1.x - a1.x; d10[5] = b1.y - a1.y; d10[6] = b1.z - a1.z; d10[7] = b1.w - a1.w;
+            }
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const uint32_t omn =
+                    basemn + (((uint32_t)(cq & 7) ^ (uint32_t)(4 * (rg & 1) + r)) << 4) + (uint32_t)(r * 128);
+                float park[16], kf[8], qf[8], kx[8], qx[8];
+                tmem_ld16(tm + lane_base + 192u + 16u * r, park);
+                const uint4 kr4 = make_uint4(__float_as_uint(park[8]), __float_as_uint(park[9]),
+                                             __float_as_uint(park[10]), __float_as_uint(park[11]));
+                const uint4 qr4 = make_uint4(__float_as_uint(park[12]), __float_as_uint(park[13]),
+                                             __float_as_uint(park[14]), __float_as_uint(park[15]));
+                unpack8(kr4, kf);
+                unpack8(qr4, qf);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float x = ex2(park[e] + d10[e]);   // 2^{G_i - G_r0} <= 1
+                    kx[e] = kf[e] * x;
+                    qx[e] = (qf[e] * p.scale) * x;
+                }
+                uint4 hi, lo;
+                st_shared_v4(sm + M::KQ3, omn, pack8(kx));
+                pack8_split(qx, hi, lo);
+                st_shared_v4(sm + M::KQ3, omn + 16384, hi);
+                st_shared_v4(sm + M::KQ3, omn + 32768, lo);
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        if (tid == 0) gram_half(0);
+    }
+    if (tid == 0 && !(!SLOW && two)) {
         if (!SLOW) {
             const uint32_t kq = sbase + M::KQ3, ky = sbase + M::KY;
 #pragma unroll
@@ -641,14 +802,22 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
     float* TF = reinterpret_cast<float*>(sm + M::TF);
     if (!SLOW) {
         // lane n = 32 sp + lane: row i of P (n < 64) or of Qp (n >= 64); columns 32 half ..
+        // (two references: lanes of rows outside column half 1's row range hold values of
+        // no meaning there, all above the diagonal and masked by selection)
         const int n = 32 * sp + lane, j0 = 32 * half;
-        float v[32], w[32];
-        tmem_ld32(tm + lane_base + TM_GRAM + j0, v);
-        tmem_ld32(tm + lane_base + TM_GRAM + 64 + j0, w);   // the hi * lo term
+        const bool tw = two_ref();
+        const uint32_t chh = tw ? 96u * half : (uint32_t)j0;              // hi * hi
+        const uint32_t chl = tw ? chh + 32u : 64u + j0;                    // hi * lo
+        const uint32_t clh = tw ? chh + 64u : 128u + j0;                   // lo * hi
+        float v[32];
+        {
+            float w[32];
+            tmem_ld32(tm + lane_base + TM_GRAM + chh, v);
+            tmem_ld32(tm + lane_base + TM_GRAM + chl, w);   // the hi * lo term
 #pragma unroll
-        for (int e = 0; e < 32; ++e) v[e] += w[e];
-        tmem_ld32(tm + lane_base + TM_GRAM + 128 + j0, w);  // lanes 64-127: the lo * hi term
-        if (n < 64) {
+            for (int e = 0; e < 32; ++e) v[e] += w[e];
+        }
+        if (n < 64) {   // warp-uniform (sub-partitions 0-1)
             const int i = n;
             const float bi = beta_s[i];
 #pragma unroll
@@ -663,6 +832,8 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
         } else {
             const int i = n - 64;
             const float dii = dq_s[i];
+            float w[32];
+            tmem_ld32(tm + lane_base + TM_GRAM + clh, w);   // the lo * hi term
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 float t8[8];
@@ -772,9 +943,24 @@ __device__ __forceinline__ int wy_job(const WyParams& p, uint8_t* sm, uint32_t t
             float v[32];
             tmem_ld32(tm + lane_base + TM_W + 64 * half + 32 * hc, v);
             if (lane < 16) {
+                // two references: W's columns take 2^{G_r0} (K e^G = (K 2^{G - G_r0}) 2^{G_r0})
+                const float4* f = reinterpret_cast<const float4*>(gref_s + 2 * DK + 64 * half + 32 * hc);
+                const bool tw = two_ref();
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
+                for (int q = 0; q < 4; ++q) {
+                    if (tw) {
+                        const float4 s0 = f[2 * q], s1 = f[2 * q + 1];
+                        v[8 * q] *= s0.x;
+                        v[8 * q + 1] *= s0.y;
+                        v[8 * q + 2] *= s0.z;
+                        v[8 * q + 3] *= s0.w;
+                        v[8 * q + 4] *= s1.x;
+                        v[8 * q + 5] *= s1.y;
+                        v[8 * q + 6] *= s1.z;
+                        v[8 * q + 7] *= s1.w;
+                    }
                     st_shared_v4(sm + M::WST, mnmaj_off(64 * half + 32 * hc + 8 * q, i, 128), pack8_f16(v + 8 * q));
+                }
             }
         }
         // U^T: lane = value row v, columns (tokens) 32 half .., hi term + lo term

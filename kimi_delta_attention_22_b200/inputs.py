@@ -10,6 +10,8 @@ the same values.  Recipe (per token and head):
   * gate g = log(alpha):
       "channel":        g = -softplus(N(0, 1)) per key channel, so alpha in (0, 1);
       "channel_strong": g = -Uniform(0, 5) per key channel;
+      "channel_extreme": g = -Uniform(0, 10) per key channel (close to the largest
+                        per-token decay the tensor-core paths hold exactly);
       "scalar":         g = -softplus(N(0, 1)) per (token, head), one value for all channels;
       "none":           no gate (alpha = 1).
   * S0 ~ N(0, s0_std^2) in fp32, or absent (zero state).
@@ -36,7 +38,7 @@ class Workload:
     d_k: int
     d_v: int
     dtype: str          # "f32" | "bf16" (q, k, v and out)
-    gate: str           # "channel" | "channel_strong" | "scalar" | "none"
+    gate: str           # "channel" | "channel_strong" | "channel_extreme" | "scalar" | "none"
     beta: str           # "sigmoid" | "one"
     chunk: int
     s0_std: float | None
@@ -128,6 +130,8 @@ def draw(B, T, H, d_k, d_v, *, dtype=torch.bfloat16, gate="channel", beta="sigmo
         g = -torch.nn.functional.softplus(torch.randn(B, T, H, d_k, **f32))
     elif gate == "channel_strong":
         g = -5.0 * torch.rand(B, T, H, d_k, **f32)
+    elif gate == "channel_extreme":
+        g = -10.0 * torch.rand(B, T, H, d_k, **f32)
     elif gate == "scalar":
         g = -torch.nn.functional.softplus(torch.randn(B, T, H, **f32))
     elif gate == "none":

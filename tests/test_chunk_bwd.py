@@ -85,9 +85,11 @@ def _mode(gate):
 
 def _gpu(d, cu=None, **kw):
     on = {k: (None if v is None else v.cuda()) for k, v in d.items()}
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
     res = kda.kda_chunk_bwd(on["q"], on["k"], on["v"], on["g"], on["beta"], on["S0"], on["d_out"],
-                            d_ST=on["d_ST"], cu_seqlens=None if cu is None else cu.cuda(), **kw)
+                            d_ST=on["d_ST"], cu_seqlens=None if cu is None else cu.cuda(), dev_status=status, **kw)
     torch.cuda.synchronize()
+    assert int(status.item()) == 0, f"device status {int(status.item()):#x}"
     return res
 
 
@@ -100,12 +102,46 @@ def _compare(got, ref, what):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("gate", ["channel", "scalar", "none", "channel_strong"])
+@pytest.mark.parametrize("gate", ["channel", "scalar", "none", "channel_strong", "channel_extreme"])
 def test_chunk_bwd_dense_matches_autograd(gate):
     d = _draw(2, 150, 2, gate, seed=3100 + len(gate))
     got = _gpu(d)
     ref = ob.backward(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], d["d_out"], d["d_ST"], gate=_mode(gate))
     _compare(got, ref, gate)
+
+
+@pytest.mark.gpu
+def test_chunk_bwd_mixed_decay_regimes():
+    """Chunks of one call needing one decay reference, two and sub-block references
+    (the gate of test_parity_gpu.mixed_decay_gate), ragged tail."""
+    from test_parity_gpu import mixed_decay_gate
+
+    d = _draw(2, 300, 2, "channel", seed=3130)
+    d["g"] = mixed_decay_gate(2, 300, 2, seed=3131)
+    got = _gpu(d)
+    ref = ob.backward(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], d["d_out"], d["d_ST"], gate="channel")
+    _compare(got, ref, "mixed")
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("gate", ["channel_extreme", "mixed"])
+def test_chunk_bwd_independent_of_scratch_contents(gate):
+    """The gradients do not depend on what the workspace held before the call: a
+    workspace of zero bytes and one of 0xFF bytes (NaN in every float format) give the
+    same, finite results."""
+    if gate == "mixed":
+        from test_parity_gpu import mixed_decay_gate
+
+        d = _draw(2, 300, 2, "channel", seed=3140)
+        d["g"] = mixed_decay_gate(2, 300, 2, seed=3141)
+    else:
+        d = _draw(2, 150, 2, gate, seed=3142)
+    sh = kda.Shape(2, d["v"].shape[1], 2, 128, 128, 2, kda.KDA_BF16, kda.KDA_GATE_CHANNEL, 64, None, 0)
+    nbytes = kda.load_library().kda_chunk_bwd_workspace_size(ctypes.byref(sh), 0)
+    res = [_gpu(d, workspace=torch.full((nbytes,), fill, dtype=torch.uint8, device="cuda")) for fill in (0, 255)]
+    for n in NAMES:
+        assert torch.isfinite(res[0][n]).all(), n
+        assert torch.equal(res[0][n], res[1][n]), n
 
 
 @pytest.mark.gpu

@@ -36,6 +36,7 @@ F32_CASES = [
     (32, 16, 64, 3, 65, 1, "none", True),
     (128, 64, 16, 1, 33, 2, "channel_strong", True),
     (48, 80, 32, 1, 1, 2, "channel", True),
+    (128, 128, 64, 1, 150, 2, "channel_extreme", True),
 ]
 
 
@@ -58,6 +59,8 @@ BF16_CASES = [
     (2, 190, 2, "channel_strong", "sigmoid", False, 64),
     (1, 1, 4, "channel", "sigmoid", True, 64),
     (2, 97, 2, "channel", "sigmoid", True, 32),
+    (2, 150, 2, "channel_extreme", "sigmoid", True, 64),
+    (1, 100, 2, "channel_extreme", "one", True, 32),
 ]
 
 
@@ -72,7 +75,7 @@ def test_bf16(B, T, H, gate, beta, s0, chunk, schedule):
     check(ST, rs, "bf16", "S_T")
 
 
-@pytest.mark.parametrize("gate,qk_div", [("channel", 1), ("channel_strong", 1), ("channel", 2)])
+@pytest.mark.parametrize("gate,qk_div", [("channel", 1), ("channel_strong", 1), ("channel_extreme", 1), ("channel", 2)])
 def test_whole_width_scan_matches_oracle(gate, qk_div):
     """More (sequence, head) pairs than SMs take the whole-width (N = 128) state
     scan: 2 x 90 heads, ragged 130-token sequences, one- and sub-block-reference
@@ -86,6 +89,50 @@ def test_whole_width_scan_matches_oracle(gate, qk_div):
     ro, rs = oracle_chunk(d, "channel")
     check(out, ro, "bf16", "out")
     check(ST, rs, "bf16", "S_T")
+
+
+def mixed_decay_gate(B, T, H, seed):
+    """Per-channel gates whose strength changes from chunk to chunk (64 tokens each):
+    -softplus(N(0,1)), -U(0,5), -U(0,10), -U(0,0.2), repeating; the tensor-core path
+    takes one decay reference, two references and sub-block references for them."""
+    gen = torch.Generator().manual_seed(seed)
+    g = torch.empty(B, T, H, 128)
+    for c0 in range(0, T, 64):
+        n = min(64, T - c0)
+        kind = (c0 // 64) % 4
+        if kind == 0:
+            g[:, c0:c0 + n] = -torch.nn.functional.softplus(torch.randn(B, n, H, 128, generator=gen))
+        else:
+            g[:, c0:c0 + n] = -(5.0, 10.0, 0.2)[kind - 1] * torch.rand(B, n, H, 128, generator=gen)
+    return g
+
+
+@pytest.mark.parametrize("schedule", ["workspace", "pool"])
+def test_mixed_decay_regimes_in_one_call(schedule):
+    """One call whose chunks need one reference, two references and sub-block
+    references (ragged tail included), against the oracle."""
+    d = inputs.draw(2, 300, 2, 128, 128, dtype=torch.bfloat16, s0_std=0.02, seed=91)
+    d["g"] = mixed_decay_gate(2, 300, 2, seed=92)
+    out, ST = run_chunk(d, 64, workspace=schedule == "workspace")
+    ro, rs = oracle_chunk(d, "channel")
+    check(out, ro, "bf16", "out")
+    check(ST, rs, "bf16", "S_T")
+
+
+def test_forward_independent_of_scratch_contents():
+    """out and S_T do not depend on what the workspace held: zero bytes and 0xFF bytes
+    (NaN in every float format) give the same, finite results (all three decay regimes)."""
+    import ctypes
+
+    d = inputs.draw(2, 300, 2, 128, 128, dtype=torch.bfloat16, s0_std=0.02, seed=93)
+    d["g"] = mixed_decay_gate(2, 300, 2, seed=94)
+    sh = kda.Shape(2, 300, 2, 128, 128, 2, kda.KDA_BF16, kda.KDA_GATE_CHANNEL, 64, None, 0)
+    nbytes = kda.load_library().kda_chunk_fwd_workspace_size(ctypes.byref(sh), 0)
+    res = [run_chunk(d, 64, workspace=torch.full((nbytes,), fill, dtype=torch.uint8, device="cuda"))
+           for fill in (0, 255)]
+    for a, b in zip(res[0], res[1]):
+        assert torch.isfinite(a.float()).all()
+        assert torch.equal(a, b)
 
 
 @pytest.mark.parametrize("schedule", ["workspace", "pool"])

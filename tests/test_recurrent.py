@@ -60,6 +60,7 @@ CASES = [
     (3, 5, 2, 96, torch.bfloat16, "scalar"),
     (2, 7, 1, 200, torch.float32, "none"),
     (1, 1, 4, 128, torch.bfloat16, "channel_strong"),
+    (2, 40, 2, 128, torch.bfloat16, "channel_extreme"),
 ]
 
 
