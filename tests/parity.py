@@ -66,10 +66,12 @@ def run_chunk(d, chunk, want_state=True, cu=None, workspace=True):
     workspace; None / False passes none, so the library draws its scratch from the
     stream-ordered pool (the same kernels either way)."""
     on = to_dev(d)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
     out, ST = kda.kda_chunk_fwd(on["q"], on["k"], on["v"], on["g"], on["beta"], S0=on["S0"],
                                 cu_seqlens=on.get("cu_seqlens") if cu is None else cu.cuda(),
-                                chunk=chunk, want_state=want_state, workspace=workspace)
+                                chunk=chunk, want_state=want_state, workspace=workspace, dev_status=status)
     torch.cuda.synchronize()
+    assert int(status.item()) == 0, f"device status {int(status.item()):#x}"
     return out, ST
 
 
