@@ -413,6 +413,9 @@ __device__ __forceinline__ bool solve_body(const GradParams& p, uint8_t* sm, uin
     // One decay reference for the whole chunk while its decay stays inside bf16's range
     // (max_c |G_last| <= 112): A = (K 2^G)(K 2^-G)^T as one tensor-core product over
     // two-term bf16 operands; otherwise the sub-block form on the CUDA cores in fp32.
+    // (The barrier first: G's last row gets its carry from another thread, and the
+    // predicate is read before __syncthreads_and synchronises.)
+    __syncthreads();
     const bool fast = __syncthreads_and(tid >= DK || sG[(C - 1) * LD + tid] >= -112.f) != 0;
     if (fast) {
 #pragma unroll
