@@ -78,12 +78,12 @@ def test_two_reference_gram_is_finite_and_close():
         checked += 1
         P = np.zeros((64, 64), dtype=np.float64)
         for h, r in ((0, 15), (1, 47)):
-            x = ex2(Gf - Gf[r])            # i-side over r (rows of half 0 or 1)
-            y = ex2(Gf[r] - Gf)            # j-side over r
             rows = np.arange(64) if h == 0 else np.arange(32, 64)
             cols = np.arange(32 * h, 32 * h + 32)
-            A = bf16(mul(k[rows], x[rows]))
-            yh, yl = split2(mul(k[cols], y[cols]))
+            x = ex2(Gf[rows] - Gf[r])      # i-side over r
+            y = ex2(Gf[r] - Gf[cols])      # j-side over r
+            A = bf16(mul(k[rows], x))
+            yh, yl = split2(mul(k[cols], y))
             assert np.all(np.isfinite(A)) and np.all(np.isfinite(yh)) and np.all(np.isfinite(yl))
             with np.errstate(over="ignore", invalid="ignore"):   # entries above the diagonal
                 part = A @ yh.T + A @ yl.T
