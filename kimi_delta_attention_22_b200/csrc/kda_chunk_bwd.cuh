@@ -1,8 +1,8 @@
 // kda_chunk_bwd.cuh -- launch interfaces and workspace layout of the chunkwise
 // backward (gradients of the tensor-core prefill; d_k = d_v = 128, chunk 64).
 //
-// The backward runs four launches on one stream:
-//   1. the forward's WY kernel: every chunk's record (kda_chunk_record.cuh);
+// The backward runs four kernels (five launches) on one stream:
+//   1. the forward's WY kernel, both launches: every chunk's record (kda_chunk_record.cuh);
 //   2. one launch of two independent scans side by side (kda_chunk_bwd_scan.cu): the
 //      forward's state scan with outputs off, keeping every chunk's incoming state
 //      S_c (fp32) in the workspace, and the reverse state scan: dS0, and per chunk
