@@ -2,8 +2,8 @@
 captured in a CUDA graph and replayed: the prefill with a caller workspace (its
 memset and programmatic-dependent launches), with pool scratch (stream-ordered
 allocation and release inside the graph), through the static scratch of the
-no-alloc entry point (after a first call outside the capture), the decode step
-and the recurrent pass, each replayed bit-identical to eager calls."""
+no-alloc entry point (after a first call outside the capture), the decode step,
+the recurrent pass and the chunkwise backward, each replayed as called eagerly."""
 import pytest
 import torch
 
@@ -83,3 +83,47 @@ def test_decode_and_recurrent_graph_replay():
     torch.cuda.synchronize()
     assert all(torch.equal(a, b) for a, b in zip(outs, outs_ref))
     assert torch.equal(S, S_ref) and torch.equal(o2, o2_ref) and torch.equal(S2, S2_ref)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("qk_heads", [None, 2])
+def test_chunk_bwd_graph_replay_equals_eager(qk_heads):
+    """The chunkwise backward with a caller workspace (five launches, the later ones
+    programmatic-dependent; grouped heads add a memset of dq, dk) replays in a graph
+    as called eagerly: bit-identical, or to fp32 rounding where grouped heads sum dq, dk
+    with atomics."""
+    import ctypes
+
+    B, T, H = 2, 150, 4
+    d = inputs.draw(B, T, H, 128, 128, dtype=torch.bfloat16, s0_std=0.02, seed=809, device="cuda",
+                    qk_heads=qk_heads)
+    gen = torch.Generator(device="cuda").manual_seed(810)
+    d_out = torch.randn(B, T, H, 128, device="cuda", generator=gen).to(torch.bfloat16)
+    d_ST = torch.randn(B, H, 128, 128, device="cuda", generator=gen)
+    sh = kda.Shape(B, T, H, 128, 128, B, kda.KDA_BF16, kda.KDA_GATE_CHANNEL, 64, None, qk_heads or 0)
+    ws = torch.empty(kda.load_library().kda_chunk_bwd_workspace_size(ctypes.byref(sh), 0), dtype=torch.uint8,
+                     device="cuda")
+
+    def call():
+        return kda.kda_chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], d_out, d_ST=d_ST,
+                                 workspace=ws)
+
+    ref = call()
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        call()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        res = call()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    for n in ("dq", "dk", "dv", "dg", "dbeta", "dS0"):
+        if qk_heads and n in ("dq", "dk"):
+            assert torch.allclose(res[n], ref[n], rtol=0, atol=1e-6 * float(ref[n].abs().max())), n
+        else:
+            assert torch.equal(res[n], ref[n]), n
