@@ -1097,8 +1097,12 @@ cudaError_t launch_wy_gate(const WyParams& p, long long slots, int sm_count, cud
     kf<<<dim3((unsigned)slots, (unsigned)p.H), NT, wy_smem_bytes<false>(), st>>>(pf);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+    // A quarter of the SMs: each of these CTAs (215 KB) holds its SM from the moment the
+    // one-reference kernel drains from it, so the state scan launched behind this kernel
+    // finds the other SMs free for its prologue while the one-reference kernel finishes.
     const long long jobs = slots * p.H;
-    const int grid = (int)(jobs < (long long)sm_count ? jobs : (long long)sm_count);
+    const int cap = sm_count / 4 > 0 ? sm_count / 4 : 1;
+    const int grid = (int)(jobs < (long long)cap ? jobs : (long long)cap);
     return launch_after(ks, dim3(grid), NT, wy_smem_bytes<true>(), st, p);
 }
 
