@@ -274,13 +274,17 @@ size_t kda_recurrent_bwd_workspace_size(const kda_shape_t* shape);
  * no backward derivation, so this is the chain rule of the chunk map that
  * kda_chunk_fwd computes (cumulative decay, decay-masked Gram products, the
  * triangular solve, the state and output products), undone chunk by chunk:
- *   1. the forward's records and, from a forward state scan, every chunk's
- *      incoming state (fp32, in the workspace);
- *   2. a reverse state scan on the tensor cores: with dS = d_ST, per chunk from
- *      the last, dE^T = dS Kd^T + dO^T Aqk and dS <- dS Diag(e^gamma) + dO^T Qg -
- *      dE^T W (the records' operands, fp16, fp32 accumulation); the final dS is dS0;
- *   3. per (chunk, head) in parallel, on CUDA cores in fp32: the triangular
- *      solve's gradient, dv and dbeta, then dq, dk and dg.
+ *   1. the forward's records;
+ *   2. in one launch, side by side: a forward state scan that keeps every chunk's
+ *      incoming state (fp32, in the workspace), and a reverse state scan on the
+ *      tensor cores: with dS = d_ST, per chunk from the last, dE^T = dS Kd^T +
+ *      dO^T Aqk and dS <- dS Diag(e^gamma) + dO^T Qg - dE^T W (the records'
+ *      operands, fp16, fp32 accumulation); the final dS is dS0;
+ *   3. per (chunk, head) in parallel: the triangular solve's gradient, dv and
+ *      dbeta, then dq, dk and dg.  The dense products run on the tensor cores over
+ *      two-term fp16 operands; the decay-weighted Gram products and their
+ *      gradients on the tensor cores over two-term bf16 operands where one decay
+ *      reference holds the chunk, on CUDA cores in fp32 otherwise.
  * Arguments as kda_chunk_fwd (dense or varlen through cu_seqlens, grouped value
  * heads through shape->qk_heads), plus:
  *   d_out  [B, T, H, d_v] bf16, 16-byte aligned
